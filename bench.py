@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of one MLA decode layer step on B200: append the step's tokens,
+absorb the queries, split-KV attention over the paged latent cache, combine with
+W^UV (libmla's three C-ABI calls).  Prints ONE JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl ours|reference]
+
+--config indexes the workloads in latent_compressed_attention_mla_b200.workloads
+(default 1: DeepSeek-V3 dims, B=1, L=4096, bf16).  With N>1 (torchrun) every
+rank runs an independent replica of the workload (weak scaling); the time is
+the max over ranks.  `--impl reference` times the CPU oracle (float64 numpy)
+on this host instead, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from latent_compressed_attention_mla_b200 import workloads as WL  # noqa: E402
+
+METRIC = "MLA decode: latent-cache TB/s, TFLOP/s and % of roofline; decode tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------
+# Algorithmic work of each kernel (bytes that must move, flops that must run)
+# ----------------------------------------------------------------------------
+def kernel_work(cfg: WL.MlaConfig, page_bytes: int) -> dict:
+    act = 4 if cfg.act_dtype == "f32" else 2
+    H, dc, dr, dn, dv, d = cfg.n_heads, cfg.d_c, cfg.d_rope, cfg.d_nope, cfg.d_v, cfg.d_model
+    D = dc + dr
+    N = cfg.B * cfg.T
+    row_bytes = page_bytes // cfg.page_size
+    seq = cfg.seq_lens.astype(np.int64)
+    keys_read = int(seq.sum())  # every cached row is read once per step
+    # (query, key) pairs: query t of sequence b sees L_b + t + 1 keys
+    pairs = int(sum(int(L) * cfg.T + cfg.T * (cfg.T + 1) // 2 for L in cfg.L))
+    return {
+        "append_project": {"bytes": D * d * act + N * d * act + N * D * 4, "flops": 2 * N * D * d},
+        "append_finalize": {"bytes": N * D * 4 + N * row_bytes, "flops": 0},
+        "plan": {"bytes": cfg.B * 8, "flops": 0},
+        "absorb": {"bytes": H * dn * dc * act + N * H * (dn + dr) * act + N * H * D * act, "flops": 2 * N * H * dn * dc},
+        "attend": {"bytes": keys_read * row_bytes + N * H * D * act, "flops": 2 * pairs * H * (D + dc),
+                   "cache_bytes": keys_read * row_bytes, "pairs": pairs},
+        "combine": {"bytes": H * dv * dc * act + N * H * dv * act, "flops": 2 * N * H * dv * dc},
+    }
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = None
+        self.gpu = gpu_index
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t0: float, t1: float) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[1].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+            except Exception:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        # samples inside the timed region (1 s granularity of the timestamp), else nearest ones
+        inside = [r for r in rows if t0 - 1.0 <= r[0] <= t1 + 1.0] or rows[-3:]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[1] for r in inside])), "sm_max_mhz": float(max(r[2] for r in inside)),
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (the reported CPU baseline and the reference arm)
+# ----------------------------------------------------------------------------
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class OracleStep:
+    """One step of the workload on the CPU oracle: the oracle's append of the
+    step's tokens and its explicit-form decode.  `heads` bounds the sample."""
+
+    def __init__(self, cfg: WL.MlaConfig, seqs, heads):
+        from oracle import mla_oracle as O
+        self.O, self.cfg, self.seqs, self.heads = O, cfg, list(seqs), list(heads)
+        self.w = {k: v.double().numpy() for k, v in WL.weights(cfg, "cpu").items()}
+        self.inp = {k: v.double().numpy() for k, v in WL.step_inputs(cfg, "cpu").items()}
+        self.seq_idx, self.pos = WL.new_token_index(cfg)
+        self.hist = {}
+        for b in self.seqs:
+            r = WL.history_rows(cfg, b, 0, int(cfg.L[b]), "cpu")
+            r = {k: (v.numpy() if v.dtype == torch.uint8 else v.double().numpy()) for k, v in r.items()}
+            self.hist[b] = O.decode_cache_rows(r)
+
+    def __call__(self):
+        O, cfg = self.O, self.cfg
+        for b in self.seqs:
+            n = np.nonzero(self.seq_idx == b)[0]
+            c, kr = O.append_latent(self.inp["h"][n], self.w["W_dkv"], self.w["W_kr"], self.pos[n], cfg.rope_base)
+            C1, KR1 = O.decode_cache_rows(O.encode_cache_rows(c, kr, cfg.cache_dtype))
+            C = np.concatenate([self.hist[b][0], C1])
+            KR = np.concatenate([self.hist[b][1], KR1])
+            O.decode_explicit(self.inp["q_nope"][b], self.inp["q_rope"][b], C, KR, self.w["W_uk"], self.w["W_uv"],
+                              int(cfg.seq_lens[b]), cfg.softmax_scale, cfg.rope_base, self.heads)
+
+    def tokens_per_call(self) -> float:
+        """Decode tokens the call covers, counting a head sample as that fraction of a token."""
+        return len(self.seqs) * self.cfg.T * len(self.heads) / self.cfg.n_heads
+
+
+def oracle_sample(cfg: WL.MlaConfig, budget_s: float):
+    """A sample of the workload sized so one call takes about budget_s: all
+    heads of a few sequences when that fits, else a head subset."""
+    rng = np.random.default_rng(0)
+    seqs = [int(np.argmin(cfg.L))] if cfg.B > 1 else [0]
+    probe = OracleStep(cfg, seqs, [0])
+    t = time.perf_counter()
+    probe()
+    per_head = max(time.perf_counter() - t, 1e-4)
+    n_heads = int(max(1, min(cfg.n_heads, budget_s / per_head)))
+    heads = sorted(rng.choice(cfg.n_heads, n_heads, replace=False).tolist()) if n_heads < cfg.n_heads else \
+        list(range(cfg.n_heads))
+    return OracleStep(cfg, seqs, heads), probe
+
+
+def describe_sample(s: OracleStep) -> str:
+    return (f"oracle append + explicit decode of sequence(s) {s.seqs} (L={[int(s.cfg.L[b]) for b in s.seqs]}), "
+            f"{len(s.heads)} of {s.cfg.n_heads} heads, {s.cfg.T} query token(s) each; "
+            f"tokens/s counts a head sample as that fraction of a token")
+
+
+def cpu_baseline(cfg: WL.MlaConfig, budget_s: float = 15.0) -> dict:
+    step, _ = oracle_sample(cfg, budget_s / 3)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        step()
+        n += 1
+        if time.perf_counter() - t0 >= budget_s or n >= 50:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n * step.tokens_per_call() / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": describe_sample(step) + f"; {n} calls in {dt:.1f} s"}
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    total = args.steps + args.warmup
+    per_step_budget = max(0.2, 150.0 / max(total, 1))
+    step, _ = oracle_sample(cfg, per_step_budget)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = args.steps * step.tokens_per_call() / dt
+    cores = blas_threads()
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(cfg, None), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": describe_sample(step)},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(cfg, extra):
+    d = {"workload": cfg.name, "batch": cfg.B, "n_q": cfg.T,
+         "context_before_step": int(cfg.L[0]) if len(set(cfg.L)) == 1 else
+         {"min": int(min(cfg.L)), "max": int(max(cfg.L)), "sum": int(sum(cfg.L))},
+         "n_heads": cfg.n_heads, "d_c": cfg.d_c, "d_rope": cfg.d_rope, "d_nope": cfg.d_nope, "d_v": cfg.d_v,
+         "d_model": cfg.d_model, "page_size": cfg.page_size, "cache": cfg.cache_dtype, "act": cfg.act_dtype,
+         "seed": cfg.seed}
+    if extra:
+        d.update(extra)
+    return d
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--flags", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = WL.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    from latent_compressed_attention_mla_b200 import binding as B
+    from latent_compressed_attention_mla_b200.decoder import MlaDecodeSession
+    from latent_compressed_attention_mla_b200.paged_cache import PagedLatentCache
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    dims = B.dims_for(cfg, args.flags)
+    page_bytes = B.cache_page_bytes(dims)
+    work = kernel_work(cfg, page_bytes)
+
+    # one copy of everything a step touches; rotate copies when one fits in L2
+    weights0 = WL.weights(cfg, dev)
+    inputs0 = WL.step_inputs(cfg, dev)
+    pt = torch.from_numpy(WL.page_table(cfg)).to(dev)
+    seq_idx, pos = (torch.from_numpy(x).to(dev) for x in WL.new_token_index(cfg))
+    seq_lens = torch.from_numpy(cfg.seq_lens.astype(np.int32)).to(dev)
+    cache0 = PagedLatentCache(dims, cfg.num_pages, dev)
+    for b in range(cfg.B):
+        L = int(cfg.L[b])
+        for s0 in range(0, L, 1 << 18):
+            s1 = min(L, s0 + (1 << 18))
+            cache0.write_rows(pt[b], torch.arange(s0, s1, device=dev), WL.history_rows(cfg, b, s0, s1, dev))
+    per_copy = sum(t.numel() * t.element_size() for t in list(weights0.values()) + list(inputs0.values()))
+    per_copy += cache0.pool.numel()
+    copies = 1 if per_copy > 3 * L2_BYTES else int(math.ceil(3 * L2_BYTES / per_copy))
+    sets = [(weights0, inputs0, cache0.pool)]
+    for _ in range(copies - 1):
+        sets.append(({k: v.clone() for k, v in weights0.items()}, {k: v.clone() for k, v in inputs0.items()},
+                     cache0.pool.clone()))
+    sess = MlaDecodeSession(dims, cfg.B, cfg.T, args.splits, dev)
+    splits = args.splits or B.auto_splits(dims, cfg.B, cfg.T)
+    path = B.decode_path(dims, cfg.T)
+
+    def step(i):
+        w, x, pool = sets[i % copies]
+        sess.step(x["h"], seq_idx, pos, x["q_nope"], x["q_rope"], seq_lens, w, pt, pool)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if B.mla_get_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    # per-kernel events: a ring of event sets, read back 32 steps behind
+    nk = len(B.TRACE_KERNELS)
+    RING = 32
+    ring = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(RING)]
+    ksum = np.zeros(nk)
+
+    def harvest(evs):
+        evs[-1].synchronize()
+        for k in range(nk):
+            ksum[k] += evs[2 * k].elapsed_time(evs[2 * k + 1])
+
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    t_start_wall = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        if i >= RING:
+            harvest(ring[i % RING])
+        B.mla_set_trace_events(ring[i % RING])
+        step(args.warmup + i)
+    e1.record()
+    torch.cuda.synchronize()
+    B.mla_set_trace_events(None)
+    t_end_wall = time.time()
+    for i in range(max(0, args.steps - RING), args.steps):
+        harvest(ring[i % RING])
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop(t_start_wall, t_end_wall)
+    ms = e0.elapsed_time(e1)
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    status = B.mla_get_status()
+
+    tokens_per_step = cfg.B * cfg.T
+    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    kms = {name: ksum[k] / args.steps for k, name in enumerate(B.TRACE_KERNELS)}  # ms per launch
+    peaks = load_peaks()
+    long_region = ms > 1000.0
+    tpeak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
+    rows = {}
+    for name, t in kms.items():
+        wk = work[name]
+        t_s = t / 1e3
+        t_bytes = wk["bytes"] / (peaks["hbm_gbs"] * 1e9)
+        t_flops = wk["flops"] / (tpeak * 1e12)
+        bound = "tensor" if t_flops > t_bytes else "hbm"
+        rows[name] = {"us": 1e3 * t, "GBps": wk["bytes"] / t_s / 1e9 if t_s > 0 else None,
+                      "TFLOPs": wk["flops"] / t_s / 1e12 if t_s > 0 else None, "bound": bound,
+                      "roofline_frac": (max(t_bytes, t_flops) / t_s) if t_s > 0 else None}
+    dom = max(kms, key=lambda k: kms[k])
+    wd, td = work[dom], kms[dom] / 1e3
+    if rows[dom]["bound"] == "tensor":
+        roof = {"bound": "tensor", "achieved": wd["flops"] / td / 1e12, "peak": tpeak, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": wd["bytes"] / td / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["peak_source"] = peaks["source"] + (" sustained" if (roof["bound"] == "tensor" and long_region) else
+                                             (" burst" if roof["bound"] == "tensor" else " copy"))
+    att = work["attend"]
+    t_att = kms["attend"] / 1e3
+    t_core = max(att["cache_bytes"] / (peaks["hbm_gbs"] * 1e9), att["flops"] / (tpeak * 1e12))
+    attend_summary = {"latent_cache_TBps": att["cache_bytes"] / t_att / 1e12, "TFLOPs": att["flops"] / t_att / 1e12,
+                      "core_roofline_us": 1e6 * t_core, "frac_of_core_roofline": t_core / t_att,
+                      "path": "tcgen05" if path == 1 else "simt", "splits": splits}
+
+    # end to end through the public API: pinned host inputs -> device -> step -> host output
+    host_in = {k: v.cpu().pin_memory() for k, v in inputs0.items()}
+    host_out = torch.empty(sess.out.shape, dtype=sess.out.dtype).pin_memory()
+    dev_in = {k: torch.empty_like(v) for k, v in inputs0.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+    for i in range(min(args.warmup, 5)):
+        w, _, pool = sets[i % copies]
+        sess.step_from_host(host_in, dev_in, seq_idx, pos, seq_lens, w, pt, pool, host_out)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for i in range(args.steps):
+        w, _, pool = sets[i % copies]
+        sess.step_from_host(host_in, dev_in, seq_idx, pos, seq_lens, w, pt, pool, host_out)
+    f1.record()
+    torch.cuda.synchronize()
+    ms_e2e = f0.elapsed_time(f1)
+    if pg:
+        t = torch.tensor([ms_e2e], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e = {"value": world * tokens_per_step * args.steps / (ms_e2e / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg)
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return
+    l2 = (f"inputs rotate over {copies} copies ({copies * per_copy / 2**20:.0f} MiB > 126 MiB L2)" if copies > 1
+          else f"inputs ({per_copy / 2**30:.2f} GiB) larger than L2")
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.act_dtype if cfg.cache_dtype != "fp8" else "bf16+e4m3-cache",
+        "data": "synthetic (seeded counter-based generator; random-init weights)",
+        "config": config_dict(cfg, {"l2": l2, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                                    "splits": splits}),
+        "roofline": roof, "attend": attend_summary, "kernels_us": {k: round(v["us"], 3) for k, v in rows.items()},
+        "kernel_roofline_frac": {k: (round(v["roofline_frac"], 4) if v["roofline_frac"] else None)
+                                 for k, v in rows.items()},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": nk * args.steps, "clocks": clocks,
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

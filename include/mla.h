@@ -1,0 +1,201 @@
+/*
+ * mla.h - C ABI of libmla: Multi-Head Latent Attention (MLA) decode on a paged
+ * latent cache, absorbed form, for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the decode step of "DeepSeek MLA Architecture: How
+ * Multi-Head Latent Attention Cuts KV Cache by 93%" (explore.n1n.ai):
+ *   - each token caches only c = W^DKV h (d_c scalars, "1. Low-Rank Key-Value
+ *     Compression") and one shared, pre-rotated RoPE key k^R = RoPE(W^KR h)
+ *     (d_rope scalars, "3. Decoupled RoPE and Matrix Absorption");
+ *   - a query is absorbed into latent space, q~_h = (W^UK_h)^T q^C_h, and
+ *     scored directly against the cached rows: score = q~_h . c_s + q^R_h . k^R_s
+ *     ("3. Decoupled RoPE and Matrix Absorption", eq. for q~ and the split
+ *     score), scaled by 1/sqrt(d_nope + d_rope);
+ *   - the softmax-weighted latent sum u_h = sum_s p_s c_s is formed in latent
+ *     space and W^UV_h is applied afterwards, o_h = W^UV_h u_h.
+ * The page's single-token decoding module appends the step's token and then
+ * attends; this library splits that step into three calls (append, decode,
+ * combine) over a caller-owned paged cache.
+ *
+ * General conventions
+ *   - Every pointer argument is a DEVICE pointer owned by the caller unless
+ *     stated otherwise.  The library allocates no device memory: scratch is the
+ *     caller's `workspace`, sized by the matching *_workspace_bytes() call.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *     is the legacy default stream).  Nothing synchronises except
+ *     mla_get_status().  Kernels run on the current CUDA device.
+ *   - Return value: MLA_OK, or an MLA_ERR_* code for errors the host can see
+ *     (bad arguments, unsupported shapes, small workspace, misalignment, a
+ *     failed launch).  Errors that depend on device-resident values (an
+ *     out-of-range page index, a sequence shorter than n_q) are recorded in a
+ *     device status word; the offending row or work item is skipped, and
+ *     mla_get_status() reports the code.
+ *   - Row-major layouts; "[a, b, c]" lists dimensions outermost first.
+ *   - Tensors of "act" type are float32 (MLA_F32) or bfloat16 (MLA_BF16)
+ *     according to mla_dims.act_dtype.
+ *
+ * Paged cache layout (`cache_pool`, num_pages pages of page_size tokens):
+ *   MLA_F32 / MLA_BF16 cache: page = [page_size][d_c + d_rope] rows of that
+ *     type; a row is [c (d_c) | k^R (d_rope)].  bf16 V3 dims: 1152 B per row.
+ *   MLA_FP8_E4M3 cache: page = [page_size][d_c] e4m3 codes of c, then
+ *     [page_size][d_rope] bf16 k^R, then [page_size][d_c/128] fp32 scales;
+ *     c[j] = e4m3(code[j]) * scale[j/128], scale = amax of the 128-wide tile
+ *     / 448 (1 for an all-zero tile).  Sub-blocks start at multiples of 128 B.
+ *   mla_cache_page_bytes() gives the page size in bytes.
+ *   Token `pos` of sequence b lives in row pos % page_size of physical page
+ *   page_table[b * max_pages + pos / page_size].
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1, MLA_FP8_E4M3 = 2 } mla_dtype;
+
+enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent dims */
+  MLA_ERR_UNSUPPORTED = 2, /* dims/dtypes with no kernel */
+  MLA_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than required */
+  MLA_ERR_ALIGNMENT = 4,   /* a pointer not 16-byte aligned */
+  MLA_ERR_LAUNCH = 5,      /* a kernel launch failed (cudaGetLastError) */
+  MLA_ERR_TIMEOUT = 6,     /* device: a bounded wait in a kernel gave up */
+  MLA_ERR_BOUNDS = 7,      /* device: page index / position / length out of range */
+  MLA_ERR_CUDA = 8         /* a CUDA runtime call failed */
+};
+
+/* mla_dims.flags */
+#define MLA_FLAG_FORCE_SIMT 1u /* use the CUDA-core kernels even where tcgen05 kernels exist */
+
+typedef struct {
+  int32_t n_heads;     /* n_h (128 for DeepSeek-V3) */
+  int32_t d_c;         /* latent rank (512); multiple of 16; multiple of 128 for FP8 */
+  int32_t d_rope;      /* decoupled RoPE width (64); even */
+  int32_t d_nope;      /* per-head content query/key width (128) */
+  int32_t d_v;         /* per-head value width (128) */
+  int32_t d_model;     /* model width d (7168); multiple of 8 */
+  int32_t page_size;   /* tokens per cache page (64) */
+  int32_t act_dtype;   /* mla_dtype: MLA_F32 or MLA_BF16 */
+  int32_t cache_dtype; /* mla_dtype: MLA_F32 (needs act F32), MLA_BF16 or MLA_FP8_E4M3 (need act BF16) */
+  float softmax_scale; /* 1/sqrt(d_nope + d_rope) in the pages' module */
+  float rope_base;     /* 10000 */
+  uint32_t flags;      /* MLA_FLAG_* */
+} mla_dims;
+
+/* Bytes of one cache page (host only, no GPU needed). 0 if dims are invalid. */
+size_t mla_cache_page_bytes(const mla_dims* dims);
+
+/* Host-side validation of dims (no GPU needed): MLA_OK or an error code. */
+int mla_check_dims(const mla_dims* dims);
+
+/* ---------------------------------------------------------------------------
+ * S1  mla_append_latent: write the latent rows of n_tokens new tokens.
+ *   c_n = W_dkv h_n                    ("1. Low-Rank Key-Value Compression")
+ *   k^R_n = RoPE(W_kr h_n, pos[n])     ("3. Decoupled RoPE and Matrix Absorption";
+ *                                       rotate-half RoPE of the decoding module,
+ *                                       angle pos * rope_base^(-i/(d_rope/2)))
+ * and store [c_n | k^R_n] at (seq_idx[n], pos[n]) of the paged cache, rounded
+ * to the cache type (fp32 accumulation; RNE to bf16; FP8 per the layout above).
+ *   h          [n_tokens, d_model] act
+ *   seq_idx    [n_tokens] int32, sequence of each token, in [0, batch)
+ *   pos        [n_tokens] int32, position of each token, >= 0
+ *   W_dkv      [d_c, d_model] act;  W_kr [d_rope, d_model] act
+ *   page_table [batch, max_pages] int32
+ *   cache_pool num_pages pages (layout above), written
+ *   workspace  >= mla_append_workspace_bytes(dims, n_tokens) bytes of scratch
+ * Out-of-range seq_idx/pos/page entries: the token is skipped and
+ * MLA_ERR_BOUNDS is recorded in the device status word.  n_tokens == 0 is a no-op.
+ * ------------------------------------------------------------------------- */
+size_t mla_append_workspace_bytes(const mla_dims* dims, int n_tokens);
+int mla_append_latent(const mla_dims* dims, const void* h, int n_tokens,
+                      const int32_t* seq_idx, const int32_t* pos,
+                      const void* W_dkv, const void* W_kr,
+                      const int32_t* page_table, int batch, int max_pages,
+                      void* cache_pool, int num_pages,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * S2+S3  mla_decode: absorb the queries and run split-KV attention over the
+ * cache, leaving per-split partial results in `workspace` for mla_combine.
+ *   For sequence b, query j (position p = seq_lens[b] - n_q + j), head h:
+ *     q~ = W_uk[h]^T q_nope[b,j,h]             (absorption, eq. for q~)
+ *     q^R = RoPE(q_rope[b,j,h], p)
+ *     a_s = softmax_scale * (q~ . c_s + q^R . k^R_s),   s = 0 .. p
+ *   and, per split of the keys, the normalised latent aggregate
+ *   u = sum_s softmax(a)_s c_s with its log-sum-exp.
+ * The query j of a sequence sees keys 0..p: causal among the n_q new tokens,
+ * which must already be in the cache (append first, then attend).
+ *   q_nope     [batch, n_q, n_heads, d_nope] act
+ *   q_rope     [batch, n_q, n_heads, d_rope] act, NOT rotated
+ *   W_uk       [n_heads, d_nope, d_c] act
+ *   cache_pool, num_pages, page_table [batch, max_pages], as above (read only)
+ *   seq_lens   [batch] int32, tokens in the cache per sequence (>= n_q)
+ *   num_splits number of key-range splits shared by all sequences; 0 = auto
+ *   workspace  >= mla_decode_workspace_bytes(dims, batch, n_q, num_splits)
+ * The workspace is consumed by the next mla_combine with the same dims, batch,
+ * n_q and num_splits.
+ * ------------------------------------------------------------------------- */
+size_t mla_decode_workspace_bytes(const mla_dims* dims, int batch, int n_q, int num_splits);
+int mla_decode(const mla_dims* dims, const void* q_nope, const void* q_rope,
+               const void* W_uk, const void* cache_pool, int num_pages,
+               const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+               int batch, int n_q, int num_splits,
+               void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * S4  mla_combine: merge the splits and apply the value up-projection.
+ *   u = sum_i exp(lse_i - LSE) u_i,  LSE = log sum_i exp(lse_i)
+ *   o_h = W_uv[h] u_h  ("value aggregation ... directly against c", with W^UV
+ *                       applied after the softmax, as in the decoding module)
+ *   W_uv    [n_heads, d_v, d_c] act
+ *   out     [batch, n_q, n_heads, d_v] act, written
+ *   lse_out [batch, n_q, n_heads] float32 natural-log softmax denominators of
+ *           the scaled scores, written; may be NULL
+ * `workspace`, `batch`, `n_q`, `num_splits` as passed to the mla_decode call
+ * whose results are combined.
+ * ------------------------------------------------------------------------- */
+int mla_combine(const mla_dims* dims, const void* W_uv, int batch, int n_q, int num_splits,
+                const void* workspace, size_t ws_bytes, void* out, float* lse_out,
+                void* stream);
+
+/* Which decode kernel mla_decode would launch for these dims on the current
+ * device: 0 = CUDA-core (SIMT) kernel, 1 = tcgen05 kernel; <0 = error code. */
+int mla_decode_path(const mla_dims* dims, int n_q);
+
+/* Number of key-range splits that num_splits = 0 selects on the current device. */
+int mla_auto_splits(const mla_dims* dims, int batch, int n_q);
+
+/* Tracing.  Kernels of the calls above, in launch order per step: */
+enum {
+  MLA_TRACE_APPEND_PROJECT = 0, /* mla_append_latent: [W_dkv; W_kr] h */
+  MLA_TRACE_APPEND_FINALIZE = 1,/* mla_append_latent: RoPE, rounding, paged store */
+  MLA_TRACE_PLAN = 2,           /* mla_decode: split plan from seq_lens */
+  MLA_TRACE_ABSORB = 3,         /* mla_decode: q~ = W_uk^T q_nope, RoPE(q_rope) */
+  MLA_TRACE_ATTEND = 4,         /* mla_decode: split-KV attention over the cache */
+  MLA_TRACE_COMBINE = 5,        /* mla_combine: split merge and W_uv */
+  MLA_TRACE_COUNT = 6
+};
+/* Install a table of 2*MLA_TRACE_COUNT cudaEvent_t (passed as void*, created
+ * by the caller with timing enabled): later calls record events[2k] before and
+ * events[2k+1] after kernel k on the launch stream.  NULL uninstalls.  The
+ * table is process-wide host state read at launch time; it is not
+ * thread-safe.  Returns MLA_OK or MLA_ERR_INVALID_ARG (n_events too small). */
+int mla_set_trace_events(void* const* events, int n_events);
+
+/* Synchronise `stream`, then read and clear the device status word of the
+ * current device into *status (MLA_OK or MLA_ERR_TIMEOUT / MLA_ERR_BOUNDS).
+ * Returns MLA_OK, or MLA_ERR_CUDA if the synchronisation failed. */
+int mla_get_status(void* stream, int* status);
+
+/* Static description of an error code (never NULL). */
+const char* mla_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_H_ */

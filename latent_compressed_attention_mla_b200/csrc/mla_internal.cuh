@@ -1,0 +1,174 @@
+// Internal declarations shared by the libmla translation units (device helpers,
+// workspace layout, kernel launchers).  Not part of the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <type_traits>
+
+#include "../../include/mla.h"
+
+namespace mla {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kE4M3Max = 448.0f;
+
+// ----------------------------------------------------------------------------
+// Device status word: kernels record errors that depend on device-resident
+// values (bad page index, short sequence, expired bounded wait) here.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void record_status(int* status, int code) {
+  if (status) atomicMax(status, code);
+}
+
+// ----------------------------------------------------------------------------
+// Element access
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Load 8 consecutive bf16 (one 16-byte vector) as floats.
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
+  uint4 v = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+// Load 8 consecutive floats (two 16-byte vectors).
+__device__ __forceinline__ void load8(const float* p, float* f) {
+  float4 a = *reinterpret_cast<const float4*>(p);
+  float4 b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+__device__ __forceinline__ float e4m3_to_float(uint8_t code) {
+  __nv_fp8_e4m3 v;
+  v.__x = code;
+  return float(v);
+}
+
+// RoPE angle cos/sin for rotation pair i of a d_rope-wide vector at position
+// pos: angle = pos * base^(-i/(d_rope/2)), evaluated in double precision and
+// rounded to float (positions reach 1.3e5, where a float angle loses ~1e-2 rad).
+__device__ __forceinline__ void rope_cos_sin(int pos, int i, int half, float base, float* c, float* s) {
+  double inv_freq = exp(-log((double)base) * (double)i / (double)half);
+  double ang = (double)pos * inv_freq;
+  *c = (float)cos(ang);
+  *s = (float)sin(ang);
+}
+
+// ----------------------------------------------------------------------------
+// Decode workspace layout (shared by mla_decode and mla_combine)
+//   plan  : int32 [batch + 1] first key tile of each sequence (prefix sum of
+//           ceil(seq_len / page_size)), then int32 [4] {total tiles, splits,
+//           batch, n_q}
+//   q_abs : [batch, n_q, n_heads, d_c + d_rope] act type (absorbed queries,
+//           rotated q^R appended)
+//   o_part: float32 [n_q, n_slots, n_heads, d_c] per-split normalised latent sums
+//   lse   : float32 [n_q, n_slots, n_heads] per-split log2-sum-exp2 of the scores
+//           scaled by softmax_scale*log2(e) (-inf for an empty split)
+// A split w covers global key tiles [w*TT/W, (w+1)*TT/W) of the concatenated
+// sequences; its piece of sequence b goes to slot w + b (n_slots = batch + W - 1).
+// ----------------------------------------------------------------------------
+struct DecodeLayout {
+  size_t off_plan, off_q, off_o, off_lse, total;
+  int splits, n_slots;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline DecodeLayout decode_layout(const mla_dims& d, int batch, int n_q, int splits) {
+  DecodeLayout L;
+  L.splits = splits;
+  L.n_slots = batch + splits - 1;
+  size_t act = d.act_dtype == MLA_F32 ? 4 : 2;
+  size_t D = (size_t)d.d_c + d.d_rope;
+  size_t off = 0;
+  L.off_plan = off;
+  off = align_up(off + sizeof(int32_t) * ((size_t)batch + 1 + 4), 256);
+  L.off_q = off;
+  off = align_up(off + act * (size_t)batch * n_q * d.n_heads * D, 256);
+  L.off_o = off;
+  off = align_up(off + 4 * (size_t)n_q * L.n_slots * d.n_heads * d.d_c, 256);
+  L.off_lse = off;
+  off = align_up(off + 4 * (size_t)n_q * L.n_slots * d.n_heads, 256);
+  L.total = off;
+  return L;
+}
+
+// Tile range of split w: [w*TT/W, (w+1)*TT/W).
+__host__ __device__ __forceinline__ long long split_tile_begin(int w, long long TT, int W) {
+  return (long long)w * TT / W;
+}
+
+// Index of the sequence that owns global tile g: the largest b with tile_start[b] <= g.
+__device__ __forceinline__ int seq_of_tile(const int32_t* tile_start, int batch, long long g) {
+  int lo = 0, hi = batch;  // tile_start[0] = 0 <= g
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if ((long long)tile_start[mid] <= g) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+struct DecodeParams {
+  mla_dims d;
+  const void* q_abs;       // workspace q_abs
+  const uint8_t* pool;     // cache pool
+  size_t page_bytes;
+  int num_pages;
+  const int32_t* page_table;
+  int max_pages;
+  const int32_t* seq_lens;
+  const int32_t* plan;     // tile_start [batch+1], then {TT, W, batch, n_q}
+  float* o_part;
+  float* lse_part;
+  int batch, n_q, splits, n_slots;
+  float scale_log2;        // softmax_scale * log2(e)
+  int* status;
+};
+
+// Tracing hook: events installed by mla_set_trace_events (may be null).
+void trace_record(int kernel, bool end, cudaStream_t st);
+
+// ----------------------------------------------------------------------------
+// Launchers (host side), each returning cudaError_t of the launch.
+// ----------------------------------------------------------------------------
+cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const int32_t* seq_idx,
+                          const int32_t* pos, const void* W_dkv, const void* W_kr,
+                          const int32_t* page_table, int batch, int max_pages, void* pool,
+                          int num_pages, size_t page_bytes, float* raw, int* status,
+                          cudaStream_t st);
+
+cudaError_t launch_plan(const int32_t* seq_lens, int batch, int n_q, int page_size, int max_pages,
+                        int splits, int32_t* plan, int* status, cudaStream_t st);
+
+cudaError_t launch_absorb(const mla_dims& d, const void* q_nope, const void* q_rope, const void* W_uk,
+                          const int32_t* seq_lens, int batch, int n_q, void* q_abs, cudaStream_t st);
+
+cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t st);
+
+bool decode_tc_supported(const mla_dims& d, int n_q);
+cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st);
+int decode_tc_auto_splits(int num_sms, int n_q);
+
+cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n_q, int splits,
+                           int n_slots, const int32_t* plan, const float* o_part,
+                           const float* lse_part, void* out, float* lse_out, cudaStream_t st);
+
+}  // namespace mla
