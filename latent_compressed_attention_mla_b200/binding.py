@@ -180,5 +180,8 @@ def mla_set_trace_events(events):
     if events is None:
         _check(lib().mla_set_trace_events(None, 0), "mla_set_trace_events")
         return
+    for e in events:  # torch creates the CUDA event lazily, on first record
+        if not e.cuda_event:
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check(lib().mla_set_trace_events(arr, len(events)), "mla_set_trace_events")

@@ -1,13 +1,632 @@
-// S3 on the 5th-generation tensor cores (tcgen05, TMEM, TMA): placeholder
-// until the kernel lands; mla_decode falls back to the CUDA-core kernel.
+// S3 on the 5th-generation tensor cores: split-KV attention of the absorbed
+// queries over the paged bf16 latent cache, DeepSeek-V3 dims (128 heads,
+// 576-wide rows = 512 latent + 64 RoPE, 64-token pages).
+//
+// What it computes ("DeepSeek MLA Architecture: How Multi-Head Latent Attention
+// Cuts KV Cache by 93%", "3. Decoupled RoPE and Matrix Absorption" and the
+// decoding module's steps 4-5): for each head, scores q~.c_s + q^R.k^R_s over
+// the cached rows (one 576-wide dot product against [c_s | k^R_s]), an online
+// softmax, and the probability-weighted sum of the latent rows c_s themselves.
+// W^UV is applied later, by the combine kernel.
+//
+// Design (B200):
+//  * A CTA pair (cluster of 2) runs one split of the keys.  The 128 heads are
+//    the M dimension of cta_group::2 tcgen05 MMAs: each CTA holds the absorbed
+//    queries of 64 heads (72 KB of shared memory); the pair's tensor cores
+//    exchange the B operand halves, so every CTA sees all keys of a tile.
+//  * Per 64-key tile (one page):
+//      QK : S[64 heads x 64 keys] = Q[64 x 576] . K^T   (M=128 pair, N=64, K=576)
+//      PV : O[64 heads x 512]    += P[64 x 64] . C[64 x 512]  (two N=256 MMAs)
+//    S (2 buffers) and O live in tensor memory (TMEM); per CTA S uses 2 x 32
+//    columns and O 2 x 128 columns of the 2-SM ("2x2") accumulator layout:
+//    row m, column n < N/2 -> lane m, column n; n >= N/2 -> lane 64+m, n-N/2.
+//  * TMA loads, 128-byte swizzle: per tile each CTA loads its 32-key half of
+//    the rows (all 576 columns, the QK B operand, K-major) and all 64 keys of
+//    its 256-column half of the latent (the PV B operand, MN-major).
+//  * Warp roles: warps 0-3 softmax + epilogue (one TMEM lane each), warp 4
+//    TMA producer, warp 5 TMEM allocation and (leader CTA) MMA issue.
+//  * Online softmax in base 2 with a lazily updated reference max: O is only
+//    rescaled when a tile's max exceeds the reference by more than 8 (in
+//    log2 units), so probabilities stay <= 2^8 and rescaling is rare.
+//  * Every mbarrier wait is bounded; on expiry the kernel records
+//    MLA_ERR_TIMEOUT in the status word and unwinds.
+#include <cuda.h>
+
 #include "mla_internal.cuh"
 
 namespace mla {
 
-bool decode_tc_supported(const mla_dims&, int) { return false; }
+namespace {
 
-int decode_tc_auto_splits(int num_sms, int n_q) { return num_sms / 2 / (n_q > 0 ? n_q : 1); }
+// ---------------------------------------------------------------------------
+// Fixed shape of this kernel
+// ---------------------------------------------------------------------------
+constexpr int kHeads = 128, kHalfHeads = 64;
+constexpr int kDC = 512, kDR = 64, kD = kDC + kDR;  // 576
+constexpr int kPage = 64;                             // keys per tile
+constexpr int kChunks = kD / 64;                      // 9 column chunks of 64 (128 B)
+constexpr int kStages = 2;
 
-cudaError_t launch_decode_tc(const DecodeParams&, cudaStream_t) { return cudaErrorNotSupported; }
+// shared memory layout (offsets from a 1024-byte aligned base)
+constexpr uint32_t kQBytes = kChunks * 64 * 128;           // 73728: 64 heads x 576 bf16
+constexpr uint32_t kKQChunk = 32 * 128;                    // 4096: 32 keys x 64 cols
+constexpr uint32_t kKQBytes = kChunks * kKQChunk;          // 36864
+constexpr uint32_t kPVChunk = 64 * 128;                    // 8192: 64 keys x 64 cols
+constexpr uint32_t kPVBytes = 4 * kPVChunk;                // 32768
+constexpr uint32_t kStageBytes = kKQBytes + kPVBytes;      // 69632
+constexpr uint32_t kPBytes = 64 * 128;                     // 8192: 64 heads x 64 keys bf16
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffStage = kOffQ + kQBytes;
+constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;  // 212992
+constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;              // 229376
+constexpr uint32_t kNumBars = 16;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kOffRedMax = kOffMisc + 16;                 // float [2][64]
+constexpr uint32_t kOffRedL = kOffRedMax + 512;                // float [2][64]
+constexpr uint32_t kSmemUsed = kOffRedL + 512;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;              // + alignment slack
+
+// barrier indices
+enum {
+  B_KV_FULL = 0,   // [2] leader: TMA bytes of both CTAs
+  B_KV_EMPTY = 2,  // [2] each CTA: stage consumed (MMA commit)
+  B_S_FULL = 4,    // [2] each CTA: S tile ready (MMA commit)
+  B_S_FREE = 6,    // [2] leader: S read by both CTAs' softmax warps (8 arrivals)
+  B_P_FULL = 8,    // [2] leader: P written + O rescaled by both CTAs (8 arrivals)
+  B_O_DONE = 10,   // each CTA: a PV group finished (MMA commit)
+  B_O_FREE = 11,   // leader: O read out by both CTAs' epilogues (8 arrivals)
+  B_Q_FULL = 12,   // leader: Q bytes of both CTAs
+  B_Q_EMPTY = 13,  // each CTA: last QK of a segment finished (MMA commit)
+};
+
+// TMEM columns (per CTA, 2x2 layout): S buffers 32 columns each, O 2 x 128
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 32, kColO0 = 128, kColO1 = 256;
+
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s
+
+// instruction descriptors (kind::f16, bf16 x bf16 -> f32, dense)
+constexpr uint32_t idesc(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+constexpr uint32_t kIdescQK = idesc(128, 64, false, false);
+constexpr uint32_t kIdescPV = idesc(128, 256, false, true);
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+// arrive on a barrier given by its shared::cluster address (own or peer CTA)
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait.  Returns false (and records MLA_ERR_TIMEOUT) if the phase does
+// not complete within the limit or another role of this CTA already gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort_flag = 1;
+      record_status(status, MLA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t cluster_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(cluster_bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc_,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc_), "r"(accumulate)
+      : "memory");
+}
+
+// arrive on the barrier at this offset in both CTAs of the pair when all
+// tcgen05 operations issued so far by this thread complete
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// ---------------------------------------------------------------------------
+// Work partition (shared by all roles): split w of query t covers global key
+// tiles [w*TT/W, (w+1)*TT/W); pieces per sequence are segments.
+// ---------------------------------------------------------------------------
+struct Segment {
+  int b, tile_lo, n_tiles, nvis;  // n_tiles: tiles with at least one visible key
+};
+
+struct SegmentWalker {
+  const int32_t* ts;
+  const int32_t* seq_lens;
+  int batch, n_q, t, b;
+  long long g, g1;
+  __device__ SegmentWalker(const DecodeParams& p, int w, int t_) {
+    ts = p.plan;
+    seq_lens = p.seq_lens;
+    batch = p.batch;
+    n_q = p.n_q;
+    t = t_;
+    const long long TT = ts[batch];
+    g = split_tile_begin(w, TT, p.splits);
+    g1 = split_tile_begin(w + 1, TT, p.splits);
+    b = g < g1 ? seq_of_tile(ts, batch, g) : 0;
+  }
+  __device__ bool next(Segment& s) {
+    if (g >= g1) return false;
+    while ((long long)ts[b + 1] <= g) ++b;
+    const long long end = min(g1, (long long)ts[b + 1]);
+    s.b = b;
+    s.tile_lo = (int)(g - ts[b]);
+    const int tile_hi = (int)(end - ts[b]);
+    s.nvis = seq_lens[b] - n_q + t + 1;
+    const int vis_tiles = (s.nvis + kPage - 1) / kPage;
+    s.n_tiles = max(0, min(tile_hi, vis_tiles) - s.tile_lo);
+    g = end;
+    return true;
+  }
+};
+
+struct TcParams {
+  DecodeParams p;
+  CUtensorMap map_q;   // q_abs [rows = batch*n_q*128][576] bf16, box 64 x 64
+  CUtensorMap map_kq;  // pool rows [num_pages*64][576] bf16, box 64 x 32
+  CUtensorMap map_pv;  // pool rows [num_pages*64][576] bf16, box 64 x 64
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    decode_tc_kernel(const __grid_constant__ TcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const DecodeParams& p = P.p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();  // 0 = leader (issues the MMAs)
+  const int pair = blockIdx.x >> 1;
+  const int t = pair % p.n_q, w = pair / p.n_q;
+
+  auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * i; };
+  auto leader_bar = [&](int i) -> uint32_t { return map_to_rank(bar(i), 0); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc + 4);
+  float* red_max = reinterpret_cast<float*>(smem + kOffRedMax);
+  float* red_l = reinterpret_cast<float*>(smem + kOffRedL);
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_KV_FULL + i), 1);
+      mbar_init(bar(B_KV_EMPTY + i), 1);
+      mbar_init(bar(B_S_FULL + i), 1);
+      mbar_init(bar(B_S_FREE + i), 8);
+      mbar_init(bar(B_P_FULL + i), 8);
+    }
+    mbar_init(bar(B_O_DONE), 1);
+    mbar_init(bar(B_O_FREE), 8);
+    mbar_init(bar(B_Q_FULL), 1);
+    mbar_init(bar(B_Q_EMPTY), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0) {
+      SegmentWalker walk(p, w, t);
+      Segment s;
+      uint32_t g = 0, seg = 0;
+      bool ok = true;
+      while (ok && walk.next(s)) {
+        if (s.n_tiles == 0) continue;
+        // absorbed queries of this CTA's 64 heads for (b, t)
+        if (seg > 0) ok = mbar_wait(bar(B_Q_EMPTY), (seg - 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        if (rank == 0) mbar_expect_tx(bar(B_Q_FULL), 2 * kQBytes);
+        const int qrow = ((s.b * p.n_q + t) * kHeads) + kHalfHeads * (int)rank;
+        const uint32_t qbar = leader_bar(B_Q_FULL);
+        for (int c = 0; c < kChunks; ++c) tma_load_2d_pair(sbase + kOffQ + c * 8192, &P.map_q, 64 * c, qrow, qbar);
+        for (int i = 0; i < s.n_tiles; ++i, ++g) {
+          const int st = g % kStages;
+          ok = mbar_wait(bar(B_KV_EMPTY + st), ((g / kStages) & 1) ^ 1, abort_flag, p.status);
+          if (!ok) break;
+          int page = p.page_table[(size_t)s.b * p.max_pages + s.tile_lo + i];
+          if (page < 0 || page >= p.num_pages) {
+            record_status(p.status, MLA_ERR_BOUNDS);
+            page = 0;
+          }
+          if (rank == 0) mbar_expect_tx(bar(B_KV_FULL + st), 2 * kStageBytes);
+          const uint32_t kbar = leader_bar(B_KV_FULL + st);
+          const uint32_t stage = sbase + kOffStage + st * kStageBytes;
+          const int row0 = page * kPage;
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_2d_pair(stage + c * kKQChunk, &P.map_kq, 64 * c, row0 + 32 * (int)rank, kbar);
+          // PV operand: chunks {2r, 2r+1} (dims 128r..) and {4+2r, 5+2r} (dims 256+128r..)
+          for (int j = 0; j < 2; ++j)
+            for (int a = 0; a < 2; ++a)
+              tma_load_2d_pair(stage + kKQBytes + (2 * j + a) * kPVChunk, &P.map_pv, 64 * (4 * j + 2 * (int)rank + a),
+                               row0, kbar);
+        }
+        ++seg;
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA
+    if (rank == 0 && lane == 0) {
+      SegmentWalker walk(p, w, t);
+      Segment s;
+      uint32_t g = 0, seg = 0;
+      bool ok = true;
+      auto do_pv = [&](uint32_t gi, bool first) -> bool {
+        if (!mbar_wait(bar(B_P_FULL + (gi & 1)), (gi >> 1) & 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const int st = gi % kStages;
+        const uint32_t pv = sbase + kOffStage + st * kStageBytes + kKQBytes;
+        const uint32_t pa = sbase + kOffP + (gi & 1) * kPBytes;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            tc_mma(tmem + (j ? kColO1 : kColO0), sdesc(pa + ks * 32, 16, 1024),
+                   sdesc(pv + 2 * j * kPVChunk + ks * 2048, kPVChunk, 1024), kIdescPV,
+                   (first && ks == 0) ? 0u : 1u);
+        tc_commit_pair(bar(B_KV_EMPTY + st));
+        tc_commit_pair(bar(B_O_DONE));
+        return true;
+      };
+      while (ok && walk.next(s)) {
+        if (s.n_tiles == 0) continue;
+        ok = mbar_wait(bar(B_Q_FULL), seg & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t g_first = g;
+        for (int i = 0; i < s.n_tiles && ok; ++i, ++g) {
+          const int st = g % kStages;
+          ok = mbar_wait(bar(B_KV_FULL + st), (g / kStages) & 1, abort_flag, p.status) &&
+               mbar_wait(bar(B_S_FREE + (g & 1)), ((g >> 1) & 1) ^ 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t kq = sbase + kOffStage + st * kStageBytes;
+#pragma unroll 4
+          for (int k = 0; k < kD / 16; ++k) {
+            const uint32_t off = (k & 3) * 32;  // 16 columns = 32 bytes into the swizzled row
+            tc_mma(tmem + ((g & 1) ? kColS1 : kColS0), sdesc(sbase + kOffQ + (k >> 2) * 8192 + off, 16, 1024),
+                   sdesc(kq + (k >> 2) * kKQChunk + off, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
+          }
+          tc_commit_pair(bar(B_S_FULL + (g & 1)));
+          if (i == s.n_tiles - 1) tc_commit_pair(bar(B_Q_EMPTY));
+          if (i > 0) {
+            if (i == 1 && seg > 0) {  // O of the previous segment must be read out first
+              ok = mbar_wait(bar(B_O_FREE), (seg - 1) & 1, abort_flag, p.status);
+              if (!ok) break;
+            }
+            ok = do_pv(g - 1, g - 1 == g_first);
+          }
+        }
+        if (!ok) break;
+        if (s.n_tiles == 1 && seg > 0) {
+          ok = mbar_wait(bar(B_O_FREE), (seg - 1) & 1, abort_flag, p.status);
+          if (!ok) break;
+        }
+        ok = do_pv(g - 1, g - 1 == g_first);
+        ++seg;
+      }
+    }
+  } else {
+    // ------------------------------------------------------- softmax, epilogue
+    const int L = warp * 32 + lane;  // TMEM lane of this thread
+    const int hl = L & 63, half = L >> 6;
+    const int head = kHalfHeads * (int)rank + hl;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    SegmentWalker walk(p, w, t);
+    Segment s;
+    uint32_t g = 0;
+    bool ok = true;
+    while (walk.next(s)) {
+      const size_t slot = (size_t)t * p.n_slots + (w + s.b);
+      float* od = p.o_part + (slot * kHeads + head) * kDC;
+      if (s.n_tiles == 0 || !ok) {
+        for (int j = 0; j < 2; ++j)
+          for (int c = 0; c < 128; c += 4)
+            *reinterpret_cast<float4*>(od + 256 * j + 128 * half + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (half == 0) p.lse_part[slot * kHeads + head] = -INFINITY;
+        continue;
+      }
+      float m_ref = -INFINITY, l_part = 0.f;
+      for (int i = 0; i < s.n_tiles; ++i, ++g) {
+        ok = mbar_wait(bar(B_S_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.status);
+        __syncwarp();
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[32];
+        tmem_ld32(tmem + lane_base + ((g & 1) ? kColS1 : kColS0), sr);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_bar(B_S_FREE + (g & 1)));
+        const int key0 = (s.tile_lo + i) * kPage + 32 * half;
+        float sv[32];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          sv[j] = key0 + j < s.nvis ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sv[j]);
+        }
+        red_max[half * 64 + hl] = mx;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const float tile_max = fmaxf(mx, red_max[(half ^ 1) * 64 + hl]);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        bool rescale = false;
+        float alpha = 1.f;
+        if (i == 0) {
+          m_ref = tile_max;
+        } else if (tile_max > m_ref + kRescaleThreshold) {
+          rescale = true;
+          alpha = fast_exp2(m_ref - tile_max);
+          m_ref = tile_max;
+        }
+        uint32_t pk[16];
+        float psum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(fast_exp2(sv[2 * j] - m_ref), fast_exp2(sv[2 * j + 1] - m_ref));
+          const float2 f2 = __bfloat1622float2(h2);
+          psum += f2.x + f2.y;
+          pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        l_part = l_part * alpha + psum;
+        if (i > 0) {  // PV of the previous tile must be done before O or its P buffer is touched
+          ok = mbar_wait(bar(B_O_DONE), (g - 1) & 1, abort_flag, p.status);
+          __syncwarp();
+          if (!ok) break;
+          tc_fence_after();
+        }
+        // tcgen05.ld/st are whole-warp instructions: rescale the warp's lanes
+        // together (alpha = 1 on lanes whose head keeps its reference max)
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+          for (int c = 0; c < 256; c += 32) {
+            const uint32_t col = (c < 128 ? kColO0 + c : kColO1 + (c - 128));
+            uint32_t orr[32];
+            tmem_ld32(tmem + lane_base + col, orr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
+            tmem_st32(tmem + lane_base + col, orr);
+          }
+          tmem_wait_st();
+        }
+        // P row hl, keys [32*half, 32*half+32): four 16-byte units, 128-byte swizzle
+        uint8_t* prow = smem + kOffP + (g & 1) * kPBytes + hl * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = (4 * half + u) ^ (hl & 7);
+          *reinterpret_cast<uint4*>(prow + unit * 16) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+        // rows past the sequence end in the last tile: zero this CTA's latent
+        // operand rows so that 0 * (whatever the pool held) cannot reach O
+        const int valid = s.nvis - (s.tile_lo + i) * kPage;
+        if (valid < kPage) {
+          uint8_t* pv = smem + kOffStage + (g % kStages) * kStageBytes + kKQBytes;
+          const int rows = kPage - valid;
+          for (int x = threadIdx.x; x < rows * 4 * 8; x += 128) {
+            const int r = valid + x / 32, rem = x % 32, c = rem / 8, u = rem % 8;
+            *reinterpret_cast<uint4*>(pv + c * kPVChunk + r * 128 + u * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (lane == 0) mbar_arrive_cluster(leader_bar(B_P_FULL + (g & 1)));
+      }
+      if (!ok) break;
+      // epilogue: wait for the last PV, normalise, write the split's partial
+      ok = mbar_wait(bar(B_O_DONE), (g - 1) & 1, abort_flag, p.status);
+      __syncwarp();
+      if (!ok) break;
+      tc_fence_after();
+      red_l[half * 64 + hl] = l_part;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const float l_tot = l_part + red_l[(half ^ 1) * 64 + hl];
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 256; c += 32) {
+        const uint32_t col = (c < 128 ? kColO0 + c : kColO1 + (c - 128));
+        uint32_t orr[32];
+        tmem_ld32(tmem + lane_base + col, orr);
+        tmem_wait_ld();
+        // lanes 0-63 hold dims [256j, 256j+128), lanes 64-127 dims [256j+128, 256j+256)
+        float* dst = od + (c < 128 ? 0 : 256) + 128 * half + (c & 127);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + j) =
+              make_float4(__uint_as_float(orr[j]) * inv, __uint_as_float(orr[j + 1]) * inv,
+                          __uint_as_float(orr[j + 2]) * inv, __uint_as_float(orr[j + 3]) * inv);
+      }
+      if (half == 0) p.lse_part[slot * kHeads + head] = l_tot > 0.f ? m_ref + __log2f(l_tot) : -INFINITY;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_bar(B_O_FREE));
+    }
+  }
+
+  // teardown: every TMEM access of both CTAs is finished before deallocation
+  tc_fence_before();
+  __syncthreads();
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  tc_fence_after();
+  if (warp == 5)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over [rows][576] with a (64 columns x box_rows) box, 128-byte swizzle
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kD, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool device_is_sm100() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  return major == 10 && minor == 0;
+}
+
+}  // namespace
+
+bool decode_tc_supported(const mla_dims& d, int n_q) {
+  return d.n_heads == kHeads && d.d_c == kDC && d.d_rope == kDR && d.page_size == kPage &&
+         d.act_dtype == MLA_BF16 && d.cache_dtype == MLA_BF16 && n_q >= 1 && n_q <= 8 && device_is_sm100();
+}
+
+int decode_tc_auto_splits(int num_sms, int n_q) {
+  const int pairs = num_sms / 2;
+  const int w = pairs / (n_q > 0 ? n_q : 1);
+  return w > 0 ? w : 1;
+}
+
+cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st) {
+  TcParams tp;
+  tp.p = p;
+  const uint64_t pool_rows = (uint64_t)p.num_pages * kPage;
+  if (!make_map(&tp.map_q, p.q_abs, (uint64_t)p.batch * p.n_q * kHeads, 64) ||
+      !make_map(&tp.map_kq, p.pool, pool_rows, 32) || !make_map(&tp.map_pv, p.pool, pool_rows, 64))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int pairs = p.splits * p.n_q;
+  decode_tc_kernel<<<2 * pairs, 192, kSmemBytes, st>>>(tp);
+  return cudaGetLastError();
+}
 
 }  // namespace mla

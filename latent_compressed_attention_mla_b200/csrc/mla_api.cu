@@ -16,8 +16,11 @@ using namespace mla;
 namespace mla {
 static cudaEvent_t g_trace[2 * MLA_TRACE_COUNT];
 static bool g_trace_on = false;
+// Called only where no launch error is pending; a failed record is dropped
+// (and cleared) so that it is never reported as a kernel launch failure.
 void trace_record(int kernel, bool end, cudaStream_t st) {
-  if (g_trace_on) cudaEventRecord(g_trace[2 * kernel + (end ? 1 : 0)], st);
+  if (g_trace_on && cudaEventRecord(g_trace[2 * kernel + (end ? 1 : 0)], st) != cudaSuccess)
+    (void)cudaGetLastError();
 }
 }  // namespace mla
 
