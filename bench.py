@@ -246,6 +246,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--flags", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch each step eagerly instead of replaying a captured CUDA graph")
     args = ap.parse_args()
     cfg = WL.CONFIGS[args.config]
     if args.impl == "reference":
@@ -298,13 +300,56 @@ def main():
         w, x, pool = sets[i % copies]
         sess.step(x["h"], seq_idx, pos, x["q_nope"], x["q_rope"], seq_lens, w, pt, pool)
 
-    for i in range(args.warmup):
+    # eager steps first: one-time set-up in the library happens outside capture
+    for i in range(min(2, copies) if args.graph else 0):
         step(i)
+    torch.cuda.synchronize()
+    graphs = []
+    if args.graph:
+        for r in range(copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(r)
+            graphs.append(g)
+
+    def run_step(i):
+        if graphs:
+            graphs[i % copies].replay()
+        else:
+            step(i)
+
+    for i in range(args.warmup):
+        run_step(i)
     torch.cuda.synchronize()
     if B.mla_get_status() != 0:
         raise RuntimeError("device status set during warm-up")
 
-    # per-kernel events: a ring of event sets, read back 32 steps behind
+    # timed region: K steps, nothing else on the stream
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    t_start_wall = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        run_step(args.warmup + i)
+    e1.record()
+    torch.cuda.synchronize()
+    t_end_wall = time.time()
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop(t_start_wall, t_end_wall)
+    ms = e0.elapsed_time(e1)
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # per-kernel durations: the same K steps again, launched eagerly with the
+    # library recording a CUDA event before and after each kernel on the launch
+    # stream (a ring of event sets, read back RING steps behind)
     nk = len(B.TRACE_KERNELS)
     RING = 32
     ring = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(RING)]
@@ -315,33 +360,15 @@ def main():
         for k in range(nk):
             ksum[k] += evs[2 * k].elapsed_time(evs[2 * k + 1])
 
-    sampler = ClockSampler(local)
-    time.sleep(0.3)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    t_start_wall = time.time()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
     for i in range(args.steps):
         if i >= RING:
             harvest(ring[i % RING])
         B.mla_set_trace_events(ring[i % RING])
         step(args.warmup + i)
-    e1.record()
     torch.cuda.synchronize()
     B.mla_set_trace_events(None)
-    t_end_wall = time.time()
     for i in range(max(0, args.steps - RING), args.steps):
         harvest(ring[i % RING])
-    if pg:
-        pg.barrier()
-    clocks = sampler.stop(t_start_wall, t_end_wall)
-    ms = e0.elapsed_time(e1)
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
     status = B.mla_get_status()
 
     tokens_per_step = cfg.B * cfg.T
@@ -427,6 +454,8 @@ def main():
         "kernel_roofline_frac": {k: (round(v["roofline_frac"], 4) if v["roofline_frac"] else None)
                                  for k, v in rows.items()},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": nk * args.steps, "clocks": clocks,
+        "timing": ("CUDA-graph replay of each step" if args.graph else "eager launches") +
+                  "; per-kernel times from a second, traced pass of the same steps",
         "device_status": status,
     }
     print(json.dumps(line), flush=True)
