@@ -112,6 +112,27 @@ int mla_check_dims(const mla_dims* dims);
  * MLA_ERR_BOUNDS is recorded in the device status word.  n_tokens == 0 is a no-op.
  * ------------------------------------------------------------------------- */
 size_t mla_append_workspace_bytes(const mla_dims* dims, int n_tokens);
+/* mla_append_latent_noalloc: mla_append_latent for callers that cannot
+ * allocate device memory at call time (a plugin or callback whose host
+ * framework owns all device memory and offers no scratch buffer, or a loop in
+ * which an allocation would synchronise the device).  The paper has no
+ * counterpart: this is a deployment variant of the S1 append.
+ * Same arguments and results as mla_append_latent, without the workspace: the
+ * fp32 scratch lives in a fixed array inside the library, 65,536 floats
+ * (256 KiB) on every GPU that loads it, held until the process exits.
+ *   - n_tokens * (d_c + d_rope) must be <= 65536 (113 tokens at DeepSeek-V3
+ *     dims); larger requests return MLA_ERR_WORKSPACE and launch nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the array: calls whose kernels overlap on the GPU race.
+ *     Nothing in it needs clearing between calls.
+ *   - It calls no cudaMalloc/cudaFree and no allocating library routine. */
+int mla_append_latent_noalloc(const mla_dims* dims, const void* h, int n_tokens,
+                              const int32_t* seq_idx, const int32_t* pos,
+                              const void* W_dkv, const void* W_kr,
+                              const int32_t* page_table, int batch, int max_pages,
+                              void* cache_pool, int num_pages, void* stream);
+
 int mla_append_latent(const mla_dims* dims, const void* h, int n_tokens,
                       const int32_t* seq_idx, const int32_t* pos,
                       const void* W_dkv, const void* W_kr,

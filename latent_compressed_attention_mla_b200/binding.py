@@ -23,6 +23,7 @@ ERRORS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "M
 
 # Every entry point declared in include/mla.h.
 EXPORTED = ("mla_cache_page_bytes", "mla_check_dims", "mla_append_workspace_bytes", "mla_append_latent",
+            "mla_append_latent_noalloc",
             "mla_decode_workspace_bytes", "mla_decode", "mla_combine", "mla_decode_path", "mla_auto_splits",
             "mla_set_trace_events", "mla_get_status", "mla_error_string")
 TRACE_KERNELS = ("append_project", "append_finalize", "plan", "absorb", "attend", "combine")
@@ -56,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.mla_append_workspace_bytes.argtypes, L.mla_append_workspace_bytes.restype = [S, I], Z
         L.mla_append_latent.argtypes = [S, P, I, P, P, P, P, P, I, I, P, I, P, Z, P]
         L.mla_append_latent.restype = I
+        L.mla_append_latent_noalloc.argtypes = [S, P, I, P, P, P, P, P, I, I, P, I, P]
+        L.mla_append_latent_noalloc.restype = I
         L.mla_decode_workspace_bytes.argtypes, L.mla_decode_workspace_bytes.restype = [S, I, I, I], Z
         L.mla_decode.argtypes = [S, P, P, P, P, I, P, I, P, I, I, I, P, Z, P]
         L.mla_decode.restype = I
@@ -144,6 +147,18 @@ def mla_append_latent(dims, h, seq_idx, pos, W_dkv, W_kr, page_table, cache_pool
                                  _ptr(cache_pool), num_pages, _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "mla_append_latent")
+
+
+def mla_append_latent_noalloc(dims, h, seq_idx, pos, W_dkv, W_kr, page_table, cache_pool, stream=None):
+    """S1 without a workspace, for callers that cannot allocate device memory
+    at call time: the library's fixed scratch array is used instead (at most
+    65,536 floats, i.e. n_tokens * (d_c + d_rope) <= 65536)."""
+    _cuda(h, seq_idx, pos, W_dkv, W_kr, page_table, cache_pool)
+    num_pages = cache_pool.numel() * cache_pool.element_size() // cache_page_bytes(dims)
+    rc = lib().mla_append_latent_noalloc(ctypes.byref(dims), _ptr(h), h.shape[0], _ptr(seq_idx), _ptr(pos),
+                                         _ptr(W_dkv), _ptr(W_kr), _ptr(page_table), page_table.shape[0],
+                                         page_table.shape[1], _ptr(cache_pool), num_pages, _stream(stream))
+    _check(rc, "mla_append_latent_noalloc")
 
 
 def mla_decode(dims, q_nope, q_rope, W_uk, cache_pool, page_table, seq_lens, workspace, num_splits=0,

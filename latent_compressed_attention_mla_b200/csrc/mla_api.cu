@@ -81,6 +81,11 @@ int launch_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_LA
 
 }  // namespace
 
+namespace mla {
+// Device status word of the current device, for entry points in other files.
+int* device_status_word() { return status_ptr(); }
+}  // namespace mla
+
 extern "C" {
 
 size_t mla_cache_page_bytes(const mla_dims* dims) {
