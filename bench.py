@@ -60,7 +60,6 @@ def kernel_work(cfg: WL.MlaConfig, page_bytes: int) -> dict:
     return {
         "append_project": {"bytes": D * d * act + N * d * act + N * D * 4, "flops": 2 * N * D * d},
         "append_finalize": {"bytes": N * D * 4 + N * row_bytes, "flops": 0},
-        "plan": {"bytes": cfg.B * 8, "flops": 0},
         "absorb": {"bytes": H * dn * dc * act + N * H * (dn + dr) * act + N * H * D * act, "flops": 2 * N * H * dn * dc},
         "attend": {"bytes": keys_read * row_bytes + N * H * D * act, "flops": 2 * pairs * H * (D + dc),
                    "cache_bytes": keys_read * row_bytes, "pairs": pairs},
@@ -293,7 +292,9 @@ def main():
         sets.append(({k: v.clone() for k, v in weights0.items()}, {k: v.clone() for k, v in inputs0.items()},
                      cache0.pool.clone()))
     sess = MlaDecodeSession(dims, cfg.B, cfg.T, args.splits, dev)
-    splits = args.splits or B.auto_splits(dims, cfg.B, cfg.T)
+    # the split count mla_decode uses: explicit, else the automatic count capped
+    # at one split per 4 key tiles of batch * max_pages
+    splits = args.splits or min(B.auto_splits(dims, cfg.B, cfg.T), max(1, -(-cfg.B * cfg.max_pages // 4)))
     path = B.decode_path(dims, cfg.T)
 
     def step(i):

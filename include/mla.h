@@ -108,6 +108,11 @@ int mla_check_dims(const mla_dims* dims);
  *   page_table [batch, max_pages] int32
  *   cache_pool num_pages pages (layout above), written
  *   workspace  >= mla_append_workspace_bytes(dims, n_tokens) bytes of scratch
+ *              (fp32 c values between the projection and the FP8 quantiser;
+ *              0 bytes, and workspace may be NULL, for fp32/bf16 caches)
+ * d_model must be a multiple of 32 and <= 8192 (bf16) / 4096 (fp32): the
+ * projection keeps a lane's slice of each weight row in registers
+ * (MLA_ERR_UNSUPPORTED otherwise).
  * Out-of-range seq_idx/pos/page entries: the token is skipped and
  * MLA_ERR_BOUNDS is recorded in the device status word.  n_tokens == 0 is a no-op.
  * ------------------------------------------------------------------------- */
@@ -193,17 +198,17 @@ int mla_auto_splits(const mla_dims* dims, int batch, int n_q);
 
 /* Tracing.  Kernels of the calls above, in launch order per step: */
 enum {
-  MLA_TRACE_APPEND_PROJECT = 0, /* mla_append_latent: [W_dkv; W_kr] h */
-  MLA_TRACE_APPEND_FINALIZE = 1,/* mla_append_latent: RoPE, rounding, paged store */
-  MLA_TRACE_PLAN = 2,           /* mla_decode: split plan from seq_lens */
-  MLA_TRACE_ABSORB = 3,         /* mla_decode: q~ = W_uk^T q_nope, RoPE(q_rope) */
-  MLA_TRACE_ATTEND = 4,         /* mla_decode: split-KV attention over the cache */
-  MLA_TRACE_COMBINE = 5,        /* mla_combine: split merge and W_uv */
-  MLA_TRACE_COUNT = 6
+  MLA_TRACE_APPEND_PROJECT = 0, /* mla_append_latent: [W_dkv; W_kr] h, RoPE, paged store */
+  MLA_TRACE_APPEND_FINALIZE = 1,/* mla_append_latent: FP8 quantiser (FP8 caches only) */
+  MLA_TRACE_ABSORB = 2,         /* mla_decode: q~ = W_uk^T q_nope, RoPE(q_rope), split plan */
+  MLA_TRACE_ATTEND = 3,         /* mla_decode: split-KV attention over the cache */
+  MLA_TRACE_COMBINE = 4,        /* mla_combine: split merge and W_uv */
+  MLA_TRACE_COUNT = 5
 };
 /* Install a table of 2*MLA_TRACE_COUNT cudaEvent_t (passed as void*, created
  * by the caller with timing enabled): later calls record events[2k] before and
- * events[2k+1] after kernel k on the launch stream.  NULL uninstalls.  The
+ * events[2k+1] after kernel k on the launch stream (both back to back when
+ * the call launches no kernel k).  NULL uninstalls.  The
  * table is process-wide host state read at launch time; it is not
  * thread-safe.  Returns MLA_OK or MLA_ERR_INVALID_ARG (n_events too small). */
 int mla_set_trace_events(void* const* events, int n_events);

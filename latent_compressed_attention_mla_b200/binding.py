@@ -26,7 +26,7 @@ EXPORTED = ("mla_cache_page_bytes", "mla_check_dims", "mla_append_workspace_byte
             "mla_append_latent_noalloc",
             "mla_decode_workspace_bytes", "mla_decode", "mla_combine", "mla_decode_path", "mla_auto_splits",
             "mla_set_trace_events", "mla_get_status", "mla_error_string")
-TRACE_KERNELS = ("append_project", "append_finalize", "plan", "absorb", "attend", "combine")
+TRACE_KERNELS = ("append_project", "append_finalize", "absorb", "attend", "combine")
 
 
 class MlaDims(ctypes.Structure):

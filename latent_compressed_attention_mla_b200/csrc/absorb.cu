@@ -5,72 +5,211 @@
 // steps 2-3).  Output row [q~ | RoPE(q^R)] per (token, head), the operand the
 // decode kernel scores against the 576-wide cached rows.
 //
-// One CTA per (head, 128-wide slice of d_c): the W^UK_h slice is read from HBM
-// once with 16-byte loads into shared memory and applied to every token of the
-// step (16 tokens per pass); fp32 accumulation.
+// One CTA per (head, 16-vector slice of d_c).  Thread (cg, dg) loads the
+// 16-byte vectors of W^UK_h for its column group cg and its rows d in group
+// dg, all loads issued up front, and keeps them in registers for every token
+// of the step; partial sums over the row groups are reduced in shared memory.
+//
+// The same launch prepares the split plan the decode and combine kernels
+// read: block (0, 0) computes the key-tile prefix sums of the sequences and,
+// per sequence, the run of splits that overlap it; all blocks fill the
+// per-split log-sum-exp slots with -inf, the value of a split that holds no
+// key of a sequence.
 #include "mla_internal.cuh"
 
 namespace mla {
 
 namespace {
 
-constexpr int kAbsTok = 16;
+constexpr int kCG = 16;        // column groups (16-byte vectors) per CTA
+constexpr int kDG = 8;         // row groups
+constexpr int kMaxRows = 16;   // rows of W^UK per thread: d_nope <= kDG * kMaxRows
+constexpr int kTokBlock = 4;
 
-template <typename T>
-__global__ void __launch_bounds__(128) absorb_kernel(
-    const T* __restrict__ q_nope, const T* __restrict__ q_rope, const T* __restrict__ W_uk,
-    const int32_t* __restrict__ seq_lens, int batch, int n_q, int n_heads, int d_nope, int d_c,
-    int d_rope, float rope_base, T* __restrict__ q_abs) {
-  extern __shared__ float smem[];
-  float* W_s = smem;                    // [d_nope][128]
-  float* q_s = smem + d_nope * 128;     // [kAbsTok][d_nope]
-  const int h = blockIdx.x, c0 = blockIdx.y * 128, tid = threadIdx.x;
-  const int D = d_c + d_rope;
-  const int M = batch * n_q;
-  const int width = min(128, d_c - c0);  // multiple of 16
+struct AbsorbArgs {
+  const void* q_nope;
+  const void* q_rope;
+  const void* W_uk;
+  const int32_t* seq_lens;
+  int batch, n_q, n_heads, d_nope, d_c, d_rope, page_size, max_pages, splits;
+  float rope_base;
+  void* q_abs;
+  int32_t* plan;
+  float* lse_part;
+  size_t lse_count;
+  int* status;
+};
 
-  // W_uk[h][d][c0 .. c0+width) -> W_s[d][0..width), 8 elements per load
-  const T* Wh = W_uk + (size_t)h * d_nope * d_c + c0;
-  const int vec_per_row = width / 8;
-  for (int i = tid; i < d_nope * vec_per_row; i += 128) {
-    const int d = i / vec_per_row, j = (i % vec_per_row) * 8;
-    float f[8];
-    load8(Wh + (size_t)d * d_c + j, f);
+template <typename T> struct VecN;
+template <> struct VecN<__nv_bfloat16> { static constexpr int n = 8; };
+template <> struct VecN<float> { static constexpr int n = 4; };
+
+__device__ __forceinline__ void unpack(const uint4& v, float* f, __nv_bfloat16*) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) W_s[d * 128 + j + k] = f[k];
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
   }
-  for (int m0 = 0; m0 < M; m0 += kAbsTok) {
-    const int mcount = min(kAbsTok, M - m0);
+}
+__device__ __forceinline__ void unpack(const uint4& v, float* f, float*) {
+  const float4 t = *reinterpret_cast<const float4*>(&v);
+  f[0] = t.x; f[1] = t.y; f[2] = t.z; f[3] = t.w;
+}
+
+// Split plan (one block).  plan layout: tile_start[batch+1], header
+// {TT, W, batch, n_q} at [batch+1 .. batch+4], then per sequence the first
+// overlapping split and the count of splits: [batch+5 + 2b], [batch+6 + 2b].
+__device__ void build_plan(const AbsorbArgs& a) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < a.batch; base += nt) {
+    const int b = base + tid;
+    int tiles = 0;
+    if (b < a.batch) {
+      const int len = a.seq_lens[b];
+      if (len >= a.n_q && len >= 1 && (long long)len <= (long long)a.max_pages * a.page_size)
+        tiles = (len + a.page_size - 1) / a.page_size;
+      else
+        record_status(a.status, MLA_ERR_BOUNDS);
+    }
+    int x = tiles;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
     __syncthreads();
-    for (int i = tid; i < mcount * d_nope; i += 128) {
-      const int mi = i / d_nope, d = i % d_nope;
-      q_s[mi * d_nope + d] = to_f(q_nope[((size_t)(m0 + mi) * n_heads + h) * d_nope + d]);
+    if (warp == 0) {
+      int s = lane < nt / 32 ? warp_sums[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      warp_sums[lane] = s;
     }
     __syncthreads();
-    if (tid < width) {
-      float acc[kAbsTok];
+    const int excl = carry + (warp ? warp_sums[warp - 1] : 0) + x - tiles;
+    if (b < a.batch) a.plan[b] = excl;
+    __syncthreads();
+    if (tid == nt - 1) carry = excl + tiles;
+    __syncthreads();
+  }
+  const long long TT = carry;
+  const int W = a.splits;
+  if (tid == 0) {
+    a.plan[a.batch] = (int32_t)TT;
+    a.plan[a.batch + 1] = (int32_t)TT;
+    a.plan[a.batch + 2] = W;
+    a.plan[a.batch + 3] = a.batch;
+    a.plan[a.batch + 4] = a.n_q;
+  }
+  __syncthreads();
+  // splits overlapping sequence b: end(w) = floor((w+1) TT / W) > ts_b and
+  // begin(w) = floor(w TT / W) < ts_{b+1}
+  for (int b = tid; b < a.batch; b += nt) {
+    const long long s0 = a.plan[b], s1 = (b + 1 < a.batch) ? a.plan[b + 1] : TT;
+    int lo = 0, n = 0;
+    if (s1 > s0 && TT > 0) {
+      lo = (int)(((s0 + 1) * W + TT - 1) / TT) - 1;
+      const int hi = (int)((s1 * W - 1) / TT);
+      n = hi - lo + 1;
+    }
+    a.plan[a.batch + 5 + 2 * b] = lo;
+    a.plan[a.batch + 6 + 2 * b] = n;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) absorb_kernel(const AbsorbArgs a) {
+  constexpr int VEC = VecN<T>::n;
+  __shared__ float q_s[kTokBlock][kDG * kMaxRows];
+  __shared__ float red[kDG][kTokBlock][kCG * 8];
+  const int h = blockIdx.x, tid = threadIdx.x;
+  const int cg = tid % kCG, dg = tid / kCG;
+  const int c0 = blockIdx.y * kCG * VEC + cg * VEC;  // first column of this thread
+  const int D = a.d_c + a.d_rope;
+  const int M = a.batch * a.n_q;
+  const int rows = (a.d_nope + kDG - 1) / kDG;
+  const bool col_ok = c0 < a.d_c;
+
+  if (blockIdx.x == 0 && blockIdx.y == 0) build_plan(a);
+  // every split's log-sum-exp slot starts empty
+  {
+    const size_t nblk = (size_t)gridDim.x * gridDim.y, bid = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+    for (size_t i = bid * 128 + tid; i < a.lse_count; i += nblk * 128) a.lse_part[i] = -INFINITY;
+  }
+
+  const T* Wh = static_cast<const T*>(a.W_uk) + (size_t)h * a.d_nope * a.d_c;
+  uint4 wv[kMaxRows];
 #pragma unroll
-      for (int mi = 0; mi < kAbsTok; ++mi) acc[mi] = 0.f;
-      for (int d = 0; d < d_nope; ++d) {
-        const float w = W_s[d * 128 + tid];
+  for (int r = 0; r < kMaxRows; ++r) {
+    const int d = dg * rows + r;
+    wv[r] = (col_ok && r < rows && d < a.d_nope) ? *reinterpret_cast<const uint4*>(Wh + (size_t)d * a.d_c + c0)
+                                                 : make_uint4(0, 0, 0, 0);
+  }
+  const T* qn = static_cast<const T*>(a.q_nope);
+  T* qa = static_cast<T*>(a.q_abs);
+  for (int m0 = 0; m0 < M; m0 += kTokBlock) {
+    const int mc = min(kTokBlock, M - m0);
+    __syncthreads();
+    for (int i = tid; i < kTokBlock * kDG * kMaxRows; i += 128) {
+      const int mi = i / (kDG * kMaxRows), d = i % (kDG * kMaxRows);
+      q_s[mi][d] = (mi < mc && d < a.d_nope) ? to_f(qn[((size_t)(m0 + mi) * a.n_heads + h) * a.d_nope + d]) : 0.f;
+    }
+    __syncthreads();
+    float acc[kTokBlock][VEC];
 #pragma unroll
-        for (int mi = 0; mi < kAbsTok; ++mi) acc[mi] = fmaf(w, q_s[mi * d_nope + d], acc[mi]);
+    for (int mi = 0; mi < kTokBlock; ++mi)
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) acc[mi][j] = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMaxRows; ++r) {
+      if (r < rows) {
+        float w[VEC];
+        unpack(wv[r], w, (T*)nullptr);
+#pragma unroll
+        for (int mi = 0; mi < kTokBlock; ++mi) {
+          const float q = q_s[mi][dg * rows + r];
+#pragma unroll
+          for (int j = 0; j < VEC; ++j) acc[mi][j] = fmaf(w[j], q, acc[mi][j]);
+        }
       }
-      for (int mi = 0; mi < mcount; ++mi)
-        q_abs[((size_t)(m0 + mi) * n_heads + h) * D + c0 + tid] = from_f<T>(acc[mi]);
+    }
+#pragma unroll
+    for (int mi = 0; mi < kTokBlock; ++mi)
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) red[dg][mi][cg * VEC + j] = acc[mi][j];
+    __syncthreads();
+    for (int i = tid; i < kTokBlock * kCG * VEC; i += 128) {
+      const int mi = i / (kCG * VEC), cc = i % (kCG * VEC);
+      const int c = blockIdx.y * kCG * VEC + cc;
+      if (mi < mc && c < a.d_c) {
+        float s = 0.f;
+#pragma unroll
+        for (int g = 0; g < kDG; ++g) s += red[g][mi][cc];
+        qa[((size_t)(m0 + mi) * a.n_heads + h) * D + c] = from_f<T>(s);
+      }
     }
   }
   if (blockIdx.y == 0) {
-    const int half = d_rope >> 1;
+    const int half = a.d_rope >> 1;
+    const T* qr = static_cast<const T*>(a.q_rope);
     for (int i = tid; i < M * half; i += 128) {
       const int m = i / half, k = i % half;
-      const int b = m / n_q, t = m % n_q;
-      const int p = seq_lens[b] - n_q + t;
+      const int b = m / a.n_q, t = m % a.n_q;
+      const int p = a.seq_lens[b] - a.n_q + t;
       float cs, sn;
-      rope_cos_sin(p, k, half, rope_base, &cs, &sn);
-      const T* src = q_rope + ((size_t)m * n_heads + h) * d_rope;
+      rope_cos_sin(p, k, half, a.rope_base, &cs, &sn);
+      const T* src = qr + ((size_t)m * a.n_heads + h) * a.d_rope;
       const float x1 = to_f(src[k]), x2 = to_f(src[half + k]);
-      T* dst = q_abs + ((size_t)m * n_heads + h) * D + d_c;
+      T* dst = qa + ((size_t)m * a.n_heads + h) * D + a.d_c;
       dst[k] = from_f<T>(x1 * cs - x2 * sn);
       dst[half + k] = from_f<T>(x2 * cs + x1 * sn);
     }
@@ -79,25 +218,38 @@ __global__ void __launch_bounds__(128) absorb_kernel(
 
 }  // namespace
 
-cudaError_t launch_absorb(const mla_dims& d, const void* q_nope, const void* q_rope, const void* W_uk,
-                          const int32_t* seq_lens, int batch, int n_q, void* q_abs, cudaStream_t st) {
-  const dim3 grid(d.n_heads, (d.d_c + 127) / 128);
-  const size_t smem = sizeof(float) * ((size_t)d.d_nope * 128 + (size_t)kAbsTok * d.d_nope);
-  cudaError_t e;
-  if (d.act_dtype == MLA_F32) {
-    e = cudaFuncSetAttribute(absorb_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    absorb_kernel<float><<<grid, 128, smem, st>>>(
-        (const float*)q_nope, (const float*)q_rope, (const float*)W_uk, seq_lens, batch, n_q, d.n_heads,
-        d.d_nope, d.d_c, d.d_rope, d.rope_base, (float*)q_abs);
-  } else {
-    e = cudaFuncSetAttribute(absorb_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    absorb_kernel<__nv_bfloat16><<<grid, 128, smem, st>>>(
-        (const __nv_bfloat16*)q_nope, (const __nv_bfloat16*)q_rope, (const __nv_bfloat16*)W_uk, seq_lens,
-        batch, n_q, d.n_heads, d.d_nope, d.d_c, d.d_rope, d.rope_base, (__nv_bfloat16*)q_abs);
-  }
+int absorb_max_d_nope() { return kDG * kMaxRows; }
+
+cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const void* q_rope, const void* W_uk,
+                                   const int32_t* seq_lens, int batch, int n_q, int max_pages, int splits,
+                                   void* q_abs, int32_t* plan, float* lse_part, size_t lse_count, int* status,
+                                   cudaStream_t st) {
+  AbsorbArgs a;
+  a.q_nope = q_nope;
+  a.q_rope = q_rope;
+  a.W_uk = W_uk;
+  a.seq_lens = seq_lens;
+  a.batch = batch;
+  a.n_q = n_q;
+  a.n_heads = d.n_heads;
+  a.d_nope = d.d_nope;
+  a.d_c = d.d_c;
+  a.d_rope = d.d_rope;
+  a.page_size = d.page_size;
+  a.max_pages = max_pages;
+  a.splits = splits;
+  a.rope_base = d.rope_base;
+  a.q_abs = q_abs;
+  a.plan = plan;
+  a.lse_part = lse_part;
+  a.lse_count = lse_count;
+  a.status = status;
+  const int vec = d.act_dtype == MLA_F32 ? 4 : 8;
+  const dim3 grid(d.n_heads, (d.d_c + kCG * vec - 1) / (kCG * vec));
+  if (d.act_dtype == MLA_F32)
+    absorb_kernel<float><<<grid, 128, 0, st>>>(a);
+  else
+    absorb_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -5,72 +5,27 @@
 // Absorption"; FP8 tile scaling after "DeepSeek Unveils DualPipe & Multi-Head
 // Latent Attention", fine-grained tile-level quantisation).
 //
-// Two kernels:
-//   project : raw[n, :] = [W_dkv; W_kr] h_n in fp32.  The stacked weight
-//             matrix (d_c + d_rope rows of d_model) is streamed once from HBM
-//             with 16-byte loads; each CTA owns 4 rows, split over two warps
-//             per row along d_model, and dots them against every token.
-//   finalize: one CTA per token; RoPE on the k^R part, rounding to the cache
-//             type (per-128-tile amax scaling for FP8) and the paged store.
+// append_project: the stacked weights [W_dkv; W_kr] (d_c + d_rope rows of
+//   d_model) are streamed from HBM once, 16 bytes per load, all of a warp's
+//   loads issued up front; each CTA owns 2 output rows (four warps per row, one
+//   per quarter of d_model) and dots them against every token.  The CTAs of
+//   the k^R rows own one rotation pair (i, i + d_rope/2) each, so they apply
+//   RoPE themselves.  For fp32/bf16 caches every value is rounded and stored into
+//   its paged slot here: one kernel per append.
+// append_fp8_finalize: FP8 caches need the amax of each 128-wide tile of c, a
+//   reduction across CTAs, so the projection leaves c in fp32 scratch and one
+//   CTA per token quantises it.
 #include "mla_internal.cuh"
 
 namespace mla {
 
 namespace {
 
-constexpr int kProjRowsPerCta = 4;
-constexpr int kProjTokGroup = 4;
+constexpr int kRows = 2;      // output rows per CTA
+constexpr int kSplitK = 4;    // warps per row, one per quarter of d_model
+constexpr int kTok = 2;       // tokens per pass
+constexpr int kMaxVec = 8;    // 16-byte vectors per lane per quarter of d_model
 
-template <typename T>
-__global__ void __launch_bounds__(256) append_project_kernel(
-    const T* __restrict__ h, int n_tokens, const T* __restrict__ W_dkv, const T* __restrict__ W_kr,
-    int d_c, int d_rope, int d_model, float* __restrict__ raw) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int D = d_c + d_rope;
-  const int row = blockIdx.x * kProjRowsPerCta + (warp & 3);
-  const int khalf = warp >> 2;
-  const int kh = d_model >> 1;
-  __shared__ float red[8][kProjTokGroup];
-  const bool active = row < D;
-  const T* wrow = nullptr;
-  if (active)
-    wrow = (row < d_c ? W_dkv + (size_t)row * d_model : W_kr + (size_t)(row - d_c) * d_model) +
-           (size_t)khalf * kh;
-  for (int n0 = 0; n0 < n_tokens; n0 += kProjTokGroup) {
-    float acc[kProjTokGroup] = {0.f, 0.f, 0.f, 0.f};
-    if (active) {
-#pragma unroll 2
-      for (int k = lane * 8; k < kh; k += 256) {
-        float wv[8];
-        load8(wrow + k, wv);
-#pragma unroll
-        for (int g = 0; g < kProjTokGroup; ++g) {
-          if (n0 + g < n_tokens) {
-            float hv[8];
-            load8(h + (size_t)(n0 + g) * d_model + (size_t)khalf * kh + k, hv);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[g] = fmaf(wv[i], hv[i], acc[g]);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < kProjTokGroup; ++g) {
-#pragma unroll
-      for (int o = 16; o; o >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], o);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int g = 0; g < kProjTokGroup; ++g) red[warp][g] = acc[g];
-    }
-    __syncthreads();
-    if (warp < 4 && lane < kProjTokGroup && active && n0 + lane < n_tokens)
-      raw[(size_t)(n0 + lane) * D + row] = red[warp][lane] + red[warp + 4][lane];
-    __syncthreads();
-  }
-}
-
-// FP8 page sub-block offsets (bytes within a page).
 struct Fp8Page {
   size_t kr_off, sc_off;
 };
@@ -80,6 +35,164 @@ __host__ __device__ inline Fp8Page fp8_page(int page_size, int d_c, int d_rope) 
   p.kr_off = a128((size_t)page_size * d_c);
   p.sc_off = a128(p.kr_off + (size_t)page_size * d_rope * 2);
   return p;
+}
+
+struct AppendArgs {
+  const void* h;
+  int n_tokens;
+  const int32_t* seq_idx;
+  const int32_t* pos;
+  const void* W_dkv;
+  const void* W_kr;
+  const int32_t* page_table;
+  int batch, max_pages;
+  uint8_t* pool;
+  int num_pages;
+  size_t page_bytes;
+  int d_c, d_rope, d_model, page_size;
+  float rope_base;
+  float* raw;  // fp32 [n_tokens][d_c] scratch (FP8 caches only)
+  int* status;
+};
+
+// Physical (page, row) of token n, or page -1 (recorded) if out of range.
+__device__ __forceinline__ int token_slot(const AppendArgs& a, int n, int* row, int* position) {
+  const int b = a.seq_idx[n], p = a.pos[n];
+  bool ok = b >= 0 && b < a.batch && p >= 0 && p / a.page_size < a.max_pages;
+  int page = ok ? a.page_table[(size_t)b * a.max_pages + p / a.page_size] : -1;
+  if (!(ok && page >= 0 && page < a.num_pages)) {
+    record_status(a.status, MLA_ERR_BOUNDS);
+    return -1;
+  }
+  *row = p % a.page_size;
+  *position = p;
+  return page;
+}
+
+template <typename T> struct Vec;
+template <> struct Vec<__nv_bfloat16> { static constexpr int n = 8; };
+template <> struct Vec<float> { static constexpr int n = 4; };
+
+__device__ __forceinline__ float dot_vec(const uint4& w, const uint4& x, __nv_bfloat16*) {
+  const __nv_bfloat162* a = reinterpret_cast<const __nv_bfloat162*>(&w);
+  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&x);
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 fa = __bfloat1622float2(a[i]), fb = __bfloat1622float2(b[i]);
+    s = fmaf(fa.x, fb.x, s);
+    s = fmaf(fa.y, fb.y, s);
+  }
+  return s;
+}
+__device__ __forceinline__ float dot_vec(const uint4& w, const uint4& x, float*) {
+  const float4 a = *reinterpret_cast<const float4*>(&w), b = *reinterpret_cast<const float4*>(&x);
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+
+template <typename T, int CACHE>
+__global__ void __launch_bounds__(256, 2) append_project_kernel(const AppendArgs a) {
+  constexpr int VEC = Vec<T>::n;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rs = warp % kRows, kq = warp / kRows;
+  const int half = a.d_rope >> 1;
+  const int c_ctas = (a.d_c + kRows - 1) / kRows;
+  const bool kr_cta = (int)blockIdx.x >= c_ctas;
+  // output row of this warp: c rows 2b, 2b+1, or the k^R pair (i, i + half)
+  int row;  // index into [W_dkv; W_kr], or -1
+  if (!kr_cta) {
+    row = blockIdx.x * kRows + rs;
+    if (row >= a.d_c) row = -1;
+  } else {
+    const int i = blockIdx.x - c_ctas;
+    row = i < half ? a.d_c + i + rs * half : -1;
+  }
+  const int kh = a.d_model / kSplitK;
+  const T* wrow = nullptr;
+  if (row >= 0)
+    wrow = (row < a.d_c ? static_cast<const T*>(a.W_dkv) + (size_t)row * a.d_model
+                        : static_cast<const T*>(a.W_kr) + (size_t)(row - a.d_c) * a.d_model) +
+           (size_t)kq * kh;
+  // this lane's slice of the weight row, kept in registers for all tokens
+  uint4 wv[kMaxVec];
+#pragma unroll
+  for (int v = 0; v < kMaxVec; ++v) {
+    const int k = (lane + 32 * v) * VEC;
+    wv[v] = (row >= 0 && k < kh) ? *reinterpret_cast<const uint4*>(wrow + k) : make_uint4(0, 0, 0, 0);
+  }
+  __shared__ float red[8][kTok];
+  const T* hb = static_cast<const T*>(a.h) + (size_t)kq * kh;
+  for (int n0 = 0; n0 < a.n_tokens; n0 += kTok) {
+    float acc[kTok];
+#pragma unroll
+    for (int g = 0; g < kTok; ++g) {
+      acc[g] = 0.f;
+      if (row >= 0 && n0 + g < a.n_tokens) {
+        const T* hr = hb + (size_t)(n0 + g) * a.d_model;
+#pragma unroll
+        for (int v = 0; v < kMaxVec; ++v) {
+          const int k = (lane + 32 * v) * VEC;
+          if (k < kh) acc[g] += dot_vec(wv[v], *reinterpret_cast<const uint4*>(hr + k), (T*)nullptr);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int g = 0; g < kTok; ++g) red[warp][g] = acc[g];
+    }
+    __syncthreads();
+    // thread t < kRows*kTok writes row slot t%kRows of token n0 + t/kRows
+    const int t = threadIdx.x;
+    if (t < kRows * kTok) {
+      const int slot = t % kRows, g = t / kRows, n = n0 + g;
+      if (n < a.n_tokens) {
+        int prow, position;
+        const int page = token_slot(a, n, &prow, &position);
+        float val = 0.f;
+#pragma unroll
+        for (int q = 0; q < kSplitK; ++q) val += red[slot + kRows * q][g];
+        if (page >= 0) {
+          uint8_t* pg = a.pool + (size_t)page * a.page_bytes;
+          if (!kr_cta) {
+            const int col = blockIdx.x * kRows + slot;
+            if (col < a.d_c) {
+              if (CACHE == MLA_FP8_E4M3) {
+                a.raw[(size_t)n * a.d_c + col] = val;
+              } else {
+                using CT = typename std::conditional<CACHE == MLA_F32, float, __nv_bfloat16>::type;
+                reinterpret_cast<CT*>(pg)[(size_t)prow * (a.d_c + a.d_rope) + col] = from_f<CT>(val);
+              }
+            }
+          } else if (slot == 0) {
+            const int i = blockIdx.x - c_ctas;
+            if (i < half) {
+              float x2 = 0.f;
+#pragma unroll
+              for (int q = 0; q < kSplitK; ++q) x2 += red[1 + kRows * q][g];
+              const float x1 = val;
+              float cs, sn;
+              rope_cos_sin(position, i, half, a.rope_base, &cs, &sn);
+              const float y1 = x1 * cs - x2 * sn, y2 = x2 * cs + x1 * sn;
+              if (CACHE == MLA_FP8_E4M3) {
+                const Fp8Page fp = fp8_page(a.page_size, a.d_c, a.d_rope);
+                __nv_bfloat16* kr = reinterpret_cast<__nv_bfloat16*>(pg + fp.kr_off) + (size_t)prow * a.d_rope;
+                kr[i] = __float2bfloat16_rn(y1);
+                kr[i + half] = __float2bfloat16_rn(y2);
+              } else {
+                using CT = typename std::conditional<CACHE == MLA_F32, float, __nv_bfloat16>::type;
+                CT* dst = reinterpret_cast<CT*>(pg) + (size_t)prow * (a.d_c + a.d_rope) + a.d_c;
+                dst[i] = from_f<CT>(y1);
+                dst[i + half] = from_f<CT>(y2);
+              }
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
 }
 
 // Block-wide max over 128 threads.
@@ -92,56 +205,26 @@ __device__ __forceinline__ float block128_max(float v, float* sh) {
   return fmaxf(fmaxf(sh[0], sh[1]), fmaxf(sh[2], sh[3]));
 }
 
-template <int CACHE>
-__global__ void __launch_bounds__(128) append_finalize_kernel(
-    const float* __restrict__ raw, const int32_t* __restrict__ seq_idx, const int32_t* __restrict__ pos,
-    const int32_t* __restrict__ page_table, int batch, int max_pages, uint8_t* __restrict__ pool,
-    int num_pages, size_t page_bytes, int d_c, int d_rope, int page_size, float rope_base,
-    int* status) {
+// One CTA (128 threads) per token: per 128-wide tile of c, scale = amax/448
+// (IEEE fp32 division; 1 for an all-zero tile) and e4m3 codes of c/scale
+// (round to nearest even, saturating).
+__global__ void __launch_bounds__(128) append_fp8_finalize_kernel(const AppendArgs a) {
   __shared__ float sh[4];
   const int n = blockIdx.x, tid = threadIdx.x;
-  const int D = d_c + d_rope, half = d_rope >> 1;
-  const int b = seq_idx[n], p = pos[n];
-  bool ok = b >= 0 && b < batch && p >= 0 && p / page_size < max_pages;
-  int page = ok ? page_table[(size_t)b * max_pages + p / page_size] : -1;
-  ok = ok && page >= 0 && page < num_pages;
-  if (!ok) {
-    if (tid == 0) record_status(status, MLA_ERR_BOUNDS);
-    return;
-  }
-  const int row = p % page_size;
-  const float* r = raw + (size_t)n * D;
-  uint8_t* pg = pool + (size_t)page * page_bytes;
-  if (CACHE == MLA_FP8_E4M3) {
-    const Fp8Page fp = fp8_page(page_size, d_c, d_rope);
-    uint8_t* codes = pg + (size_t)row * d_c;
-    __nv_bfloat16* kr = reinterpret_cast<__nv_bfloat16*>(pg + fp.kr_off) + (size_t)row * d_rope;
-    float* sc = reinterpret_cast<float*>(pg + fp.sc_off) + (size_t)row * (d_c / 128);
-    for (int t0 = 0; t0 < d_c; t0 += 128) {
-      const float v = r[t0 + tid];
-      const float amax = block128_max(fabsf(v), sh);
-      const float scale = amax > 0.f ? amax / kE4M3Max : 1.0f;  // IEEE division
-      codes[t0 + tid] = (uint8_t)__nv_cvt_float_to_fp8(v / scale, __NV_SATFINITE, __NV_E4M3);
-      if (tid == 0) sc[t0 / 128] = scale;
-    }
-    for (int i = tid; i < half; i += 128) {
-      float cs, sn;
-      rope_cos_sin(p, i, half, rope_base, &cs, &sn);
-      const float x1 = r[d_c + i], x2 = r[d_c + half + i];
-      kr[i] = __float2bfloat16_rn(x1 * cs - x2 * sn);
-      kr[half + i] = __float2bfloat16_rn(x2 * cs + x1 * sn);
-    }
-  } else {
-    using CT = typename std::conditional<CACHE == MLA_F32, float, __nv_bfloat16>::type;
-    CT* dst = reinterpret_cast<CT*>(pg) + (size_t)row * D;
-    for (int j = tid; j < d_c; j += 128) dst[j] = from_f<CT>(r[j]);
-    for (int i = tid; i < half; i += 128) {
-      float cs, sn;
-      rope_cos_sin(p, i, half, rope_base, &cs, &sn);
-      const float x1 = r[d_c + i], x2 = r[d_c + half + i];
-      dst[d_c + i] = from_f<CT>(x1 * cs - x2 * sn);
-      dst[d_c + half + i] = from_f<CT>(x2 * cs + x1 * sn);
-    }
+  int prow, position;
+  const int page = token_slot(a, n, &prow, &position);
+  if (page < 0) return;
+  const Fp8Page fp = fp8_page(a.page_size, a.d_c, a.d_rope);
+  uint8_t* pg = a.pool + (size_t)page * a.page_bytes;
+  uint8_t* codes = pg + (size_t)prow * a.d_c;
+  float* sc = reinterpret_cast<float*>(pg + fp.sc_off) + (size_t)prow * (a.d_c / 128);
+  const float* r = a.raw + (size_t)n * a.d_c;
+  for (int t0 = 0; t0 < a.d_c; t0 += 128) {
+    const float v = r[t0 + tid];
+    const float amax = block128_max(fabsf(v), sh);
+    const float scale = amax > 0.f ? amax / kE4M3Max : 1.0f;
+    codes[t0 + tid] = (uint8_t)__nv_cvt_float_to_fp8(v / scale, __NV_SATFINITE, __NV_E4M3);
+    if (tid == 0) sc[t0 / 128] = scale;
   }
 }
 
@@ -155,34 +238,61 @@ size_t cache_page_bytes(const mla_dims& d) {
   return a128(fp.sc_off + (size_t)d.page_size * (d.d_c / 128) * 4);
 }
 
+// Largest d_model the projection kernel holds in registers (four quarters of
+// kMaxVec 16-byte vectors per lane).
+int append_max_d_model(int act_dtype) { return kSplitK * kMaxVec * 32 * (act_dtype == MLA_F32 ? 4 : 8); }
+
+size_t append_scratch_floats(const mla_dims& d, int n_tokens) {
+  return d.cache_dtype == MLA_FP8_E4M3 ? (size_t)n_tokens * d.d_c : 0;
+}
+
 cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const int32_t* seq_idx,
                           const int32_t* pos, const void* W_dkv, const void* W_kr,
                           const int32_t* page_table, int batch, int max_pages, void* pool,
                           int num_pages, size_t page_bytes, float* raw, int* status,
                           cudaStream_t st) {
-  const int D = d.d_c + d.d_rope;
-  const dim3 pgrid((D + kProjRowsPerCta - 1) / kProjRowsPerCta);
+  AppendArgs a;
+  a.h = h;
+  a.n_tokens = n_tokens;
+  a.seq_idx = seq_idx;
+  a.pos = pos;
+  a.W_dkv = W_dkv;
+  a.W_kr = W_kr;
+  a.page_table = page_table;
+  a.batch = batch;
+  a.max_pages = max_pages;
+  a.pool = static_cast<uint8_t*>(pool);
+  a.num_pages = num_pages;
+  a.page_bytes = page_bytes;
+  a.d_c = d.d_c;
+  a.d_rope = d.d_rope;
+  a.d_model = d.d_model;
+  a.page_size = d.page_size;
+  a.rope_base = d.rope_base;
+  a.raw = raw;
+  a.status = status;
+  const int grid = (d.d_c + kRows - 1) / kRows + d.d_rope / 2;
   trace_record(MLA_TRACE_APPEND_PROJECT, false, st);
-  if (d.act_dtype == MLA_F32)
-    append_project_kernel<float><<<pgrid, 256, 0, st>>>(
-        (const float*)h, n_tokens, (const float*)W_dkv, (const float*)W_kr, d.d_c, d.d_rope, d.d_model, raw);
-  else
-    append_project_kernel<__nv_bfloat16><<<pgrid, 256, 0, st>>>(
-        (const __nv_bfloat16*)h, n_tokens, (const __nv_bfloat16*)W_dkv, (const __nv_bfloat16*)W_kr,
-        d.d_c, d.d_rope, d.d_model, raw);
+#define MLA_PROJ(T, K) append_project_kernel<T, K><<<grid, 256, 0, st>>>(a)
+  if (d.act_dtype == MLA_F32) {
+    if (d.cache_dtype == MLA_F32) MLA_PROJ(float, MLA_F32);
+    else if (d.cache_dtype == MLA_BF16) MLA_PROJ(float, MLA_BF16);
+    else MLA_PROJ(float, MLA_FP8_E4M3);
+  } else {
+    if (d.cache_dtype == MLA_F32) MLA_PROJ(__nv_bfloat16, MLA_F32);
+    else if (d.cache_dtype == MLA_BF16) MLA_PROJ(__nv_bfloat16, MLA_BF16);
+    else MLA_PROJ(__nv_bfloat16, MLA_FP8_E4M3);
+  }
+#undef MLA_PROJ
   cudaError_t e = cudaGetLastError();
   trace_record(MLA_TRACE_APPEND_PROJECT, true, st);
   if (e != cudaSuccess) return e;
   trace_record(MLA_TRACE_APPEND_FINALIZE, false, st);
-#define MLA_FIN(K)                                                                               \
-  append_finalize_kernel<K><<<n_tokens, 128, 0, st>>>(raw, seq_idx, pos, page_table, batch,      \
-                                                      max_pages, (uint8_t*)pool, num_pages,      \
-                                                      page_bytes, d.d_c, d.d_rope, d.page_size,  \
-                                                      d.rope_base, status)
-  if (d.cache_dtype == MLA_F32) MLA_FIN(MLA_F32);
-  else if (d.cache_dtype == MLA_BF16) MLA_FIN(MLA_BF16);
-  else MLA_FIN(MLA_FP8_E4M3);
-#undef MLA_FIN
+  if (d.cache_dtype != MLA_FP8_E4M3) {
+    trace_record(MLA_TRACE_APPEND_FINALIZE, true, st);
+    return e;
+  }
+  append_fp8_finalize_kernel<<<n_tokens, 128, 0, st>>>(a);
   e = cudaGetLastError();
   trace_record(MLA_TRACE_APPEND_FINALIZE, true, st);
   return e;

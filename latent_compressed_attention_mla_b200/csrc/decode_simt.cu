@@ -9,68 +9,11 @@
 // passed through an online (running max / running sum) softmax in base 2, and
 // the probabilities aggregate the latent c_s itself (decoding module step 5),
 // so W^UV is applied later, in the combine step.
-//
-// Also here: the plan kernel that turns device-resident sequence lengths into
-// the tile prefix sums every split and the combine step read.
 #include "mla_internal.cuh"
 
 namespace mla {
 
 namespace {
-
-// One block: tile_start[b] = sum_{b'<b} ceil(len_b' / page_size) for valid
-// sequences (n_q <= len <= max_pages * page_size), 0 tiles for invalid ones
-// (recorded as MLA_ERR_BOUNDS).  Then the header {TT, W, batch, n_q}.
-__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ seq_lens, int batch,
-                                                    int n_q, int page_size, int max_pages, int splits,
-                                                    int32_t* __restrict__ plan, int* status) {
-  __shared__ int32_t warp_sums[32];
-  __shared__ int32_t carry;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) carry = 0;
-  __syncthreads();
-  for (int base = 0; base < batch; base += 1024) {
-    const int b = base + tid;
-    int tiles = 0;
-    if (b < batch) {
-      const int len = seq_lens[b];
-      if (len >= n_q && len >= 1 && (long long)len <= (long long)max_pages * page_size)
-        tiles = (len + page_size - 1) / page_size;
-      else
-        record_status(status, MLA_ERR_BOUNDS);
-    }
-    int x = tiles;  // inclusive warp scan
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_sums[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int s = warp_sums[lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, s, o);
-        if (lane >= o) s += y;
-      }
-      warp_sums[lane] = s;  // inclusive
-    }
-    __syncthreads();
-    const int excl = carry + (warp ? warp_sums[warp - 1] : 0) + x - tiles;
-    if (b < batch) plan[b] = excl;
-    __syncthreads();
-    if (tid == 1023) carry = excl + tiles;
-    __syncthreads();
-  }
-  if (tid == 0) {
-    plan[batch] = carry;
-    plan[batch + 1] = carry;
-    plan[batch + 2] = splits;
-    plan[batch + 3] = batch;
-    plan[batch + 4] = n_q;
-  }
-}
 
 // Cache row element loaders into fp32 shared memory.
 template <int CACHE>
@@ -229,12 +172,6 @@ bool decode_simt_supported(const mla_dims& d) {
   const size_t D = (size_t)d.d_c + d.d_rope;
   const size_t smem = 4 * (HG * (D + 1) + TPH * (D + 1) + HG * TPH);
   return smem <= 200 * 1024;
-}
-
-cudaError_t launch_plan(const int32_t* seq_lens, int batch, int n_q, int page_size, int max_pages,
-                        int splits, int32_t* plan, int* status, cudaStream_t st) {
-  plan_kernel<<<1, 1024, 0, st>>>(seq_lens, batch, n_q, page_size, max_pages, splits, plan, status);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t st) {

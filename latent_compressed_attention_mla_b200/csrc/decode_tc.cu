@@ -20,9 +20,14 @@
 //    S (2 buffers) and O live in tensor memory (TMEM); per CTA S uses 2 x 32
 //    columns and O 2 x 128 columns of the 2-SM ("2x2") accumulator layout:
 //    row m, column n < N/2 -> lane m, column n; n >= N/2 -> lane 64+m, n-N/2.
-//  * TMA loads, 128-byte swizzle: per tile each CTA loads its 32-key half of
-//    the rows (all 576 columns, the QK B operand, K-major) and all 64 keys of
-//    its 256-column half of the latent (the PV B operand, MN-major).
+//  * Operands stream through a ring of 4 KB units (TMA, 128-byte swizzle) in
+//    the order the MMAs consume them: the 9 QK units of tile g (this CTA's
+//    32-key half of the rows x 64 columns each, K-major), then the 8 PV units
+//    of tile g-1 (16 keys x this CTA's 128 latent columns of one N=256 MMA,
+//    MN-major).  Each unit has its own full/empty barrier, so loads run about
+//    two tiles ahead of the MMAs.  Rows past a sequence's end in its last page
+//    are loaded from outside the tensor (TMA zero fill), never from the pool,
+//    so 0 * (whatever the pool held) cannot reach O.
 //  * Warp roles: warps 0-3 softmax + epilogue (one TMEM lane each), warp 4
 //    TMA producer, warp 5 TMEM allocation and (leader CTA) MMA issue.
 //  * Online softmax in base 2 with a lazily updated reference max: O is only
@@ -45,21 +50,19 @@ constexpr int kHeads = 128, kHalfHeads = 64;
 constexpr int kDC = 512, kDR = 64, kD = kDC + kDR;  // 576
 constexpr int kPage = 64;                             // keys per tile
 constexpr int kChunks = kD / 64;                      // 9 column chunks of 64 (128 B)
-constexpr int kStages = 2;
+constexpr uint32_t kUnitBytes = 4096;                      // one ring unit
+constexpr int kUnits = 32;                                   // ring depth (128 KB)
+constexpr int kQKUnits = kChunks;                            // 9 per tile
+constexpr int kPVUnits = 8;                                  // 2 MMAs x 4 K-steps per tile
 
 // shared memory layout (offsets from a 1024-byte aligned base)
 constexpr uint32_t kQBytes = kChunks * 64 * 128;           // 73728: 64 heads x 576 bf16
-constexpr uint32_t kKQChunk = 32 * 128;                    // 4096: 32 keys x 64 cols
-constexpr uint32_t kKQBytes = kChunks * kKQChunk;          // 36864
-constexpr uint32_t kPVChunk = 64 * 128;                    // 8192: 64 keys x 64 cols
-constexpr uint32_t kPVBytes = 4 * kPVChunk;                // 32768
-constexpr uint32_t kStageBytes = kKQBytes + kPVBytes;      // 69632
 constexpr uint32_t kPBytes = 64 * 128;                     // 8192: 64 heads x 64 keys bf16
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffStage = kOffQ + kQBytes;
-constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;  // 212992
-constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;              // 229376
-constexpr uint32_t kNumBars = 16;
+constexpr uint32_t kOffRing = kOffQ + kQBytes;
+constexpr uint32_t kOffP = kOffRing + kUnits * kUnitBytes;   // 204800
+constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;            // 221184
+constexpr uint32_t kNumBars = 2 * kUnits + 16;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffRedMax = kOffMisc + 16;                 // float [2][64]
 constexpr uint32_t kOffRedL = kOffRedMax + 512;                // float [2][64]
@@ -68,15 +71,15 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;              // + alignment sl
 
 // barrier indices
 enum {
-  B_KV_FULL = 0,   // [2] leader: TMA bytes of both CTAs
-  B_KV_EMPTY = 2,  // [2] each CTA: stage consumed (MMA commit)
-  B_S_FULL = 4,    // [2] each CTA: S tile ready (MMA commit)
-  B_S_FREE = 6,    // [2] leader: S read by both CTAs' softmax warps (8 arrivals)
-  B_P_FULL = 8,    // [2] leader: P written + O rescaled by both CTAs (8 arrivals)
-  B_O_DONE = 10,   // each CTA: a PV group finished (MMA commit)
-  B_O_FREE = 11,   // leader: O read out by both CTAs' epilogues (8 arrivals)
-  B_Q_FULL = 12,   // leader: Q bytes of both CTAs
-  B_Q_EMPTY = 13,  // each CTA: last QK of a segment finished (MMA commit)
+  B_UNIT_FULL = 0,          // [kUnits] leader: TMA bytes of both CTAs
+  B_UNIT_EMPTY = kUnits,    // [kUnits] each CTA: unit consumed (MMA commit)
+  B_S_FULL = 2 * kUnits,    // [2] each CTA: S tile ready (MMA commit)
+  B_S_FREE = B_S_FULL + 2,  // [2] leader: S read by both CTAs' softmax warps (8 arrivals)
+  B_P_FULL = B_S_FREE + 2,  // [2] leader: P written + O rescaled by both CTAs (8 arrivals)
+  B_O_DONE = B_P_FULL + 2,  // [2] each CTA: PV(g) finished, g's P buffer parity (MMA commit)
+  B_O_FREE = B_O_DONE + 2,  // leader: O read out by both CTAs' epilogues (8 arrivals)
+  B_Q_FULL,                 // leader: Q bytes of both CTAs
+  B_Q_EMPTY,                // each CTA: last QK of a segment finished (MMA commit)
 };
 
 // TMEM columns (per CTA, 2x2 layout): S buffers 32 columns each, O 2 x 128
@@ -93,6 +96,25 @@ constexpr uint32_t idesc(int M, int N, bool a_mn, bool b_mn) {
 }
 constexpr uint32_t kIdescQK = idesc(128, 64, false, false);
 constexpr uint32_t kIdescPV = idesc(128, 256, false, true);
+
+// ---------------------------------------------------------------------------
+// Protocol timestamps for development builds (-DMLA_TC_TRACE): event e of
+// tile g in CTA b, read back with mla_tc_trace_read.  Absent otherwise.
+// ---------------------------------------------------------------------------
+#ifdef MLA_TC_TRACE
+constexpr int kTrCtas = 8, kTrTiles = 48, kTrEvents = 8;
+__device__ unsigned long long g_tc_trace[kTrCtas * kTrTiles * kTrEvents];
+__device__ __forceinline__ void tc_trace(int e, uint32_t g) {
+  if (blockIdx.x < kTrCtas && g < kTrTiles) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    g_tc_trace[(blockIdx.x * kTrTiles + g) * kTrEvents + e] = t;
+  }
+}
+#define TC_TRACE(e, g) tc_trace((e), (g))
+#else
+#define TC_TRACE(e, g) ((void)0)
+#endif
 
 // ---------------------------------------------------------------------------
 // PTX helpers
@@ -264,8 +286,9 @@ struct SegmentWalker {
 struct TcParams {
   DecodeParams p;
   CUtensorMap map_q;   // q_abs [rows = batch*n_q*128][576] bf16, box 64 x 64
-  CUtensorMap map_kq;  // pool rows [num_pages*64][576] bf16, box 64 x 32
-  CUtensorMap map_pv;  // pool rows [num_pages*64][576] bf16, box 64 x 64
+  CUtensorMap map_kq;  // pool rows [num_pages*64][576] bf16, box 64 x 32 (QK units)
+  CUtensorMap map_pv;  // pool rows, box 64 x 16 (PV unit halves)
+  CUtensorMap map_row; // pool rows, box 64 x 1 (PV rows of a partial 16-key step)
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
@@ -288,14 +311,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
+    for (int i = 0; i < kUnits; ++i) {
+      mbar_init(bar(B_UNIT_FULL + i), 1);
+      mbar_init(bar(B_UNIT_EMPTY + i), 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(B_KV_FULL + i), 1);
-      mbar_init(bar(B_KV_EMPTY + i), 1);
       mbar_init(bar(B_S_FULL + i), 1);
       mbar_init(bar(B_S_FREE + i), 8);
       mbar_init(bar(B_P_FULL + i), 8);
     }
     mbar_init(bar(B_O_DONE), 1);
+    mbar_init(bar(B_O_DONE + 1), 1);
     mbar_init(bar(B_O_FREE), 8);
     mbar_init(bar(B_Q_FULL), 1);
     mbar_init(bar(B_Q_EMPTY), 1);
@@ -317,8 +343,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     if (lane == 0) {
       SegmentWalker walk(p, w, t);
       Segment s;
-      uint32_t g = 0, seg = 0;
+      uint32_t U = 0, seg = 0, gtile = 0;
       bool ok = true;
+      (void)gtile;
+      const int y_half = 32 * (int)rank;  // this CTA's half of a tile's keys (QK units)
+      const int x_pv = 128 * (int)rank;   // this CTA's half of an N=256 MMA's columns (PV units)
+      // wait for ring unit U to be free; the leader expects both CTAs' bytes
+      auto acquire = [&](uint32_t& dst, uint32_t& fullbar) -> bool {
+        const uint32_t u = U % kUnits;
+        if (!mbar_wait(bar(B_UNIT_EMPTY + u), ((U / kUnits) & 1) ^ 1, abort_flag, p.status)) return false;
+        if (rank == 0) mbar_expect_tx(bar(B_UNIT_FULL + u), 2 * kUnitBytes);
+        dst = sbase + kOffRing + u * kUnitBytes;
+        fullbar = leader_bar(B_UNIT_FULL + u);
+        ++U;
+        return true;
+      };
+      auto load_qk = [&](int page) -> bool {
+        for (int c = 0; c < kQKUnits; ++c) {
+          uint32_t dst, fb;
+          if (!acquire(dst, fb)) return false;
+          tma_load_2d_pair(dst, &P.map_kq, 64 * c, page * kPage + y_half, fb);
+        }
+        return true;
+      };
+      // PV units of a tile whose first `valid` keys are visible: rows past
+      // them come from outside the tensor (zero fill)
+      auto load_pv = [&](int page, int valid) -> bool {
+        for (int j = 0; j < 2; ++j)
+          for (int ks = 0; ks < 4; ++ks) {
+            uint32_t dst, fb;
+            if (!acquire(dst, fb)) return false;
+            for (int a = 0; a < 2; ++a) {
+              const int x = 256 * j + x_pv + 64 * a;
+              const uint32_t d = dst + a * 2048;
+              if (16 * ks + 16 <= valid) {
+                tma_load_2d_pair(d, &P.map_pv, x, page * kPage + 16 * ks, fb);
+              } else if (16 * ks >= valid) {
+                tma_load_2d_pair(d, &P.map_pv, x, -16, fb);
+              } else {
+                for (int i = 0; i < 16; ++i)
+                  tma_load_2d_pair(d + i * 128, &P.map_row, x, 16 * ks + i < valid ? page * kPage + 16 * ks + i : -1,
+                                   fb);
+              }
+            }
+          }
+        return true;
+      };
+      auto page_of = [&](int b, int tile) -> int {
+        int page = p.page_table[(size_t)b * p.max_pages + tile];
+        if (page < 0 || page >= p.num_pages) {
+          record_status(p.status, MLA_ERR_BOUNDS);
+          page = 0;
+        }
+        return page;
+      };
       while (ok && walk.next(s)) {
         if (s.n_tiles == 0) continue;
         // absorbed queries of this CTA's 64 heads for (b, t)
@@ -328,27 +406,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         const int qrow = ((s.b * p.n_q + t) * kHeads) + kHalfHeads * (int)rank;
         const uint32_t qbar = leader_bar(B_Q_FULL);
         for (int c = 0; c < kChunks; ++c) tma_load_2d_pair(sbase + kOffQ + c * 8192, &P.map_q, 64 * c, qrow, qbar);
-        for (int i = 0; i < s.n_tiles; ++i, ++g) {
-          const int st = g % kStages;
-          ok = mbar_wait(bar(B_KV_EMPTY + st), ((g / kStages) & 1) ^ 1, abort_flag, p.status);
-          if (!ok) break;
-          int page = p.page_table[(size_t)s.b * p.max_pages + s.tile_lo + i];
-          if (page < 0 || page >= p.num_pages) {
-            record_status(p.status, MLA_ERR_BOUNDS);
-            page = 0;
-          }
-          if (rank == 0) mbar_expect_tx(bar(B_KV_FULL + st), 2 * kStageBytes);
-          const uint32_t kbar = leader_bar(B_KV_FULL + st);
-          const uint32_t stage = sbase + kOffStage + st * kStageBytes;
-          const int row0 = page * kPage;
-          for (int c = 0; c < kChunks; ++c)
-            tma_load_2d_pair(stage + c * kKQChunk, &P.map_kq, 64 * c, row0 + 32 * (int)rank, kbar);
-          // PV operand: chunks {2r, 2r+1} (dims 128r..) and {4+2r, 5+2r} (dims 256+128r..)
-          for (int j = 0; j < 2; ++j)
-            for (int a = 0; a < 2; ++a)
-              tma_load_2d_pair(stage + kKQBytes + (2 * j + a) * kPVChunk, &P.map_pv, 64 * (4 * j + 2 * (int)rank + a),
-                               row0, kbar);
+        int prev_page = 0, prev_valid = 0;
+        for (int i = 0; i < s.n_tiles && ok; ++i) {
+          const int tile = s.tile_lo + i;
+          const int page = page_of(s.b, tile);
+          TC_TRACE(0, gtile++);
+          ok = load_qk(page);
+          if (ok && i > 0) ok = load_pv(prev_page, prev_valid);
+          prev_page = page;
+          prev_valid = min(kPage, s.nvis - tile * kPage);
         }
+        if (ok) ok = load_pv(prev_page, prev_valid);
         ++seg;
       }
     }
@@ -357,23 +425,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     if (rank == 0 && lane == 0) {
       SegmentWalker walk(p, w, t);
       Segment s;
-      uint32_t g = 0, seg = 0;
+      uint32_t U = 0, g = 0, seg = 0;
       bool ok = true;
+      auto unit_ready = [&](uint32_t& addr) -> bool {
+        const uint32_t u = U % kUnits;
+        if (!mbar_wait(bar(B_UNIT_FULL + u), (U / kUnits) & 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        addr = sbase + kOffRing + u * kUnitBytes;
+        return true;
+      };
+      auto unit_done = [&]() {
+        tc_commit_pair(bar(B_UNIT_EMPTY + (U % kUnits)));
+        ++U;
+      };
       auto do_pv = [&](uint32_t gi, bool first) -> bool {
         if (!mbar_wait(bar(B_P_FULL + (gi & 1)), (gi >> 1) & 1, abort_flag, p.status)) return false;
+        TC_TRACE(2, gi);
         tc_fence_after();
-        const int st = gi % kStages;
-        const uint32_t pv = sbase + kOffStage + st * kStageBytes + kKQBytes;
         const uint32_t pa = sbase + kOffP + (gi & 1) * kPBytes;
-#pragma unroll
         for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            tc_mma(tmem + (j ? kColO1 : kColO0), sdesc(pa + ks * 32, 16, 1024),
-                   sdesc(pv + 2 * j * kPVChunk + ks * 2048, kPVChunk, 1024), kIdescPV,
+          for (int ks = 0; ks < 4; ++ks) {
+            uint32_t unit;
+            if (!unit_ready(unit)) return false;
+            tc_mma(tmem + (j ? kColO1 : kColO0), sdesc(pa + ks * 32, 16, 1024), sdesc(unit, 2048, 1024), kIdescPV,
                    (first && ks == 0) ? 0u : 1u);
-        tc_commit_pair(bar(B_KV_EMPTY + st));
-        tc_commit_pair(bar(B_O_DONE));
+            unit_done();
+          }
+        tc_commit_pair(bar(B_O_DONE + (gi & 1)));
+        TC_TRACE(3, gi);
         return true;
       };
       while (ok && walk.next(s)) {
@@ -383,19 +462,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t g_first = g;
         for (int i = 0; i < s.n_tiles && ok; ++i, ++g) {
-          const int st = g % kStages;
-          ok = mbar_wait(bar(B_KV_FULL + st), (g / kStages) & 1, abort_flag, p.status) &&
-               mbar_wait(bar(B_S_FREE + (g & 1)), ((g >> 1) & 1) ^ 1, abort_flag, p.status);
+          ok = mbar_wait(bar(B_S_FREE + (g & 1)), ((g >> 1) & 1) ^ 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t kq = sbase + kOffStage + st * kStageBytes;
-#pragma unroll 4
-          for (int k = 0; k < kD / 16; ++k) {
-            const uint32_t off = (k & 3) * 32;  // 16 columns = 32 bytes into the swizzled row
-            tc_mma(tmem + ((g & 1) ? kColS1 : kColS0), sdesc(sbase + kOffQ + (k >> 2) * 8192 + off, 16, 1024),
-                   sdesc(kq + (k >> 2) * kKQChunk + off, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
+          const uint32_t sd = tmem + ((g & 1) ? kColS1 : kColS0);
+          TC_TRACE(7, g);
+          for (int c = 0; c < kQKUnits && ok; ++c) {
+            uint32_t unit;
+            ok = unit_ready(unit);
+            if (!ok) break;
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)  // 16 columns = 32 bytes into the swizzled rows
+              tc_mma(sd, sdesc(sbase + kOffQ + c * 8192 + k4 * 32, 16, 1024), sdesc(unit + k4 * 32, 16, 1024),
+                     kIdescQK, (c | k4) ? 1u : 0u);
+            unit_done();
           }
+          if (!ok) break;
           tc_commit_pair(bar(B_S_FULL + (g & 1)));
+          TC_TRACE(1, g);
           if (i == s.n_tiles - 1) tc_commit_pair(bar(B_Q_EMPTY));
           if (i > 0) {
             if (i == 1 && seg > 0) {  // O of the previous segment must be read out first
@@ -439,10 +523,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         ok = mbar_wait(bar(B_S_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.status);
         __syncwarp();
         if (!ok) break;
+        if (threadIdx.x == 0) TC_TRACE(4, g);
         tc_fence_after();
         uint32_t sr[32];
         tmem_ld32(tmem + lane_base + ((g & 1) ? kColS1 : kColS0), sr);
         tmem_wait_ld();
+        if (threadIdx.x == 0) TC_TRACE(5, g);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_bar(B_S_FREE + (g & 1)));
@@ -477,15 +563,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
         }
         l_part = l_part * alpha + psum;
-        if (i > 0) {  // PV of the previous tile must be done before O or its P buffer is touched
-          ok = mbar_wait(bar(B_O_DONE), (g - 1) & 1, abort_flag, p.status);
+        // P buffer g&1 was last read by PV(g-2)
+        if (g >= 2) {
+          ok = mbar_wait(bar(B_O_DONE + (g & 1)), ((g - 2) >> 1) & 1, abort_flag, p.status);
+          __syncwarp();
+          if (!ok) break;
+        }
+        // tcgen05.ld/st are whole-warp instructions: rescale the warp's lanes
+        // together (alpha = 1 on lanes whose head keeps its reference max),
+        // after PV(g-1), the last MMA writing O, has finished
+        const bool warp_rescale = __any_sync(0xffffffffu, rescale);
+        if (warp_rescale) {
+          ok = mbar_wait(bar(B_O_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, p.status);
           __syncwarp();
           if (!ok) break;
           tc_fence_after();
         }
-        // tcgen05.ld/st are whole-warp instructions: rescale the warp's lanes
-        // together (alpha = 1 on lanes whose head keeps its reference max)
-        if (__any_sync(0xffffffffu, rescale)) {
+        if (warp_rescale) {
 #pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
             const uint32_t col = (c < 128 ? kColO0 + c : kColO1 + (c - 128));
@@ -505,25 +599,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           const int unit = (4 * half + u) ^ (hl & 7);
           *reinterpret_cast<uint4*>(prow + unit * 16) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
-        // rows past the sequence end in the last tile: zero this CTA's latent
-        // operand rows so that 0 * (whatever the pool held) cannot reach O
-        const int valid = s.nvis - (s.tile_lo + i) * kPage;
-        if (valid < kPage) {
-          uint8_t* pv = smem + kOffStage + (g % kStages) * kStageBytes + kKQBytes;
-          const int rows = kPage - valid;
-          for (int x = threadIdx.x; x < rows * 4 * 8; x += 128) {
-            const int r = valid + x / 32, rem = x % 32, c = rem / 8, u = rem % 8;
-            *reinterpret_cast<uint4*>(pv + c * kPVChunk + r * 128 + u * 16) = make_uint4(0, 0, 0, 0);
-          }
-        }
         fence_proxy_async();
         tc_fence_before();
         asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (threadIdx.x == 0) TC_TRACE(6, g);
         if (lane == 0) mbar_arrive_cluster(leader_bar(B_P_FULL + (g & 1)));
       }
       if (!ok) break;
       // epilogue: wait for the last PV, normalise, write the split's partial
-      ok = mbar_wait(bar(B_O_DONE), (g - 1) & 1, abort_flag, p.status);
+      ok = mbar_wait(bar(B_O_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, p.status);
       __syncwarp();
       if (!ok) break;
       tc_fence_after();
@@ -620,7 +704,8 @@ cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st) {
   tp.p = p;
   const uint64_t pool_rows = (uint64_t)p.num_pages * kPage;
   if (!make_map(&tp.map_q, p.q_abs, (uint64_t)p.batch * p.n_q * kHeads, 64) ||
-      !make_map(&tp.map_kq, p.pool, pool_rows, 32) || !make_map(&tp.map_pv, p.pool, pool_rows, 64))
+      !make_map(&tp.map_kq, p.pool, pool_rows, 32) || !make_map(&tp.map_pv, p.pool, pool_rows, 16) ||
+      !make_map(&tp.map_row, p.pool, pool_rows, 1))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -630,3 +715,9 @@ cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st) {
 }
 
 }  // namespace mla
+
+#ifdef MLA_TC_TRACE
+extern "C" int mla_tc_trace_read(void* host, size_t bytes) {
+  return cudaMemcpyFromSymbol(host, mla::g_tc_trace, bytes) == cudaSuccess ? 0 : 8;
+}
+#endif

@@ -9,6 +9,11 @@
 namespace mla {
 size_t cache_page_bytes(const mla_dims& d);
 bool decode_simt_supported(const mla_dims& d);
+int append_max_d_model(int act_dtype);
+size_t append_scratch_floats(const mla_dims& d, int n_tokens);
+int absorb_max_d_nope();
+int combine_max_splits();
+int combine_max_d_c(int act_dtype);
 }  // namespace mla
 
 using namespace mla;
@@ -30,6 +35,7 @@ static __device__ int g_mla_status;
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kMinTilesPerSplit = 4;
 int* g_status_ptr[kMaxDevices] = {nullptr};
 
 int* status_ptr() {
@@ -54,7 +60,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int check_dims(const mla_dims* d) {
   if (!d) return MLA_ERR_INVALID_ARG;
   if (d->n_heads < 1 || d->d_c < 16 || d->d_c % 16 || d->d_rope < 0 || d->d_rope % 2 || d->d_nope < 1 ||
-      d->d_v < 1 || d->d_model < 16 || d->d_model % 16 || d->page_size < 1)
+      d->d_v < 1 || d->d_model < 32 || d->d_model % 32 || d->page_size < 1)
     return MLA_ERR_INVALID_ARG;
   if (!(d->softmax_scale > 0.f) || !isfinite(d->softmax_scale) || !(d->rope_base > 0.f) || !isfinite(d->rope_base))
     return MLA_ERR_INVALID_ARG;
@@ -64,6 +70,8 @@ int check_dims(const mla_dims* d) {
   if (d->cache_dtype == MLA_F32 && d->act_dtype != MLA_F32) return MLA_ERR_UNSUPPORTED;
   if (d->cache_dtype == MLA_FP8_E4M3 && d->d_c % 128) return MLA_ERR_UNSUPPORTED;
   if (d->d_nope % 8 || d->d_v > 1024) return MLA_ERR_UNSUPPORTED;
+  if (d->d_model > append_max_d_model(d->act_dtype)) return MLA_ERR_UNSUPPORTED;
+  if (d->d_nope > absorb_max_d_nope() || d->d_c > combine_max_d_c(d->act_dtype)) return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
 }
 
@@ -74,7 +82,7 @@ int auto_splits(const mla_dims& d, int batch, int n_q) {
   const int hg = d.n_heads % 8 == 0 && d.d_c / 16 <= 32 ? 8 : 4;
   const int per_split = n_q * (d.n_heads / hg);
   int w = (4 * sms + per_split - 1) / per_split;
-  return w < 1 ? 1 : (w > 512 ? 512 : w);
+  return w < 1 ? 1 : (w > combine_max_splits() ? combine_max_splits() : w);
 }
 
 int launch_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_LAUNCH; }
@@ -97,7 +105,7 @@ int mla_check_dims(const mla_dims* dims) { return check_dims(dims); }
 
 size_t mla_append_workspace_bytes(const mla_dims* dims, int n_tokens) {
   if (check_dims(dims) != MLA_OK || n_tokens < 0) return 0;
-  return align_up(sizeof(float) * (size_t)n_tokens * (dims->d_c + dims->d_rope), 256);
+  return align_up(sizeof(float) * append_scratch_floats(*dims, n_tokens), 256);
 }
 
 int mla_append_latent(const mla_dims* dims, const void* h, int n_tokens, const int32_t* seq_idx,
@@ -109,8 +117,10 @@ int mla_append_latent(const mla_dims* dims, const void* h, int n_tokens, const i
   if (n_tokens < 0 || batch < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
   if (n_tokens == 0) return MLA_OK;
   if (!h || !seq_idx || !pos || !W_dkv || !W_kr || !page_table || !cache_pool) return MLA_ERR_INVALID_ARG;
-  if (!workspace || ws_bytes < mla_append_workspace_bytes(dims, n_tokens)) return MLA_ERR_WORKSPACE;
-  if (!aligned16(h) || !aligned16(W_dkv) || !aligned16(W_kr) || !aligned16(cache_pool) || !aligned16(workspace))
+  const size_t need = mla_append_workspace_bytes(dims, n_tokens);
+  if (need > 0 && (!workspace || ws_bytes < need)) return MLA_ERR_WORKSPACE;
+  if (!aligned16(h) || !aligned16(W_dkv) || !aligned16(W_kr) || !aligned16(cache_pool) ||
+      (need > 0 && !aligned16(workspace)))
     return MLA_ERR_ALIGNMENT;
   return launch_status(launch_append(*dims, h, n_tokens, seq_idx, pos, W_dkv, W_kr, page_table, batch,
                                      max_pages, cache_pool, num_pages, cache_page_bytes(*dims),
@@ -143,24 +153,34 @@ int mla_decode(const mla_dims* dims, const void* q_nope, const void* q_rope, con
                void* stream) {
   int rc = check_dims(dims);
   if (rc != MLA_OK) return rc;
-  if (batch < 1 || n_q < 1 || num_pages < 1 || max_pages < 1 || num_splits < 0) return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || n_q < 1 || num_pages < 1 || max_pages < 1 || num_splits < 0 ||
+      num_splits > combine_max_splits())
+    return MLA_ERR_INVALID_ARG;
   if (!q_nope || !q_rope || !W_uk || !cache_pool || !page_table || !seq_lens) return MLA_ERR_INVALID_ARG;
   const int path = mla_decode_path(dims, n_q);
   if (path < 0) return -path;
-  const int W = num_splits > 0 ? num_splits : auto_splits(*dims, batch, n_q);
-  const DecodeLayout L = decode_layout(*dims, batch, n_q, W);
+  // The workspace layout is the one of the requested (or automatic) split
+  // count; with num_splits = 0 short contexts use fewer splits (at least
+  // kMinTilesPerSplit key tiles each, counted on batch * max_pages), which the
+  // plan records for mla_combine.
+  const int W_layout = num_splits > 0 ? num_splits : auto_splits(*dims, batch, n_q);
+  const DecodeLayout L = decode_layout(*dims, batch, n_q, W_layout);
+  int W = W_layout;
+  if (num_splits == 0) {
+    const long long cap = ((long long)batch * max_pages + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
+    if (cap < W) W = (int)(cap > 0 ? cap : 1);
+  }
   if (!workspace || ws_bytes < L.total) return MLA_ERR_WORKSPACE;
   if (!aligned16(W_uk) || !aligned16(cache_pool) || !aligned16(workspace)) return MLA_ERR_ALIGNMENT;
   cudaStream_t st = (cudaStream_t)stream;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* plan = reinterpret_cast<int32_t*>(ws + L.off_plan);
   int* status = status_ptr();
-  trace_record(MLA_TRACE_PLAN, false, st);
-  cudaError_t e = launch_plan(seq_lens, batch, n_q, dims->page_size, max_pages, W, plan, status, st);
-  trace_record(MLA_TRACE_PLAN, true, st);
-  if (e != cudaSuccess) return MLA_ERR_LAUNCH;
   trace_record(MLA_TRACE_ABSORB, false, st);
-  e = launch_absorb(*dims, q_nope, q_rope, W_uk, seq_lens, batch, n_q, ws + L.off_q, st);
+  const int n_slots = batch + W - 1;
+  cudaError_t e = launch_absorb_and_plan(*dims, q_nope, q_rope, W_uk, seq_lens, batch, n_q, max_pages, W, ws + L.off_q,
+                                         plan, reinterpret_cast<float*>(ws + L.off_lse),
+                                         (size_t)n_q * n_slots * dims->n_heads, status, st);
   trace_record(MLA_TRACE_ABSORB, true, st);
   if (e != cudaSuccess) return MLA_ERR_LAUNCH;
   DecodeParams p;
@@ -178,7 +198,7 @@ int mla_decode(const mla_dims* dims, const void* q_nope, const void* q_rope, con
   p.batch = batch;
   p.n_q = n_q;
   p.splits = W;
-  p.n_slots = L.n_slots;
+  p.n_slots = n_slots;
   p.scale_log2 = dims->softmax_scale * kLog2e;
   p.status = status;
   trace_record(MLA_TRACE_ATTEND, false, st);
@@ -199,11 +219,9 @@ int mla_combine(const mla_dims* dims, const void* W_uv, int batch, int n_q, int 
   if (!aligned16(W_uv) || !aligned16(workspace)) return MLA_ERR_ALIGNMENT;
   const uint8_t* ws = static_cast<const uint8_t*>(workspace);
   trace_record(MLA_TRACE_COMBINE, false, (cudaStream_t)stream);
-  cudaError_t e = launch_combine(*dims, W_uv, batch, n_q, W, L.n_slots,
-                                 reinterpret_cast<const int32_t*>(ws + L.off_plan),
+  cudaError_t e = launch_combine(*dims, W_uv, batch, n_q, reinterpret_cast<const int32_t*>(ws + L.off_plan),
                                  reinterpret_cast<const float*>(ws + L.off_o),
-                                 reinterpret_cast<const float*>(ws + L.off_lse), out, lse_out,
-                                 (cudaStream_t)stream);
+                                 reinterpret_cast<const float*>(ws + L.off_lse), out, lse_out, (cudaStream_t)stream);
   trace_record(MLA_TRACE_COMBINE, true, (cudaStream_t)stream);
   return launch_status(e);
 }

@@ -76,7 +76,8 @@ __device__ __forceinline__ void rope_cos_sin(int pos, int i, int half, float bas
 // Decode workspace layout (shared by mla_decode and mla_combine)
 //   plan  : int32 [batch + 1] first key tile of each sequence (prefix sum of
 //           ceil(seq_len / page_size)), then int32 [4] {total tiles, splits,
-//           batch, n_q}
+//           batch, n_q}, then int32 [batch][2] {first split, split count}
+//           overlapping each sequence
 //   q_abs : [batch, n_q, n_heads, d_c + d_rope] act type (absorbed queries,
 //           rotated q^R appended)
 //   o_part: float32 [n_q, n_slots, n_heads, d_c] per-split normalised latent sums
@@ -100,7 +101,7 @@ inline DecodeLayout decode_layout(const mla_dims& d, int batch, int n_q, int spl
   size_t D = (size_t)d.d_c + d.d_rope;
   size_t off = 0;
   L.off_plan = off;
-  off = align_up(off + sizeof(int32_t) * ((size_t)batch + 1 + 4), 256);
+  off = align_up(off + sizeof(int32_t) * ((size_t)batch + 1 + 4 + 2 * (size_t)batch), 256);
   L.off_q = off;
   off = align_up(off + act * (size_t)batch * n_q * d.n_heads * D, 256);
   L.off_o = off;
@@ -155,11 +156,11 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
                           int num_pages, size_t page_bytes, float* raw, int* status,
                           cudaStream_t st);
 
-cudaError_t launch_plan(const int32_t* seq_lens, int batch, int n_q, int page_size, int max_pages,
-                        int splits, int32_t* plan, int* status, cudaStream_t st);
-
-cudaError_t launch_absorb(const mla_dims& d, const void* q_nope, const void* q_rope, const void* W_uk,
-                          const int32_t* seq_lens, int batch, int n_q, void* q_abs, cudaStream_t st);
+// absorb + split plan (+ empty-split initialisation of the lse slots)
+cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const void* q_rope, const void* W_uk,
+                                   const int32_t* seq_lens, int batch, int n_q, int max_pages, int splits,
+                                   void* q_abs, int32_t* plan, float* lse_part, size_t lse_count, int* status,
+                                   cudaStream_t st);
 
 cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t st);
 
@@ -167,8 +168,7 @@ bool decode_tc_supported(const mla_dims& d, int n_q);
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st);
 int decode_tc_auto_splits(int num_sms, int n_q);
 
-cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n_q, int splits,
-                           int n_slots, const int32_t* plan, const float* o_part,
-                           const float* lse_part, void* out, float* lse_out, cudaStream_t st);
+cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n_q, const int32_t* plan,
+                           const float* o_part, const float* lse_part, void* out, float* lse_out, cudaStream_t st);
 
 }  // namespace mla

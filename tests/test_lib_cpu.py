@@ -93,11 +93,17 @@ def test_host_side_argument_errors_return_before_any_launch():
     assert L.mla_combine(ref, fake, 1, 1, 4, fake, ws_need, None, None, None) == 1
     # append: zero tokens is a no-op, workspace checked otherwise
     assert L.mla_append_latent(ref, None, 0, None, None, None, None, None, 1, 1, None, 1, None, 0, None) == 0
-    need = B.append_workspace_bytes(d, 3)
-    assert need >= 3 * 576 * 4
-    assert L.mla_append_latent(ref, fake, 3, fake, fake, fake, fake, fake, 1, 1, fake, 1, fake, need - 1, None) == 3
-    assert L.mla_append_latent(ref, _p(0x10002), 3, fake, fake, fake, fake, fake, 1, 1, fake, 1, fake, need,
+    # bf16/fp32 caches: the projection writes the cache directly, no scratch
+    assert B.append_workspace_bytes(d, 3) == 0
+    assert L.mla_append_latent(ref, _p(0x10002), 3, fake, fake, fake, fake, fake, 1, 1, fake, 1, None, 0,
                                None) == 4
+    # FP8 caches keep fp32 c between the projection and the quantiser
+    d8 = B.dims_for(W.CONFIGS[4])
+    ref8 = ctypes.byref(d8)
+    need = B.append_workspace_bytes(d8, 3)
+    assert need >= 3 * 512 * 4
+    assert L.mla_append_latent(ref8, fake, 3, fake, fake, fake, fake, fake, 1, 1, fake, 1, fake, need - 1, None) == 3
+    assert L.mla_append_latent(ref8, fake, 3, fake, fake, fake, fake, fake, 1, 1, fake, 1, None, need, None) == 3
 
 
 def test_workspace_layout_grows_with_splits():
