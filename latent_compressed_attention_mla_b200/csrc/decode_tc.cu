@@ -48,21 +48,26 @@ namespace {
 // ---------------------------------------------------------------------------
 constexpr int kHeads = 128, kHalfHeads = 64;
 constexpr int kDC = 512, kDR = 64, kD = kDC + kDR;  // 576
-constexpr int kPage = 64;                             // keys per tile
+constexpr int kPage = 64;                             // keys per cache page
+constexpr int kTilePages = 4;                         // pages per tile: 256 keys = N of the QK MMA
 constexpr int kChunks = kD / 64;                      // 9 column chunks of 64 (128 B)
-constexpr uint32_t kUnitBytes = 4096;                      // one ring unit
-constexpr int kUnits = 32;                                   // ring depth (128 KB)
-constexpr int kQKUnits = kChunks;                            // 9 per tile
-constexpr int kPVUnits = 8;                                  // 2 MMAs x 4 K-steps per tile
+
+// Ring units: 16 KB each, this CTA's share of one MMA group
+//   QK unit c : its 128 keys of the tile (32 per page) x columns [64c, 64c+64), K-major
+//   PV unit   : one page's 64 keys x its 128 latent columns of one N=256 half, MN-major
+constexpr uint32_t kUnitBytes = 16384;
+constexpr int kUnits = 7;
+constexpr int kQKUnits = kChunks;                     // 9 per tile
+constexpr int kPVUnits = 2 * kTilePages;              // 8 per tile
 
 // shared memory layout (offsets from a 1024-byte aligned base)
-constexpr uint32_t kQBytes = kChunks * 64 * 128;           // 73728: 64 heads x 576 bf16
-constexpr uint32_t kPBytes = 64 * 128;                     // 8192: 64 heads x 64 keys bf16
+constexpr uint32_t kQBytes = kChunks * 64 * 128;      // 73728: 64 heads x 576 bf16
+constexpr uint32_t kPBytes = kTilePages * 64 * 128;   // 32768: 64 heads x 256 keys bf16, 4 sub-tiles
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffRing = kOffQ + kQBytes;
-constexpr uint32_t kOffP = kOffRing + kUnits * kUnitBytes;   // 204800
-constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;            // 221184
-constexpr uint32_t kNumBars = 2 * kUnits + 16;
+constexpr uint32_t kOffP = kOffQ + kQBytes;
+constexpr uint32_t kOffRing = kOffP + kPBytes;                // 106496
+constexpr uint32_t kOffBar = kOffRing + kUnits * kUnitBytes;  // 221184
+constexpr uint32_t kNumBars = 2 * kUnits + 10;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffRedMax = kOffMisc + 16;                 // float [2][64]
 constexpr uint32_t kOffRedL = kOffRedMax + 512;                // float [2][64]
@@ -75,16 +80,16 @@ enum {
   B_UNIT_EMPTY = kUnits,    // [kUnits] each CTA: unit consumed (MMA commit)
   B_S_FULL = 2 * kUnits,    // [2] each CTA: S tile ready (MMA commit)
   B_S_FREE = B_S_FULL + 2,  // [2] leader: S read by both CTAs' softmax warps (8 arrivals)
-  B_P_FULL = B_S_FREE + 2,  // [2] leader: P written + O rescaled by both CTAs (8 arrivals)
-  B_O_DONE = B_P_FULL + 2,  // [2] each CTA: PV(g) finished, g's P buffer parity (MMA commit)
-  B_O_FREE = B_O_DONE + 2,  // leader: O read out by both CTAs' epilogues (8 arrivals)
+  B_P_FULL = B_S_FREE + 2,  // leader: P written + O rescaled by both CTAs (8 arrivals)
+  B_O_DONE,                 // each CTA: the tile's PV MMAs finished (MMA commit)
+  B_O_FREE,                 // leader: O read out by both CTAs' epilogues (8 arrivals)
   B_Q_FULL,                 // leader: Q bytes of both CTAs
   B_Q_EMPTY,                // each CTA: last QK of a segment finished (MMA commit)
 };
 
-// TMEM columns (per CTA, 2x2 layout): S buffers 32 columns each, O 2 x 128
+// TMEM columns (per CTA, 2x2 layout): S buffers 128 columns each, O 2 x 128
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 32, kColO0 = 128, kColO1 = 256;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s
@@ -94,7 +99,7 @@ constexpr uint32_t idesc(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-constexpr uint32_t kIdescQK = idesc(128, 64, false, false);
+constexpr uint32_t kIdescQK = idesc(128, 256, false, false);
 constexpr uint32_t kIdescPV = idesc(128, 256, false, true);
 
 // ---------------------------------------------------------------------------
@@ -102,7 +107,7 @@ constexpr uint32_t kIdescPV = idesc(128, 256, false, true);
 // tile g in CTA b, read back with mla_tc_trace_read.  Absent otherwise.
 // ---------------------------------------------------------------------------
 #ifdef MLA_TC_TRACE
-constexpr int kTrCtas = 8, kTrTiles = 48, kTrEvents = 8;
+constexpr int kTrCtas = 8, kTrTiles = 48, kTrEvents = 12;
 __device__ unsigned long long g_tc_trace[kTrCtas * kTrTiles * kTrEvents];
 __device__ __forceinline__ void tc_trace(int e, uint32_t g) {
   if (blockIdx.x < kTrCtas && g < kTrTiles) {
@@ -144,14 +149,14 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 
 // arrive on a barrier given by its shared::cluster address (own or peer CTA)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -249,7 +254,7 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
 // tiles [w*TT/W, (w+1)*TT/W); pieces per sequence are segments.
 // ---------------------------------------------------------------------------
 struct Segment {
-  int b, tile_lo, n_tiles, nvis;  // n_tiles: tiles with at least one visible key
+  int b, page_lo, n_pages, nvis;  // n_pages: pages with at least one visible key
 };
 
 struct SegmentWalker {
@@ -273,11 +278,11 @@ struct SegmentWalker {
     while ((long long)ts[b + 1] <= g) ++b;
     const long long end = min(g1, (long long)ts[b + 1]);
     s.b = b;
-    s.tile_lo = (int)(g - ts[b]);
-    const int tile_hi = (int)(end - ts[b]);
+    s.page_lo = (int)(g - ts[b]);
+    const int page_hi = (int)(end - ts[b]);
     s.nvis = seq_lens[b] - n_q + t + 1;
-    const int vis_tiles = (s.nvis + kPage - 1) / kPage;
-    s.n_tiles = max(0, min(tile_hi, vis_tiles) - s.tile_lo);
+    const int vis_pages = (s.nvis + kPage - 1) / kPage;
+    s.n_pages = max(0, min(page_hi, vis_pages) - s.page_lo);
     g = end;
     return true;
   }
@@ -285,10 +290,11 @@ struct SegmentWalker {
 
 struct TcParams {
   DecodeParams p;
-  CUtensorMap map_q;   // q_abs [rows = batch*n_q*128][576] bf16, box 64 x 64
-  CUtensorMap map_kq;  // pool rows [num_pages*64][576] bf16, box 64 x 32 (QK units)
-  CUtensorMap map_pv;  // pool rows, box 64 x 16 (PV unit halves)
-  CUtensorMap map_row; // pool rows, box 64 x 1 (PV rows of a partial 16-key step)
+  CUtensorMap map_q;    // q_abs [rows = batch*n_q*128][576] bf16, box 64 x 64
+  CUtensorMap map_kq;   // pool rows [num_pages*64][576] bf16, box 64 x 32 (QK unit, one page)
+  CUtensorMap map_pv;   // pool rows, box 64 x 64 (PV unit atom, one page)
+  CUtensorMap map_pv16; // pool rows, box 64 x 16 (16-key group of a partial page)
+  CUtensorMap map_row;  // pool rows, box 64 x 1 (one row of a partial 16-key group)
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
@@ -318,10 +324,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_S_FULL + i), 1);
       mbar_init(bar(B_S_FREE + i), 8);
-      mbar_init(bar(B_P_FULL + i), 8);
     }
+    mbar_init(bar(B_P_FULL), 8);
     mbar_init(bar(B_O_DONE), 1);
-    mbar_init(bar(B_O_DONE + 1), 1);
     mbar_init(bar(B_O_FREE), 8);
     mbar_init(bar(B_Q_FULL), 1);
     mbar_init(bar(B_Q_EMPTY), 1);
@@ -343,54 +348,82 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     if (lane == 0) {
       SegmentWalker walk(p, w, t);
       Segment s;
-      uint32_t U = 0, seg = 0, gtile = 0;
+      uint32_t slot = 0, phase = 0, seg = 0, gtile = 0;  // ring position
       bool ok = true;
       (void)gtile;
-      const int y_half = 32 * (int)rank;  // this CTA's half of a tile's keys (QK units)
-      const int x_pv = 128 * (int)rank;   // this CTA's half of an N=256 MMA's columns (PV units)
-      // wait for ring unit U to be free; the leader expects both CTAs' bytes
+      const int y_half = 32 * (int)rank;  // this CTA's 32 keys of each page (QK units)
+      const int x_pv = 128 * (int)rank;   // this CTA's 128 columns of an N=256 half (PV units)
+      const uint32_t empty0 = bar(B_UNIT_EMPTY), full0 = bar(B_UNIT_FULL);
+      const uint32_t leader_full0 = leader_bar(B_UNIT_FULL), ring0 = sbase + kOffRing;
+      // wait for the next ring unit to be free; the leader expects both CTAs' bytes
+#ifdef MLA_TC_TRACE
+      unsigned long long wait_ns = 0;
+#endif
       auto acquire = [&](uint32_t& dst, uint32_t& fullbar) -> bool {
-        const uint32_t u = U % kUnits;
-        if (!mbar_wait(bar(B_UNIT_EMPTY + u), ((U / kUnits) & 1) ^ 1, abort_flag, p.status)) return false;
-        if (rank == 0) mbar_expect_tx(bar(B_UNIT_FULL + u), 2 * kUnitBytes);
-        dst = sbase + kOffRing + u * kUnitBytes;
-        fullbar = leader_bar(B_UNIT_FULL + u);
-        ++U;
-        return true;
-      };
-      auto load_qk = [&](int page) -> bool {
-        for (int c = 0; c < kQKUnits; ++c) {
-          uint32_t dst, fb;
-          if (!acquire(dst, fb)) return false;
-          tma_load_2d_pair(dst, &P.map_kq, 64 * c, page * kPage + y_half, fb);
+#ifdef MLA_TC_TRACE
+        unsigned long long ta, tb;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(ta));
+#endif
+        if (!mbar_wait(empty0 + 8 * slot, phase ^ 1, abort_flag, p.status)) return false;
+#ifdef MLA_TC_TRACE
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tb));
+        wait_ns += tb - ta;
+#endif
+        if (rank == 0) mbar_expect_tx(full0 + 8 * slot, 2 * kUnitBytes);
+        dst = ring0 + slot * kUnitBytes;
+        fullbar = leader_full0 + 8 * slot;
+        if (++slot == kUnits) {
+          slot = 0;
+          phase ^= 1;
         }
         return true;
       };
-      // PV units of a tile whose first `valid` keys are visible: rows past
-      // them come from outside the tensor (zero fill)
-      auto load_pv = [&](int page, int valid) -> bool {
-        for (int j = 0; j < 2; ++j)
-          for (int ks = 0; ks < 4; ++ks) {
+      // QK units of a tile: page i's 32 keys at rows 32i..32i+31; pages past
+      // the tile's end come from outside the tensor (zero fill)
+      auto load_qk = [&](const int* pages, int npg) -> bool {
+        for (int c = 0; c < kQKUnits; ++c) {
+          uint32_t dst, fb;
+          if (!acquire(dst, fb)) return false;
+          for (int i = 0; i < kTilePages; ++i)
+            tma_load_2d_pair(dst + i * 4096, &P.map_kq, 64 * c, i < npg ? pages[i] * kPage + y_half : -32, fb);
+        }
+        return true;
+      };
+      // PV units of a tile (page i outer, N-half j inner).  Rows past the
+      // visible keys and pages past the tile's end come from outside the
+      // tensor (zero fill), so 0 * (whatever the pool held) cannot reach O.
+      auto load_pv = [&](const int* pages, int npg, int valid_last) -> bool {
+        for (int i = 0; i < kTilePages; ++i)
+          for (int j = 0; j < 2; ++j) {
             uint32_t dst, fb;
             if (!acquire(dst, fb)) return false;
             for (int a = 0; a < 2; ++a) {
               const int x = 256 * j + x_pv + 64 * a;
-              const uint32_t d = dst + a * 2048;
-              if (16 * ks + 16 <= valid) {
-                tma_load_2d_pair(d, &P.map_pv, x, page * kPage + 16 * ks, fb);
-              } else if (16 * ks >= valid) {
-                tma_load_2d_pair(d, &P.map_pv, x, -16, fb);
+              const uint32_t d = dst + a * 8192;
+              const int valid = i < npg ? (i == npg - 1 ? valid_last : kPage) : 0;
+              if (valid == kPage) {
+                tma_load_2d_pair(d, &P.map_pv, x, pages[i] * kPage, fb);
+              } else if (valid == 0) {
+                tma_load_2d_pair(d, &P.map_pv, x, -kPage, fb);
               } else {
-                for (int i = 0; i < 16; ++i)
-                  tma_load_2d_pair(d + i * 128, &P.map_row, x, 16 * ks + i < valid ? page * kPage + 16 * ks + i : -1,
-                                   fb);
+                for (int q = 0; q < 4; ++q) {
+                  if (16 * q + 16 <= valid) {
+                    tma_load_2d_pair(d + q * 2048, &P.map_pv16, x, pages[i] * kPage + 16 * q, fb);
+                  } else if (16 * q >= valid) {
+                    tma_load_2d_pair(d + q * 2048, &P.map_pv16, x, -16, fb);
+                  } else {
+                    for (int k = 0; k < 16; ++k)
+                      tma_load_2d_pair(d + (16 * q + k) * 128, &P.map_row, x,
+                                       16 * q + k < valid ? pages[i] * kPage + 16 * q + k : -1, fb);
+                  }
+                }
               }
             }
           }
         return true;
       };
-      auto page_of = [&](int b, int tile) -> int {
-        int page = p.page_table[(size_t)b * p.max_pages + tile];
+      auto page_of = [&](int b, int pg) -> int {
+        int page = p.page_table[(size_t)b * p.max_pages + pg];
         if (page < 0 || page >= p.num_pages) {
           record_status(p.status, MLA_ERR_BOUNDS);
           page = 0;
@@ -398,7 +431,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         return page;
       };
       while (ok && walk.next(s)) {
-        if (s.n_tiles == 0) continue;
+        if (s.n_pages == 0) continue;
         // absorbed queries of this CTA's 64 heads for (b, t)
         if (seg > 0) ok = mbar_wait(bar(B_Q_EMPTY), (seg - 1) & 1, abort_flag, p.status);
         if (!ok) break;
@@ -406,17 +439,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         const int qrow = ((s.b * p.n_q + t) * kHeads) + kHalfHeads * (int)rank;
         const uint32_t qbar = leader_bar(B_Q_FULL);
         for (int c = 0; c < kChunks; ++c) tma_load_2d_pair(sbase + kOffQ + c * 8192, &P.map_q, 64 * c, qrow, qbar);
-        int prev_page = 0, prev_valid = 0;
-        for (int i = 0; i < s.n_tiles && ok; ++i) {
-          const int tile = s.tile_lo + i;
-          const int page = page_of(s.b, tile);
-          TC_TRACE(0, gtile++);
-          ok = load_qk(page);
-          if (ok && i > 0) ok = load_pv(prev_page, prev_valid);
-          prev_page = page;
-          prev_valid = min(kPage, s.nvis - tile * kPage);
+        const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
+        int prev[kTilePages] = {0, 0, 0, 0}, prev_npg = 0, prev_valid = 0;
+        for (int it = 0; it < n_tiles && ok; ++it) {
+          int pages[kTilePages];
+          const int pg0 = s.page_lo + it * kTilePages;
+          const int npg = min(kTilePages, s.n_pages - it * kTilePages);
+          for (int i = 0; i < kTilePages; ++i) pages[i] = i < npg ? page_of(s.b, pg0 + i) : 0;
+          TC_TRACE(0, gtile);
+#ifdef MLA_TC_TRACE
+          wait_ns = 0;
+#endif
+          ok = load_qk(pages, npg);
+          if (ok && it > 0) ok = load_pv(prev, prev_npg, prev_valid);
+#ifdef MLA_TC_TRACE
+          if (blockIdx.x < kTrCtas && gtile < kTrTiles) {
+            g_tc_trace[(blockIdx.x * kTrTiles + gtile) * kTrEvents + 9] = wait_ns;
+            unsigned long long te;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(te));
+            g_tc_trace[(blockIdx.x * kTrTiles + gtile) * kTrEvents + 8] = te;
+          }
+#endif
+          ++gtile;
+          for (int i = 0; i < kTilePages; ++i) prev[i] = pages[i];
+          prev_npg = npg;
+          prev_valid = min(kPage, s.nvis - (pg0 + npg - 1) * kPage);
         }
-        if (ok) ok = load_pv(prev_page, prev_valid);
+        if (ok) ok = load_pv(prev, prev_npg, prev_valid);
         ++seg;
       }
     }
@@ -425,64 +474,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     if (rank == 0 && lane == 0) {
       SegmentWalker walk(p, w, t);
       Segment s;
-      uint32_t U = 0, g = 0, seg = 0;
+      uint32_t slot = 0, phase = 0, g = 0, seg = 0;  // ring position, tile counter
       bool ok = true;
-      auto unit_ready = [&](uint32_t& addr) -> bool {
-        const uint32_t u = U % kUnits;
-        if (!mbar_wait(bar(B_UNIT_FULL + u), (U / kUnits) & 1, abort_flag, p.status)) return false;
-        tc_fence_after();
-        addr = sbase + kOffRing + u * kUnitBytes;
-        return true;
-      };
-      auto unit_done = [&]() {
-        tc_commit_pair(bar(B_UNIT_EMPTY + (U % kUnits)));
-        ++U;
+      const uint32_t full0 = bar(B_UNIT_FULL), empty0 = bar(B_UNIT_EMPTY);
+      // descriptors advance by adding (byte offset >> 4) to the start-address field
+      const uint64_t qdesc = sdesc(sbase + kOffQ, 16, 1024);       // chunk c: + 512 c; K-step: + 2
+      const uint64_t kdesc = sdesc(sbase + kOffRing, 16, 1024);    // unit: + 1024 slot
+      const uint64_t vdesc = sdesc(sbase + kOffRing, 8192, 1024);  // unit: + 1024 slot; K-step: + 128
+      const uint64_t pdesc = sdesc(sbase + kOffP, 16, 1024);       // page sub-tile: + 512 i; K-step: + 2
+      auto release_unit = [&]() {
+        tc_commit_pair(empty0 + 8 * slot);
+        if (++slot == kUnits) {
+          slot = 0;
+          phase ^= 1;
+        }
       };
       auto do_pv = [&](uint32_t gi, bool first) -> bool {
-        if (!mbar_wait(bar(B_P_FULL + (gi & 1)), (gi >> 1) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(bar(B_P_FULL), gi & 1, abort_flag, p.status)) return false;
         TC_TRACE(2, gi);
         tc_fence_after();
-        const uint32_t pa = sbase + kOffP + (gi & 1) * kPBytes;
-        for (int j = 0; j < 2; ++j)
-          for (int ks = 0; ks < 4; ++ks) {
-            uint32_t unit;
-            if (!unit_ready(unit)) return false;
-            tc_mma(tmem + (j ? kColO1 : kColO0), sdesc(pa + ks * 32, 16, 1024), sdesc(unit, 2048, 1024), kIdescPV,
-                   (first && ks == 0) ? 0u : 1u);
-            unit_done();
+#pragma unroll 1
+        for (int i = 0; i < kTilePages; ++i)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (!mbar_wait(full0 + 8 * slot, phase, abort_flag, p.status)) return false;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              tc_mma(tmem + (j ? kColO1 : kColO0), pdesc + 512 * i + 2 * ks, vdesc + 1024 * slot + 128 * ks, kIdescPV,
+                     (first && i == 0 && ks == 0) ? 0u : 1u);
+            release_unit();
           }
-        tc_commit_pair(bar(B_O_DONE + (gi & 1)));
+        tc_commit_pair(bar(B_O_DONE));
         TC_TRACE(3, gi);
         return true;
       };
       while (ok && walk.next(s)) {
-        if (s.n_tiles == 0) continue;
+        if (s.n_pages == 0) continue;
         ok = mbar_wait(bar(B_Q_FULL), seg & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         const uint32_t g_first = g;
-        for (int i = 0; i < s.n_tiles && ok; ++i, ++g) {
+        const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
+        for (int it = 0; it < n_tiles && ok; ++it, ++g) {
           ok = mbar_wait(bar(B_S_FREE + (g & 1)), ((g >> 1) & 1) ^ 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
           const uint32_t sd = tmem + ((g & 1) ? kColS1 : kColS0);
           TC_TRACE(7, g);
-          for (int c = 0; c < kQKUnits && ok; ++c) {
-            uint32_t unit;
-            ok = unit_ready(unit);
+#pragma unroll 1
+          for (int c = 0; c < kQKUnits; ++c) {
+            ok = mbar_wait(full0 + 8 * slot, phase, abort_flag, p.status);
             if (!ok) break;
+            const uint64_t a = qdesc + 512 * c, bb = kdesc + 1024 * slot;
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)  // 16 columns = 32 bytes into the swizzled rows
-              tc_mma(sd, sdesc(sbase + kOffQ + c * 8192 + k4 * 32, 16, 1024), sdesc(unit + k4 * 32, 16, 1024),
-                     kIdescQK, (c | k4) ? 1u : 0u);
-            unit_done();
+              tc_mma(sd, a + 2 * k4, bb + 2 * k4, kIdescQK, (c | k4) ? 1u : 0u);
+            release_unit();
           }
           if (!ok) break;
           tc_commit_pair(bar(B_S_FULL + (g & 1)));
           TC_TRACE(1, g);
-          if (i == s.n_tiles - 1) tc_commit_pair(bar(B_Q_EMPTY));
-          if (i > 0) {
-            if (i == 1 && seg > 0) {  // O of the previous segment must be read out first
+          if (it == n_tiles - 1) tc_commit_pair(bar(B_Q_EMPTY));
+          if (it > 0) {
+            if (it == 1 && seg > 0) {  // O of the previous segment must be read out first
               ok = mbar_wait(bar(B_O_FREE), (seg - 1) & 1, abort_flag, p.status);
               if (!ok) break;
             }
@@ -490,7 +544,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           }
         }
         if (!ok) break;
-        if (s.n_tiles == 1 && seg > 0) {
+        if (n_tiles == 1 && seg > 0) {
           ok = mbar_wait(bar(B_O_FREE), (seg - 1) & 1, abort_flag, p.status);
           if (!ok) break;
         }
@@ -500,7 +554,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------- softmax, epilogue
-    const int L = warp * 32 + lane;  // TMEM lane of this thread
+    // Thread L (TMEM lane) holds head hl of this CTA; lanes 0-63 see keys
+    // 0-31 of each page of a tile, lanes 64-127 keys 32-63 (2x2 layout).
+    const int L = warp * 32 + lane;
     const int hl = L & 63, half = L >> 6;
     const int head = kHalfHeads * (int)rank + hl;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -511,7 +567,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     while (walk.next(s)) {
       const size_t slot = (size_t)t * p.n_slots + (w + s.b);
       float* od = p.o_part + (slot * kHeads + head) * kDC;
-      if (s.n_tiles == 0 || !ok) {
+      if (s.n_pages == 0 || !ok) {
         for (int j = 0; j < 2; ++j)
           for (int c = 0; c < 128; c += 4)
             *reinterpret_cast<float4*>(od + 256 * j + 128 * half + c) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -519,26 +575,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         continue;
       }
       float m_ref = -INFINITY, l_part = 0.f;
-      for (int i = 0; i < s.n_tiles; ++i, ++g) {
+      const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
+      for (int it = 0; it < n_tiles; ++it, ++g) {
         ok = mbar_wait(bar(B_S_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.status);
         __syncwarp();
         if (!ok) break;
         if (threadIdx.x == 0) TC_TRACE(4, g);
         tc_fence_after();
-        uint32_t sr[32];
-        tmem_ld32(tmem + lane_base + ((g & 1) ? kColS1 : kColS0), sr);
-        tmem_wait_ld();
-        if (threadIdx.x == 0) TC_TRACE(5, g);
+        float sv[4 * 32];
+        {
+          uint32_t sr[32];
+#pragma unroll
+          for (int q = 0; q < kTilePages; ++q) {
+            tmem_ld32(tmem + lane_base + ((g & 1) ? kColS1 : kColS0) + 32 * q, sr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sv[32 * q + j] = __uint_as_float(sr[j]);
+          }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_bar(B_S_FREE + (g & 1)));
-        const int key0 = (s.tile_lo + i) * kPage + 32 * half;
-        float sv[32];
+        if (threadIdx.x == 0) TC_TRACE(5, g);
+        // keys of this thread: page q of the tile, in-page 32*half + j
+        const int pg0 = s.page_lo + it * kTilePages;
         float mx = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          sv[j] = key0 + j < s.nvis ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
-          mx = fmaxf(mx, sv[j]);
+        for (int q = 0; q < kTilePages; ++q) {
+          const int key0 = (pg0 + q) * kPage + 32 * half;
+          const bool page_ok = pg0 + q < s.page_lo + s.n_pages;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float v = (page_ok && key0 + j < s.nvis) ? sv[32 * q + j] * p.scale_log2 : -INFINITY;
+            sv[32 * q + j] = v;
+            mx = fmaxf(mx, v);
+          }
         }
         red_max[half * 64 + hl] = mx;
         asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -546,40 +617,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         asm volatile("bar.sync 1, 128;" ::: "memory");
         bool rescale = false;
         float alpha = 1.f;
-        if (i == 0) {
+        if (it == 0) {
           m_ref = tile_max;
         } else if (tile_max > m_ref + kRescaleThreshold) {
           rescale = true;
           alpha = fast_exp2(m_ref - tile_max);
           m_ref = tile_max;
         }
-        uint32_t pk[16];
+        uint32_t pk[64];
         float psum = 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(fast_exp2(sv[2 * j] - m_ref), fast_exp2(sv[2 * j + 1] - m_ref));
+        for (int j = 0; j < 64; ++j) {
+          const __nv_bfloat162 h2 =
+              __floats2bfloat162_rn(fast_exp2(sv[2 * j] - m_ref), fast_exp2(sv[2 * j + 1] - m_ref));
           const float2 f2 = __bfloat1622float2(h2);
           psum += f2.x + f2.y;
           pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
         }
         l_part = l_part * alpha + psum;
-        // P buffer g&1 was last read by PV(g-2)
-        if (g >= 2) {
-          ok = mbar_wait(bar(B_O_DONE + (g & 1)), ((g - 2) >> 1) & 1, abort_flag, p.status);
-          __syncwarp();
-          if (!ok) break;
-        }
-        // tcgen05.ld/st are whole-warp instructions: rescale the warp's lanes
-        // together (alpha = 1 on lanes whose head keeps its reference max),
-        // after PV(g-1), the last MMA writing O, has finished
-        const bool warp_rescale = __any_sync(0xffffffffu, rescale);
-        if (warp_rescale) {
-          ok = mbar_wait(bar(B_O_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, p.status);
+        if (threadIdx.x == 0) TC_TRACE(10, g);
+        // the previous tile's PV MMAs read P and write O: wait for them
+        if (g >= 1) {
+          ok = mbar_wait(bar(B_O_DONE), (g - 1) & 1, abort_flag, p.status);
           __syncwarp();
           if (!ok) break;
           tc_fence_after();
         }
-        if (warp_rescale) {
+        // tcgen05.ld/st are whole-warp instructions: rescale the warp's lanes
+        // together (alpha = 1 on lanes whose head keeps its reference max)
+        if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
             const uint32_t col = (c < 128 ? kColO0 + c : kColO1 + (c - 128));
@@ -592,22 +658,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           }
           tmem_wait_st();
         }
-        // P row hl, keys [32*half, 32*half+32): four 16-byte units, 128-byte swizzle
-        uint8_t* prow = smem + kOffP + (g & 1) * kPBytes + hl * 128;
+        // P row hl: page q is sub-tile q (64 keys, 128 B per row, 128-byte
+        // swizzle); this thread's 32 keys are 16-byte units 4*half .. 4*half+3
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = (4 * half + u) ^ (hl & 7);
-          *reinterpret_cast<uint4*>(prow + unit * 16) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        for (int q = 0; q < kTilePages; ++q) {
+          uint8_t* prow = smem + kOffP + q * 8192 + hl * 128;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int unit = (4 * half + u) ^ (hl & 7);
+            *reinterpret_cast<uint4*>(prow + unit * 16) =
+                make_uint4(pk[16 * q + 4 * u], pk[16 * q + 4 * u + 1], pk[16 * q + 4 * u + 2], pk[16 * q + 4 * u + 3]);
+          }
         }
+        if (threadIdx.x == 0) TC_TRACE(11, g);
         fence_proxy_async();
         tc_fence_before();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (threadIdx.x == 0) TC_TRACE(6, g);
-        if (lane == 0) mbar_arrive_cluster(leader_bar(B_P_FULL + (g & 1)));
+        if (lane == 0) mbar_arrive_cluster(leader_bar(B_P_FULL));
       }
       if (!ok) break;
       // epilogue: wait for the last PV, normalise, write the split's partial
-      ok = mbar_wait(bar(B_O_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, p.status);
+      ok = mbar_wait(bar(B_O_DONE), (g - 1) & 1, abort_flag, p.status);
       __syncwarp();
       if (!ok) break;
       tc_fence_after();
@@ -704,8 +776,8 @@ cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st) {
   tp.p = p;
   const uint64_t pool_rows = (uint64_t)p.num_pages * kPage;
   if (!make_map(&tp.map_q, p.q_abs, (uint64_t)p.batch * p.n_q * kHeads, 64) ||
-      !make_map(&tp.map_kq, p.pool, pool_rows, 32) || !make_map(&tp.map_pv, p.pool, pool_rows, 16) ||
-      !make_map(&tp.map_row, p.pool, pool_rows, 1))
+      !make_map(&tp.map_kq, p.pool, pool_rows, 32) || !make_map(&tp.map_pv, p.pool, pool_rows, 64) ||
+      !make_map(&tp.map_pv16, p.pool, pool_rows, 16) || !make_map(&tp.map_row, p.pool, pool_rows, 1))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
