@@ -14,22 +14,25 @@
 //    the M dimension of cta_group::2 tcgen05 MMAs: each CTA holds the absorbed
 //    queries of 64 heads (72 KB of shared memory); the pair's tensor cores
 //    exchange the B operand halves, so every CTA sees all keys of a tile.
-//  * Per 64-key tile (one page):
-//      QK : S[64 heads x 64 keys] = Q[64 x 576] . K^T   (M=128 pair, N=64, K=576)
-//      PV : O[64 heads x 512]    += P[64 x 64] . C[64 x 512]  (two N=256 MMAs)
-//    S (2 buffers) and O live in tensor memory (TMEM); per CTA S uses 2 x 32
-//    columns and O 2 x 128 columns of the 2-SM ("2x2") accumulator layout:
-//    row m, column n < N/2 -> lane m, column n; n >= N/2 -> lane 64+m, n-N/2.
-//  * Operands stream through a ring of 4 KB units (TMA, 128-byte swizzle) in
-//    the order the MMAs consume them: the 9 QK units of tile g (this CTA's
-//    32-key half of the rows x 64 columns each, K-major), then the 8 PV units
-//    of tile g-1 (16 keys x this CTA's 128 latent columns of one N=256 MMA,
-//    MN-major).  Each unit has its own full/empty barrier, so loads run about
-//    two tiles ahead of the MMAs.  Rows past a sequence's end in its last page
-//    are loaded from outside the tensor (TMA zero fill), never from the pool,
-//    so 0 * (whatever the pool held) cannot reach O.
+//  * Per 256-key tile (four pages):
+//      QK : S[128 heads x 256 keys] = Q[128 x 576] . K^T   (M=128 pair, N=256, K=576)
+//      PV : O[128 heads x 512]     += P[128 x 256] . C[256 x 512]  (two N=256 MMAs)
+//    The leader CTA supplies pages 0-1 of the tile as its half of the QK B
+//    operand, the peer pages 2-3.  S (2 buffers) and O live in tensor memory
+//    (TMEM), 2x2 layout: row m, column n < N/2 -> lane m, column n;
+//    n >= N/2 -> lane 64+m, column n-N/2.
+//  * Operands stream through a ring of 16 KB units (TMA, 128-byte swizzle) in
+//    the order the MMAs consume them: the 9 QK units of tile g (this CTA's two
+//    pages x 64 columns each, K-major), then the 8 PV units of tile g-1 (one
+//    page x this CTA's 128 latent columns of one N=256 MMA, MN-major).  Each
+//    unit has its own full/empty barrier.  Rows past a sequence's end in its
+//    last page are loaded from outside the tensor (TMA zero fill), never from
+//    the pool, so 0 * (whatever the pool held) cannot reach O.
+//  * Three producer warps take the units in turn: one thread's TMA issue rate
+//    is bounded by its own barrier wait/arm cycle, and several issuing warps
+//    keep enough loads in flight to stream at the HBM rate.
 //  * Warp roles: warps 0-3 softmax + epilogue (one TMEM lane each), warp 4
-//    TMA producer, warp 5 TMEM allocation and (leader CTA) MMA issue.
+//    TMEM allocation and (leader CTA) MMA issue, warps 5-7 TMA producers.
 //  * Online softmax in base 2 with a lazily updated reference max: O is only
 //    rescaled when a tile's max exceeds the reference by more than 8 (in
 //    log2 units), so probabilities stay <= 2^8 and rescaling is rare.
@@ -52,44 +55,59 @@ constexpr int kPage = 64;                             // keys per cache page
 constexpr int kTilePages = 4;                         // pages per tile: 256 keys = N of the QK MMA
 constexpr int kChunks = kD / 64;                      // 9 column chunks of 64 (128 B)
 
-// Ring units: 16 KB each, this CTA's share of one MMA group
-//   QK unit c : its 128 keys of the tile (32 per page) x columns [64c, 64c+64), K-major
+// Operand units: 16 KB each, this CTA's share of one group of four MMAs
+//   QK unit c : its two pages of the tile (128 keys) x columns [64c, 64c+64), K-major
 //   PV unit   : one page's 64 keys x its 128 latent columns of one N=256 half, MN-major
+// QK and PV units stream through rings of their own, each consumed by its own
+// MMA-issuing thread: an MMA issue returns only once the tensor pipe takes
+// it, so one issuer's barrier waits and commits are covered by the other's
+// MMAs.
 constexpr uint32_t kUnitBytes = 16384;
-constexpr int kUnits = 7;
-constexpr int kQKUnits = kChunks;                     // 9 per tile
-constexpr int kPVUnits = 2 * kTilePages;              // 8 per tile
+constexpr int kQKSlots = 3, kPVSlots = 4;
+constexpr int kQKUnits = kChunks;         // 9 per tile
 
 // shared memory layout (offsets from a 1024-byte aligned base)
 constexpr uint32_t kQBytes = kChunks * 64 * 128;      // 73728: 64 heads x 576 bf16
 constexpr uint32_t kPBytes = kTilePages * 64 * 128;   // 32768: 64 heads x 256 keys bf16, 4 sub-tiles
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffP = kOffQ + kQBytes;
-constexpr uint32_t kOffRing = kOffP + kPBytes;                // 106496
-constexpr uint32_t kOffBar = kOffRing + kUnits * kUnitBytes;  // 221184
-constexpr uint32_t kNumBars = 2 * kUnits + 10;
+constexpr uint32_t kOffQKRing = kOffP + kPBytes;                   // 106496
+constexpr uint32_t kOffPVRing = kOffQKRing + kQKSlots * kUnitBytes;
+constexpr uint32_t kOffBar = kOffPVRing + kPVSlots * kUnitBytes;
+constexpr uint32_t kNumBars = 2 * kQKSlots + 2 * kPVSlots + 9;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kOffRedMax = kOffMisc + 16;                 // float [2][64]
-constexpr uint32_t kOffRedL = kOffRedMax + 512;                // float [2][64]
+constexpr uint32_t kOffRedMax = kOffMisc + 16;                     // float [2][64]
+constexpr uint32_t kOffRedL = kOffRedMax + 512;                    // float [2][64]
 constexpr uint32_t kSmemUsed = kOffRedL + 512;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;              // + alignment slack
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;                  // + alignment slack
 
 // barrier indices
 enum {
-  B_UNIT_FULL = 0,          // [kUnits] leader: TMA bytes of both CTAs
-  B_UNIT_EMPTY = kUnits,    // [kUnits] each CTA: unit consumed (MMA commit)
-  B_S_FULL = 2 * kUnits,    // [2] each CTA: S tile ready (MMA commit)
-  B_S_FREE = B_S_FULL + 2,  // [2] leader: S read by both CTAs' softmax warps (8 arrivals)
-  B_P_FULL = B_S_FREE + 2,  // leader: P written + O rescaled by both CTAs (8 arrivals)
-  B_O_DONE,                 // each CTA: the tile's PV MMAs finished (MMA commit)
-  B_O_FREE,                 // leader: O read out by both CTAs' epilogues (8 arrivals)
-  B_Q_FULL,                 // leader: Q bytes of both CTAs
-  B_Q_EMPTY,                // each CTA: last QK of a segment finished (MMA commit)
+  B_QK_FULL = 0,                        // [kQKSlots] leader: TMA bytes of both CTAs
+  B_QK_EMPTY = kQKSlots,                // [kQKSlots] each CTA: unit consumed (MMA commit)
+  B_PV_FULL = 2 * kQKSlots,             // [kPVSlots] leader: TMA bytes of both CTAs
+  B_PV_EMPTY = B_PV_FULL + kPVSlots,    // [kPVSlots] each CTA: unit consumed (MMA commit)
+  B_S_FULL = B_PV_EMPTY + kPVSlots,     // [2] each CTA: S tile ready (MMA commit)
+  B_S_FREE = B_S_FULL + 2,              // [2] leader: S read by both CTAs' softmax warps (8 arrivals)
+  B_P_FULL = B_S_FREE + 2,              // leader: P written + O rescaled by both CTAs (8 arrivals)
+  B_O_DONE,                             // each CTA: the tile's PV MMAs finished (MMA commit)
+  B_O_FREE,                             // leader: O read out by both CTAs' epilogues (8 arrivals)
+  B_Q_FULL,                             // leader: Q bytes of both CTAs
+  B_Q_EMPTY,                            // each CTA: last QK of a segment finished (MMA commit)
+  B_COUNT
 };
+static_assert(B_COUNT == (int)kNumBars, "barrier count");
 
 // TMEM columns (per CTA, 2x2 layout): S buffers 128 columns each, O 2 x 128
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
+
+// warp roles
+constexpr int kQKWarp = 4;                         // TMEM allocation; leader lane 0 issues the QK MMAs
+constexpr int kPVWarp = 5;                         // leader lane 0 issues the PV MMAs
+constexpr int kQKProdWarp = 6, kQKProducers = 2;   // load Q and the QK units
+constexpr int kPVProdWarp = 8, kPVProducers = 2;   // load the PV units
+constexpr int kThreads = 32 * (kPVProdWarp + kPVProducers);  // 320
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s
@@ -107,7 +125,7 @@ constexpr uint32_t kIdescPV = idesc(128, 256, false, true);
 // tile g in CTA b, read back with mla_tc_trace_read.  Absent otherwise.
 // ---------------------------------------------------------------------------
 #ifdef MLA_TC_TRACE
-constexpr int kTrCtas = 8, kTrTiles = 48, kTrEvents = 12;
+constexpr int kTrCtas = 8, kTrTiles = 48, kTrEvents = 16;
 __device__ unsigned long long g_tc_trace[kTrCtas * kTrTiles * kTrEvents];
 __device__ __forceinline__ void tc_trace(int e, uint32_t g) {
   if (blockIdx.x < kTrCtas && g < kTrTiles) {
@@ -117,6 +135,11 @@ __device__ __forceinline__ void tc_trace(int e, uint32_t g) {
   }
 }
 #define TC_TRACE(e, g) tc_trace((e), (g))
+__device__ __forceinline__ unsigned long long tc_now() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 #else
 #define TC_TRACE(e, g) ((void)0)
 #endif
@@ -291,13 +314,60 @@ struct SegmentWalker {
 struct TcParams {
   DecodeParams p;
   CUtensorMap map_q;    // q_abs [rows = batch*n_q*128][576] bf16, box 64 x 64
-  CUtensorMap map_kq;   // pool rows [num_pages*64][576] bf16, box 64 x 32 (QK unit, one page)
-  CUtensorMap map_pv;   // pool rows, box 64 x 64 (PV unit atom, one page)
+  CUtensorMap map_pv;   // pool rows, box 64 x 64 (one page x 64 columns: QK and PV boxes)
   CUtensorMap map_pv16; // pool rows, box 64 x 16 (16-key group of a partial page)
   CUtensorMap map_row;  // pool rows, box 64 x 1 (one row of a partial 16-key group)
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+// Producer side of one operand ring: producer pid of n issues every n-th unit
+// of the ring's consumption order; every producer walks the same schedule, so
+// the ring position of each unit is known to all of them.
+struct RingProducer {
+  uint32_t full0, empty0, leader_full0, ring0;
+  int slots, producers, pid;
+  uint32_t slot = 0, phase = 0, unit = 0;
+  // Claim the next unit.  Returns true when this producer issues it, after the
+  // slot is free and (leader) the barrier expects both CTAs' bytes.
+  __device__ bool claim(uint32_t rank, uint32_t& dst, uint32_t& fullbar, bool& ok, volatile int* abort_flag,
+                        int* status) {
+    const bool mine = (int)(unit % (uint32_t)producers) == pid;
+    const uint32_t my_slot = slot, my_phase = phase;
+    ++unit;
+    if (++slot == (uint32_t)slots) {
+      slot = 0;
+      phase ^= 1;
+    }
+    if (!mine || !ok) return false;
+    if (!mbar_wait(empty0 + 8 * my_slot, my_phase ^ 1, abort_flag, status)) {
+      ok = false;
+      return false;
+    }
+    if (rank == 0) mbar_expect_tx(full0 + 8 * my_slot, 2 * kUnitBytes);
+    dst = ring0 + my_slot * kUnitBytes;
+    fullbar = leader_full0 + 8 * my_slot;
+    return true;
+  }
+};
+
+// Consumer side of one operand ring (the MMA-issuing thread of the leader).
+struct RingConsumer {
+  uint32_t full0, empty0, ring0;
+  int slots;
+  uint32_t slot = 0, phase = 0;
+  __device__ bool wait_full(volatile int* abort_flag, int* status) {
+    return mbar_wait(full0 + 8 * slot, phase, abort_flag, status);
+  }
+  // the unit's MMAs are issued: free the slot in both CTAs once they complete
+  __device__ void release() {
+    tc_commit_pair(empty0 + 8 * slot);
+    if (++slot == (uint32_t)slots) {
+      slot = 0;
+      phase ^= 1;
+    }
+  }
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -317,9 +387,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    for (int i = 0; i < kUnits; ++i) {
-      mbar_init(bar(B_UNIT_FULL + i), 1);
-      mbar_init(bar(B_UNIT_EMPTY + i), 1);
+    for (int i = 0; i < kQKSlots; ++i) {
+      mbar_init(bar(B_QK_FULL + i), 1);
+      mbar_init(bar(B_QK_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kPVSlots; ++i) {
+      mbar_init(bar(B_PV_FULL + i), 1);
+      mbar_init(bar(B_PV_EMPTY + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_S_FULL + i), 1);
@@ -332,7 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     mbar_init(bar(B_Q_EMPTY), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 5) {
+  if (warp == kQKWarp) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols)
                  : "memory");
@@ -343,177 +417,120 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------------ TMA
+  auto page_of = [&](int b, int pg) -> int {
+    int page = p.page_table[(size_t)b * p.max_pages + pg];
+    if (page < 0 || page >= p.num_pages) {
+      record_status(p.status, MLA_ERR_BOUNDS);
+      page = 0;
+    }
+    return page;
+  };
+
+  if (warp >= kQKProdWarp && warp < kQKProdWarp + kQKProducers) {
+    // -------------------------------------------------------------- TMA: Q, QK
     if (lane == 0) {
+      RingProducer ring{bar(B_QK_FULL), bar(B_QK_EMPTY), leader_bar(B_QK_FULL), sbase + kOffQKRing, kQKSlots,
+                        kQKProducers, warp - kQKProdWarp};
+      const bool q_loader = ring.pid == 0;
+      const int y_pages = 2 * (int)rank;  // this CTA's two pages of a tile
       SegmentWalker walk(p, w, t);
       Segment s;
-      uint32_t slot = 0, phase = 0, seg = 0, gtile = 0;  // ring position
+      uint32_t seg = 0;
       bool ok = true;
-      (void)gtile;
-      const int y_half = 32 * (int)rank;  // this CTA's 32 keys of each page (QK units)
-      const int x_pv = 128 * (int)rank;   // this CTA's 128 columns of an N=256 half (PV units)
-      const uint32_t empty0 = bar(B_UNIT_EMPTY), full0 = bar(B_UNIT_FULL);
-      const uint32_t leader_full0 = leader_bar(B_UNIT_FULL), ring0 = sbase + kOffRing;
-      // wait for the next ring unit to be free; the leader expects both CTAs' bytes
-#ifdef MLA_TC_TRACE
-      unsigned long long wait_ns = 0;
-#endif
-      auto acquire = [&](uint32_t& dst, uint32_t& fullbar) -> bool {
-#ifdef MLA_TC_TRACE
-        unsigned long long ta, tb;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(ta));
-#endif
-        if (!mbar_wait(empty0 + 8 * slot, phase ^ 1, abort_flag, p.status)) return false;
-#ifdef MLA_TC_TRACE
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tb));
-        wait_ns += tb - ta;
-#endif
-        if (rank == 0) mbar_expect_tx(full0 + 8 * slot, 2 * kUnitBytes);
-        dst = ring0 + slot * kUnitBytes;
-        fullbar = leader_full0 + 8 * slot;
-        if (++slot == kUnits) {
-          slot = 0;
-          phase ^= 1;
+      while (ok && walk.next(s)) {
+        if (s.n_pages == 0) continue;
+        // absorbed queries of this CTA's 64 heads for (b, t)
+        if (q_loader) {
+          if (seg > 0) ok = mbar_wait(bar(B_Q_EMPTY), (seg - 1) & 1, abort_flag, p.status);
+          if (!ok) break;
+          if (rank == 0) mbar_expect_tx(bar(B_Q_FULL), 2 * kQBytes);
+          const int qrow = ((s.b * p.n_q + t) * kHeads) + kHalfHeads * (int)rank;
+          const uint32_t qbar = leader_bar(B_Q_FULL);
+          for (int c = 0; c < kChunks; ++c) tma_load_2d_pair(sbase + kOffQ + c * 8192, &P.map_q, 64 * c, qrow, qbar);
         }
-        return true;
-      };
-      // QK units of a tile: page i's 32 keys at rows 32i..32i+31; pages past
-      // the tile's end come from outside the tensor (zero fill)
-      auto load_qk = [&](const int* pages, int npg) -> bool {
-        for (int c = 0; c < kQKUnits; ++c) {
-          uint32_t dst, fb;
-          if (!acquire(dst, fb)) return false;
-          for (int i = 0; i < kTilePages; ++i)
-            tma_load_2d_pair(dst + i * 4096, &P.map_kq, 64 * c, i < npg ? pages[i] * kPage + y_half : -32, fb);
-        }
-        return true;
-      };
-      // PV units of a tile (page i outer, N-half j inner).  Rows past the
-      // visible keys and pages past the tile's end come from outside the
-      // tensor (zero fill), so 0 * (whatever the pool held) cannot reach O.
-      auto load_pv = [&](const int* pages, int npg, int valid_last) -> bool {
-        for (int i = 0; i < kTilePages; ++i)
-          for (int j = 0; j < 2; ++j) {
+        const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
+        for (int it = 0; it < n_tiles && ok; ++it) {
+          const int pg0 = s.page_lo + it * kTilePages;
+          const int npg = min(kTilePages, s.n_pages - it * kTilePages);
+          // rows of this CTA's pages; pages past the tile's end come from
+          // outside the tensor (zero fill)
+          int y[2];
+          for (int i = 0; i < 2; ++i) y[i] = y_pages + i < npg ? page_of(s.b, pg0 + y_pages + i) * kPage : -kPage;
+          for (int c = 0; c < kQKUnits; ++c) {
             uint32_t dst, fb;
-            if (!acquire(dst, fb)) return false;
-            for (int a = 0; a < 2; ++a) {
-              const int x = 256 * j + x_pv + 64 * a;
-              const uint32_t d = dst + a * 8192;
-              const int valid = i < npg ? (i == npg - 1 ? valid_last : kPage) : 0;
-              if (valid == kPage) {
-                tma_load_2d_pair(d, &P.map_pv, x, pages[i] * kPage, fb);
-              } else if (valid == 0) {
-                tma_load_2d_pair(d, &P.map_pv, x, -kPage, fb);
-              } else {
-                for (int q = 0; q < 4; ++q) {
-                  if (16 * q + 16 <= valid) {
-                    tma_load_2d_pair(d + q * 2048, &P.map_pv16, x, pages[i] * kPage + 16 * q, fb);
-                  } else if (16 * q >= valid) {
-                    tma_load_2d_pair(d + q * 2048, &P.map_pv16, x, -16, fb);
-                  } else {
-                    for (int k = 0; k < 16; ++k)
-                      tma_load_2d_pair(d + (16 * q + k) * 128, &P.map_row, x,
-                                       16 * q + k < valid ? pages[i] * kPage + 16 * q + k : -1, fb);
+            if (!ring.claim(rank, dst, fb, ok, abort_flag, p.status)) continue;
+            for (int i = 0; i < 2; ++i) tma_load_2d_pair(dst + i * 8192, &P.map_pv, 64 * c, y[i], fb);
+          }
+        }
+        ++seg;
+      }
+    }
+  } else if (warp >= kPVProdWarp) {
+    // ------------------------------------------------------------------ TMA: PV
+    if (lane == 0) {
+      RingProducer ring{bar(B_PV_FULL), bar(B_PV_EMPTY), leader_bar(B_PV_FULL), sbase + kOffPVRing, kPVSlots,
+                        kPVProducers, warp - kPVProdWarp};
+      const int x_pv = 128 * (int)rank;  // this CTA's 128 columns of an N=256 half
+      SegmentWalker walk(p, w, t);
+      Segment s;
+      bool ok = true;
+      while (ok && walk.next(s)) {
+        if (s.n_pages == 0) continue;
+        const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
+        for (int it = 0; it < n_tiles && ok; ++it) {
+          const int pg0 = s.page_lo + it * kTilePages;
+          const int npg = min(kTilePages, s.n_pages - it * kTilePages);
+          // page i outer, N-half j inner.  Rows past the visible keys and
+          // pages past the tile's end come from outside the tensor (zero
+          // fill), so 0 * (whatever the pool held) cannot reach O.
+          for (int i = 0; i < kTilePages; ++i) {
+            const int valid = i < npg ? min(kPage, s.nvis - (pg0 + i) * kPage) : 0;
+            const int page = valid > 0 ? page_of(s.b, pg0 + i) : 0;
+            for (int j = 0; j < 2; ++j) {
+              uint32_t dst, fb;
+              if (!ring.claim(rank, dst, fb, ok, abort_flag, p.status)) continue;
+              for (int a = 0; a < 2; ++a) {
+                const int x = 256 * j + x_pv + 64 * a;
+                const uint32_t d = dst + a * 8192;
+                if (valid == kPage) {
+                  tma_load_2d_pair(d, &P.map_pv, x, page * kPage, fb);
+                } else if (valid <= 0) {
+                  tma_load_2d_pair(d, &P.map_pv, x, -kPage, fb);
+                } else {
+                  for (int q = 0; q < 4; ++q) {
+                    if (16 * q + 16 <= valid) {
+                      tma_load_2d_pair(d + q * 2048, &P.map_pv16, x, page * kPage + 16 * q, fb);
+                    } else if (16 * q >= valid) {
+                      tma_load_2d_pair(d + q * 2048, &P.map_pv16, x, -16, fb);
+                    } else {
+                      for (int k = 0; k < 16; ++k)
+                        tma_load_2d_pair(d + (16 * q + k) * 128, &P.map_row, x,
+                                         16 * q + k < valid ? page * kPage + 16 * q + k : -1, fb);
+                    }
                   }
                 }
               }
             }
           }
-        return true;
-      };
-      auto page_of = [&](int b, int pg) -> int {
-        int page = p.page_table[(size_t)b * p.max_pages + pg];
-        if (page < 0 || page >= p.num_pages) {
-          record_status(p.status, MLA_ERR_BOUNDS);
-          page = 0;
         }
-        return page;
-      };
-      while (ok && walk.next(s)) {
-        if (s.n_pages == 0) continue;
-        // absorbed queries of this CTA's 64 heads for (b, t)
-        if (seg > 0) ok = mbar_wait(bar(B_Q_EMPTY), (seg - 1) & 1, abort_flag, p.status);
-        if (!ok) break;
-        if (rank == 0) mbar_expect_tx(bar(B_Q_FULL), 2 * kQBytes);
-        const int qrow = ((s.b * p.n_q + t) * kHeads) + kHalfHeads * (int)rank;
-        const uint32_t qbar = leader_bar(B_Q_FULL);
-        for (int c = 0; c < kChunks; ++c) tma_load_2d_pair(sbase + kOffQ + c * 8192, &P.map_q, 64 * c, qrow, qbar);
-        const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
-        int prev[kTilePages] = {0, 0, 0, 0}, prev_npg = 0, prev_valid = 0;
-        for (int it = 0; it < n_tiles && ok; ++it) {
-          int pages[kTilePages];
-          const int pg0 = s.page_lo + it * kTilePages;
-          const int npg = min(kTilePages, s.n_pages - it * kTilePages);
-          for (int i = 0; i < kTilePages; ++i) pages[i] = i < npg ? page_of(s.b, pg0 + i) : 0;
-          TC_TRACE(0, gtile);
-#ifdef MLA_TC_TRACE
-          wait_ns = 0;
-#endif
-          ok = load_qk(pages, npg);
-          if (ok && it > 0) ok = load_pv(prev, prev_npg, prev_valid);
-#ifdef MLA_TC_TRACE
-          if (blockIdx.x < kTrCtas && gtile < kTrTiles) {
-            g_tc_trace[(blockIdx.x * kTrTiles + gtile) * kTrEvents + 9] = wait_ns;
-            unsigned long long te;
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(te));
-            g_tc_trace[(blockIdx.x * kTrTiles + gtile) * kTrEvents + 8] = te;
-          }
-#endif
-          ++gtile;
-          for (int i = 0; i < kTilePages; ++i) prev[i] = pages[i];
-          prev_npg = npg;
-          prev_valid = min(kPage, s.nvis - (pg0 + npg - 1) * kPage);
-        }
-        if (ok) ok = load_pv(prev, prev_npg, prev_valid);
-        ++seg;
       }
     }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA
+  } else if (warp == kQKWarp) {
+    // ----------------------------------------------------------- MMA: S = Q K^T
     if (rank == 0 && lane == 0) {
+      RingConsumer ring{bar(B_QK_FULL), bar(B_QK_EMPTY), sbase + kOffQKRing, kQKSlots};
       SegmentWalker walk(p, w, t);
       Segment s;
-      uint32_t slot = 0, phase = 0, g = 0, seg = 0;  // ring position, tile counter
+      uint32_t g = 0, seg = 0;
       bool ok = true;
-      const uint32_t full0 = bar(B_UNIT_FULL), empty0 = bar(B_UNIT_EMPTY);
       // descriptors advance by adding (byte offset >> 4) to the start-address field
-      const uint64_t qdesc = sdesc(sbase + kOffQ, 16, 1024);       // chunk c: + 512 c; K-step: + 2
-      const uint64_t kdesc = sdesc(sbase + kOffRing, 16, 1024);    // unit: + 1024 slot
-      const uint64_t vdesc = sdesc(sbase + kOffRing, 8192, 1024);  // unit: + 1024 slot; K-step: + 128
-      const uint64_t pdesc = sdesc(sbase + kOffP, 16, 1024);       // page sub-tile: + 512 i; K-step: + 2
-      auto release_unit = [&]() {
-        tc_commit_pair(empty0 + 8 * slot);
-        if (++slot == kUnits) {
-          slot = 0;
-          phase ^= 1;
-        }
-      };
-      auto do_pv = [&](uint32_t gi, bool first) -> bool {
-        if (!mbar_wait(bar(B_P_FULL), gi & 1, abort_flag, p.status)) return false;
-        TC_TRACE(2, gi);
-        tc_fence_after();
-#pragma unroll 1
-        for (int i = 0; i < kTilePages; ++i)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            if (!mbar_wait(full0 + 8 * slot, phase, abort_flag, p.status)) return false;
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-              tc_mma(tmem + (j ? kColO1 : kColO0), pdesc + 512 * i + 2 * ks, vdesc + 1024 * slot + 128 * ks, kIdescPV,
-                     (first && i == 0 && ks == 0) ? 0u : 1u);
-            release_unit();
-          }
-        tc_commit_pair(bar(B_O_DONE));
-        TC_TRACE(3, gi);
-        return true;
-      };
+      const uint64_t qdesc = sdesc(sbase + kOffQ, 16, 1024);      // chunk c: + 512 c; K-step: + 2
+      const uint64_t kdesc = sdesc(sbase + kOffQKRing, 16, 1024);  // slot: + 1024 slot
       while (ok && walk.next(s)) {
         if (s.n_pages == 0) continue;
         ok = mbar_wait(bar(B_Q_FULL), seg & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t g_first = g;
         const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
         for (int it = 0; it < n_tiles && ok; ++it, ++g) {
           ok = mbar_wait(bar(B_S_FREE + (g & 1)), ((g >> 1) & 1) ^ 1, abort_flag, p.status);
@@ -523,39 +540,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           TC_TRACE(7, g);
 #pragma unroll 1
           for (int c = 0; c < kQKUnits; ++c) {
-            ok = mbar_wait(full0 + 8 * slot, phase, abort_flag, p.status);
+            ok = ring.wait_full(abort_flag, p.status);
             if (!ok) break;
-            const uint64_t a = qdesc + 512 * c, bb = kdesc + 1024 * slot;
+            tc_fence_after();
+            const uint64_t a = qdesc + 512 * c, bb = kdesc + 1024 * ring.slot;
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)  // 16 columns = 32 bytes into the swizzled rows
               tc_mma(sd, a + 2 * k4, bb + 2 * k4, kIdescQK, (c | k4) ? 1u : 0u);
-            release_unit();
+            ring.release();
           }
           if (!ok) break;
           tc_commit_pair(bar(B_S_FULL + (g & 1)));
           TC_TRACE(1, g);
           if (it == n_tiles - 1) tc_commit_pair(bar(B_Q_EMPTY));
-          if (it > 0) {
-            if (it == 1 && seg > 0) {  // O of the previous segment must be read out first
-              ok = mbar_wait(bar(B_O_FREE), (seg - 1) & 1, abort_flag, p.status);
-              if (!ok) break;
-            }
-            ok = do_pv(g - 1, g - 1 == g_first);
-          }
         }
-        if (!ok) break;
-        if (n_tiles == 1 && seg > 0) {
-          ok = mbar_wait(bar(B_O_FREE), (seg - 1) & 1, abort_flag, p.status);
+        ++seg;
+      }
+    }
+  } else if (warp == kPVWarp) {
+    // ---------------------------------------------------------- MMA: O += P C
+    if (rank == 0 && lane == 0) {
+      RingConsumer ring{bar(B_PV_FULL), bar(B_PV_EMPTY), sbase + kOffPVRing, kPVSlots};
+      SegmentWalker walk(p, w, t);
+      Segment s;
+      uint32_t g = 0, seg = 0;
+      bool ok = true;
+      const uint64_t vdesc = sdesc(sbase + kOffPVRing, 8192, 1024);  // slot: + 1024 slot; K-step: + 128
+      const uint64_t pdesc = sdesc(sbase + kOffP, 16, 1024);         // page sub-tile: + 512 i; K-step: + 2
+      while (ok && walk.next(s)) {
+        if (s.n_pages == 0) continue;
+        const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
+        for (int it = 0; it < n_tiles && ok; ++it, ++g) {
+          ok = mbar_wait(bar(B_P_FULL), g & 1, abort_flag, p.status);
           if (!ok) break;
+          if (it == 0 && seg > 0) {  // O of the previous segment must be read out first
+            ok = mbar_wait(bar(B_O_FREE), (seg - 1) & 1, abort_flag, p.status);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          TC_TRACE(2, g);
+#pragma unroll 1
+          for (int i = 0; i < kTilePages && ok; ++i)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              ok = ring.wait_full(abort_flag, p.status);
+              if (!ok) break;
+              tc_fence_after();
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                tc_mma(tmem + (j ? kColO1 : kColO0), pdesc + 512 * i + 2 * ks, vdesc + 1024 * ring.slot + 128 * ks,
+                       kIdescPV, (it == 0 && i == 0 && ks == 0) ? 0u : 1u);
+              ring.release();
+            }
+          if (!ok) break;
+          tc_commit_pair(bar(B_O_DONE));
+          TC_TRACE(3, g);
         }
-        ok = do_pv(g - 1, g - 1 == g_first);
         ++seg;
       }
     }
   } else {
     // ------------------------------------------------------- softmax, epilogue
-    // Thread L (TMEM lane) holds head hl of this CTA; lanes 0-63 see keys
-    // 0-31 of each page of a tile, lanes 64-127 keys 32-63 (2x2 layout).
+    // Thread L (TMEM lane) holds head hl of this CTA; lanes 0-63 see the
+    // keys of pages 0-1 of a tile, lanes 64-127 those of pages 2-3 (the QK B
+    // operand holds the leader's two pages in N columns [0,128), the peer's in
+    // [128,256); 2x2 layout).  S is read twice from TMEM: once for the max,
+    // once for the probabilities, so that few registers hold scores at a time.
     const int L = warp * 32 + lane;
     const int hl = L & 63, half = L >> 6;
     const int head = kHalfHeads * (int)rank + hl;
@@ -582,35 +632,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         if (!ok) break;
         if (threadIdx.x == 0) TC_TRACE(4, g);
         tc_fence_after();
-        float sv[4 * 32];
-        {
-          uint32_t sr[32];
-#pragma unroll
-          for (int q = 0; q < kTilePages; ++q) {
-            tmem_ld32(tmem + lane_base + ((g & 1) ? kColS1 : kColS0) + 32 * q, sr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) sv[32 * q + j] = __uint_as_float(sr[j]);
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_bar(B_S_FREE + (g & 1)));
-        if (threadIdx.x == 0) TC_TRACE(5, g);
-        // keys of this thread: page q of the tile, in-page 32*half + j
+        const uint32_t s_addr = tmem + lane_base + ((g & 1) ? kColS1 : kColS0);
+        // visible keys of this thread's two pages (page 2*half + q of the tile)
         const int pg0 = s.page_lo + it * kTilePages;
+        int nv[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int pg = pg0 + 2 * half + q;
+          nv[q] = pg < s.page_lo + s.n_pages ? max(0, min(kPage, s.nvis - pg * kPage)) : 0;
+        }
+        // pass 1: the tile's max (scale > 0 commutes with max)
         float mx = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < kTilePages; ++q) {
-          const int key0 = (pg0 + q) * kPage + 32 * half;
-          const bool page_ok = pg0 + q < s.page_lo + s.n_pages;
+        for (int q = 0; q < 2; ++q) {
+          uint32_t sr[64];
+          tmem_ld32(s_addr + 64 * q, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(s_addr + 64 * q + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float v = (page_ok && key0 + j < s.nvis) ? sv[32 * q + j] * p.scale_log2 : -INFINITY;
-            sv[32 * q + j] = v;
-            mx = fmaxf(mx, v);
-          }
+          for (int j = 0; j < 64; ++j)
+            if (j < nv[q]) mx = fmaxf(mx, __uint_as_float(sr[j]));
         }
+        mx = mx * p.scale_log2;
         red_max[half * 64 + hl] = mx;
         asm volatile("bar.sync 1, 128;" ::: "memory");
         const float tile_max = fmaxf(mx, red_max[(half ^ 1) * 64 + hl]);
@@ -624,18 +667,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           alpha = fast_exp2(m_ref - tile_max);
           m_ref = tile_max;
         }
-        uint32_t pk[64];
-        float psum = 0.f;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const __nv_bfloat162 h2 =
-              __floats2bfloat162_rn(fast_exp2(sv[2 * j] - m_ref), fast_exp2(sv[2 * j + 1] - m_ref));
-          const float2 f2 = __bfloat1622float2(h2);
-          psum += f2.x + f2.y;
-          pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
-        l_part = l_part * alpha + psum;
-        if (threadIdx.x == 0) TC_TRACE(10, g);
         // the previous tile's PV MMAs read P and write O: wait for them
         if (g >= 1) {
           ok = mbar_wait(bar(B_O_DONE), (g - 1) & 1, abort_flag, p.status);
@@ -658,21 +689,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           }
           tmem_wait_st();
         }
-        // P row hl: page q is sub-tile q (64 keys, 128 B per row, 128-byte
-        // swizzle); this thread's 32 keys are 16-byte units 4*half .. 4*half+3
+        // pass 2: probabilities, written as P row hl of sub-tiles 2*half + q
+        // (64 keys, 128 B per row, 128-byte swizzle)
+        float psum = 0.f;
 #pragma unroll
-        for (int q = 0; q < kTilePages; ++q) {
-          uint8_t* prow = smem + kOffP + q * 8192 + hl * 128;
+        for (int q = 0; q < 2; ++q) {
+          uint32_t sr[64];
+          tmem_ld32(s_addr + 64 * q, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(s_addr + 64 * q + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_wait_ld();
+          uint32_t pk[32];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int unit = (4 * half + u) ^ (hl & 7);
-            *reinterpret_cast<uint4*>(prow + unit * 16) =
-                make_uint4(pk[16 * q + 4 * u], pk[16 * q + 4 * u + 1], pk[16 * q + 4 * u + 2], pk[16 * q + 4 * u + 3]);
+          for (int j = 0; j < 32; ++j) {
+            const float e0 = 2 * j < nv[q] ? fast_exp2(__uint_as_float(sr[2 * j]) * p.scale_log2 - m_ref) : 0.f;
+            const float e1 = 2 * j + 1 < nv[q] ? fast_exp2(__uint_as_float(sr[2 * j + 1]) * p.scale_log2 - m_ref) : 0.f;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+            const float2 f2 = __bfloat1622float2(h2);
+            psum += f2.x + f2.y;
+            pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
           }
+          uint8_t* prow = smem + kOffP + (2 * half + q) * 8192 + hl * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(prow + ((u ^ (hl & 7)) * 16)) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
-        if (threadIdx.x == 0) TC_TRACE(11, g);
-        fence_proxy_async();
+        l_part = l_part * alpha + psum;
+        // S of this tile is consumed
         tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_bar(B_S_FREE + (g & 1)));
+        fence_proxy_async();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (threadIdx.x == 0) TC_TRACE(6, g);
         if (lane == 0) mbar_arrive_cluster(leader_bar(B_P_FULL));
@@ -714,7 +761,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   __syncthreads();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   tc_fence_after();
-  if (warp == 5)
+  if (warp == kQKWarp)
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
@@ -776,13 +823,13 @@ cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st) {
   tp.p = p;
   const uint64_t pool_rows = (uint64_t)p.num_pages * kPage;
   if (!make_map(&tp.map_q, p.q_abs, (uint64_t)p.batch * p.n_q * kHeads, 64) ||
-      !make_map(&tp.map_kq, p.pool, pool_rows, 32) || !make_map(&tp.map_pv, p.pool, pool_rows, 64) ||
+      !make_map(&tp.map_pv, p.pool, pool_rows, 64) ||
       !make_map(&tp.map_pv16, p.pool, pool_rows, 16) || !make_map(&tp.map_row, p.pool, pool_rows, 1))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const int pairs = p.splits * p.n_q;
-  decode_tc_kernel<<<2 * pairs, 192, kSmemBytes, st>>>(tp);
+  decode_tc_kernel<<<2 * pairs, kThreads, kSmemBytes, st>>>(tp);
   return cudaGetLastError();
 }
 
