@@ -5,6 +5,9 @@
 // steps 2-3).  Output row [q~ | RoPE(q^R)] per (token, head), the operand the
 // decode kernel scores against the 576-wide cached rows.
 //
+// The output is in the activation type, or f16 when the decode path reads
+// f16 queries (FP8 cache on the tensor cores).
+//
 // One CTA per (head, 16-vector slice of d_c).  Thread (cg, dg) loads the
 // 16-byte vectors of W^UK_h for its column group cg and its rows d in group
 // dg, all loads issued up front, and keeps them in registers for every token
@@ -126,7 +129,7 @@ __device__ void build_plan(const AbsorbArgs& a) {
   }
 }
 
-template <typename T>
+template <typename T, typename TO>
 __global__ void __launch_bounds__(128) absorb_kernel(const AbsorbArgs a) {
   constexpr int VEC = VecN<T>::n;
   __shared__ float q_s[kTokBlock][kDG * kMaxRows];
@@ -155,7 +158,7 @@ __global__ void __launch_bounds__(128) absorb_kernel(const AbsorbArgs a) {
                                                  : make_uint4(0, 0, 0, 0);
   }
   const T* qn = static_cast<const T*>(a.q_nope);
-  T* qa = static_cast<T*>(a.q_abs);
+  TO* qa = static_cast<TO*>(a.q_abs);
   for (int m0 = 0; m0 < M; m0 += kTokBlock) {
     const int mc = min(kTokBlock, M - m0);
     __syncthreads();
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(128) absorb_kernel(const AbsorbArgs a) {
         float s = 0.f;
 #pragma unroll
         for (int g = 0; g < kDG; ++g) s += red[g][mi][cc];
-        qa[((size_t)(m0 + mi) * a.n_heads + h) * D + c] = from_f<T>(s);
+        qa[((size_t)(m0 + mi) * a.n_heads + h) * D + c] = from_f<TO>(s);
       }
     }
   }
@@ -209,9 +212,9 @@ __global__ void __launch_bounds__(128) absorb_kernel(const AbsorbArgs a) {
       rope_cos_sin(p, k, half, a.rope_base, &cs, &sn);
       const T* src = qr + ((size_t)m * a.n_heads + h) * a.d_rope;
       const float x1 = to_f(src[k]), x2 = to_f(src[half + k]);
-      T* dst = qa + ((size_t)m * a.n_heads + h) * D + a.d_c;
-      dst[k] = from_f<T>(x1 * cs - x2 * sn);
-      dst[half + k] = from_f<T>(x2 * cs + x1 * sn);
+      TO* dst = qa + ((size_t)m * a.n_heads + h) * D + a.d_c;
+      dst[k] = from_f<TO>(x1 * cs - x2 * sn);
+      dst[half + k] = from_f<TO>(x2 * cs + x1 * sn);
     }
   }
 }
@@ -222,8 +225,8 @@ int absorb_max_d_nope() { return kDG * kMaxRows; }
 
 cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const void* q_rope, const void* W_uk,
                                    const int32_t* seq_lens, int batch, int n_q, int max_pages, int splits,
-                                   void* q_abs, int32_t* plan, float* lse_part, size_t lse_count, int* status,
-                                   cudaStream_t st) {
+                                   void* q_abs, bool q_abs_f16, int32_t* plan, float* lse_part, size_t lse_count,
+                                   int* status, cudaStream_t st) {
   AbsorbArgs a;
   a.q_nope = q_nope;
   a.q_rope = q_rope;
@@ -247,9 +250,11 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
   const int vec = d.act_dtype == MLA_F32 ? 4 : 8;
   const dim3 grid(d.n_heads, (d.d_c + kCG * vec - 1) / (kCG * vec));
   if (d.act_dtype == MLA_F32)
-    absorb_kernel<float><<<grid, 128, 0, st>>>(a);
+    absorb_kernel<float, float><<<grid, 128, 0, st>>>(a);
+  else if (q_abs_f16)
+    absorb_kernel<__nv_bfloat16, __half><<<grid, 128, 0, st>>>(a);
   else
-    absorb_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(a);
+    absorb_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 128, 0, st>>>(a);
   return cudaGetLastError();
 }
 

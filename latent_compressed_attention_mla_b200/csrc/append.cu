@@ -26,16 +26,6 @@ constexpr int kSplitK = 4;    // warps per row, one per quarter of d_model
 constexpr int kTok = 2;       // tokens per pass
 constexpr int kMaxVec = 8;    // 16-byte vectors per lane per quarter of d_model
 
-struct Fp8Page {
-  size_t kr_off, sc_off;
-};
-__host__ __device__ inline size_t a128(size_t x) { return (x + 127) / 128 * 128; }
-__host__ __device__ inline Fp8Page fp8_page(int page_size, int d_c, int d_rope) {
-  Fp8Page p;
-  p.kr_off = a128((size_t)page_size * d_c);
-  p.sc_off = a128(p.kr_off + (size_t)page_size * d_rope * 2);
-  return p;
-}
 
 struct AppendArgs {
   const void* h;

@@ -1,6 +1,7 @@
 // S3 on the 5th-generation tensor cores: split-KV attention of the absorbed
-// queries over the paged bf16 latent cache, DeepSeek-V3 dims (128 heads,
-// 576-wide rows = 512 latent + 64 RoPE, 64-token pages).
+// queries over the paged latent cache, DeepSeek-V3 dims (128 heads, 576-wide
+// rows = 512 latent + 64 RoPE, 64-token pages), for a bf16 cache and for an
+// FP8 (e4m3 + per-128-column fp32 scales, bf16 k^R) cache.
 //
 // What it computes ("DeepSeek MLA Architecture: How Multi-Head Latent Attention
 // Cuts KV Cache by 93%", "3. Decoupled RoPE and Matrix Absorption" and the
@@ -21,24 +22,36 @@
 //    operand, the peer pages 2-3.  S (2 buffers) and O live in tensor memory
 //    (TMEM), 2x2 layout: row m, column n < N/2 -> lane m, column n;
 //    n >= N/2 -> lane 64+m, column n-N/2.
-//  * Operands stream through a ring of 16 KB units (TMA, 128-byte swizzle) in
-//    the order the MMAs consume them: the 9 QK units of tile g (this CTA's two
-//    pages x 64 columns each, K-major), then the 8 PV units of tile g-1 (one
-//    page x this CTA's 128 latent columns of one N=256 MMA, MN-major).  Each
-//    unit has its own full/empty barrier.  Rows past a sequence's end in its
-//    last page are loaded from outside the tensor (TMA zero fill), never from
-//    the pool, so 0 * (whatever the pool held) cannot reach O.
-//  * Three producer warps take the units in turn: one thread's TMA issue rate
-//    is bounded by its own barrier wait/arm cycle, and several issuing warps
-//    keep enough loads in flight to stream at the HBM rate.
-//  * Warp roles: warps 0-3 softmax + epilogue (one TMEM lane each), warp 4
-//    TMEM allocation and (leader CTA) MMA issue, warps 5-7 TMA producers.
+//  * Operands stream through two rings of 16 KB units (128-byte swizzle) in
+//    the order the MMAs consume them: QK units (this CTA's two pages x 64
+//    columns, K-major) and PV units (one page x this CTA's 128 latent columns
+//    of one N=256 MMA, MN-major).  Each ring has its own MMA-issuing thread:
+//    an MMA issue returns only once the tensor pipe takes it, so one issuer's
+//    barrier waits and commits are covered by the other's MMAs.
+//  * bf16 cache: TMA writes the units directly; two producer warps per ring
+//    keep enough loads in flight (one thread's issue rate is bounded by its
+//    barrier wait/arm cycle).  Rows past a sequence's end in its last page
+//    are loaded from outside the tensor (TMA zero fill), never from the pool,
+//    so 0 * (whatever the pool held) cannot reach O.
+//  * FP8 cache: TMA brings the raw page data (codes, k^R) into staging slots;
+//    converter warps write the operand units as f16, code * scale with the
+//    scale of the row's 128-column tile (f16 keeps more mantissa than bf16,
+//    and one cvt + one multiply per element pair), and zero the rows past a
+//    sequence's end.  Queries and probabilities are f16 on this path, so both
+//    MMA operands share the type (kind::f16).
+//  * Warp roles: 0-3 softmax + epilogue (one TMEM lane each), 4 TMEM
+//    allocation and (leader) QK issue, 5 (leader) PV issue, 6-7 TMA for Q and
+//    QK data, 8-9 TMA for PV data, and for the FP8 cache 10-11 / 12-13
+//    converters of QK / PV units.
 //  * Online softmax in base 2 with a lazily updated reference max: O is only
 //    rescaled when a tile's max exceeds the reference by more than 8 (in
 //    log2 units), so probabilities stay <= 2^8 and rescaling is rare.
 //  * Every mbarrier wait is bounded; on expiry the kernel records
 //    MLA_ERR_TIMEOUT in the status word and unwinds.
 #include <cuda.h>
+#include <cuda_fp16.h>
+
+#include <cstring>
 
 #include "mla_internal.cuh"
 
@@ -54,71 +67,77 @@ constexpr int kDC = 512, kDR = 64, kD = kDC + kDR;  // 576
 constexpr int kPage = 64;                             // keys per cache page
 constexpr int kTilePages = 4;                         // pages per tile: 256 keys = N of the QK MMA
 constexpr int kChunks = kD / 64;                      // 9 column chunks of 64 (128 B)
+constexpr int kQKUnits = kChunks;                     // QK units per tile
 
-// Operand units: 16 KB each, this CTA's share of one group of four MMAs
-//   QK unit c : its two pages of the tile (128 keys) x columns [64c, 64c+64), K-major
-//   PV unit   : one page's 64 keys x its 128 latent columns of one N=256 half, MN-major
-// QK and PV units stream through rings of their own, each consumed by its own
-// MMA-issuing thread: an MMA issue returns only once the tensor pipe takes
-// it, so one issuer's barrier waits and commits are covered by the other's
-// MMAs.
-constexpr uint32_t kUnitBytes = 16384;
-constexpr int kQKSlots = 3, kPVSlots = 4;
-constexpr int kQKUnits = kChunks;         // 9 per tile
+constexpr uint32_t kUnitBytes = 16384;                // operand unit: this CTA's share of four MMAs
+constexpr uint32_t kStageBytes = 8192;                // FP8 staging slot: raw page data of one unit
+constexpr uint32_t kSclBytes = kTilePages * 64 * 4 * 4;  // FP8: [4 pages][64 rows][4] fp32 scales of a tile
+constexpr uint32_t kQBytes = kChunks * 64 * 128;      // 73728: 64 heads x 576 (16-bit)
+constexpr uint32_t kPBytes = kTilePages * 64 * 128;   // 32768: 64 heads x 256 keys (16-bit), 4 sub-tiles
 
-// shared memory layout (offsets from a 1024-byte aligned base)
-constexpr uint32_t kQBytes = kChunks * 64 * 128;      // 73728: 64 heads x 576 bf16
-constexpr uint32_t kPBytes = kTilePages * 64 * 128;   // 32768: 64 heads x 256 keys bf16, 4 sub-tiles
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffP = kOffQ + kQBytes;
-constexpr uint32_t kOffQKRing = kOffP + kPBytes;                   // 106496
-constexpr uint32_t kOffPVRing = kOffQKRing + kQKSlots * kUnitBytes;
-constexpr uint32_t kOffBar = kOffPVRing + kPVSlots * kUnitBytes;
-constexpr uint32_t kNumBars = 2 * kQKSlots + 2 * kPVSlots + 9;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kOffRedMax = kOffMisc + 16;                     // float [2][64]
-constexpr uint32_t kOffRedL = kOffRedMax + 512;                    // float [2][64]
-constexpr uint32_t kSmemUsed = kOffRedL + 512;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;                  // + alignment slack
-
-// barrier indices
-enum {
-  B_QK_FULL = 0,                        // [kQKSlots] leader: TMA bytes of both CTAs
-  B_QK_EMPTY = kQKSlots,                // [kQKSlots] each CTA: unit consumed (MMA commit)
-  B_PV_FULL = 2 * kQKSlots,             // [kPVSlots] leader: TMA bytes of both CTAs
-  B_PV_EMPTY = B_PV_FULL + kPVSlots,    // [kPVSlots] each CTA: unit consumed (MMA commit)
-  B_S_FULL = B_PV_EMPTY + kPVSlots,     // [2] each CTA: S tile ready (MMA commit)
-  B_S_FREE = B_S_FULL + 2,              // [2] leader: S read by both CTAs' softmax warps (8 arrivals)
-  B_P_FULL = B_S_FREE + 2,              // leader: P written + O rescaled by both CTAs (8 arrivals)
-  B_O_DONE,                             // each CTA: the tile's PV MMAs finished (MMA commit)
-  B_O_FREE,                             // leader: O read out by both CTAs' epilogues (8 arrivals)
-  B_Q_FULL,                             // leader: Q bytes of both CTAs
-  B_Q_EMPTY,                            // each CTA: last QK of a segment finished (MMA commit)
-  B_COUNT
+// Shared memory layout and warp roles of the two variants (offsets from a
+// 1024-byte aligned base).
+template <bool kFp8>
+struct TcLayout {
+  static constexpr int QKSlots = kFp8 ? 2 : 3, PVSlots = kFp8 ? 2 : 4;
+  static constexpr int QStSlots = kFp8 ? 3 : 0, PStSlots = kFp8 ? 3 : 0;
+  static constexpr int SclBufs = kFp8 ? 2 : 0;  // per-tile scales of the four pages (4 KB each)
+  static constexpr uint32_t OffQ = 0;
+  static constexpr uint32_t OffP = OffQ + kQBytes;
+  static constexpr uint32_t OffQKRing = OffP + kPBytes;
+  static constexpr uint32_t OffPVRing = OffQKRing + QKSlots * kUnitBytes;
+  static constexpr uint32_t OffQSt = OffPVRing + PVSlots * kUnitBytes;
+  static constexpr uint32_t OffPSt = OffQSt + QStSlots * kStageBytes;
+  static constexpr uint32_t OffScl = OffPSt + PStSlots * kStageBytes;
+  static constexpr uint32_t OffBar = OffScl + SclBufs * kSclBytes;
+  // barrier indices
+  static constexpr int QK_FULL = 0;                     // [QKSlots] leader: unit written in both CTAs
+  static constexpr int QK_EMPTY = QK_FULL + QKSlots;    // [QKSlots] each CTA: unit consumed (MMA commit)
+  static constexpr int PV_FULL = QK_EMPTY + QKSlots;    // [PVSlots]
+  static constexpr int PV_EMPTY = PV_FULL + PVSlots;    // [PVSlots]
+  static constexpr int S_FULL = PV_EMPTY + PVSlots;     // [2] each CTA: S tile ready (MMA commit)
+  static constexpr int S_FREE = S_FULL + 2;             // [2] leader: S read by both CTAs' softmax warps
+  static constexpr int P_FULL = S_FREE + 2;             // leader: P written + O rescaled by both CTAs
+  static constexpr int O_DONE = P_FULL + 1;             // each CTA: the tile's PV MMAs finished
+  static constexpr int O_FREE = O_DONE + 1;             // leader: O read out by both CTAs' epilogues
+  static constexpr int Q_FULL = O_FREE + 1;             // leader: Q bytes of both CTAs
+  static constexpr int Q_EMPTY = Q_FULL + 1;            // each CTA: last QK of a segment finished
+  static constexpr int QST_FULL = Q_EMPTY + 1;          // [QStSlots] local: staged bytes landed
+  static constexpr int QST_EMPTY = QST_FULL + QStSlots; // [QStSlots] local: both converter warps done
+  static constexpr int PST_FULL = QST_EMPTY + QStSlots; // [PStSlots]
+  static constexpr int PST_EMPTY = PST_FULL + PStSlots; // [PStSlots]
+  static constexpr int SCL_FULL = PST_EMPTY + PStSlots;  // [SclBufs] local: a tile's scales landed
+  static constexpr int SCL_EMPTY = SCL_FULL + SclBufs;   // [SclBufs] local: all converter warps done
+  static constexpr int NumBars = SCL_EMPTY + SclBufs;
+  static constexpr uint32_t OffMisc = OffBar + NumBars * 8;
+  static constexpr uint32_t OffRedMax = OffMisc + 16;   // float [2][64]
+  static constexpr uint32_t OffRedL = OffRedMax + 512;  // float [2][64]
+  static constexpr uint32_t SmemBytes = OffRedL + 512 + 1024;  // + alignment slack
+  // warp roles
+  static constexpr int QKWarp = 4, PVWarp = 5;          // TMEM alloc (QKWarp); leader lane 0 issues the MMAs
+  static constexpr int QKProdWarp = 6, PVProdWarp = 8, Producers = 2;
+  static constexpr int QKConvWarp = 10, PVConvWarp = 12, ConvWarps = 2;
+  static constexpr int Threads = 32 * (kFp8 ? 14 : 10);
+  // arrivals completing one phase of a unit's FULL barrier: the leader's
+  // expect-tx arrival (bf16), or every converter warp of both CTAs (FP8)
+  static constexpr int UnitFullCount = kFp8 ? 2 * ConvWarps : 1;
 };
-static_assert(B_COUNT == (int)kNumBars, "barrier count");
+static_assert(TcLayout<false>::SmemBytes <= 232448, "shared memory");
+static_assert(TcLayout<true>::SmemBytes <= 232448, "shared memory");
 
 // TMEM columns (per CTA, 2x2 layout): S buffers 128 columns each, O 2 x 128
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 
-// warp roles
-constexpr int kQKWarp = 4;                         // TMEM allocation; leader lane 0 issues the QK MMAs
-constexpr int kPVWarp = 5;                         // leader lane 0 issues the PV MMAs
-constexpr int kQKProdWarp = 6, kQKProducers = 2;   // load Q and the QK units
-constexpr int kPVProdWarp = 8, kPVProducers = 2;   // load the PV units
-constexpr int kThreads = 32 * (kPVProdWarp + kPVProducers);  // 320
-
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s
 
-// instruction descriptors (kind::f16, bf16 x bf16 -> f32, dense)
-constexpr uint32_t idesc(int M, int N, bool a_mn, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+// instruction descriptors (kind::f16, dense, f32 accumulator; operands bf16
+// or f16, the same for A and B)
+constexpr uint32_t idesc(int M, int N, bool a_mn, bool b_mn, bool f16) {
+  return (1u << 4) | (f16 ? 0u : ((1u << 7) | (1u << 10))) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-constexpr uint32_t kIdescQK = idesc(128, 256, false, false);
-constexpr uint32_t kIdescPV = idesc(128, 256, false, true);
 
 // ---------------------------------------------------------------------------
 // Protocol timestamps for development builds (-DMLA_TC_TRACE): event e of
@@ -135,6 +154,11 @@ __device__ __forceinline__ void tc_trace(int e, uint32_t g) {
   }
 }
 #define TC_TRACE(e, g) tc_trace((e), (g))
+#define TC_TRACE_VAL(e, g, v)                                                        \
+  do {                                                                               \
+    if (blockIdx.x < kTrCtas && (g) < kTrTiles)                                      \
+      g_tc_trace[(blockIdx.x * kTrTiles + (g)) * kTrEvents + (e)] = (unsigned long long)(v); \
+  } while (0)
 __device__ __forceinline__ unsigned long long tc_now() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -142,6 +166,7 @@ __device__ __forceinline__ unsigned long long tc_now() {
 }
 #else
 #define TC_TRACE(e, g) ((void)0)
+#define TC_TRACE_VAL(e, g, v) ((void)0)
 #endif
 
 // ---------------------------------------------------------------------------
@@ -272,6 +297,40 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// arrive on a barrier of this CTA with an expected transaction count
+__device__ __forceinline__ void mbar_arrive_tx_local(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_local(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Four e4m3 codes (one 32-bit word, first code in the low byte) times a
+// scale -> four f16 values packed as two f16x2 words.
+__device__ __forceinline__ void e4m3x4_scaled(uint32_t w, __half2 s2, uint32_t& lo, uint32_t& hi) {
+  const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+  const __half2 x = __hmul2(__half2(a), s2), y = __hmul2(__half2(b), s2);
+  lo = *reinterpret_cast<const uint32_t*>(&x);
+  hi = *reinterpret_cast<const uint32_t*>(&y);
+}
+
+// Two bf16 (one 32-bit word) -> two f16 (round to nearest).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+  const __half2 h = __float22half2_rn(f);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // ---------------------------------------------------------------------------
 // Work partition (shared by all roles): split w of query t covers global key
 // tiles [w*TT/W, (w+1)*TT/W); pieces per sequence are segments.
@@ -313,62 +372,75 @@ struct SegmentWalker {
 
 struct TcParams {
   DecodeParams p;
-  CUtensorMap map_q;    // q_abs [rows = batch*n_q*128][576] bf16, box 64 x 64
-  CUtensorMap map_pv;   // pool rows, box 64 x 64 (one page x 64 columns: QK and PV boxes)
-  CUtensorMap map_pv16; // pool rows, box 64 x 16 (16-key group of a partial page)
-  CUtensorMap map_row;  // pool rows, box 64 x 1 (one row of a partial 16-key group)
+  CUtensorMap map_q;     // q_abs [rows = batch*n_q*128][576], box 64 x 64 (bf16, or f16 for the FP8 cache)
+  // bf16 cache
+  CUtensorMap map_pv;    // pool rows, box 64 x 64 (one page x 64 columns: QK and PV boxes)
+  CUtensorMap map_pv16;  // pool rows, box 64 x 16 (16-key group of a partial page)
+  CUtensorMap map_row;   // pool rows, box 64 x 1 (one row of a partial 16-key group)
+  // FP8 cache: [pages][64 rows][...] views of the page sub-blocks
+  CUtensorMap map_codes_qk;  // e4m3 codes, box 64 codes x 64 rows (one page's part of a QK unit)
+  CUtensorMap map_codes_pv;  // e4m3 codes, box 128 codes x 64 rows (one PV unit)
+  CUtensorMap map_kr;        // bf16 k^R, box 64 x 64 rows
+  CUtensorMap map_scl;       // fp32 scales, box 4 x 64 rows (one page)
 };
 
-// Producer side of one operand ring: producer pid of n issues every n-th unit
-// of the ring's consumption order; every producer walks the same schedule, so
-// the ring position of each unit is known to all of them.
-struct RingProducer {
-  uint32_t full0, empty0, leader_full0, ring0;
-  int slots, producers, pid;
-  uint32_t slot = 0, phase = 0, unit = 0;
-  // Claim the next unit.  Returns true when this producer issues it, after the
-  // slot is free and (leader) the barrier expects both CTAs' bytes.
-  __device__ bool claim(uint32_t rank, uint32_t& dst, uint32_t& fullbar, bool& ok, volatile int* abort_flag,
-                        int* status) {
-    const bool mine = (int)(unit % (uint32_t)producers) == pid;
-    const uint32_t my_slot = slot, my_phase = phase;
-    ++unit;
+// Position in a ring of `slots` slots: slot index and the parity of its use.
+struct RingPos {
+  uint32_t slot = 0, phase = 0;
+  __device__ void advance(int slots) {
     if (++slot == (uint32_t)slots) {
       slot = 0;
       phase ^= 1;
     }
+  }
+};
+
+// Producer side of one ring: producer pid of n issues every n-th entry of the
+// ring's consumption order; every producer walks the same schedule, so the
+// ring position of each entry is known to all of them.
+struct RingProducer {
+  int slots, producers, pid;
+  RingPos pos;
+  uint32_t entry = 0;
+  // Claim the next entry: returns true (with its slot) when this producer
+  // issues it, after waiting for the slot to be free.
+  __device__ bool claim(uint32_t empty0, uint32_t& slot, bool& ok, volatile int* abort_flag, int* status) {
+    const bool mine = (int)(entry % (uint32_t)producers) == pid;
+    const RingPos cur = pos;
+    ++entry;
+    pos.advance(slots);
     if (!mine || !ok) return false;
-    if (!mbar_wait(empty0 + 8 * my_slot, my_phase ^ 1, abort_flag, status)) {
+    if (!mbar_wait(empty0 + 8 * cur.slot, cur.phase ^ 1, abort_flag, status)) {
       ok = false;
       return false;
     }
-    if (rank == 0) mbar_expect_tx(full0 + 8 * my_slot, 2 * kUnitBytes);
-    dst = ring0 + my_slot * kUnitBytes;
-    fullbar = leader_full0 + 8 * my_slot;
+    slot = cur.slot;
     return true;
   }
 };
 
 // Consumer side of one operand ring (the MMA-issuing thread of the leader).
 struct RingConsumer {
-  uint32_t full0, empty0, ring0;
+  uint32_t full0, empty0;
   int slots;
-  uint32_t slot = 0, phase = 0;
+  RingPos pos;
   __device__ bool wait_full(volatile int* abort_flag, int* status) {
-    return mbar_wait(full0 + 8 * slot, phase, abort_flag, status);
+    return mbar_wait(full0 + 8 * pos.slot, pos.phase, abort_flag, status);
   }
   // the unit's MMAs are issued: free the slot in both CTAs once they complete
   __device__ void release() {
-    tc_commit_pair(empty0 + 8 * slot);
-    if (++slot == (uint32_t)slots) {
-      slot = 0;
-      phase ^= 1;
-    }
+    tc_commit_pair(empty0 + 8 * pos.slot);
+    pos.advance(slots);
   }
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <bool kFp8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Threads, 1)
     decode_tc_kernel(const __grid_constant__ TcParams P) {
+  using L = TcLayout<kFp8>;
+  using PT = typename std::conditional<kFp8, __half2, __nv_bfloat162>::type;  // P element pair
+  constexpr uint32_t kIdescQK = idesc(128, 256, false, false, kFp8);
+  constexpr uint32_t kIdescPV = idesc(128, 256, false, true, kFp8);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -378,35 +450,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int pair = blockIdx.x >> 1;
   const int t = pair % p.n_q, w = pair / p.n_q;
 
-  auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * i; };
+  auto bar = [&](int i) -> uint32_t { return sbase + L::OffBar + 8u * i; };
   auto leader_bar = [&](int i) -> uint32_t { return map_to_rank(bar(i), 0); };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc + 4);
-  float* red_max = reinterpret_cast<float*>(smem + kOffRedMax);
-  float* red_l = reinterpret_cast<float*>(smem + kOffRedL);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OffMisc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OffMisc + 4);
+  float* red_max = reinterpret_cast<float*>(smem + L::OffRedMax);
+  float* red_l = reinterpret_cast<float*>(smem + L::OffRedL);
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    for (int i = 0; i < kQKSlots; ++i) {
-      mbar_init(bar(B_QK_FULL + i), 1);
-      mbar_init(bar(B_QK_EMPTY + i), 1);
+    for (int i = 0; i < L::QKSlots; ++i) {
+      mbar_init(bar(L::QK_FULL + i), L::UnitFullCount);
+      mbar_init(bar(L::QK_EMPTY + i), 1);
     }
-    for (int i = 0; i < kPVSlots; ++i) {
-      mbar_init(bar(B_PV_FULL + i), 1);
-      mbar_init(bar(B_PV_EMPTY + i), 1);
+    for (int i = 0; i < L::PVSlots; ++i) {
+      mbar_init(bar(L::PV_FULL + i), L::UnitFullCount);
+      mbar_init(bar(L::PV_EMPTY + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(B_S_FULL + i), 1);
-      mbar_init(bar(B_S_FREE + i), 8);
+      mbar_init(bar(L::S_FULL + i), 1);
+      mbar_init(bar(L::S_FREE + i), 8);
     }
-    mbar_init(bar(B_P_FULL), 8);
-    mbar_init(bar(B_O_DONE), 1);
-    mbar_init(bar(B_O_FREE), 8);
-    mbar_init(bar(B_Q_FULL), 1);
-    mbar_init(bar(B_Q_EMPTY), 1);
+    mbar_init(bar(L::P_FULL), 8);
+    mbar_init(bar(L::O_DONE), 1);
+    mbar_init(bar(L::O_FREE), 8);
+    mbar_init(bar(L::Q_FULL), 1);
+    mbar_init(bar(L::Q_EMPTY), 1);
+    for (int i = 0; i < L::QStSlots; ++i) {
+      mbar_init(bar(L::QST_FULL + i), 1);
+      mbar_init(bar(L::QST_EMPTY + i), L::ConvWarps);
+    }
+    for (int i = 0; i < L::PStSlots; ++i) {
+      mbar_init(bar(L::PST_FULL + i), 1);
+      mbar_init(bar(L::PST_EMPTY + i), L::ConvWarps);
+    }
+    for (int i = 0; i < L::SclBufs; ++i) {
+      mbar_init(bar(L::SCL_FULL + i), 1);
+      mbar_init(bar(L::SCL_EMPTY + i), 2 * L::ConvWarps);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == kQKWarp) {
+  if (warp == L::QKWarp) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols)
                  : "memory");
@@ -426,50 +510,86 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     return page;
   };
 
-  if (warp >= kQKProdWarp && warp < kQKProdWarp + kQKProducers) {
+  if (warp >= L::QKProdWarp && warp < L::QKProdWarp + L::Producers) {
     // -------------------------------------------------------------- TMA: Q, QK
     if (lane == 0) {
-      RingProducer ring{bar(B_QK_FULL), bar(B_QK_EMPTY), leader_bar(B_QK_FULL), sbase + kOffQKRing, kQKSlots,
-                        kQKProducers, warp - kQKProdWarp};
-      const bool q_loader = ring.pid == 0;
+      const int pid = warp - L::QKProdWarp;
+      RingProducer ring{kFp8 ? L::QStSlots : L::QKSlots, L::Producers, pid};
+      const uint32_t empty0 = kFp8 ? bar(L::QST_EMPTY) : bar(L::QK_EMPTY);
       const int y_pages = 2 * (int)rank;  // this CTA's two pages of a tile
       SegmentWalker walk(p, w, t);
       Segment s;
-      uint32_t seg = 0;
+      uint32_t seg = 0, gtile = 0;
       bool ok = true;
       while (ok && walk.next(s)) {
         if (s.n_pages == 0) continue;
         // absorbed queries of this CTA's 64 heads for (b, t)
-        if (q_loader) {
-          if (seg > 0) ok = mbar_wait(bar(B_Q_EMPTY), (seg - 1) & 1, abort_flag, p.status);
+        if (pid == 0) {
+          if (seg > 0) ok = mbar_wait(bar(L::Q_EMPTY), (seg - 1) & 1, abort_flag, p.status);
           if (!ok) break;
-          if (rank == 0) mbar_expect_tx(bar(B_Q_FULL), 2 * kQBytes);
+          if (rank == 0) mbar_expect_tx(bar(L::Q_FULL), 2 * kQBytes);
           const int qrow = ((s.b * p.n_q + t) * kHeads) + kHalfHeads * (int)rank;
-          const uint32_t qbar = leader_bar(B_Q_FULL);
-          for (int c = 0; c < kChunks; ++c) tma_load_2d_pair(sbase + kOffQ + c * 8192, &P.map_q, 64 * c, qrow, qbar);
+          const uint32_t qbar = leader_bar(L::Q_FULL);
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_2d_pair(sbase + L::OffQ + c * 8192, &P.map_q, 64 * c, qrow, qbar);
         }
         const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
         for (int it = 0; it < n_tiles && ok; ++it) {
           const int pg0 = s.page_lo + it * kTilePages;
           const int npg = min(kTilePages, s.n_pages - it * kTilePages);
-          // rows of this CTA's pages; pages past the tile's end come from
-          // outside the tensor (zero fill)
-          int y[2];
-          for (int i = 0; i < 2; ++i) y[i] = y_pages + i < npg ? page_of(s.b, pg0 + y_pages + i) * kPage : -kPage;
+          // this CTA's pages; pages past the tile's end come from outside the
+          // tensor (zero fill)
+          int pg[2];
+          for (int i = 0; i < 2; ++i) pg[i] = y_pages + i < npg ? page_of(s.b, pg0 + y_pages + i) : -1;
+          if constexpr (kFp8) {
+            // scales of the tile's four pages (zero for pages past its end)
+            if (pid == 0) {
+              const uint32_t sb = gtile & 1;
+              ok = mbar_wait(bar(L::SCL_EMPTY + sb), ((gtile >> 1) & 1) ^ 1, abort_flag, p.status);
+              if (!ok) break;
+              const uint32_t fb = bar(L::SCL_FULL + sb);
+              mbar_arrive_tx_local(fb, kSclBytes);
+              for (int i = 0; i < kTilePages; ++i)
+                tma_load_3d(sbase + L::OffScl + sb * kSclBytes + i * 1024, &P.map_scl, 0, 0,
+                            i < npg ? page_of(s.b, pg0 + i) : -1, fb);
+            }
+            ++gtile;
+          }
           for (int c = 0; c < kQKUnits; ++c) {
-            uint32_t dst, fb;
-            if (!ring.claim(rank, dst, fb, ok, abort_flag, p.status)) continue;
-            for (int i = 0; i < 2; ++i) tma_load_2d_pair(dst + i * 8192, &P.map_pv, 64 * c, y[i], fb);
+            if constexpr (!kFp8) {
+              uint32_t slot;
+              if (!ring.claim(empty0, slot, ok, abort_flag, p.status)) continue;
+              if (rank == 0) mbar_expect_tx(bar(L::QK_FULL + slot), 2 * kUnitBytes);
+              const uint32_t dst = sbase + L::OffQKRing + slot * kUnitBytes, fb = leader_bar(L::QK_FULL + slot);
+              for (int i = 0; i < 2; ++i)
+                tma_load_2d_pair(dst + i * 8192, &P.map_pv, 64 * c, pg[i] >= 0 ? pg[i] * kPage : -kPage, fb);
+            } else if (c < kChunks - 1) {
+              // codes of columns [64c, 64c+64) of both pages: one staging slot
+              uint32_t slot;
+              if (!ring.claim(empty0, slot, ok, abort_flag, p.status)) continue;
+              const uint32_t dst = sbase + L::OffQSt + slot * kStageBytes, fb = bar(L::QST_FULL + slot);
+              mbar_arrive_tx_local(fb, kStageBytes);
+              for (int i = 0; i < 2; ++i) tma_load_3d(dst + i * 4096, &P.map_codes_qk, 64 * c, 0, pg[i], fb);
+            } else {
+              // k^R: one staging slot per page
+              for (int i = 0; i < 2; ++i) {
+                uint32_t slot;
+                if (!ring.claim(empty0, slot, ok, abort_flag, p.status)) continue;
+                const uint32_t dst = sbase + L::OffQSt + slot * kStageBytes, fb = bar(L::QST_FULL + slot);
+                mbar_arrive_tx_local(fb, kStageBytes);
+                tma_load_3d(dst, &P.map_kr, 0, 0, pg[i], fb);
+              }
+            }
           }
         }
         ++seg;
       }
     }
-  } else if (warp >= kPVProdWarp) {
+  } else if (warp >= L::PVProdWarp && warp < L::PVProdWarp + L::Producers) {
     // ------------------------------------------------------------------ TMA: PV
     if (lane == 0) {
-      RingProducer ring{bar(B_PV_FULL), bar(B_PV_EMPTY), leader_bar(B_PV_FULL), sbase + kOffPVRing, kPVSlots,
-                        kPVProducers, warp - kPVProdWarp};
+      RingProducer ring{kFp8 ? L::PStSlots : L::PVSlots, L::Producers, warp - L::PVProdWarp};
+      const uint32_t empty0 = kFp8 ? bar(L::PST_EMPTY) : bar(L::PV_EMPTY);
       const int x_pv = 128 * (int)rank;  // this CTA's 128 columns of an N=256 half
       SegmentWalker walk(p, w, t);
       Segment s;
@@ -480,32 +600,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int it = 0; it < n_tiles && ok; ++it) {
           const int pg0 = s.page_lo + it * kTilePages;
           const int npg = min(kTilePages, s.n_pages - it * kTilePages);
-          // page i outer, N-half j inner.  Rows past the visible keys and
-          // pages past the tile's end come from outside the tensor (zero
-          // fill), so 0 * (whatever the pool held) cannot reach O.
+          // page i outer, N-half j inner
           for (int i = 0; i < kTilePages; ++i) {
             const int valid = i < npg ? min(kPage, s.nvis - (pg0 + i) * kPage) : 0;
             const int page = valid > 0 ? page_of(s.b, pg0 + i) : 0;
             for (int j = 0; j < 2; ++j) {
-              uint32_t dst, fb;
-              if (!ring.claim(rank, dst, fb, ok, abort_flag, p.status)) continue;
-              for (int a = 0; a < 2; ++a) {
-                const int x = 256 * j + x_pv + 64 * a;
-                const uint32_t d = dst + a * 8192;
-                if (valid == kPage) {
-                  tma_load_2d_pair(d, &P.map_pv, x, page * kPage, fb);
-                } else if (valid <= 0) {
-                  tma_load_2d_pair(d, &P.map_pv, x, -kPage, fb);
-                } else {
-                  for (int q = 0; q < 4; ++q) {
-                    if (16 * q + 16 <= valid) {
-                      tma_load_2d_pair(d + q * 2048, &P.map_pv16, x, page * kPage + 16 * q, fb);
-                    } else if (16 * q >= valid) {
-                      tma_load_2d_pair(d + q * 2048, &P.map_pv16, x, -16, fb);
-                    } else {
-                      for (int k = 0; k < 16; ++k)
-                        tma_load_2d_pair(d + (16 * q + k) * 128, &P.map_row, x,
-                                         16 * q + k < valid ? page * kPage + 16 * q + k : -1, fb);
+              uint32_t slot;
+              if (!ring.claim(empty0, slot, ok, abort_flag, p.status)) continue;
+              const int x0 = 256 * j + x_pv;
+              if constexpr (kFp8) {
+                // the converters zero the rows past the visible keys
+                const uint32_t fb = bar(L::PST_FULL + slot);
+                mbar_arrive_tx_local(fb, kStageBytes);
+                tma_load_3d(sbase + L::OffPSt + slot * kStageBytes, &P.map_codes_pv, x0, 0, valid > 0 ? page : -1, fb);
+              } else {
+                // Rows past the visible keys and pages past the tile's end
+                // come from outside the tensor (zero fill), so 0 * (whatever
+                // the pool held) cannot reach O.
+                if (rank == 0) mbar_expect_tx(bar(L::PV_FULL + slot), 2 * kUnitBytes);
+                const uint32_t dst = sbase + L::OffPVRing + slot * kUnitBytes, fb = leader_bar(L::PV_FULL + slot);
+                for (int a = 0; a < 2; ++a) {
+                  const int x = x0 + 64 * a;
+                  const uint32_t d = dst + a * 8192;
+                  if (valid == kPage) {
+                    tma_load_2d_pair(d, &P.map_pv, x, page * kPage, fb);
+                  } else if (valid <= 0) {
+                    tma_load_2d_pair(d, &P.map_pv, x, -kPage, fb);
+                  } else {
+                    for (int q = 0; q < 4; ++q) {
+                      if (16 * q + 16 <= valid) {
+                        tma_load_2d_pair(d + q * 2048, &P.map_pv16, x, page * kPage + 16 * q, fb);
+                      } else if (16 * q >= valid) {
+                        tma_load_2d_pair(d + q * 2048, &P.map_pv16, x, -16, fb);
+                      } else {
+                        for (int k = 0; k < 16; ++k)
+                          tma_load_2d_pair(d + (16 * q + k) * 128, &P.map_row, x,
+                                           16 * q + k < valid ? page * kPage + 16 * q + k : -1, fb);
+                      }
                     }
                   }
                 }
@@ -515,25 +646,203 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == kQKWarp) {
+  } else if (kFp8 && warp >= L::QKConvWarp && warp < L::QKConvWarp + L::ConvWarps) {
+    // ------------------------------------------------- FP8: QK unit conversion
+    // Thread ct of the two warps converts 16-byte groups ct, ct+64, ... of
+    // the staged data into the unit (128-byte swizzle).
+    const int ct = (warp - L::QKConvWarp) * 32 + lane;
+    RingPos unit, stage;
+    uint32_t gt = 0;
+    const int y_pages = 2 * (int)rank;
+    SegmentWalker walk(p, w, t);
+    Segment s;
+    bool ok = true;
+    while (ok && walk.next(s)) {
+      if (s.n_pages == 0) continue;
+      const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
+      for (int it = 0; it < n_tiles && ok; ++it, ++gt) {
+        ok = mbar_wait(bar(L::SCL_FULL + (gt & 1)), (gt >> 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        const float* scl = reinterpret_cast<const float*>(smem + L::OffScl + (gt & 1) * kSclBytes) + y_pages * 256;
+#ifdef MLA_TC_TRACE
+        long long w_unit = 0, w_stage = 0, t_tile = clock64();
+#endif
+        for (int c = 0; c < kQKUnits && ok; ++c) {
+#ifdef MLA_TC_TRACE
+          long long tw = clock64();
+#endif
+          ok = mbar_wait(bar(L::QK_EMPTY + unit.slot), unit.phase ^ 1, abort_flag, p.status);
+#ifdef MLA_TC_TRACE
+          w_unit += clock64() - tw;
+          tw = clock64();
+#endif
+          if (!ok) break;
+          uint8_t* dstu = smem + L::OffQKRing + unit.slot * kUnitBytes;
+          if (c < kChunks - 1) {
+            // [2 pages][64 rows][64 codes]; the scale of columns [64c, 64c+64) is tile c/2
+            ok = mbar_wait(bar(L::QST_FULL + stage.slot), stage.phase, abort_flag, p.status);
+#ifdef MLA_TC_TRACE
+            w_stage += clock64() - tw;
+#endif
+            if (!ok) break;
+            const uint8_t* src = smem + L::OffQSt + stage.slot * kStageBytes;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int gi = k * 64 + ct, r = gi >> 2, q = gi & 3;  // r: unit row (page r/64)
+              const uint4 v = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
+              const __half2 s2 = __float2half2_rn(scl[r * 4 + (c >> 1)]);
+              uint32_t o[8];
+              e4m3x4_scaled(v.x, s2, o[0], o[1]);
+              e4m3x4_scaled(v.y, s2, o[2], o[3]);
+              e4m3x4_scaled(v.z, s2, o[4], o[5]);
+              e4m3x4_scaled(v.w, s2, o[6], o[7]);
+              uint8_t* rp = dstu + r * 128;
+              *reinterpret_cast<uint4*>(rp + (((2 * q) ^ (r & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+              *reinterpret_cast<uint4*>(rp + (((2 * q + 1) ^ (r & 7)) * 16)) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_local(bar(L::QST_EMPTY + stage.slot));
+            stage.advance(L::QStSlots);
+          } else {
+            // k^R: one staged page (64 rows x 64 bf16) per half of the unit
+            for (int i = 0; i < 2 && ok; ++i) {
+              ok = mbar_wait(bar(L::QST_FULL + stage.slot), stage.phase, abort_flag, p.status);
+              if (!ok) break;
+              const uint8_t* src = smem + L::OffQSt + stage.slot * kStageBytes;
+              uint8_t* dst = dstu + i * 8192;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int gi = k * 64 + ct, row = gi >> 3, u = gi & 7;
+                const uint4 v = *reinterpret_cast<const uint4*>(src + row * 128 + u * 16);
+                *reinterpret_cast<uint4*>(dst + row * 128 + ((u ^ (row & 7)) * 16)) =
+                    make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+              }
+              fence_proxy_async();
+              __syncwarp();
+              if (lane == 0) mbar_arrive_local(bar(L::QST_EMPTY + stage.slot));
+              stage.advance(L::QStSlots);
+            }
+            if (!ok) break;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(leader_bar(L::QK_FULL + unit.slot));
+          unit.advance(L::QKSlots);
+        }
+        if (!ok) break;
+#ifdef MLA_TC_TRACE
+        if (ct == 0) {
+          TC_TRACE_VAL(8, gt, w_unit);
+          TC_TRACE_VAL(9, gt, w_stage);
+          TC_TRACE_VAL(10, gt, clock64() - t_tile);
+          TC_TRACE(11, gt);
+        }
+#endif
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(bar(L::SCL_EMPTY + (gt & 1)));
+      }
+    }
+  } else if (kFp8 && warp >= L::PVConvWarp && warp < L::PVConvWarp + L::ConvWarps) {
+    // ------------------------------------------------- FP8: PV unit conversion
+    const int ct = (warp - L::PVConvWarp) * 32 + lane;
+    const int blk = (int)rank;  // + 2j: this CTA's 128 columns of half j are scale tile 2j + rank
+    RingPos unit, stage;
+    uint32_t gt = 0;
+    SegmentWalker walk(p, w, t);
+    Segment s;
+    bool ok = true;
+    while (ok && walk.next(s)) {
+      if (s.n_pages == 0) continue;
+      const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
+      for (int it = 0; it < n_tiles && ok; ++it, ++gt) {
+        ok = mbar_wait(bar(L::SCL_FULL + (gt & 1)), (gt >> 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        const float* scl_t = reinterpret_cast<const float*>(smem + L::OffScl + (gt & 1) * kSclBytes);
+        const int pg0 = s.page_lo + it * kTilePages;
+        const int npg = min(kTilePages, s.n_pages - it * kTilePages);
+#ifdef MLA_TC_TRACE
+        long long w_unit = 0, w_stage = 0, t_tile = clock64();
+#endif
+        for (int i = 0; i < kTilePages && ok; ++i) {
+          const int valid = i < npg ? min(kPage, s.nvis - (pg0 + i) * kPage) : 0;
+          const float* scl = scl_t + i * 256;
+          for (int j = 0; j < 2 && ok; ++j) {
+#ifdef MLA_TC_TRACE
+            long long tw = clock64();
+#endif
+            ok = mbar_wait(bar(L::PV_EMPTY + unit.slot), unit.phase ^ 1, abort_flag, p.status);
+            if (!ok) break;
+#ifdef MLA_TC_TRACE
+            w_unit += clock64() - tw;
+            tw = clock64();
+#endif
+            ok = mbar_wait(bar(L::PST_FULL + stage.slot), stage.phase, abort_flag, p.status);
+            if (!ok) break;
+#ifdef MLA_TC_TRACE
+            w_stage += clock64() - tw;
+#endif
+            const uint8_t* src = smem + L::OffPSt + stage.slot * kStageBytes;
+            uint8_t* dst = smem + L::OffPVRing + unit.slot * kUnitBytes;
+            // 64 rows x 128 codes -> two 64-column atoms (8 KB apart); rows
+            // past the visible keys are zero
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int gi = k * 64 + ct, row = gi >> 3, q = gi & 7;
+              uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+              if (row < valid) {
+                const uint4 v = *reinterpret_cast<const uint4*>(src + row * 128 + q * 16);
+                const __half2 s2 = __float2half2_rn(scl[row * 4 + 2 * j + blk]);
+                e4m3x4_scaled(v.x, s2, o[0], o[1]);
+                e4m3x4_scaled(v.y, s2, o[2], o[3]);
+                e4m3x4_scaled(v.z, s2, o[4], o[5]);
+                e4m3x4_scaled(v.w, s2, o[6], o[7]);
+              }
+              uint8_t* rp = dst + (q >> 2) * 8192 + row * 128;
+              const int u0 = 2 * (q & 3);
+              *reinterpret_cast<uint4*>(rp + ((u0 ^ (row & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+              *reinterpret_cast<uint4*>(rp + (((u0 + 1) ^ (row & 7)) * 16)) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive_local(bar(L::PST_EMPTY + stage.slot));
+              mbar_arrive_cluster(leader_bar(L::PV_FULL + unit.slot));
+            }
+            stage.advance(L::PStSlots);
+            unit.advance(L::PVSlots);
+          }
+        }
+        if (!ok) break;
+#ifdef MLA_TC_TRACE
+        if (ct == 0) {
+          TC_TRACE_VAL(12, gt, w_unit);
+          TC_TRACE_VAL(13, gt, w_stage);
+          TC_TRACE_VAL(14, gt, clock64() - t_tile);
+        }
+#endif
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(bar(L::SCL_EMPTY + (gt & 1)));
+      }
+    }
+  } else if (warp == L::QKWarp) {
     // ----------------------------------------------------------- MMA: S = Q K^T
     if (rank == 0 && lane == 0) {
-      RingConsumer ring{bar(B_QK_FULL), bar(B_QK_EMPTY), sbase + kOffQKRing, kQKSlots};
+      RingConsumer ring{bar(L::QK_FULL), bar(L::QK_EMPTY), L::QKSlots};
       SegmentWalker walk(p, w, t);
       Segment s;
       uint32_t g = 0, seg = 0;
       bool ok = true;
       // descriptors advance by adding (byte offset >> 4) to the start-address field
-      const uint64_t qdesc = sdesc(sbase + kOffQ, 16, 1024);      // chunk c: + 512 c; K-step: + 2
-      const uint64_t kdesc = sdesc(sbase + kOffQKRing, 16, 1024);  // slot: + 1024 slot
+      const uint64_t qdesc = sdesc(sbase + L::OffQ, 16, 1024);      // chunk c: + 512 c; K-step: + 2
+      const uint64_t kdesc = sdesc(sbase + L::OffQKRing, 16, 1024);  // slot: + 1024 slot
       while (ok && walk.next(s)) {
         if (s.n_pages == 0) continue;
-        ok = mbar_wait(bar(B_Q_FULL), seg & 1, abort_flag, p.status);
+        ok = mbar_wait(bar(L::Q_FULL), seg & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
         for (int it = 0; it < n_tiles && ok; ++it, ++g) {
-          ok = mbar_wait(bar(B_S_FREE + (g & 1)), ((g >> 1) & 1) ^ 1, abort_flag, p.status);
+          ok = mbar_wait(bar(L::S_FREE + (g & 1)), ((g >> 1) & 1) ^ 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
           const uint32_t sd = tmem + ((g & 1) ? kColS1 : kColS0);
@@ -543,38 +852,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = ring.wait_full(abort_flag, p.status);
             if (!ok) break;
             tc_fence_after();
-            const uint64_t a = qdesc + 512 * c, bb = kdesc + 1024 * ring.slot;
+            const uint64_t a = qdesc + 512 * c, bb = kdesc + 1024 * ring.pos.slot;
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)  // 16 columns = 32 bytes into the swizzled rows
               tc_mma(sd, a + 2 * k4, bb + 2 * k4, kIdescQK, (c | k4) ? 1u : 0u);
             ring.release();
           }
           if (!ok) break;
-          tc_commit_pair(bar(B_S_FULL + (g & 1)));
+          tc_commit_pair(bar(L::S_FULL + (g & 1)));
           TC_TRACE(1, g);
-          if (it == n_tiles - 1) tc_commit_pair(bar(B_Q_EMPTY));
+          if (it == n_tiles - 1) tc_commit_pair(bar(L::Q_EMPTY));
         }
         ++seg;
       }
     }
-  } else if (warp == kPVWarp) {
+  } else if (warp == L::PVWarp) {
     // ---------------------------------------------------------- MMA: O += P C
     if (rank == 0 && lane == 0) {
-      RingConsumer ring{bar(B_PV_FULL), bar(B_PV_EMPTY), sbase + kOffPVRing, kPVSlots};
+      RingConsumer ring{bar(L::PV_FULL), bar(L::PV_EMPTY), L::PVSlots};
       SegmentWalker walk(p, w, t);
       Segment s;
       uint32_t g = 0, seg = 0;
       bool ok = true;
-      const uint64_t vdesc = sdesc(sbase + kOffPVRing, 8192, 1024);  // slot: + 1024 slot; K-step: + 128
-      const uint64_t pdesc = sdesc(sbase + kOffP, 16, 1024);         // page sub-tile: + 512 i; K-step: + 2
+      const uint64_t vdesc = sdesc(sbase + L::OffPVRing, 8192, 1024);  // slot: + 1024 slot; K-step: + 128
+      const uint64_t pdesc = sdesc(sbase + L::OffP, 16, 1024);         // page sub-tile: + 512 i; K-step: + 2
       while (ok && walk.next(s)) {
         if (s.n_pages == 0) continue;
         const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
         for (int it = 0; it < n_tiles && ok; ++it, ++g) {
-          ok = mbar_wait(bar(B_P_FULL), g & 1, abort_flag, p.status);
+          ok = mbar_wait(bar(L::P_FULL), g & 1, abort_flag, p.status);
           if (!ok) break;
           if (it == 0 && seg > 0) {  // O of the previous segment must be read out first
-            ok = mbar_wait(bar(B_O_FREE), (seg - 1) & 1, abort_flag, p.status);
+            ok = mbar_wait(bar(L::O_FREE), (seg - 1) & 1, abort_flag, p.status);
             if (!ok) break;
           }
           tc_fence_after();
@@ -588,26 +897,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               tc_fence_after();
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                tc_mma(tmem + (j ? kColO1 : kColO0), pdesc + 512 * i + 2 * ks, vdesc + 1024 * ring.slot + 128 * ks,
-                       kIdescPV, (it == 0 && i == 0 && ks == 0) ? 0u : 1u);
+                tc_mma(tmem + (j ? kColO1 : kColO0), pdesc + 512 * i + 2 * ks,
+                       vdesc + 1024 * ring.pos.slot + 128 * ks, kIdescPV, (it == 0 && i == 0 && ks == 0) ? 0u : 1u);
               ring.release();
             }
           if (!ok) break;
-          tc_commit_pair(bar(B_O_DONE));
+          tc_commit_pair(bar(L::O_DONE));
           TC_TRACE(3, g);
         }
         ++seg;
       }
     }
-  } else {
+  } else if (warp < 4) {
     // ------------------------------------------------------- softmax, epilogue
     // Thread L (TMEM lane) holds head hl of this CTA; lanes 0-63 see the
     // keys of pages 0-1 of a tile, lanes 64-127 those of pages 2-3 (the QK B
     // operand holds the leader's two pages in N columns [0,128), the peer's in
     // [128,256); 2x2 layout).  S is read twice from TMEM: once for the max,
     // once for the probabilities, so that few registers hold scores at a time.
-    const int L = warp * 32 + lane;
-    const int hl = L & 63, half = L >> 6;
+    const int Lt = warp * 32 + lane;
+    const int hl = Lt & 63, half = Lt >> 6;
     const int head = kHalfHeads * (int)rank + hl;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     SegmentWalker walk(p, w, t);
@@ -627,7 +936,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       float m_ref = -INFINITY, l_part = 0.f;
       const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
       for (int it = 0; it < n_tiles; ++it, ++g) {
-        ok = mbar_wait(bar(B_S_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.status);
+        ok = mbar_wait(bar(L::S_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.status);
         __syncwarp();
         if (!ok) break;
         if (threadIdx.x == 0) TC_TRACE(4, g);
@@ -669,7 +978,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         // the previous tile's PV MMAs read P and write O: wait for them
         if (g >= 1) {
-          ok = mbar_wait(bar(B_O_DONE), (g - 1) & 1, abort_flag, p.status);
+          ok = mbar_wait(bar(L::O_DONE), (g - 1) & 1, abort_flag, p.status);
           __syncwarp();
           if (!ok) break;
           tc_fence_after();
@@ -703,12 +1012,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j) {
             const float e0 = 2 * j < nv[q] ? fast_exp2(__uint_as_float(sr[2 * j]) * p.scale_log2 - m_ref) : 0.f;
             const float e1 = 2 * j + 1 < nv[q] ? fast_exp2(__uint_as_float(sr[2 * j + 1]) * p.scale_log2 - m_ref) : 0.f;
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-            const float2 f2 = __bfloat1622float2(h2);
+            PT h2;
+            float2 f2;
+            if constexpr (kFp8) {
+              h2 = __floats2half2_rn(e0, e1);
+              f2 = __half22float2(h2);
+            } else {
+              h2 = __floats2bfloat162_rn(e0, e1);
+              f2 = __bfloat1622float2(h2);
+            }
             psum += f2.x + f2.y;
             pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
           }
-          uint8_t* prow = smem + kOffP + (2 * half + q) * 8192 + hl * 128;
+          uint8_t* prow = smem + L::OffP + (2 * half + q) * 8192 + hl * 128;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             *reinterpret_cast<uint4*>(prow + ((u ^ (hl & 7)) * 16)) =
@@ -718,15 +1034,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // S of this tile is consumed
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_bar(B_S_FREE + (g & 1)));
+        if (lane == 0) mbar_arrive_cluster(leader_bar(L::S_FREE + (g & 1)));
         fence_proxy_async();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (threadIdx.x == 0) TC_TRACE(6, g);
-        if (lane == 0) mbar_arrive_cluster(leader_bar(B_P_FULL));
+        if (lane == 0) mbar_arrive_cluster(leader_bar(L::P_FULL));
       }
       if (!ok) break;
       // epilogue: wait for the last PV, normalise, write the split's partial
-      ok = mbar_wait(bar(B_O_DONE), (g - 1) & 1, abort_flag, p.status);
+      ok = mbar_wait(bar(L::O_DONE), (g - 1) & 1, abort_flag, p.status);
       __syncwarp();
       if (!ok) break;
       tc_fence_after();
@@ -752,7 +1068,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (half == 0) p.lse_part[slot * kHeads + head] = l_tot > 0.f ? m_ref + __log2f(l_tot) : -INFINITY;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_bar(B_O_FREE));
+      if (lane == 0) mbar_arrive_cluster(leader_bar(L::O_FREE));
     }
   }
 
@@ -761,7 +1077,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   tc_fence_after();
-  if (warp == kQKWarp)
+  if (warp == L::QKWarp)
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
@@ -784,17 +1100,33 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 map over [rows][576] with a (64 columns x box_rows) box, 128-byte swizzle
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+// 2-D 16-bit map over [rows][576] with a (64 columns x box_rows) box, 128-byte swizzle
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows,
+              CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)kD, rows};
   const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
   const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// 3-D map over a page sub-block: [pages][64 rows][row_elems], unswizzled box
+// (box_x x 64 rows x 1 page)
+bool make_page_map(CUtensorMap* m, const void* base, CUtensorMapDataType type, uint32_t elem_bytes,
+                   uint64_t row_elems, uint64_t num_pages, uint64_t page_bytes, uint32_t box_x) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {row_elems, (cuuint64_t)kPage, num_pages};
+  const cuuint64_t strides[2] = {row_elems * elem_bytes, page_bytes};
+  const cuuint32_t box[3] = {box_x, (cuuint32_t)kPage, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, type, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 bool device_is_sm100() {
@@ -805,12 +1137,25 @@ bool device_is_sm100() {
   return major == 10 && minor == 0;
 }
 
+template <bool kFp8>
+cudaError_t launch_variant(const TcParams& tp, int pairs, cudaStream_t st) {
+  using L = TcLayout<kFp8>;
+  cudaError_t e =
+      cudaFuncSetAttribute(decode_tc_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SmemBytes);
+  if (e != cudaSuccess) return e;
+  decode_tc_kernel<kFp8><<<2 * pairs, L::Threads, L::SmemBytes, st>>>(tp);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool decode_tc_supported(const mla_dims& d, int n_q) {
   return d.n_heads == kHeads && d.d_c == kDC && d.d_rope == kDR && d.page_size == kPage &&
-         d.act_dtype == MLA_BF16 && d.cache_dtype == MLA_BF16 && n_q >= 1 && n_q <= 8 && device_is_sm100();
+         d.act_dtype == MLA_BF16 && (d.cache_dtype == MLA_BF16 || d.cache_dtype == MLA_FP8_E4M3) && n_q >= 1 &&
+         n_q <= 8 && device_is_sm100();
 }
+
+bool decode_tc_wants_f16_queries(const mla_dims& d) { return d.cache_dtype == MLA_FP8_E4M3; }
 
 int decode_tc_auto_splits(int num_sms, int n_q) {
   const int pairs = num_sms / 2;
@@ -820,17 +1165,29 @@ int decode_tc_auto_splits(int num_sms, int n_q) {
 
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st) {
   TcParams tp;
+  memset(&tp, 0, sizeof(tp));
   tp.p = p;
+  const bool fp8 = p.d.cache_dtype == MLA_FP8_E4M3;
+  const uint64_t q_rows = (uint64_t)p.batch * p.n_q * kHeads;
+  if (fp8) {
+    const Fp8Page fp = fp8_page(kPage, kDC, kDR);
+    if (!make_map(&tp.map_q, p.q_abs, q_rows, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !make_page_map(&tp.map_codes_qk, p.pool, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kDC, p.num_pages, p.page_bytes,
+                       64) ||
+        !make_page_map(&tp.map_codes_pv, p.pool, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kDC, p.num_pages, p.page_bytes,
+                       128) ||
+        !make_page_map(&tp.map_kr, p.pool + fp.kr_off, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDR, p.num_pages,
+                       p.page_bytes, 64) ||
+        !make_page_map(&tp.map_scl, p.pool + fp.sc_off, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDC / 128, p.num_pages,
+                       p.page_bytes, kDC / 128))
+      return cudaErrorInvalidValue;
+    return launch_variant<true>(tp, p.splits * p.n_q, st);
+  }
   const uint64_t pool_rows = (uint64_t)p.num_pages * kPage;
-  if (!make_map(&tp.map_q, p.q_abs, (uint64_t)p.batch * p.n_q * kHeads, 64) ||
-      !make_map(&tp.map_pv, p.pool, pool_rows, 64) ||
+  if (!make_map(&tp.map_q, p.q_abs, q_rows, 64) || !make_map(&tp.map_pv, p.pool, pool_rows, 64) ||
       !make_map(&tp.map_pv16, p.pool, pool_rows, 16) || !make_map(&tp.map_row, p.pool, pool_rows, 1))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  const int pairs = p.splits * p.n_q;
-  decode_tc_kernel<<<2 * pairs, kThreads, kSmemBytes, st>>>(tp);
-  return cudaGetLastError();
+  return launch_variant<false>(tp, p.splits * p.n_q, st);
 }
 
 }  // namespace mla

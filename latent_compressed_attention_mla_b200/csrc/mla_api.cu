@@ -178,8 +178,9 @@ int mla_decode(const mla_dims* dims, const void* q_nope, const void* q_rope, con
   int* status = status_ptr();
   trace_record(MLA_TRACE_ABSORB, false, st);
   const int n_slots = batch + W - 1;
+  const bool q_f16 = path == 1 && decode_tc_wants_f16_queries(*dims);
   cudaError_t e = launch_absorb_and_plan(*dims, q_nope, q_rope, W_uk, seq_lens, batch, n_q, max_pages, W, ws + L.off_q,
-                                         plan, reinterpret_cast<float*>(ws + L.off_lse),
+                                         q_f16, plan, reinterpret_cast<float*>(ws + L.off_lse),
                                          (size_t)n_q * n_slots * dims->n_heads, status, st);
   trace_record(MLA_TRACE_ABSORB, true, st);
   if (e != cudaSuccess) return MLA_ERR_LAUNCH;

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -26,6 +27,21 @@ __device__ __forceinline__ void record_status(int* status, int code) {
 }
 
 // ----------------------------------------------------------------------------
+// FP8 cache page: [page_size][d_c] e4m3 codes, then [page_size][d_rope] bf16
+// k^R, then [page_size][d_c/128] fp32 scales, each sub-block 128-byte aligned.
+// ----------------------------------------------------------------------------
+struct Fp8Page {
+  size_t kr_off, sc_off;
+};
+__host__ __device__ inline size_t a128(size_t x) { return (x + 127) / 128 * 128; }
+__host__ __device__ inline Fp8Page fp8_page(int page_size, int d_c, int d_rope) {
+  Fp8Page p;
+  p.kr_off = a128((size_t)page_size * d_c);
+  p.sc_off = a128(p.kr_off + (size_t)page_size * d_rope * 2);
+  return p;
+}
+
+// ----------------------------------------------------------------------------
 // Element access
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ float to_f(float x) { return x; }
@@ -36,6 +52,7 @@ template <> __device__ __forceinline__ float from_f<float>(float x) { return x; 
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
+template <> __device__ __forceinline__ __half from_f<__half>(float x) { return __float2half_rn(x); }
 
 // Load 8 consecutive bf16 (one 16-byte vector) as floats.
 __device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
@@ -159,12 +176,14 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
 // absorb + split plan (+ empty-split initialisation of the lse slots)
 cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const void* q_rope, const void* W_uk,
                                    const int32_t* seq_lens, int batch, int n_q, int max_pages, int splits,
-                                   void* q_abs, int32_t* plan, float* lse_part, size_t lse_count, int* status,
-                                   cudaStream_t st);
+                                   void* q_abs, bool q_abs_f16, int32_t* plan, float* lse_part, size_t lse_count,
+                                   int* status, cudaStream_t st);
 
 cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t st);
 
 bool decode_tc_supported(const mla_dims& d, int n_q);
+// the tensor-core path for this cache reads the absorbed queries as f16
+bool decode_tc_wants_f16_queries(const mla_dims& d);
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st);
 int decode_tc_auto_splits(int num_sms, int n_q);
 
