@@ -8,7 +8,13 @@
 // The output is in the activation type, or f16 when the decode path reads
 // f16 queries (FP8 cache on the tensor cores).
 //
-// One CTA per (head, 16-vector slice of d_c).  Thread (cg, dg) loads the
+// bf16 activations (absorb_tc_kernel): one CTA per head stages W^UK_h (d_nope x
+// d_c, 128 KB at DeepSeek-V3 dims) and the head's q^C rows in swizzled shared
+// memory with cp.async and multiplies them with mma.sync m16n8k16 (fp32
+// accumulation); the eight warps split the d_c output columns.  The kernel is
+// bound by the 16.8 MB of W^UK read once from HBM.
+//
+// fp32 activations (absorb_kernel): one CTA per (head, 16-vector slice of d_c).  Thread (cg, dg) loads the
 // 16-byte vectors of W^UK_h for its column group cg and its rows d in group
 // dg, all loads issued up front, and keeps them in registers for every token
 // of the step; partial sums over the row groups are reduced in shared memory.
@@ -19,6 +25,7 @@
 // per-split log-sum-exp slots with -inf, the value of a split that holds no
 // key of a sequence.
 #include "mla_internal.cuh"
+#include "mma_tile.cuh"
 
 namespace mla {
 
@@ -219,9 +226,118 @@ __global__ void __launch_bounds__(128) absorb_kernel(const AbsorbArgs a) {
   }
 }
 
+// RoPE of q^R at the query's own position for head h (all tokens).
+template <typename T, typename TO>
+__device__ void rope_queries(const AbsorbArgs& a, int h) {
+  const int D = a.d_c + a.d_rope, M = a.batch * a.n_q, half = a.d_rope >> 1;
+  const T* qr = static_cast<const T*>(a.q_rope);
+  TO* qa = static_cast<TO*>(a.q_abs);
+  for (int i = threadIdx.x; i < M * half; i += blockDim.x) {
+    const int m = i / half, k = i % half;
+    const int b = m / a.n_q, t = m % a.n_q;
+    const int p = a.seq_lens[b] - a.n_q + t;
+    float cs, sn;
+    rope_cos_sin(p, k, half, a.rope_base, &cs, &sn);
+    const T* src = qr + ((size_t)m * a.n_heads + h) * a.d_rope;
+    const float x1 = to_f(src[k]), x2 = to_f(src[half + k]);
+    TO* dst = qa + ((size_t)m * a.n_heads + h) * D + a.d_c;
+    dst[k] = from_f<TO>(x1 * cs - x2 * sn);
+    dst[half + k] = from_f<TO>(x2 * cs + x1 * sn);
+  }
+}
+
+constexpr int kTcThreads = 256;
+constexpr int kTcMaxTok = 256;  // query rows staged per pass
+
+__device__ __forceinline__ void store2(__nv_bfloat16* p, float x, float y) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(x, y);
+}
+__device__ __forceinline__ void store2(__half* p, float x, float y) {
+  *reinterpret_cast<__half2*>(p) = __floats2half2_rn(x, y);
+}
+
+// q~[m, h, :] = q^C[m, h, :] . W^UK_h for bf16 activations; d_nope % 64 == 0
+// (swizzle groups), d_c % 128 == 0 and <= 1024 (eight warps, at most eight
+// 16-column pairs each), W^UK_h in shared memory.
+template <typename TO>
+__global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const AbsorbArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int h = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int dn = a.d_nope, dc = a.d_c, D = a.d_c + a.d_rope, M = a.batch * a.n_q;
+  const int wu = dc / 8, au = dn / 8;  // 16-byte units per row of W^UK_h and of q^C
+  uint8_t* Ws = smem;
+  uint8_t* As = smem + (size_t)dn * dc * 2;
+
+  if (h == 0) build_plan(a);
+  {
+    const size_t nblk = gridDim.x, bid = blockIdx.x;
+    for (size_t i = bid * kTcThreads + tid; i < a.lse_count; i += nblk * kTcThreads) a.lse_part[i] = -INFINITY;
+  }
+  // W^UK_h, rows d (K) x columns c (N)
+  const __nv_bfloat16* Wh = static_cast<const __nv_bfloat16*>(a.W_uk) + (size_t)h * dn * dc;
+  for (int i = tid; i < dn * wu; i += kTcThreads) {
+    const int r = i / wu, u = i % wu;
+    cp_async16(smem_addr(Ws) + swz(r, u, wu), Wh + (size_t)r * dc + u * 8);
+  }
+  cp_async_commit();
+  const __nv_bfloat16* qn = static_cast<const __nv_bfloat16*>(a.q_nope);
+  TO* qa = static_cast<TO*>(a.q_abs);
+  const int ncols = dc / 8;  // columns per warp
+  for (int m0 = 0; m0 < M; m0 += kTcMaxTok) {
+    const int mc = min(kTcMaxTok, M - m0), mpad = (mc + 15) & ~15;
+    __syncthreads();  // previous pass done with As
+    for (int i = tid; i < mpad * au; i += kTcThreads) {
+      const int r = i / au, u = i % au;
+      const uint32_t dst = smem_addr(As) + swz(r, u, au);
+      if (r < mc)
+        cp_async16(dst, qn + ((size_t)(m0 + r) * a.n_heads + h) * dn + u * 8);
+      else
+        *reinterpret_cast<uint4*>(As + swz(r, u, au)) = make_uint4(0, 0, 0, 0);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    for (int mt = 0; mt < mpad; mt += 16) {
+      float acc[16][4];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+      for (int k0 = 0; k0 < dn; k0 += 16) {
+        uint32_t af[4];
+        load_a(As, au, mt, k0, lane, af);
+#pragma unroll
+        for (int np = 0; np < 8; ++np) {
+          if (np * 16 >= ncols) break;
+          uint32_t b00, b01, b10, b11;
+          load_b_kn(Ws, wu, k0, warp * ncols + np * 16, lane, b00, b01, b10, b11);
+          mma_bf16(acc[2 * np], af, b00, b01);
+          mma_bf16(acc[2 * np + 1], af, b10, b11);
+        }
+      }
+      // accumulator (row g / g+8, columns 2q, 2q+1 of each n8 tile)
+      const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j * 8 >= ncols) break;
+        const int col = warp * ncols + j * 8 + 2 * q;
+        const int r0 = mt + g, r1 = mt + g + 8;
+        if (r0 < mc) store2(qa + ((size_t)(m0 + r0) * a.n_heads + h) * D + col, acc[j][0], acc[j][1]);
+        if (r1 < mc) store2(qa + ((size_t)(m0 + r1) * a.n_heads + h) * D + col, acc[j][2], acc[j][3]);
+      }
+    }
+  }
+  rope_queries<__nv_bfloat16, TO>(a, h);
+}
+
 }  // namespace
 
 int absorb_max_d_nope() { return kDG * kMaxRows; }
+
+// shapes of the tensor-core absorption: W^UK_h and 256 staged query rows fit
+// in shared memory, columns split over eight warps in 16-column pairs
+bool absorb_tc_fits(const mla_dims& d) {
+  return d.d_nope % 64 == 0 && d.d_c % 128 == 0 && d.d_c <= 1024 &&
+         (size_t)d.d_nope * d.d_c * 2 + (size_t)kTcMaxTok * d.d_nope * 2 <= 227 * 1024;
+}
 
 cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const void* q_rope, const void* W_uk,
                                    const int32_t* seq_lens, int batch, int n_q, int max_pages, int splits,
@@ -247,6 +363,22 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
   a.lse_part = lse_part;
   a.lse_count = lse_count;
   a.status = status;
+  // the tensor-core kernel stages q^C with 16-byte copies
+  if (d.act_dtype == MLA_BF16 && absorb_tc_fits(d) && (reinterpret_cast<uintptr_t>(q_nope) & 15u) == 0) {
+    const size_t smem = (size_t)d.d_nope * d.d_c * 2 + (size_t)kTcMaxTok * d.d_nope * 2;
+    cudaError_t e;
+    if (q_abs_f16) {
+      e = cudaFuncSetAttribute(absorb_tc_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      absorb_tc_kernel<__half><<<d.n_heads, kTcThreads, smem, st>>>(a);
+    } else {
+      e = cudaFuncSetAttribute(absorb_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+      if (e != cudaSuccess) return e;
+      absorb_tc_kernel<__nv_bfloat16><<<d.n_heads, kTcThreads, smem, st>>>(a);
+    }
+    return cudaGetLastError();
+  }
   const int vec = d.act_dtype == MLA_F32 ? 4 : 8;
   const dim3 grid(d.n_heads, (d.d_c + kCG * vec - 1) / (kCG * vec));
   if (d.act_dtype == MLA_F32)

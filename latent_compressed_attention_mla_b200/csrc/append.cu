@@ -12,10 +12,22 @@
 //   the k^R rows own one rotation pair (i, i + d_rope/2) each, so they apply
 //   RoPE themselves.  For fp32/bf16 caches every value is rounded and stored into
 //   its paged slot here: one kernel per append.
+// append_tc (bf16 activations, bf16 or FP8 cache): the same projection as a
+//   split-K GEMM on the tensor cores.  The d_c + d_rope outputs form 32-wide
+//   tiles; a cluster of eight CTAs owns a tile, each CTA one eighth of
+//   d_model: its weight slice and the tokens' h slice are staged in swizzled
+//   shared memory with cp.async and multiplied with mma.sync m16n8k16 (fp32
+//   accumulation).  The eight partial sums are reduced over distributed shared
+//   memory, each CTA finishing 1/8 of the tokens (RoPE, rounding, paged store),
+//   so no workspace is needed.  The k^R tiles hold rotation pairs (i, i +
+//   d_rope/2) in columns (j, j + 16), so RoPE stays inside a tile.
 // append_fp8_finalize: FP8 caches need the amax of each 128-wide tile of c, a
 //   reduction across CTAs, so the projection leaves c in fp32 scratch and one
 //   CTA per token quantises it.
+#include <cooperative_groups.h>
+
 #include "mla_internal.cuh"
+#include "mma_tile.cuh"
 
 namespace mla {
 
@@ -218,6 +230,132 @@ __global__ void __launch_bounds__(128) append_fp8_finalize_kernel(const AppendAr
   }
 }
 
+constexpr int kTcCluster = 8;   // CTAs per output tile (d_model split)
+constexpr int kTcTile = 32;     // outputs per tile
+constexpr int kTcThreads = 256;
+constexpr int kTcMb = 64;       // tokens per pass
+
+size_t append_tc_smem(const mla_dims& d) {
+  const size_t ks = (size_t)d.d_model / kTcCluster;
+  return (size_t)kTcTile * ks * 2 + (size_t)kTcMb * ks * 2 + (size_t)4 * kTcMb * kTcTile * 4;
+}
+
+// bf16 activations; d_model % (8 * 64) == 0, d_c % 32 == 0, d_rope % 32 == 0.
+template <int CACHE>
+__global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads, 1)
+    append_tc_kernel(const AppendArgs a) {
+  namespace cg = cooperative_groups;
+  extern __shared__ __align__(128) uint8_t smem_tc[];
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank(), tile = blockIdx.x / kTcCluster;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int K = a.d_model, ks = K / kTcCluster, ku = ks / 8, k_lo = rank * ks;
+  const int n_c_tiles = a.d_c / kTcTile, half = a.d_rope / 2;
+  const bool is_kr = tile >= n_c_tiles;
+  const int kr_tile = tile - n_c_tiles;
+  uint8_t* Ws = smem_tc;
+  uint8_t* Hs = Ws + (size_t)kTcTile * ks * 2;
+  float* Ps = reinterpret_cast<float*>(Hs + (size_t)kTcMb * ks * 2);  // [4][kTcMb][kTcTile]
+  const __nv_bfloat16* Wd = static_cast<const __nv_bfloat16*>(a.W_dkv);
+  const __nv_bfloat16* Wk = static_cast<const __nv_bfloat16*>(a.W_kr);
+  const __nv_bfloat16* H = static_cast<const __nv_bfloat16*>(a.h);
+  // output index of tile column j: a row of W_dkv, or a rotation pair member of W_kr
+  auto out_idx = [&](int j) -> int { return is_kr ? (j < 16 ? 16 * kr_tile + j : half + 16 * kr_tile + j - 16)
+                                                  : tile * kTcTile + j; };
+  for (int i = tid; i < kTcTile * ku; i += kTcThreads) {
+    const int r = i / ku, u = i % ku;
+    const __nv_bfloat16* src = (is_kr ? Wk : Wd) + (size_t)out_idx(r) * K + k_lo + u * 8;
+    cp_async16(smem_addr(Ws) + swz(r, u, ku), src);
+  }
+  cp_async_commit();
+  const Fp8Page fp = fp8_page(a.page_size, a.d_c, a.d_rope);
+  const int M = a.n_tokens, nk = ks / 16;
+  for (int m0 = 0; m0 < M; m0 += kTcMb) {
+    const int mc = min(kTcMb, M - m0), mpad = (mc + 15) & ~15;
+    const int combos = (mpad / 16) * 2, kparts = 8 / combos;  // warps per (m16, n16) pair split the K slice
+    for (int i = tid; i < mpad * ku; i += kTcThreads) {
+      const int r = i / ku, u = i % ku;
+      if (r < mc)
+        cp_async16(smem_addr(Hs) + swz(r, u, ku), H + (size_t)(m0 + r) * K + k_lo + u * 8);
+      else
+        *reinterpret_cast<uint4*>(Hs + swz(r, u, ku)) = make_uint4(0, 0, 0, 0);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    {
+      const int combo = warp % combos, kp = warp / combos;
+      if (kp < kparts) {
+        const int mt = (combo >> 1) * 16, nt = (combo & 1) * 16, per = nk / kparts;
+        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int kk = kp * per; kk < (kp + 1) * per; ++kk) {
+          uint32_t af[4], b00, b01, b10, b11;
+          load_a(Hs, ku, mt, kk * 16, lane, af);
+          load_b_nk(Ws, ku, kk * 16, nt, lane, b00, b01, b10, b11);
+          mma_bf16(acc0, af, b00, b01);
+          mma_bf16(acc1, af, b10, b11);
+        }
+        const int g = lane >> 2, q = lane & 3;
+        float* P = Ps + (size_t)kp * kTcMb * kTcTile;
+        const int c0 = nt + 2 * q;
+        P[(mt + g) * kTcTile + c0] = acc0[0];
+        P[(mt + g) * kTcTile + c0 + 1] = acc0[1];
+        P[(mt + g + 8) * kTcTile + c0] = acc0[2];
+        P[(mt + g + 8) * kTcTile + c0 + 1] = acc0[3];
+        P[(mt + g) * kTcTile + c0 + 8] = acc1[0];
+        P[(mt + g) * kTcTile + c0 + 9] = acc1[1];
+        P[(mt + g + 8) * kTcTile + c0 + 8] = acc1[2];
+        P[(mt + g + 8) * kTcTile + c0 + 9] = acc1[3];
+      }
+    }
+    __syncthreads();
+    if (kparts > 1)
+      for (int i = tid; i < mpad * kTcTile; i += kTcThreads) {
+        float v = Ps[i];
+        for (int kp = 1; kp < kparts; ++kp) v += Ps[(size_t)kp * kTcMb * kTcTile + i];
+        Ps[i] = v;
+      }
+    cl.sync();  // every CTA's partial tile is complete
+    // this CTA finishes rows [rank * rows, (rank + 1) * rows) of the tile
+    const int rows = mpad / kTcCluster;
+    const int per_row = is_kr ? kTcTile / 2 : kTcTile;
+    for (int e = tid; e < rows * per_row; e += kTcThreads) {
+      const int r = rank * rows + e / per_row, j = e % per_row;
+      if (r >= mc) continue;
+      float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+      for (int src = 0; src < kTcCluster; ++src) {
+        const float* P = cl.map_shared_rank(Ps, src);
+        v0 += P[r * kTcTile + j];
+        if (is_kr) v1 += P[r * kTcTile + j + 16];
+      }
+      const int n = m0 + r;
+      int prow = 0, position = 0;
+      const int page = token_slot(a, n, &prow, &position);
+      if (page < 0) continue;
+      uint8_t* pg = a.pool + (size_t)page * a.page_bytes;
+      if (!is_kr) {
+        const int c = tile * kTcTile + j;
+        if (CACHE == MLA_FP8_E4M3)
+          a.raw[(size_t)n * a.d_c + c] = v0;
+        else
+          reinterpret_cast<__nv_bfloat16*>(pg)[(size_t)prow * (a.d_c + a.d_rope) + c] = __float2bfloat16_rn(v0);
+      } else {
+        const int i = 16 * kr_tile + j;
+        float cs, sn;
+        rope_cos_sin(position, i, half, a.rope_base, &cs, &sn);
+        const float y1 = v0 * cs - v1 * sn, y2 = v1 * cs + v0 * sn;
+        __nv_bfloat16* kr = CACHE == MLA_FP8_E4M3
+                                ? reinterpret_cast<__nv_bfloat16*>(pg + fp.kr_off) + (size_t)prow * a.d_rope
+                                : reinterpret_cast<__nv_bfloat16*>(pg) + (size_t)prow * (a.d_c + a.d_rope) + a.d_c;
+        kr[i] = __float2bfloat16_rn(y1);
+        kr[i + half] = __float2bfloat16_rn(y2);
+      }
+    }
+    cl.sync();  // peers are done reading this CTA's partials before the next pass
+  }
+}
+
 }  // namespace
 
 size_t cache_page_bytes(const mla_dims& d) {
@@ -264,7 +402,19 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
   const int grid = (d.d_c + kRows - 1) / kRows + d.d_rope / 2;
   trace_record(MLA_TRACE_APPEND_PROJECT, false, st);
 #define MLA_PROJ(T, K) append_project_kernel<T, K><<<grid, 256, 0, st>>>(a)
-  if (d.act_dtype == MLA_F32) {
+  const bool tc = d.act_dtype == MLA_BF16 && d.cache_dtype != MLA_F32 && d.d_model % (kTcCluster * 64) == 0 &&
+                  d.d_c % kTcTile == 0 && d.d_rope % kTcTile == 0 && append_tc_smem(d) <= 227 * 1024;
+  if (tc) {
+    const size_t smem = append_tc_smem(d);
+    const int tgrid = (d.d_c / kTcTile + d.d_rope / kTcTile) * kTcCluster;
+    if (d.cache_dtype == MLA_BF16) {
+      cudaFuncSetAttribute(append_tc_kernel<MLA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      append_tc_kernel<MLA_BF16><<<tgrid, kTcThreads, smem, st>>>(a);
+    } else {
+      cudaFuncSetAttribute(append_tc_kernel<MLA_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      append_tc_kernel<MLA_FP8_E4M3><<<tgrid, kTcThreads, smem, st>>>(a);
+    }
+  } else if (d.act_dtype == MLA_F32) {
     if (d.cache_dtype == MLA_F32) MLA_PROJ(float, MLA_F32);
     else if (d.cache_dtype == MLA_BF16) MLA_PROJ(float, MLA_BF16);
     else MLA_PROJ(float, MLA_FP8_E4M3);

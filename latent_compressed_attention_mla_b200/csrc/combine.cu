@@ -6,7 +6,14 @@
 // Cache by 93%", "3. Decoupled RoPE and Matrix Absorption"; decoding module
 // step 5).
 //
-// One CTA (8 warps) per head, kTok tokens per pass:
+// bf16 activations (combine_tc_kernel): one CTA per head stages W^UV_h (d_v x
+// d_c, 128 KB at DeepSeek-V3 dims) in swizzled shared memory with cp.async
+// while its warps merge the splits of 64 tokens at a time (warp per token,
+// lanes over latent columns) into a bf16 u tile; mma.sync m16n8k16 then forms
+// o = u . W^UV_h^T with fp32 accumulation.
+//
+// fp32 activations (combine_kernel): one CTA (8 warps) per head, kTok tokens
+// per pass:
 //   1. warp m merges token m: the run of splits overlapping the token's
 //      sequence comes from the plan; lanes take splits, warp max / sum give
 //      the weights (empty splits hold lse = -inf and weigh 0);
@@ -14,6 +21,7 @@
 //   3. warps take rows of W^UV_h, each lane holding 16-byte vectors of the row,
 //      and dot them with every token's u (warp-shuffle reduction).
 #include "mla_internal.cuh"
+#include "mma_tile.cuh"
 
 namespace mla {
 
@@ -119,6 +127,117 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(
   }
 }
 
+constexpr int kTcTok = 64;  // tokens merged per pass (rows of the u tile)
+
+size_t combine_tc_smem(const mla_dims& d) {
+  return (size_t)d.d_v * d.d_c * 2 + (size_t)kTcTok * d.d_c * 2 + (size_t)(kThreads / 32) * kMaxSplits * 4;
+}
+
+// bf16 activations: d_c % 128 == 0 (lanes x 4 columns, swizzle groups),
+// d_v % 16 == 0 (16-column pairs over the eight warps).
+__global__ void __launch_bounds__(kThreads) combine_tc_kernel(
+    const __nv_bfloat16* __restrict__ W_uv, int n_heads, int d_c, int d_v, int batch, int n_q,
+    const int32_t* __restrict__ plan, const float* __restrict__ o_part, const float* __restrict__ lse_part,
+    __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out) {
+  extern __shared__ __align__(128) uint8_t smem_tc[];
+  const int h = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cu = d_c / 8;  // 16-byte units per row of W^UV_h and of u
+  uint8_t* Ws = smem_tc;
+  uint8_t* Us = smem_tc + (size_t)d_v * d_c * 2;
+  float* wgt = reinterpret_cast<float*>(Us + (size_t)kTcTok * d_c * 2) + warp * kMaxSplits;
+  const int M = batch * n_q;
+  const int splits = plan[batch + 2];
+  const int n_slots = batch + splits - 1;  // slot stride of the decode that wrote the partials
+
+  // W^UV_h: rows j (N) x columns c (K)
+  const __nv_bfloat16* Wh = W_uv + (size_t)h * d_v * d_c;
+  for (int i = tid; i < d_v * cu; i += kThreads) {
+    const int r = i / cu, u = i % cu;
+    cp_async16(smem_addr(Ws) + swz(r, u, cu), Wh + (size_t)r * d_c + u * 8);
+  }
+  cp_async_commit();
+
+  for (int m0 = 0; m0 < M; m0 += kTcTok) {
+    const int mc = min(kTcTok, M - m0), mpad = (mc + 15) & ~15;
+    __syncthreads();  // previous pass done with Us
+    // merge: warp per token
+    for (int mi = warp; mi < mpad; mi += kThreads / 32) {
+      if (mi >= mc) {
+        for (int u = lane; u < cu; u += 32) *reinterpret_cast<uint4*>(Us + swz(mi, u, cu)) = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      const int m = m0 + mi, b = m / n_q, t = m % n_q;
+      const int lo = plan[batch + 5 + 2 * b], n = min(plan[batch + 6 + 2 * b], kMaxSplits);
+      const size_t s0 = (size_t)t * n_slots + lo + b;
+      const float* lse = lse_part + s0 * n_heads + h;
+      float mx = -INFINITY;
+      for (int k = lane; k < n; k += 32) mx = fmaxf(mx, lse[(size_t)k * n_heads]);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float sum = 0.f;
+      for (int k = lane; k < n; k += 32) {
+        const float e = mx > -INFINITY ? exp2f(lse[(size_t)k * n_heads] - mx) : 0.f;
+        wgt[k] = e;
+        sum += e;
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      const float inv = sum > 0.f ? 1.f / sum : 0.f;
+      if (lane == 0 && lse_out) lse_out[(size_t)m * n_heads + h] = sum > 0.f ? (mx + log2f(sum)) * kLn2 : -INFINITY;
+      __syncwarp();
+      // u[c] = sum_k w_k o_k[c]; lane holds columns 4*lane + 128*i
+      for (int c0 = 4 * lane; c0 < d_c; c0 += 128) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float* op = o_part + (s0 * n_heads + h) * d_c + c0;
+        for (int k = 0; k < n; ++k) {
+          const float wk = wgt[k];
+          if (wk != 0.f) {
+            const float4 v = *reinterpret_cast<const float4*>(op + (size_t)k * n_heads * d_c);
+            acc.x = fmaf(wk, v.x, acc.x);
+            acc.y = fmaf(wk, v.y, acc.y);
+            acc.z = fmaf(wk, v.z, acc.z);
+            acc.w = fmaf(wk, v.w, acc.w);
+          }
+        }
+        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
+        pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
+        *reinterpret_cast<uint2*>(Us + swz(mi, c0 >> 3, cu) + (c0 & 7) * 2) = pk;
+      }
+      __syncwarp();
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    // o[m, j] = sum_c u[m, c] W^UV_h[j, c]
+    const int g = lane >> 2, q = lane & 3;
+    for (int np = warp; np * 16 < d_v; np += kThreads / 32) {
+      for (int mt = 0; mt < mpad; mt += 16) {
+        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k0 = 0; k0 < d_c; k0 += 16) {
+          uint32_t af[4], b00, b01, b10, b11;
+          load_a(Us, cu, mt, k0, lane, af);
+          load_b_nk(Ws, cu, k0, np * 16, lane, b00, b01, b10, b11);
+          mma_bf16(acc0, af, b00, b01);
+          mma_bf16(acc1, af, b10, b11);
+        }
+        const int r0 = mt + g, r1 = mt + g + 8, col = np * 16 + 2 * q;
+        __nv_bfloat16* o0 = out + ((size_t)(m0 + r0) * n_heads + h) * d_v + col;
+        __nv_bfloat16* o1 = out + ((size_t)(m0 + r1) * n_heads + h) * d_v + col;
+        if (r0 < mc) {
+          *reinterpret_cast<__nv_bfloat162*>(o0) = __floats2bfloat162_rn(acc0[0], acc0[1]);
+          *reinterpret_cast<__nv_bfloat162*>(o0 + 8) = __floats2bfloat162_rn(acc1[0], acc1[1]);
+        }
+        if (r1 < mc) {
+          *reinterpret_cast<__nv_bfloat162*>(o1) = __floats2bfloat162_rn(acc0[2], acc0[3]);
+          *reinterpret_cast<__nv_bfloat162*>(o1 + 8) = __floats2bfloat162_rn(acc1[2], acc1[3]);
+        }
+      }
+    }
+  }
+}
+
 }  // namespace
 
 size_t combine_smem_bytes(const mla_dims& d) { return 4 * ((size_t)kTok * d.d_c + (size_t)kTok * kMaxSplits); }
@@ -134,6 +253,13 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
     if (e != cudaSuccess) return e;
     combine_kernel<float><<<d.n_heads, kThreads, smem, st>>>((const float*)W_uv, d.n_heads, d.d_c, d.d_v, batch, n_q,
                                                               plan, o_part, lse_part, (float*)out, lse_out);
+  } else if (d.d_c % 128 == 0 && d.d_v % 16 == 0 && combine_tc_smem(d) <= 227 * 1024 &&
+             (reinterpret_cast<uintptr_t>(out) & 3u) == 0) {  // paired bf16 stores
+    const size_t tsm = combine_tc_smem(d);
+    e = cudaFuncSetAttribute(combine_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+    if (e != cudaSuccess) return e;
+    combine_tc_kernel<<<d.n_heads, kThreads, tsm, st>>>((const __nv_bfloat16*)W_uv, d.n_heads, d.d_c, d.d_v, batch,
+                                                        n_q, plan, o_part, lse_part, (__nv_bfloat16*)out, lse_out);
   } else {
     e = cudaFuncSetAttribute(combine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
