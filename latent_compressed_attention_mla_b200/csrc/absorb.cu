@@ -268,11 +268,7 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const AbsorbArgs 
   uint8_t* Ws = smem;
   uint8_t* As = smem + (size_t)dn * dc * 2;
 
-  if (h == 0) build_plan(a);
-  {
-    const size_t nblk = gridDim.x, bid = blockIdx.x;
-    for (size_t i = bid * kTcThreads + tid; i < a.lse_count; i += nblk * kTcThreads) a.lse_part[i] = -INFINITY;
-  }
+  pdl_trigger();
   // W^UK_h, rows d (K) x columns c (N)
   const __nv_bfloat16* Wh = static_cast<const __nv_bfloat16*>(a.W_uk) + (size_t)h * dn * dc;
   for (int i = tid; i < dn * wu; i += kTcThreads) {
@@ -280,6 +276,12 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const AbsorbArgs 
     cp_async16(smem_addr(Ws) + swz(r, u, wu), Wh + (size_t)r * dc + u * 8);
   }
   cp_async_commit();
+  pdl_wait();
+  if (h == 0) build_plan(a);
+  {
+    const size_t nblk = gridDim.x, bid = blockIdx.x;
+    for (size_t i = bid * kTcThreads + tid; i < a.lse_count; i += nblk * kTcThreads) a.lse_part[i] = -INFINITY;
+  }
   const __nv_bfloat16* qn = static_cast<const __nv_bfloat16*>(a.q_nope);
   TO* qa = static_cast<TO*>(a.q_abs);
   const int ncols = dc / 8;  // columns per warp
@@ -370,12 +372,12 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
     if (q_abs_f16) {
       e = cudaFuncSetAttribute(absorb_tc_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      absorb_tc_kernel<__half><<<d.n_heads, kTcThreads, smem, st>>>(a);
+      launch_pdl(absorb_tc_kernel<__half>, dim3(d.n_heads), dim3(kTcThreads), smem, st, a);
     } else {
       e = cudaFuncSetAttribute(absorb_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)smem);
       if (e != cudaSuccess) return e;
-      absorb_tc_kernel<__nv_bfloat16><<<d.n_heads, kTcThreads, smem, st>>>(a);
+      launch_pdl(absorb_tc_kernel<__nv_bfloat16>, dim3(d.n_heads), dim3(kTcThreads), smem, st, a);
     }
     return cudaGetLastError();
   }

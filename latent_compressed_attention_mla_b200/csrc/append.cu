@@ -211,6 +211,8 @@ __device__ __forceinline__ float block128_max(float v, float* sh) {
 // (IEEE fp32 division; 1 for an all-zero tile) and e4m3 codes of c/scale
 // (round to nearest even, saturating).
 __global__ void __launch_bounds__(128) append_fp8_finalize_kernel(const AppendArgs a) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sh[4];
   const int n = blockIdx.x, tid = threadIdx.x;
   int prow, position;
@@ -262,12 +264,14 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
   // output index of tile column j: a row of W_dkv, or a rotation pair member of W_kr
   auto out_idx = [&](int j) -> int { return is_kr ? (j < 16 ? 16 * kr_tile + j : half + 16 * kr_tile + j - 16)
                                                   : tile * kTcTile + j; };
+  pdl_trigger();
   for (int i = tid; i < kTcTile * ku; i += kTcThreads) {
     const int r = i / ku, u = i % ku;
     const __nv_bfloat16* src = (is_kr ? Wk : Wd) + (size_t)out_idx(r) * K + k_lo + u * 8;
     cp_async16(smem_addr(Ws) + swz(r, u, ku), src);
   }
   cp_async_commit();
+  pdl_wait();
   const Fp8Page fp = fp8_page(a.page_size, a.d_c, a.d_rope);
   const int M = a.n_tokens, nk = ks / 16;
   for (int m0 = 0; m0 < M; m0 += kTcMb) {
@@ -409,10 +413,10 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
     const int tgrid = (d.d_c / kTcTile + d.d_rope / kTcTile) * kTcCluster;
     if (d.cache_dtype == MLA_BF16) {
       cudaFuncSetAttribute(append_tc_kernel<MLA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      append_tc_kernel<MLA_BF16><<<tgrid, kTcThreads, smem, st>>>(a);
+      launch_pdl(append_tc_kernel<MLA_BF16>, dim3(tgrid), dim3(kTcThreads), smem, st, a);
     } else {
       cudaFuncSetAttribute(append_tc_kernel<MLA_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      append_tc_kernel<MLA_FP8_E4M3><<<tgrid, kTcThreads, smem, st>>>(a);
+      launch_pdl(append_tc_kernel<MLA_FP8_E4M3>, dim3(tgrid), dim3(kTcThreads), smem, st, a);
     }
   } else if (d.act_dtype == MLA_F32) {
     if (d.cache_dtype == MLA_F32) MLA_PROJ(float, MLA_F32);
@@ -432,8 +436,8 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
     trace_record(MLA_TRACE_APPEND_FINALIZE, true, st);
     return e;
   }
-  append_fp8_finalize_kernel<<<n_tokens, 128, 0, st>>>(a);
-  e = cudaGetLastError();
+  e = launch_pdl(append_fp8_finalize_kernel, dim3(n_tokens), dim3(128), 0, st, a);
+  if (e == cudaSuccess) e = cudaGetLastError();
   trace_record(MLA_TRACE_APPEND_FINALIZE, true, st);
   return e;
 }

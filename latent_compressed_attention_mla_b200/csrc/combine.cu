@@ -8,9 +8,10 @@
 //
 // bf16 activations (combine_tc_kernel): one CTA per head stages W^UV_h (d_v x
 // d_c, 128 KB at DeepSeek-V3 dims) in swizzled shared memory with cp.async
-// while its warps merge the splits of 64 tokens at a time (warp per token,
-// lanes over latent columns) into a bf16 u tile; mma.sync m16n8k16 then forms
-// o = u . W^UV_h^T with fp32 accumulation.
+// while it merges the splits of 64 tokens at a time into a bf16 u tile (a
+// warp per token for the weights, then every thread over (token, 4 columns)
+// items, eight splits' loads in flight at a time); mma.sync m16n8k16 then
+// forms o = u . W^UV_h^T with fp32 accumulation.
 //
 // fp32 activations (combine_kernel): one CTA (8 warps) per head, kTok tokens
 // per pass:
@@ -129,9 +130,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(
 
 constexpr int kTcTok = 64;  // tokens merged per pass (rows of the u tile)
 
-size_t combine_tc_smem(const mla_dims& d) {
-  return (size_t)d.d_v * d.d_c * 2 + (size_t)kTcTok * d.d_c * 2 + (size_t)(kThreads / 32) * kMaxSplits * 4;
-}
+size_t combine_tc_smem(const mla_dims& d) { return (size_t)d.d_v * d.d_c * 2 + (size_t)kTcTok * d.d_c * 2; }
 
 // bf16 activations: d_c % 128 == 0 (lanes x 4 columns, swizzle groups),
 // d_v % 16 == 0 (16-column pairs over the eight warps).
@@ -144,11 +143,10 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(
   const int cu = d_c / 8;  // 16-byte units per row of W^UV_h and of u
   uint8_t* Ws = smem_tc;
   uint8_t* Us = smem_tc + (size_t)d_v * d_c * 2;
-  float* wgt = reinterpret_cast<float*>(Us + (size_t)kTcTok * d_c * 2) + warp * kMaxSplits;
+  __shared__ float s_mx[kTcTok], s_inv[kTcTok];
   const int M = batch * n_q;
-  const int splits = plan[batch + 2];
-  const int n_slots = batch + splits - 1;  // slot stride of the decode that wrote the partials
 
+  pdl_trigger();
   // W^UV_h: rows j (N) x columns c (K)
   const __nv_bfloat16* Wh = W_uv + (size_t)h * d_v * d_c;
   for (int i = tid; i < d_v * cu; i += kThreads) {
@@ -156,57 +154,77 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(
     cp_async16(smem_addr(Ws) + swz(r, u, cu), Wh + (size_t)r * d_c + u * 8);
   }
   cp_async_commit();
+  pdl_wait();
+  const int splits = plan[batch + 2];
+  const int n_slots = batch + splits - 1;  // slot stride of the decode that wrote the partials
 
   for (int m0 = 0; m0 < M; m0 += kTcTok) {
     const int mc = min(kTcTok, M - m0), mpad = (mc + 15) & ~15;
     __syncthreads();  // previous pass done with Us
-    // merge: warp per token
-    for (int mi = warp; mi < mpad; mi += kThreads / 32) {
-      if (mi >= mc) {
-        for (int u = lane; u < cu; u += 32) *reinterpret_cast<uint4*>(Us + swz(mi, u, cu)) = make_uint4(0, 0, 0, 0);
-        continue;
-      }
+    // merge weights: warp per token computes the reference max and 1/sum
+    for (int mi = warp; mi < mc; mi += kThreads / 32) {
       const int m = m0 + mi, b = m / n_q, t = m % n_q;
       const int lo = plan[batch + 5 + 2 * b], n = min(plan[batch + 6 + 2 * b], kMaxSplits);
-      const size_t s0 = (size_t)t * n_slots + lo + b;
-      const float* lse = lse_part + s0 * n_heads + h;
+      const float* lse = lse_part + ((size_t)t * n_slots + lo + b) * n_heads + h;
       float mx = -INFINITY;
       for (int k = lane; k < n; k += 32) mx = fmaxf(mx, lse[(size_t)k * n_heads]);
 #pragma unroll
       for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       float sum = 0.f;
-      for (int k = lane; k < n; k += 32) {
-        const float e = mx > -INFINITY ? exp2f(lse[(size_t)k * n_heads] - mx) : 0.f;
-        wgt[k] = e;
-        sum += e;
-      }
+      for (int k = lane; k < n; k += 32) sum += mx > -INFINITY ? exp2f(lse[(size_t)k * n_heads] - mx) : 0.f;
 #pragma unroll
       for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      const float inv = sum > 0.f ? 1.f / sum : 0.f;
-      if (lane == 0 && lse_out) lse_out[(size_t)m * n_heads + h] = sum > 0.f ? (mx + log2f(sum)) * kLn2 : -INFINITY;
-      __syncwarp();
-      // u[c] = sum_k w_k o_k[c]; lane holds columns 4*lane + 128*i
-      for (int c0 = 4 * lane; c0 < d_c; c0 += 128) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (lane == 0) {
+        s_mx[mi] = mx;
+        s_inv[mi] = sum > 0.f ? 1.f / sum : 0.f;
+        if (lse_out) lse_out[(size_t)m * n_heads + h] = sum > 0.f ? (mx + log2f(sum)) * kLn2 : -INFINITY;
+      }
+    }
+    __syncthreads();
+    // u[m, c..c+3] = sum_k w_k o_k[c..c+3]: one item per (token, 4 columns)
+    // over every thread of the CTA; the splits are read eight at a time with
+    // all loads issued before any is used
+    const int c4n = d_c / 4, n_items = mpad * c4n;
+    for (int it = tid; it < n_items; it += kThreads) {
+      const int mi = it / c4n, c0 = (it % c4n) * 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (mi < mc && s_mx[mi] > -INFINITY) {
+        const int m = m0 + mi, b = m / n_q, t = m % n_q;
+        const int lo = plan[batch + 5 + 2 * b], n = min(plan[batch + 6 + 2 * b], kMaxSplits);
+        const size_t s0 = (size_t)t * n_slots + lo + b;
+        const float* lp = lse_part + s0 * n_heads + h;
         const float* op = o_part + (s0 * n_heads + h) * d_c + c0;
-        for (int k = 0; k < n; ++k) {
-          const float wk = wgt[k];
-          if (wk != 0.f) {
-            const float4 v = *reinterpret_cast<const float4*>(op + (size_t)k * n_heads * d_c);
-            acc.x = fmaf(wk, v.x, acc.x);
-            acc.y = fmaf(wk, v.y, acc.y);
-            acc.z = fmaf(wk, v.z, acc.z);
-            acc.w = fmaf(wk, v.w, acc.w);
+        const float mx = s_mx[mi], inv = s_inv[mi];
+        constexpr int kU = 8;
+        for (int k0 = 0; k0 < n; k0 += kU) {
+          float4 v[kU];
+          float l[kU];
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int k = min(k0 + u, n - 1);  // in-range duplicate for the tail, weight zeroed below
+            v[u] = *reinterpret_cast<const float4*>(op + (size_t)k * n_heads * d_c);
+            l[u] = lp[(size_t)k * n_heads];
+          }
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            // a split holding no key of the sequence has lse = -inf and an
+            // unwritten partial: its weight is 0 and its values are not used
+            const float wk = k0 + u < n ? exp2f(l[u] - mx) * inv : 0.f;
+            if (wk != 0.f) {
+              acc.x = fmaf(wk, v[u].x, acc.x);
+              acc.y = fmaf(wk, v[u].y, acc.y);
+              acc.z = fmaf(wk, v[u].z, acc.z);
+              acc.w = fmaf(wk, v[u].w, acc.w);
+            }
           }
         }
-        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-        const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-        uint2 pk;
-        pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
-        pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
-        *reinterpret_cast<uint2*>(Us + swz(mi, c0 >> 3, cu) + (c0 & 7) * 2) = pk;
       }
-      __syncwarp();
+      const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y);
+      const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
+      pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
+      *reinterpret_cast<uint2*>(Us + swz(mi, c0 >> 3, cu) + (c0 & 7) * 2) = pk;
     }
     cp_async_wait<0>();
     __syncthreads();
@@ -258,8 +276,9 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
     const size_t tsm = combine_tc_smem(d);
     e = cudaFuncSetAttribute(combine_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e != cudaSuccess) return e;
-    combine_tc_kernel<<<d.n_heads, kThreads, tsm, st>>>((const __nv_bfloat16*)W_uv, d.n_heads, d.d_c, d.d_v, batch,
-                                                        n_q, plan, o_part, lse_part, (__nv_bfloat16*)out, lse_out);
+    e = launch_pdl(combine_tc_kernel, dim3(d.n_heads), dim3(kThreads), tsm, st, (const __nv_bfloat16*)W_uv,
+                   d.n_heads, d.d_c, d.d_v, batch, n_q, plan, o_part, lse_part, (__nv_bfloat16*)out, lse_out);
+    if (e != cudaSuccess) return e;
   } else {
     e = cudaFuncSetAttribute(combine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);

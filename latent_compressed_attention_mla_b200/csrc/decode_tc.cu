@@ -305,6 +305,20 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// shared -> global tensor store (bulk group of this thread)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // arrive on a barrier of this CTA with an expected transaction count
 __device__ __forceinline__ void mbar_arrive_tx_local(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
@@ -373,6 +387,7 @@ struct SegmentWalker {
 struct TcParams {
   DecodeParams p;
   CUtensorMap map_q;     // q_abs [rows = batch*n_q*128][576], box 64 x 64 (bf16, or f16 for the FP8 cache)
+  CUtensorMap map_o;     // o_part [rows = n_q*n_slots*128][512] fp32, box 32 x 64, 128-byte swizzle
   // bf16 cache
   CUtensorMap map_pv;    // pool rows, box 64 x 64 (one page x 64 columns: QK and PV boxes)
   CUtensorMap map_pv16;  // pool rows, box 64 x 16 (16-key group of a partial page)
@@ -457,6 +472,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
   float* red_max = reinterpret_cast<float*>(smem + L::OffRedMax);
   float* red_l = reinterpret_cast<float*>(smem + L::OffRedL);
 
+  pdl_trigger();
+  if (threadIdx.x == 0) TC_TRACE(12, 0);
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int i = 0; i < L::QKSlots; ++i) {
@@ -500,6 +517,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything below reads the absorbed queries, the plan and the cache, or
+  // writes the split partials
+  if (threadIdx.x == 0) TC_TRACE(13, 0);
+  pdl_wait();
+  if (threadIdx.x == 0) TC_TRACE(14, 0);
 
   auto page_of = [&](int b, int pg) -> int {
     int page = p.page_table[(size_t)b * p.max_pages + pg];
@@ -1051,21 +1073,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       const float l_tot = l_part + red_l[(half ^ 1) * 64 + hl];
       asm volatile("bar.sync 1, 128;" ::: "memory");
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      // O leaves through the (free) P buffer as 32-column x 64-head boxes,
+      // stored by TMA: lanes 0-63 hold dims [256j, 256j+128), lanes 64-127
+      // dims [256j+128, 256j+256).  Four 8 KB staging slots: two iterations
+      // of both halves in flight.
+      {
+        const bool issuer = hl == 0;  // thread 0 of each half
+        const int orow = (int)((((size_t)t * p.n_slots + w + s.b) * kHeads) + kHalfHeads * rank);
 #pragma unroll 1
-      for (int c = 0; c < 256; c += 32) {
-        const uint32_t col = (c < 128 ? kColO0 + c : kColO1 + (c - 128));
-        uint32_t orr[32];
-        tmem_ld32(tmem + lane_base + col, orr);
-        tmem_wait_ld();
-        // lanes 0-63 hold dims [256j, 256j+128), lanes 64-127 dims [256j+128, 256j+256)
-        float* dst = od + (c < 128 ? 0 : 256) + 128 * half + (c & 127);
+        for (int i = 0; i < 8; ++i) {
+          const int c = 32 * i;
+          if (i >= 2) {
+            if (issuer) bulk_wait_read<1>();
+            asm volatile("bar.sync %0, 64;" ::"r"(2 + half) : "memory");
+          }
+          const uint32_t col = (c < 128 ? kColO0 + c : kColO1 + (c - 128));
+          uint32_t orr[32];
+          tmem_ld32(tmem + lane_base + col, orr);
+          tmem_wait_ld();
+          uint8_t* box = smem + L::OffP + ((i & 1) * 2 + half) * 8192 + hl * 128;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + j) =
-              make_float4(__uint_as_float(orr[j]) * inv, __uint_as_float(orr[j + 1]) * inv,
-                          __uint_as_float(orr[j + 2]) * inv, __uint_as_float(orr[j + 3]) * inv);
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(box + ((q ^ (hl & 7)) * 16)) =
+                make_float4(__uint_as_float(orr[4 * q]) * inv, __uint_as_float(orr[4 * q + 1]) * inv,
+                            __uint_as_float(orr[4 * q + 2]) * inv, __uint_as_float(orr[4 * q + 3]) * inv);
+          fence_proxy_async();
+          asm volatile("bar.sync %0, 64;" ::"r"(2 + half) : "memory");
+          if (issuer) {
+            tma_store_2d(&P.map_o, (c < 128 ? 0 : 256) + 128 * half + (c & 127), orow,
+                         sbase + L::OffP + ((i & 1) * 2 + half) * 8192);
+            bulk_commit();
+          }
+        }
+        // the stores have read the staging slots (the next segment writes P
+        // there) and written the partials
+        if (issuer) bulk_wait_all();
+        asm volatile("bar.sync %0, 64;" ::"r"(2 + half) : "memory");
       }
       if (half == 0) p.lse_part[slot * kHeads + head] = l_tot > 0.f ? m_ref + __log2f(l_tot) : -INFINITY;
+      if (threadIdx.x == 0) TC_TRACE(15, 0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_bar(L::O_FREE));
@@ -1137,14 +1183,27 @@ bool device_is_sm100() {
   return major == 10 && minor == 0;
 }
 
+// o_part as a 2-D fp32 tensor [rows][512], box 32 x 64, 128-byte swizzle
+bool make_o_map(CUtensorMap* m, void* base, uint64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kDC, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kDC * 4};
+  const cuuint32_t box[2] = {32, (cuuint32_t)kHalfHeads};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 template <bool kFp8>
 cudaError_t launch_variant(const TcParams& tp, int pairs, cudaStream_t st) {
   using L = TcLayout<kFp8>;
   cudaError_t e =
       cudaFuncSetAttribute(decode_tc_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SmemBytes);
   if (e != cudaSuccess) return e;
-  decode_tc_kernel<kFp8><<<2 * pairs, L::Threads, L::SmemBytes, st>>>(tp);
-  return cudaGetLastError();
+  e = launch_pdl(decode_tc_kernel<kFp8>, dim3(2 * pairs), dim3(L::Threads), L::SmemBytes, st, tp);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
@@ -1169,6 +1228,7 @@ cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st) {
   tp.p = p;
   const bool fp8 = p.d.cache_dtype == MLA_FP8_E4M3;
   const uint64_t q_rows = (uint64_t)p.batch * p.n_q * kHeads;
+  if (!make_o_map(&tp.map_o, p.o_part, (uint64_t)p.n_q * p.n_slots * kHeads)) return cudaErrorInvalidValue;
   if (fp8) {
     const Fp8Page fp = fp8_page(kPage, kDC, kDR);
     if (!make_map(&tp.map_q, p.q_abs, q_rows, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||

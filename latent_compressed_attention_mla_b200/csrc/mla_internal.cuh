@@ -42,6 +42,33 @@ __host__ __device__ inline Fp8Page fp8_page(int page_size, int d_c, int d_rope) 
 }
 
 // ----------------------------------------------------------------------------
+// Programmatic dependent launch.  The tensor-core kernels are launched with
+// programmatic stream serialization: a kernel may start while the previous
+// one drains, stages what does not depend on it (weights), and then waits.
+// Every such kernel calls pdl_wait() before it reads or writes anything the
+// previous kernels of the stream touch, so it also completes after them (the
+// ordering stays transitive along the stream).
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// ----------------------------------------------------------------------------
 // Element access
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ float to_f(float x) { return x; }
