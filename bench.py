@@ -14,6 +14,7 @@ on this host instead, rank 0 only.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -32,6 +33,39 @@ from latent_compressed_attention_mla_b200 import workloads as WL  # noqa: E402
 
 METRIC = "MLA decode: latent-cache TB/s, TFLOP/s and % of roofline; decode tokens/s"
 L2_BYTES = 126 * 1024 * 1024
+
+
+# kernel (bench name) -> sources whose content decides its DRAM counters
+KERNEL_SOURCES = {
+    "append_project": ["csrc/append.cu"], "append_finalize": ["csrc/append.cu"], "absorb": ["csrc/absorb.cu"],
+    "attend": ["csrc/decode_tc.cu", "csrc/decode_simt.cu"], "combine": ["csrc/combine.cu"],
+}
+COMMON_SOURCES = ["csrc/mla_internal.cuh", "csrc/mma_tile.cuh"]
+
+
+def source_digest(kernel: str) -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kernel] + COMMON_SOURCES:
+        with open(os.path.join(ROOT, "latent_compressed_attention_mla_b200", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch (read + write) of `kernel` on `workload` from the
+    committed ncu counters, or None when none were taken or the kernel's
+    sources changed since."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            table = json.load(f)
+    except Exception:
+        return None
+    for e in table.get("entries", []):
+        if e["workload"] == workload and e["kernel"] == kernel:
+            if e["source_sha256"] != source_digest(kernel):
+                return None
+            return (e["dram_read_bytes"] + e["dram_write_bytes"]) / e["launches"]
+    return None
 
 
 def load_peaks():
@@ -247,8 +281,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch each step eagerly instead of replaying a captured CUDA graph")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="keep only the first N sequences of the workload (smaller case of the same kernels, "
+                         "e.g. for profiler captures); the workload name records it")
     args = ap.parse_args()
     cfg = WL.CONFIGS[args.config]
+    if 0 < args.batch < cfg.B:
+        cfg = cfg.with_(name=f"{cfg.name}[:{args.batch}]", B=args.batch, L=tuple(cfg.L[:args.batch]))
     if args.impl == "reference":
         return run_reference(args, cfg)
 
@@ -375,6 +414,9 @@ def main():
     tokens_per_step = cfg.B * cfg.T
     value = world * tokens_per_step * args.steps / (ms / 1e3)
     kms = {name: ksum[k] / args.steps for k, name in enumerate(B.TRACE_KERNELS)}  # ms per launch
+    if cfg.cache_dtype != "fp8":
+        kms.pop("append_finalize")  # only FP8 caches launch it; its events bracket nothing here
+    launches_per_step = len(kms)
     peaks = load_peaks()
     long_region = ms > 1000.0
     tpeak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
@@ -395,7 +437,7 @@ def main():
     else:
         roof = {"bound": "hbm", "achieved": wd["bytes"] / td / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(cfg.name, dom)
     roof["kernel"] = dom
     roof["peak_source"] = peaks["source"] + (" sustained" if (roof["bound"] == "tensor" and long_region) else
                                              (" burst" if roof["bound"] == "tensor" else " copy"))
@@ -454,7 +496,7 @@ def main():
         "roofline": roof, "attend": attend_summary, "kernels_us": {k: round(v["us"], 3) for k, v in rows.items()},
         "kernel_roofline_frac": {k: (round(v["roofline_frac"], 4) if v["roofline_frac"] else None)
                                  for k, v in rows.items()},
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": nk * args.steps, "clocks": clocks,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
         "timing": ("CUDA-graph replay of each step" if args.graph else "eager launches") +
                   "; per-kernel times from a second, traced pass of the same steps",
         "device_status": status,
