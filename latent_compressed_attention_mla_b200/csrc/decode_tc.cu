@@ -40,9 +40,9 @@
 //    sequence's end.  Queries and probabilities are f16 on this path, so both
 //    MMA operands share the type (kind::f16).
 //  * Warp roles: 0-3 softmax + epilogue (one TMEM lane each), 4 TMEM
-//    allocation and (leader) QK issue, 5 (leader) PV issue, 6-7 TMA for Q and
-//    QK data, 8-9 TMA for PV data, and for the FP8 cache 10-11 / 12-13
-//    converters of QK / PV units.
+//    allocation and (leader) QK issue, 5 (leader) PV issue; bf16 cache: 6-7
+//    TMA for Q and QK data, 8-9 TMA for PV data; FP8 cache: 6 / 7 TMA for
+//    Q and QK / PV data, 8-9 / 10-11 converters of QK / PV units.
 //  * Online softmax in base 2 with a lazily updated reference max: O is only
 //    rescaled when a tile's max exceeds the reference by more than 8 (in
 //    log2 units), so probabilities stay <= 2^8 and rescaling is rare.
@@ -113,11 +113,13 @@ struct TcLayout {
   static constexpr uint32_t OffRedMax = OffMisc + 16;   // float [2][64]
   static constexpr uint32_t OffRedL = OffRedMax + 512;  // float [2][64]
   static constexpr uint32_t SmemBytes = OffRedL + 512 + 1024;  // + alignment slack
-  // warp roles
+  // warp roles: the FP8 cache moves half the bytes through its producers, so
+  // one producer per ring keeps up and leaves registers for the converters
   static constexpr int QKWarp = 4, PVWarp = 5;          // TMEM alloc (QKWarp); leader lane 0 issues the MMAs
-  static constexpr int QKProdWarp = 6, PVProdWarp = 8, Producers = 2;
-  static constexpr int QKConvWarp = 10, PVConvWarp = 12, ConvWarps = 2;
-  static constexpr int Threads = 32 * (kFp8 ? 14 : 10);
+  static constexpr int Producers = kFp8 ? 1 : 2, ConvWarps = 4;
+  static constexpr int QKProdWarp = 6, PVProdWarp = QKProdWarp + Producers;
+  static constexpr int QKConvWarp = PVProdWarp + Producers, PVConvWarp = QKConvWarp + ConvWarps;
+  static constexpr int Threads = 32 * (kFp8 ? PVConvWarp + ConvWarps : PVProdWarp + Producers);
   // arrivals completing one phase of a unit's FULL barrier: the leader's
   // expect-tx arrival (bf16), or every converter warp of both CTAs (FP8)
   static constexpr int UnitFullCount = kFp8 ? 2 * ConvWarps : 1;
@@ -454,6 +456,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
     decode_tc_kernel(const __grid_constant__ TcParams P) {
   using L = TcLayout<kFp8>;
   using PT = typename std::conditional<kFp8, __half2, __nv_bfloat162>::type;  // P element pair
+  constexpr int kConvThreads = 32 * L::ConvWarps;  // threads converting one ring's units
   constexpr uint32_t kIdescQK = idesc(128, 256, false, false, kFp8);
   constexpr uint32_t kIdescPV = idesc(128, 256, false, true, kFp8);
   extern __shared__ uint8_t smem_raw[];
@@ -670,8 +673,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
     }
   } else if (kFp8 && warp >= L::QKConvWarp && warp < L::QKConvWarp + L::ConvWarps) {
     // ------------------------------------------------- FP8: QK unit conversion
-    // Thread ct of the two warps converts 16-byte groups ct, ct+64, ... of
-    // the staged data into the unit (128-byte swizzle).
+    // Thread ct of the converter warps converts 16-byte groups ct,
+    // ct + kConvThreads, ... of the staged data into the unit (128-byte swizzle).
     const int ct = (warp - L::QKConvWarp) * 32 + lane;
     RingPos unit, stage;
     uint32_t gt = 0;
@@ -709,8 +712,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
             if (!ok) break;
             const uint8_t* src = smem + L::OffQSt + stage.slot * kStageBytes;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int gi = k * 64 + ct, r = gi >> 2, q = gi & 3;  // r: unit row (page r/64)
+            for (int k = 0; k < 512 / kConvThreads; ++k) {
+              const int gi = k * kConvThreads + ct, r = gi >> 2, q = gi & 3;  // r: unit row (page r/64)
               const uint4 v = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
               const __half2 s2 = __float2half2_rn(scl[r * 4 + (c >> 1)]);
               uint32_t o[8];
@@ -734,8 +737,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
               const uint8_t* src = smem + L::OffQSt + stage.slot * kStageBytes;
               uint8_t* dst = dstu + i * 8192;
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const int gi = k * 64 + ct, row = gi >> 3, u = gi & 7;
+              for (int k = 0; k < 512 / kConvThreads; ++k) {
+                const int gi = k * kConvThreads + ct, row = gi >> 3, u = gi & 7;
                 const uint4 v = *reinterpret_cast<const uint4*>(src + row * 128 + u * 16);
                 *reinterpret_cast<uint4*>(dst + row * 128 + ((u ^ (row & 7)) * 16)) =
                     make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
@@ -808,8 +811,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
             // 64 rows x 128 codes -> two 64-column atoms (8 KB apart); rows
             // past the visible keys are zero
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int gi = k * 64 + ct, row = gi >> 3, q = gi & 7;
+            for (int k = 0; k < 512 / kConvThreads; ++k) {
+              const int gi = k * kConvThreads + ct, row = gi >> 3, q = gi & 7;
               uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
               if (row < valid) {
                 const uint4 v = *reinterpret_cast<const uint4*>(src + row * 128 + q * 16);
@@ -819,10 +822,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
                 e4m3x4_scaled(v.z, s2, o[4], o[5]);
                 e4m3x4_scaled(v.w, s2, o[6], o[7]);
               }
+              // the eight threads of a row cover both 64-column atoms; threads
+              // of the second atom store their odd unit first, so the two
+              // stores of each phase fall on distinct banks
               uint8_t* rp = dst + (q >> 2) * 8192 + row * 128;
-              const int u0 = 2 * (q & 3);
-              *reinterpret_cast<uint4*>(rp + ((u0 ^ (row & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
-              *reinterpret_cast<uint4*>(rp + (((u0 + 1) ^ (row & 7)) * 16)) = make_uint4(o[4], o[5], o[6], o[7]);
+              const int u0 = 2 * (q & 3), odd = q >> 2;
+              const uint4 ev = make_uint4(o[0], o[1], o[2], o[3]), od = make_uint4(o[4], o[5], o[6], o[7]);
+              *reinterpret_cast<uint4*>(rp + (((u0 + odd) ^ (row & 7)) * 16)) = odd ? od : ev;
+              *reinterpret_cast<uint4*>(rp + (((u0 + 1 - odd) ^ (row & 7)) * 16)) = odd ? ev : od;
             }
             fence_proxy_async();
             __syncwarp();
