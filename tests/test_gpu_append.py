@@ -1,0 +1,110 @@
+"""GPU parity of the latent append (S1) against the oracle's append: the rows
+land in their paged slots and nowhere else (bit-exact placement), and the
+stored values are the fp64 projection within the storage format's rounding.
+
+Both sides use the same bf16 inputs, so the device's sums differ from the
+oracle's only in fp32 accumulation order (d_model terms); after rounding to
+bf16 a value may sit one ulp from the oracle's nearest-even result, and an FP8
+code one e4m3 step, when the exact value lies next to a rounding boundary."""
+import numpy as np
+import pytest
+import torch
+
+from latent_compressed_attention_mla_b200 import binding as B
+from latent_compressed_attention_mla_b200 import workloads as W
+from oracle import mla_oracle as O
+from tests.gpu_harness import GpuProblem, OracleProblem
+
+pytestmark = pytest.mark.gpu
+
+V3 = W.CONFIGS[1]
+CASES = [
+    ("bf16-t1", dict(B=3, T=1, L=(0, 63, 700), cache_dtype="bf16")),
+    ("bf16-t2", dict(B=5, T=2, L=(1, 64, 127, 128, 4000), cache_dtype="bf16")),
+    ("fp8-t2", dict(B=5, T=2, L=(1, 64, 127, 128, 4000), cache_dtype="fp8")),
+    # more tokens than one 64-token pass of the tensor-core projection
+    ("bf16-70-tokens", dict(B=70, T=1, L=tuple(int(x) for x in np.arange(70) * 37 % 300), cache_dtype="bf16")),
+    ("fp8-70-tokens", dict(B=35, T=2, L=tuple(int(x) for x in np.arange(35) * 53 % 400), cache_dtype="fp8")),
+]
+
+
+def appended_slots(cfg, pt_host, seq_idx, pos):
+    return [(int(n), int(b), int(p), *O.paged_slot(pt_host, int(b), int(p), cfg.page_size))
+            for n, (b, p) in enumerate(zip(seq_idx, pos))]
+
+
+def row_byte_ranges(cfg, page_bytes, page, row):
+    if cfg.cache_dtype != "fp8":
+        w = (cfg.d_c + cfg.d_rope) * (4 if cfg.cache_dtype == "f32" else 2)
+        return [(page * page_bytes + row * w, w)]
+    kr_off = -(-cfg.page_size * cfg.d_c // 128) * 128
+    sc_off = -(-(kr_off + cfg.page_size * cfg.d_rope * 2) // 128) * 128
+    base = page * page_bytes
+    return [(base + row * cfg.d_c, cfg.d_c), (base + kr_off + row * cfg.d_rope * 2, cfg.d_rope * 2),
+            (base + sc_off + row * (cfg.d_c // 128) * 4, (cfg.d_c // 128) * 4)]
+
+
+@pytest.mark.parametrize("name,kw", CASES, ids=[c[0] for c in CASES])
+def test_append_rows_match_oracle(name, kw):
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    cfg = V3.with_(name=name, seed=70 + len(name), **kw)
+    g = GpuProblem(cfg)
+    before = g.cache.pool.clone()
+    g.session.append(g.inputs["h"], g.seq_idx, g.pos, g.weights["W_dkv"], g.weights["W_kr"], g.page_table,
+                     g.cache.pool)
+    torch.cuda.synchronize()
+    assert g.status() == 0
+    after = g.cache.pool
+    o = OracleProblem(cfg)
+    slots = appended_slots(cfg, g.pt_host, o.seq_idx, o.pos)
+
+    # placement: every changed byte belongs to an appended row
+    allowed = torch.zeros_like(before, dtype=torch.bool)
+    for _, _, _, page, row in slots:
+        for off, n in row_byte_ranges(cfg, g.cache.page_bytes, page, row):
+            allowed[off:off + n] = True
+    changed = before != after
+    assert not bool((changed & ~allowed).any()), "bytes outside the appended rows changed"
+
+    # values: oracle projection in fp64 at the token's own position
+    c, kr = O.append_latent(o.inp["h"], o.w["W_dkv"], o.w["W_kr"], o.pos, cfg.rope_base)
+    v = g.cache.views()
+    pages = torch.tensor([s[3] for s in slots], device=after.device)
+    rows = torch.tensor([s[4] for s in slots], device=after.device)
+    kr_gpu = v["kr"][pages, rows].double().cpu().numpy()
+    ulp_bound = lambda x, rel: rel * np.abs(x) + 2.0 ** -12 * np.abs(x).max(axis=1, keepdims=True)
+    assert (np.abs(kr_gpu - kr) <= ulp_bound(kr, 2.0 ** -7)).all()
+    if cfg.cache_dtype == "fp8":
+        codes = v["codes"][pages, rows].cpu().numpy()
+        scales = v["scales"][pages, rows].double().cpu().numpy()
+        ref_codes, ref_scales = O.fp8_quantise_latent(c)
+        assert np.allclose(scales, ref_scales, rtol=1e-5, atol=0)
+        got = O.fp8_dequantise_latent(codes, scales)
+        step = np.repeat(scales, 128, axis=1)
+        assert (np.abs(got - c) <= 2.0 ** -3 * np.abs(c) + 2.0 ** -9 * step).all()
+        assert (codes == ref_codes).mean() >= 0.99
+    else:
+        c_gpu = v["c"][pages, rows].double().cpu().numpy()
+        assert (np.abs(c_gpu - c) <= ulp_bound(c, 2.0 ** -7)).all()
+        assert (c_gpu == O.to_bf16(c)).mean() >= 0.99
+        assert (kr_gpu == O.to_bf16(kr)).mean() >= 0.99
+
+
+def test_append_f32_cache_matches_oracle():
+    """fp32 activations and cache (the tiny configuration): within fp32 rounding."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    cfg = W.CONFIGS[0].with_(name="append-f32", B=3, T=2, L=(0, 100, 255), seed=77)
+    g = GpuProblem(cfg)
+    g.session.append(g.inputs["h"], g.seq_idx, g.pos, g.weights["W_dkv"], g.weights["W_kr"], g.page_table,
+                     g.cache.pool)
+    torch.cuda.synchronize()
+    o = OracleProblem(cfg)
+    slots = appended_slots(cfg, g.pt_host, o.seq_idx, o.pos)
+    c, kr = O.append_latent(o.inp["h"], o.w["W_dkv"], o.w["W_kr"], o.pos, cfg.rope_base)
+    v = g.cache.views()
+    pages = torch.tensor([s[3] for s in slots], device="cuda")
+    rows = torch.tensor([s[4] for s in slots], device="cuda")
+    assert np.abs(v["c"][pages, rows].double().cpu().numpy() - c).max() <= 1e-5 * np.abs(c).max()
+    assert np.abs(v["kr"][pages, rows].double().cpu().numpy() - kr).max() <= 1e-5 * np.abs(kr).max()
