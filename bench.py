@@ -40,7 +40,7 @@ KERNEL_SOURCES = {
     "append_project": ["csrc/append.cu"], "append_finalize": ["csrc/append.cu"], "absorb": ["csrc/absorb.cu"],
     "attend": ["csrc/decode_tc.cu", "csrc/decode_simt.cu"], "combine": ["csrc/combine.cu"],
 }
-COMMON_SOURCES = ["csrc/mla_internal.cuh", "csrc/mma_tile.cuh"]
+COMMON_SOURCES = ["csrc/mla_internal.cuh", "csrc/mma_tile.cuh", "csrc/tensor_map.cu"]
 
 
 def source_digest(kernel: str) -> str:

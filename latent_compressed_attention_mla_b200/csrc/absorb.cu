@@ -8,11 +8,12 @@
 // The output is in the activation type, or f16 when the decode path reads
 // f16 queries (FP8 cache on the tensor cores).
 //
-// bf16 activations (absorb_tc_kernel): one CTA per head stages W^UK_h (d_nope x
-// d_c, 128 KB at DeepSeek-V3 dims) and the head's q^C rows in swizzled shared
-// memory with cp.async and multiplies them with mma.sync m16n8k16 (fp32
-// accumulation); the eight warps split the d_c output columns.  The kernel is
-// bound by the 16.8 MB of W^UK read once from HBM.
+// bf16 activations at DeepSeek-V3 dims (absorb_tc_kernel): one CTA per head
+// brings W^UK_h (d_nope x d_c, 128 KB) into shared memory with eight TMA
+// boxes (issued before the programmatic-launch wait, so the fetch overlaps the
+// previous kernel), stages the head's q^C rows, and multiplies them with
+// mma.sync m16n8k16 (fp32 accumulation); the eight warps split the d_c output
+// columns.  The kernel is bound by the 16.8 MB of W^UK read once from HBM.
 //
 // fp32 activations (absorb_kernel): one CTA per (head, 16-vector slice of d_c).  Thread (cg, dg) loads the
 // 16-byte vectors of W^UK_h for its column group cg and its rows d in group
@@ -24,6 +25,8 @@
 // per sequence, the run of splits that overlap it; all blocks fill the
 // per-split log-sum-exp slots with -inf, the value of a split that holds no
 // key of a sequence.
+#include <cuda.h>
+
 #include "mla_internal.cuh"
 #include "mma_tile.cuh"
 
@@ -248,6 +251,13 @@ __device__ void rope_queries(const AbsorbArgs& a, int h) {
 
 constexpr int kTcThreads = 256;
 constexpr int kTcMaxTok = 256;  // query rows staged per pass
+constexpr int kTcDn = 128, kTcDc = 512;  // DeepSeek-V3 shape of W^UK_h
+constexpr uint32_t kTcWBytes = kTcDn * kTcDc * 2;  // 128 KB
+
+struct AbsorbTcArgs {
+  AbsorbArgs a;
+  CUtensorMap map_w;  // W_uk as [n_heads * d_nope rows][d_c] bf16, box 64 x 128, 128-byte swizzle
+};
 
 __device__ __forceinline__ void store2(__nv_bfloat16* p, float x, float y) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(x, y);
@@ -256,26 +266,30 @@ __device__ __forceinline__ void store2(__half* p, float x, float y) {
   *reinterpret_cast<__half2*>(p) = __floats2half2_rn(x, y);
 }
 
-// q~[m, h, :] = q^C[m, h, :] . W^UK_h for bf16 activations; d_nope % 64 == 0
-// (swizzle groups), d_c % 128 == 0 and <= 1024 (eight warps, at most eight
-// 16-column pairs each), W^UK_h in shared memory.
+// q~[m, h, :] = q^C[m, h, :] . W^UK_h for bf16 activations at DeepSeek-V3
+// dims.  W^UK_h (d_nope rows x d_c columns) arrives by eight TMA boxes into
+// [8 column blocks][128 rows][128 B] with the 128-byte swizzle; the query rows
+// are staged by cp.async in the same layout.  Warp w owns columns [64w,
+// 64w + 64) and runs two 16-row query tiles at a time over them.
 template <typename TO>
-__global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const AbsorbArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
+__global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_constant__ AbsorbTcArgs P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t wbar;
+  const AbsorbArgs& a = P.a;
   const int h = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int dn = a.d_nope, dc = a.d_c, D = a.d_c + a.d_rope, M = a.batch * a.n_q;
-  const int wu = dc / 8, au = dn / 8;  // 16-byte units per row of W^UK_h and of q^C
-  uint8_t* Ws = smem;
-  uint8_t* As = smem + (size_t)dn * dc * 2;
-
+  const int D = a.d_c + a.d_rope, M = a.batch * a.n_q;
+  uint8_t* Ws = smem;              // [8][128][128 B]
+  uint8_t* As = smem + kTcWBytes;  // [2][kTcMaxTok][128 B]
+  const uint32_t bar = smem_addr(&wbar);
+  if (tid == 0) mbar_init_local(bar, 1);
+  __syncthreads();
   pdl_trigger();
-  // W^UK_h, rows d (K) x columns c (N)
-  const __nv_bfloat16* Wh = static_cast<const __nv_bfloat16*>(a.W_uk) + (size_t)h * dn * dc;
-  for (int i = tid; i < dn * wu; i += kTcThreads) {
-    const int r = i / wu, u = i % wu;
-    cp_async16(smem_addr(Ws) + swz(r, u, wu), Wh + (size_t)r * dc + u * 8);
+  if (tid == 0) {
+    mbar_expect_local(bar, kTcWBytes);
+    for (int cb = 0; cb < kTcDc / 64; ++cb)
+      tma_load_2d(smem_addr(Ws) + cb * kTcDn * 128, &P.map_w, 64 * cb, h * kTcDn, bar);
   }
-  cp_async_commit();
   pdl_wait();
   if (h == 0) build_plan(a);
   {
@@ -284,47 +298,59 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const AbsorbArgs 
   }
   const __nv_bfloat16* qn = static_cast<const __nv_bfloat16*>(a.q_nope);
   TO* qa = static_cast<TO*>(a.q_abs);
-  const int ncols = dc / 8;  // columns per warp
+  bool w_ready = false;
   for (int m0 = 0; m0 < M; m0 += kTcMaxTok) {
-    const int mc = min(kTcMaxTok, M - m0), mpad = (mc + 15) & ~15;
+    const int mc = min(kTcMaxTok, M - m0), mpad = (mc + 31) & ~31;
     __syncthreads();  // previous pass done with As
-    for (int i = tid; i < mpad * au; i += kTcThreads) {
-      const int r = i / au, u = i % au;
-      const uint32_t dst = smem_addr(As) + swz(r, u, au);
+    for (int i = tid; i < mpad * (kTcDn / 8); i += kTcThreads) {
+      const int r = i / (kTcDn / 8), u = i % (kTcDn / 8);
+      const uint32_t off = swz_cb(r, u, kTcMaxTok);
       if (r < mc)
-        cp_async16(dst, qn + ((size_t)(m0 + r) * a.n_heads + h) * dn + u * 8);
+        cp_async16(smem_addr(As) + off, qn + ((size_t)(m0 + r) * a.n_heads + h) * kTcDn + u * 8);
       else
-        *reinterpret_cast<uint4*>(As + swz(r, u, au)) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(As + off) = make_uint4(0, 0, 0, 0);
     }
     cp_async_commit();
     cp_async_wait<0>();
+    if (!w_ready) {
+      if (!mbar_wait_bounded(bar, 0)) {
+        record_status(a.status, MLA_ERR_TIMEOUT);
+        return;
+      }
+      w_ready = true;
+    }
     __syncthreads();
-    for (int mt = 0; mt < mpad; mt += 16) {
-      float acc[16][4];
+    const int g = lane >> 2, q = lane & 3;
+    for (int mt = 0; mt < mpad; mt += 32) {
+      float acc[2][8][4];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-      for (int k0 = 0; k0 < dn; k0 += 16) {
-        uint32_t af[4];
-        load_a(As, au, mt, k0, lane, af);
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
-        for (int np = 0; np < 8; ++np) {
-          if (np * 16 >= ncols) break;
+        for (int j = 0; j < 8; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+#pragma unroll
+      for (int k0 = 0; k0 < kTcDn; k0 += 16) {
+        uint32_t a0[4], a1[4];
+        load_a_cb(As, kTcMaxTok, mt, k0, lane, a0);
+        load_a_cb(As, kTcMaxTok, mt + 16, k0, lane, a1);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
           uint32_t b00, b01, b10, b11;
-          load_b_kn(Ws, wu, k0, warp * ncols + np * 16, lane, b00, b01, b10, b11);
-          mma_bf16(acc[2 * np], af, b00, b01);
-          mma_bf16(acc[2 * np + 1], af, b10, b11);
+          load_b_kn_cb(Ws, kTcDn, k0, warp * 64 + np * 16, lane, b00, b01, b10, b11);
+          mma_bf16(acc[0][2 * np], a0, b00, b01);
+          mma_bf16(acc[0][2 * np + 1], a0, b10, b11);
+          mma_bf16(acc[1][2 * np], a1, b00, b01);
+          mma_bf16(acc[1][2 * np + 1], a1, b10, b11);
         }
       }
-      // accumulator (row g / g+8, columns 2q, 2q+1 of each n8 tile)
-      const int g = lane >> 2, q = lane & 3;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j * 8 >= ncols) break;
-        const int col = warp * ncols + j * 8 + 2 * q;
-        const int r0 = mt + g, r1 = mt + g + 8;
-        if (r0 < mc) store2(qa + ((size_t)(m0 + r0) * a.n_heads + h) * D + col, acc[j][0], acc[j][1]);
-        if (r1 < mc) store2(qa + ((size_t)(m0 + r1) * a.n_heads + h) * D + col, acc[j][2], acc[j][3]);
-      }
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int col = warp * 64 + j * 8 + 2 * q;
+          const int r0 = mt + 16 * i + g, r1 = r0 + 8;
+          if (r0 < mc) store2(qa + ((size_t)(m0 + r0) * a.n_heads + h) * D + col, acc[i][j][0], acc[i][j][1]);
+          if (r1 < mc) store2(qa + ((size_t)(m0 + r1) * a.n_heads + h) * D + col, acc[i][j][2], acc[i][j][3]);
+        }
     }
   }
   rope_queries<__nv_bfloat16, TO>(a, h);
@@ -334,12 +360,9 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const AbsorbArgs 
 
 int absorb_max_d_nope() { return kDG * kMaxRows; }
 
-// shapes of the tensor-core absorption: W^UK_h and 256 staged query rows fit
-// in shared memory, columns split over eight warps in 16-column pairs
-bool absorb_tc_fits(const mla_dims& d) {
-  return d.d_nope % 64 == 0 && d.d_c % 128 == 0 && d.d_c <= 1024 &&
-         (size_t)d.d_nope * d.d_c * 2 + (size_t)kTcMaxTok * d.d_nope * 2 <= 227 * 1024;
-}
+// the tensor-core absorption runs at DeepSeek-V3 dims (its tile shapes are
+// compile-time)
+bool absorb_tc_fits(const mla_dims& d) { return d.d_nope == kTcDn && d.d_c == kTcDc; }
 
 cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const void* q_rope, const void* W_uk,
                                    const int32_t* seq_lens, int batch, int n_q, int max_pages, int splits,
@@ -367,19 +390,23 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
   a.status = status;
   // the tensor-core kernel stages q^C with 16-byte copies
   if (d.act_dtype == MLA_BF16 && absorb_tc_fits(d) && (reinterpret_cast<uintptr_t>(q_nope) & 15u) == 0) {
-    const size_t smem = (size_t)d.d_nope * d.d_c * 2 + (size_t)kTcMaxTok * d.d_nope * 2;
+    AbsorbTcArgs p;
+    p.a = a;
+    if (!make_tile_map_bf16(&p.map_w, W_uk, kTcDc, (uint64_t)d.n_heads * kTcDn, (uint64_t)kTcDc * 2, 64, kTcDn))
+      return cudaErrorInvalidValue;
+    const size_t smem = kTcWBytes + (size_t)kTcMaxTok * kTcDn * 2 + 1024;
     cudaError_t e;
     if (q_abs_f16) {
       e = cudaFuncSetAttribute(absorb_tc_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      launch_pdl(absorb_tc_kernel<__half>, dim3(d.n_heads), dim3(kTcThreads), smem, st, a);
+      e = launch_pdl(absorb_tc_kernel<__half>, dim3(d.n_heads), dim3(kTcThreads), smem, st, p);
     } else {
       e = cudaFuncSetAttribute(absorb_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)smem);
       if (e != cudaSuccess) return e;
-      launch_pdl(absorb_tc_kernel<__nv_bfloat16>, dim3(d.n_heads), dim3(kTcThreads), smem, st, a);
+      e = launch_pdl(absorb_tc_kernel<__nv_bfloat16>, dim3(d.n_heads), dim3(kTcThreads), smem, st, p);
     }
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
   }
   const int vec = d.act_dtype == MLA_F32 ? 4 : 8;
   const dim3 grid(d.n_heads, (d.d_c + kCG * vec - 1) / (kCG * vec));

@@ -15,9 +15,10 @@
 // append_tc (bf16 activations, bf16 or FP8 cache): the same projection as a
 //   split-K GEMM on the tensor cores.  The d_c + d_rope outputs form 32-wide
 //   tiles; a cluster of eight CTAs owns a tile, each CTA one eighth of
-//   d_model: its weight slice and the tokens' h slice are staged in swizzled
-//   shared memory with cp.async and multiplied with mma.sync m16n8k16 (fp32
-//   accumulation).  The eight partial sums are reduced over distributed shared
+//   d_model: its weight slice (fetched by TMA before the programmatic-launch
+//   wait) and the tokens' h slice (TMA, rows past the last token zero-filled)
+//   sit in 128-byte-swizzled shared memory and are multiplied with mma.sync
+//   m16n8k16 (fp32 accumulation).  The eight partial sums are reduced over distributed shared
 //   memory, each CTA finishing 1/8 of the tokens (RoPE, rounding, paged store),
 //   so no workspace is needed.  The k^R tiles hold rotation pairs (i, i +
 //   d_rope/2) in columns (j, j + 16), so RoPE stays inside a tile.
@@ -25,6 +26,7 @@
 //   reduction across CTAs, so the projection leaves c in fp32 scratch and one
 //   CTA per token quantises it.
 #include <cooperative_groups.h>
+#include <cuda.h>
 
 #include "mla_internal.cuh"
 #include "mma_tile.cuh"
@@ -237,65 +239,90 @@ constexpr int kTcTile = 32;     // outputs per tile
 constexpr int kTcThreads = 256;
 constexpr int kTcMb = 64;       // tokens per pass
 
+struct AppendTcArgs {
+  AppendArgs a;
+  CUtensorMap map_wd;  // W_dkv [d_c rows][d_model], box 64 x 32, 128-byte swizzle
+  CUtensorMap map_wk;  // W_kr [d_rope rows][d_model], box 64 x 16
+  CUtensorMap map_h;   // h [n_tokens rows][d_model], box 64 x 64 (rows past n_tokens read as zero)
+  CUtensorMap map_h16; // the same with 16-row boxes, for passes of at most 16 tokens
+};
+
 size_t append_tc_smem(const mla_dims& d) {
   const size_t ks = (size_t)d.d_model / kTcCluster;
-  return (size_t)kTcTile * ks * 2 + (size_t)kTcMb * ks * 2 + (size_t)4 * kTcMb * kTcTile * 4;
+  return (size_t)kTcTile * ks * 2 + (size_t)kTcMb * ks * 2 + (size_t)4 * kTcMb * kTcTile * 4 + 1024;
 }
 
 // bf16 activations; d_model % (8 * 64) == 0, d_c % 32 == 0, d_rope % 32 == 0.
+// Shared memory: the weight slice [ks/64 column blocks][32 rows][128 B] and
+// the h slice [ks/64][64 rows][128 B], both written by TMA with the 128-byte
+// swizzle, then fp32 partial tiles [4][64][32].
 template <int CACHE>
 __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads, 1)
-    append_tc_kernel(const AppendArgs a) {
+    append_tc_kernel(const __grid_constant__ AppendTcArgs T) {
   namespace cg = cooperative_groups;
-  extern __shared__ __align__(128) uint8_t smem_tc[];
+  extern __shared__ uint8_t smem_tc[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_tc) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t wbar, hbar;
+  const AppendArgs& a = T.a;
   cg::cluster_group cl = cg::this_cluster();
   const int rank = (int)cl.block_rank(), tile = blockIdx.x / kTcCluster;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int K = a.d_model, ks = K / kTcCluster, ku = ks / 8, k_lo = rank * ks;
+  const int K = a.d_model, ks = K / kTcCluster, ncb = ks / 64, k_lo = rank * ks;
   const int n_c_tiles = a.d_c / kTcTile, half = a.d_rope / 2;
   const bool is_kr = tile >= n_c_tiles;
   const int kr_tile = tile - n_c_tiles;
-  uint8_t* Ws = smem_tc;
+  uint8_t* Ws = smem;
   uint8_t* Hs = Ws + (size_t)kTcTile * ks * 2;
   float* Ps = reinterpret_cast<float*>(Hs + (size_t)kTcMb * ks * 2);  // [4][kTcMb][kTcTile]
-  const __nv_bfloat16* Wd = static_cast<const __nv_bfloat16*>(a.W_dkv);
-  const __nv_bfloat16* Wk = static_cast<const __nv_bfloat16*>(a.W_kr);
-  const __nv_bfloat16* H = static_cast<const __nv_bfloat16*>(a.h);
-  // output index of tile column j: a row of W_dkv, or a rotation pair member of W_kr
-  auto out_idx = [&](int j) -> int { return is_kr ? (j < 16 ? 16 * kr_tile + j : half + 16 * kr_tile + j - 16)
-                                                  : tile * kTcTile + j; };
-  pdl_trigger();
-  for (int i = tid; i < kTcTile * ku; i += kTcThreads) {
-    const int r = i / ku, u = i % ku;
-    const __nv_bfloat16* src = (is_kr ? Wk : Wd) + (size_t)out_idx(r) * K + k_lo + u * 8;
-    cp_async16(smem_addr(Ws) + swz(r, u, ku), src);
+  const uint32_t wb = smem_addr(&wbar), hb = smem_addr(&hbar);
+  if (tid == 0) {
+    mbar_init_local(wb, 1);
+    mbar_init_local(hb, 1);
   }
-  cp_async_commit();
+  __syncthreads();
+  pdl_trigger();
+  if (tid == 0) {
+    // weight slice: tile column j is W_dkv row tile*32 + j, or for a k^R tile
+    // W_kr rows 16*kr_tile + j (j < 16) and d_rope/2 + 16*kr_tile + j - 16
+    mbar_expect_local(wb, (uint32_t)kTcTile * ks * 2);
+    for (int cb = 0; cb < ncb; ++cb) {
+      const uint32_t dst = smem_addr(Ws) + cb * kTcTile * 128;
+      if (!is_kr) {
+        tma_load_2d(dst, &T.map_wd, k_lo + 64 * cb, tile * kTcTile, wb);
+      } else {
+        tma_load_2d(dst, &T.map_wk, k_lo + 64 * cb, 16 * kr_tile, wb);
+        tma_load_2d(dst + 16 * 128, &T.map_wk, k_lo + 64 * cb, half + 16 * kr_tile, wb);
+      }
+    }
+  }
   pdl_wait();
   const Fp8Page fp = fp8_page(a.page_size, a.d_c, a.d_rope);
   const int M = a.n_tokens, nk = ks / 16;
-  for (int m0 = 0; m0 < M; m0 += kTcMb) {
+  uint32_t pass = 0;
+  for (int m0 = 0; m0 < M; m0 += kTcMb, ++pass) {
     const int mc = min(kTcMb, M - m0), mpad = (mc + 15) & ~15;
     const int combos = (mpad / 16) * 2, kparts = 8 / combos;  // warps per (m16, n16) pair split the K slice
-    for (int i = tid; i < mpad * ku; i += kTcThreads) {
-      const int r = i / ku, u = i % ku;
-      if (r < mc)
-        cp_async16(smem_addr(Hs) + swz(r, u, ku), H + (size_t)(m0 + r) * K + k_lo + u * 8);
-      else
-        *reinterpret_cast<uint4*>(Hs + swz(r, u, ku)) = make_uint4(0, 0, 0, 0);
+    if (tid == 0) {
+      // h rows of the pass (16-row boxes when the pass has at most 16 tokens)
+      const bool small = mpad == 16;
+      mbar_expect_local(hb, (uint32_t)(small ? 16 : kTcMb) * ks * 2);
+      for (int cb = 0; cb < ncb; ++cb)
+        tma_load_2d(smem_addr(Hs) + cb * kTcMb * 128, small ? &T.map_h16 : &T.map_h, k_lo + 64 * cb, m0, hb);
     }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
+    if ((pass == 0 && !mbar_wait_bounded(wb, 0)) || !mbar_wait_bounded(hb, pass & 1)) {
+      record_status(a.status, MLA_ERR_TIMEOUT);
+      return;
+    }
     {
       const int combo = warp % combos, kp = warp / combos;
       if (kp < kparts) {
         const int mt = (combo >> 1) * 16, nt = (combo & 1) * 16, per = nk / kparts;
         float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
         for (int kk = kp * per; kk < (kp + 1) * per; ++kk) {
           uint32_t af[4], b00, b01, b10, b11;
-          load_a(Hs, ku, mt, kk * 16, lane, af);
-          load_b_nk(Ws, ku, kk * 16, nt, lane, b00, b01, b10, b11);
+          load_a_cb(Hs, kTcMb, mt, kk * 16, lane, af);
+          load_b_nk_cb(Ws, kTcTile, kk * 16, nt, lane, b00, b01, b10, b11);
           mma_bf16(acc0, af, b00, b01);
           mma_bf16(acc1, af, b10, b11);
         }
@@ -319,7 +346,7 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
         for (int kp = 1; kp < kparts; ++kp) v += Ps[(size_t)kp * kTcMb * kTcTile + i];
         Ps[i] = v;
       }
-    cl.sync();  // every CTA's partial tile is complete
+    cl.sync();  // every CTA's partial tile is complete (and this CTA is done reading Hs)
     // this CTA finishes rows [rank * rows, (rank + 1) * rows) of the tile
     const int rows = mpad / kTcCluster;
     const int per_row = is_kr ? kTcTile / 2 : kTcTile;
@@ -409,14 +436,22 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
   const bool tc = d.act_dtype == MLA_BF16 && d.cache_dtype != MLA_F32 && d.d_model % (kTcCluster * 64) == 0 &&
                   d.d_c % kTcTile == 0 && d.d_rope % kTcTile == 0 && append_tc_smem(d) <= 227 * 1024;
   if (tc) {
+    AppendTcArgs t;
+    t.a = a;
+    const uint64_t row_bytes = (uint64_t)d.d_model * 2;
+    if (!make_tile_map_bf16(&t.map_wd, W_dkv, d.d_model, d.d_c, row_bytes, 64, kTcTile) ||
+        !make_tile_map_bf16(&t.map_wk, W_kr, d.d_model, d.d_rope, row_bytes, 64, 16) ||
+        !make_tile_map_bf16(&t.map_h, h, d.d_model, n_tokens, row_bytes, 64, kTcMb) ||
+        !make_tile_map_bf16(&t.map_h16, h, d.d_model, n_tokens, row_bytes, 64, 16))
+      return cudaErrorInvalidValue;
     const size_t smem = append_tc_smem(d);
     const int tgrid = (d.d_c / kTcTile + d.d_rope / kTcTile) * kTcCluster;
     if (d.cache_dtype == MLA_BF16) {
       cudaFuncSetAttribute(append_tc_kernel<MLA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      launch_pdl(append_tc_kernel<MLA_BF16>, dim3(tgrid), dim3(kTcThreads), smem, st, a);
+      launch_pdl(append_tc_kernel<MLA_BF16>, dim3(tgrid), dim3(kTcThreads), smem, st, t);
     } else {
       cudaFuncSetAttribute(append_tc_kernel<MLA_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      launch_pdl(append_tc_kernel<MLA_FP8_E4M3>, dim3(tgrid), dim3(kTcThreads), smem, st, a);
+      launch_pdl(append_tc_kernel<MLA_FP8_E4M3>, dim3(tgrid), dim3(kTcThreads), smem, st, t);
     }
   } else if (d.act_dtype == MLA_F32) {
     if (d.cache_dtype == MLA_F32) MLA_PROJ(float, MLA_F32);

@@ -21,6 +21,8 @@
 //   2. threads over (token, latent column) form u from the split partials;
 //   3. warps take rows of W^UV_h, each lane holding 16-byte vectors of the row,
 //      and dot them with every token's u (warp-shuffle reduction).
+#include <cuda.h>
+
 #include "mla_internal.cuh"
 #include "mma_tile.cuh"
 
@@ -128,44 +130,61 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(
   }
 }
 
-constexpr int kTcTok = 64;  // tokens merged per pass (rows of the u tile)
+constexpr int kTcTok = 64;                 // tokens merged per pass (rows of the u tile)
+constexpr int kTcDc = 512, kTcDv = 128;   // DeepSeek-V3 shape of W^UV_h
+constexpr uint32_t kTcWBytes = kTcDv * kTcDc * 2;  // 128 KB
 
-size_t combine_tc_smem(const mla_dims& d) { return (size_t)d.d_v * d.d_c * 2 + (size_t)kTcTok * d.d_c * 2; }
+struct CombineTcArgs {
+  const int32_t* plan;
+  const float* o_part;
+  const float* lse_part;
+  __nv_bfloat16* out;
+  float* lse_out;
+  int* status;
+  int n_heads, batch, n_q;
+  CUtensorMap map_w;  // W_uv as [n_heads * d_v rows][d_c] bf16, box 64 x 128, 128-byte swizzle
+};
 
-// bf16 activations: d_c % 128 == 0 (lanes x 4 columns, swizzle groups),
-// d_v % 16 == 0 (16-column pairs over the eight warps).
-__global__ void __launch_bounds__(kThreads) combine_tc_kernel(
-    const __nv_bfloat16* __restrict__ W_uv, int n_heads, int d_c, int d_v, int batch, int n_q,
-    const int32_t* __restrict__ plan, const float* __restrict__ o_part, const float* __restrict__ lse_part,
-    __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out) {
-  extern __shared__ __align__(128) uint8_t smem_tc[];
-  const int h = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cu = d_c / 8;  // 16-byte units per row of W^UV_h and of u
-  uint8_t* Ws = smem_tc;
-  uint8_t* Us = smem_tc + (size_t)d_v * d_c * 2;
+size_t combine_tc_smem() { return kTcWBytes + (size_t)kTcTok * kTcDc * 2 + 1024; }
+
+// bf16 activations at DeepSeek-V3 dims.  W^UV_h (d_v rows x d_c columns)
+// arrives by eight TMA boxes into [8 column blocks][128 rows][128 B]
+// (128-byte swizzle) while the CTA merges the splits into the bf16 u tile
+// [8 column blocks][64 tokens][128 B] in the same layout; warp w then owns
+// output columns [16w, 16w + 16) for four 16-token tiles at a time.
+__global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_constant__ CombineTcArgs P) {
+  extern __shared__ uint8_t smem_tc[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_tc) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t wbar;
   __shared__ float s_mx[kTcTok], s_inv[kTcTok];
+  const int h = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_heads = P.n_heads, batch = P.batch, n_q = P.n_q;
+  const int32_t* plan = P.plan;
+  uint8_t* Ws = smem;              // [8][d_v][128 B]
+  uint8_t* Us = smem + kTcWBytes;  // [8][kTcTok][128 B]
   const int M = batch * n_q;
-
+  const uint32_t bar = smem_addr(&wbar);
+  if (tid == 0) mbar_init_local(bar, 1);
+  __syncthreads();
   pdl_trigger();
-  // W^UV_h: rows j (N) x columns c (K)
-  const __nv_bfloat16* Wh = W_uv + (size_t)h * d_v * d_c;
-  for (int i = tid; i < d_v * cu; i += kThreads) {
-    const int r = i / cu, u = i % cu;
-    cp_async16(smem_addr(Ws) + swz(r, u, cu), Wh + (size_t)r * d_c + u * 8);
+  if (tid == 0) {
+    mbar_expect_local(bar, kTcWBytes);
+    for (int cb = 0; cb < kTcDc / 64; ++cb)
+      tma_load_2d(smem_addr(Ws) + cb * kTcDv * 128, &P.map_w, 64 * cb, h * kTcDv, bar);
   }
-  cp_async_commit();
   pdl_wait();
   const int splits = plan[batch + 2];
   const int n_slots = batch + splits - 1;  // slot stride of the decode that wrote the partials
+  bool w_ready = false;
 
   for (int m0 = 0; m0 < M; m0 += kTcTok) {
     const int mc = min(kTcTok, M - m0), mpad = (mc + 15) & ~15;
-    __syncthreads();  // previous pass done with Us
+    __syncthreads();  // previous pass done with Us and the weights
     // merge weights: warp per token computes the reference max and 1/sum
     for (int mi = warp; mi < mc; mi += kThreads / 32) {
       const int m = m0 + mi, b = m / n_q, t = m % n_q;
       const int lo = plan[batch + 5 + 2 * b], n = min(plan[batch + 6 + 2 * b], kMaxSplits);
-      const float* lse = lse_part + ((size_t)t * n_slots + lo + b) * n_heads + h;
+      const float* lse = P.lse_part + ((size_t)t * n_slots + lo + b) * n_heads + h;
       float mx = -INFINITY;
       for (int k = lane; k < n; k += 32) mx = fmaxf(mx, lse[(size_t)k * n_heads]);
 #pragma unroll
@@ -177,23 +196,23 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(
       if (lane == 0) {
         s_mx[mi] = mx;
         s_inv[mi] = sum > 0.f ? 1.f / sum : 0.f;
-        if (lse_out) lse_out[(size_t)m * n_heads + h] = sum > 0.f ? (mx + log2f(sum)) * kLn2 : -INFINITY;
+        if (P.lse_out) P.lse_out[(size_t)m * n_heads + h] = sum > 0.f ? (mx + log2f(sum)) * kLn2 : -INFINITY;
       }
     }
     __syncthreads();
     // u[m, c..c+3] = sum_k w_k o_k[c..c+3]: one item per (token, 4 columns)
     // over every thread of the CTA; the splits are read eight at a time with
     // all loads issued before any is used
-    const int c4n = d_c / 4, n_items = mpad * c4n;
-    for (int it = tid; it < n_items; it += kThreads) {
+    constexpr int c4n = kTcDc / 4;
+    for (int it = tid; it < mpad * c4n; it += kThreads) {
       const int mi = it / c4n, c0 = (it % c4n) * 4;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       if (mi < mc && s_mx[mi] > -INFINITY) {
         const int m = m0 + mi, b = m / n_q, t = m % n_q;
         const int lo = plan[batch + 5 + 2 * b], n = min(plan[batch + 6 + 2 * b], kMaxSplits);
         const size_t s0 = (size_t)t * n_slots + lo + b;
-        const float* lp = lse_part + s0 * n_heads + h;
-        const float* op = o_part + (s0 * n_heads + h) * d_c + c0;
+        const float* lp = P.lse_part + s0 * n_heads + h;
+        const float* op = P.o_part + (s0 * n_heads + h) * kTcDc + c0;
         const float mx = s_mx[mi], inv = s_inv[mi];
         constexpr int kU = 8;
         for (int k0 = 0; k0 < n; k0 += kU) {
@@ -202,7 +221,7 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(
 #pragma unroll
           for (int u = 0; u < kU; ++u) {
             const int k = min(k0 + u, n - 1);  // in-range duplicate for the tail, weight zeroed below
-            v[u] = *reinterpret_cast<const float4*>(op + (size_t)k * n_heads * d_c);
+            v[u] = *reinterpret_cast<const float4*>(op + (size_t)k * n_heads * kTcDc);
             l[u] = lp[(size_t)k * n_heads];
           }
 #pragma unroll
@@ -224,33 +243,48 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(
       uint2 pk;
       pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
       pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
-      *reinterpret_cast<uint2*>(Us + swz(mi, c0 >> 3, cu) + (c0 & 7) * 2) = pk;
+      *reinterpret_cast<uint2*>(Us + swz_cb(mi, c0 >> 3, kTcTok) + (c0 & 7) * 2) = pk;
     }
-    cp_async_wait<0>();
+    if (!w_ready) {
+      if (!mbar_wait_bounded(bar, 0)) {
+        record_status(P.status, MLA_ERR_TIMEOUT);
+        return;
+      }
+      w_ready = true;
+    }
     __syncthreads();
-    // o[m, j] = sum_c u[m, c] W^UV_h[j, c]
-    const int g = lane >> 2, q = lane & 3;
-    for (int np = warp; np * 16 < d_v; np += kThreads / 32) {
-      for (int mt = 0; mt < mpad; mt += 16) {
-        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int k0 = 0; k0 < d_c; k0 += 16) {
-          uint32_t af[4], b00, b01, b10, b11;
-          load_a(Us, cu, mt, k0, lane, af);
-          load_b_nk(Ws, cu, k0, np * 16, lane, b00, b01, b10, b11);
-          mma_bf16(acc0, af, b00, b01);
-          mma_bf16(acc1, af, b10, b11);
-        }
-        const int r0 = mt + g, r1 = mt + g + 8, col = np * 16 + 2 * q;
-        __nv_bfloat16* o0 = out + ((size_t)(m0 + r0) * n_heads + h) * d_v + col;
-        __nv_bfloat16* o1 = out + ((size_t)(m0 + r1) * n_heads + h) * d_v + col;
-        if (r0 < mc) {
-          *reinterpret_cast<__nv_bfloat162*>(o0) = __floats2bfloat162_rn(acc0[0], acc0[1]);
-          *reinterpret_cast<__nv_bfloat162*>(o0 + 8) = __floats2bfloat162_rn(acc1[0], acc1[1]);
-        }
-        if (r1 < mc) {
-          *reinterpret_cast<__nv_bfloat162*>(o1) = __floats2bfloat162_rn(acc0[2], acc0[3]);
-          *reinterpret_cast<__nv_bfloat162*>(o1 + 8) = __floats2bfloat162_rn(acc1[2], acc1[3]);
-        }
+    // o[m, j] = sum_c u[m, c] W^UV_h[j, c]: warp w, columns [16w, 16w + 16)
+    const int g = lane >> 2, q = lane & 3, n0 = warp * 16;
+    float acc[4][2][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+#pragma unroll 4
+    for (int k0 = 0; k0 < kTcDc; k0 += 16) {
+      uint32_t b00, b01, b10, b11;
+      load_b_nk_cb(Ws, kTcDv, k0, n0, lane, b00, b01, b10, b11);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (16 * i >= mpad) break;
+        uint32_t af[4];
+        load_a_cb(Us, kTcTok, 16 * i, k0, lane, af);
+        mma_bf16(acc[i][0], af, b00, b01);
+        mma_bf16(acc[i][1], af, b10, b11);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r0 = 16 * i + g, r1 = r0 + 8, col = n0 + 2 * q;
+      __nv_bfloat16* o0 = P.out + ((size_t)(m0 + r0) * n_heads + h) * kTcDv + col;
+      __nv_bfloat16* o1 = P.out + ((size_t)(m0 + r1) * n_heads + h) * kTcDv + col;
+      if (r0 < mc) {
+        *reinterpret_cast<__nv_bfloat162*>(o0) = __floats2bfloat162_rn(acc[i][0][0], acc[i][0][1]);
+        *reinterpret_cast<__nv_bfloat162*>(o0 + 8) = __floats2bfloat162_rn(acc[i][1][0], acc[i][1][1]);
+      }
+      if (r1 < mc) {
+        *reinterpret_cast<__nv_bfloat162*>(o1) = __floats2bfloat162_rn(acc[i][0][2], acc[i][0][3]);
+        *reinterpret_cast<__nv_bfloat162*>(o1 + 8) = __floats2bfloat162_rn(acc[i][1][2], acc[i][1][3]);
       }
     }
   }
@@ -263,7 +297,8 @@ int combine_max_splits() { return kMaxSplits; }
 int combine_max_d_c(int act_dtype) { return kMaxVecPerLane * 32 * (act_dtype == MLA_F32 ? 4 : 8); }
 
 cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n_q, const int32_t* plan,
-                           const float* o_part, const float* lse_part, void* out, float* lse_out, cudaStream_t st) {
+                           const float* o_part, const float* lse_part, void* out, float* lse_out, int* status,
+                           cudaStream_t st) {
   const size_t smem = combine_smem_bytes(d);
   cudaError_t e;
   if (d.act_dtype == MLA_F32) {
@@ -271,13 +306,24 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
     if (e != cudaSuccess) return e;
     combine_kernel<float><<<d.n_heads, kThreads, smem, st>>>((const float*)W_uv, d.n_heads, d.d_c, d.d_v, batch, n_q,
                                                               plan, o_part, lse_part, (float*)out, lse_out);
-  } else if (d.d_c % 128 == 0 && d.d_v % 16 == 0 && combine_tc_smem(d) <= 227 * 1024 &&
-             (reinterpret_cast<uintptr_t>(out) & 3u) == 0) {  // paired bf16 stores
-    const size_t tsm = combine_tc_smem(d);
+  } else if (d.d_c == kTcDc && d.d_v == kTcDv && (reinterpret_cast<uintptr_t>(out) & 3u) == 0) {
+    // paired bf16 stores; tile shapes are compile-time (DeepSeek-V3 dims)
+    CombineTcArgs p;
+    p.plan = plan;
+    p.o_part = o_part;
+    p.lse_part = lse_part;
+    p.out = (__nv_bfloat16*)out;
+    p.lse_out = lse_out;
+    p.status = status;
+    p.n_heads = d.n_heads;
+    p.batch = batch;
+    p.n_q = n_q;
+    if (!make_tile_map_bf16(&p.map_w, W_uv, kTcDc, (uint64_t)d.n_heads * kTcDv, (uint64_t)kTcDc * 2, 64, kTcDv))
+      return cudaErrorInvalidValue;
+    const size_t tsm = combine_tc_smem();
     e = cudaFuncSetAttribute(combine_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(combine_tc_kernel, dim3(d.n_heads), dim3(kThreads), tsm, st, (const __nv_bfloat16*)W_uv,
-                   d.n_heads, d.d_c, d.d_v, batch, n_q, plan, o_part, lse_part, (__nv_bfloat16*)out, lse_out);
+    e = launch_pdl(combine_tc_kernel, dim3(d.n_heads), dim3(kThreads), tsm, st, p);
     if (e != cudaSuccess) return e;
   } else {
     e = cudaFuncSetAttribute(combine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -222,7 +222,8 @@ int mla_combine(const mla_dims* dims, const void* W_uv, int batch, int n_q, int 
   trace_record(MLA_TRACE_COMBINE, false, (cudaStream_t)stream);
   cudaError_t e = launch_combine(*dims, W_uv, batch, n_q, reinterpret_cast<const int32_t*>(ws + L.off_plan),
                                  reinterpret_cast<const float*>(ws + L.off_o),
-                                 reinterpret_cast<const float*>(ws + L.off_lse), out, lse_out, (cudaStream_t)stream);
+                                 reinterpret_cast<const float*>(ws + L.off_lse), out, lse_out, status_ptr(),
+                                 (cudaStream_t)stream);
   trace_record(MLA_TRACE_COMBINE, true, (cudaStream_t)stream);
   return launch_status(e);
 }

@@ -68,6 +68,12 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// 2-D bf16 TMA tensor map with the 128-byte swizzle (box_cols * 2 == 128),
+// written into `map` (a 64-byte aligned CUtensorMap).  False if the driver
+// entry point is missing or the encoder rejects the shape.
+bool make_tile_map_bf16(void* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                        uint32_t box_cols, uint32_t box_rows);
+
 // ----------------------------------------------------------------------------
 // Element access
 // ----------------------------------------------------------------------------
@@ -215,6 +221,6 @@ cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st);
 int decode_tc_auto_splits(int num_sms, int n_q);
 
 cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n_q, const int32_t* plan,
-                           const float* o_part, const float* lse_part, void* out, float* lse_out, cudaStream_t st);
+                           const float* o_part, const float* lse_part, void* out, float* lse_out, int* status, cudaStream_t st);
 
 }  // namespace mla

@@ -72,3 +72,65 @@ __device__ __forceinline__ void load_b_nk(const void* tile, int row_units, int k
 }
 
 }  // namespace mla
+
+// ----------------------------------------------------------------------------
+// Tiles written by TMA with the 128-byte swizzle: a K-contiguous (or
+// N-contiguous) matrix is stored as [row_units/8 column blocks][rows][128 B],
+// the 16-byte unit index inside each 128-byte row XOR-ed with (row & 7).
+// ----------------------------------------------------------------------------
+namespace mla {
+
+__device__ __forceinline__ uint32_t swz_cb(int r, int u, int rows) {
+  return (uint32_t)((((u >> 3) * rows + r) << 7) + ((((u & 7) ^ (r & 7))) << 4));
+}
+
+__device__ __forceinline__ void load_a_cb(const void* tile, int rows, int m0, int k0, int lane, uint32_t (&a)[4]) {
+  const int j = lane >> 3, r = m0 + (j & 1) * 8 + (lane & 7), u = (k0 >> 3) + (j >> 1);
+  ldsm_x4(smem_addr(tile) + swz_cb(r, u, rows), a[0], a[1], a[2], a[3]);
+}
+
+// B fragments of two n8 tiles from a K x N tile (N contiguous), rows = K
+__device__ __forceinline__ void load_b_kn_cb(const void* tile, int rows, int k0, int n0, int lane, uint32_t& b00,
+                                             uint32_t& b01, uint32_t& b10, uint32_t& b11) {
+  const int j = lane >> 3, r = k0 + (j & 1) * 8 + (lane & 7), u = (n0 >> 3) + (j >> 1);
+  ldsm_x4_t(smem_addr(tile) + swz_cb(r, u, rows), b00, b01, b10, b11);
+}
+
+// B fragments of two n8 tiles from an N x K tile (K contiguous), rows = N
+__device__ __forceinline__ void load_b_nk_cb(const void* tile, int rows, int k0, int n0, int lane, uint32_t& b00,
+                                             uint32_t& b01, uint32_t& b10, uint32_t& b11) {
+  const int j = lane >> 3, r = n0 + (j >> 1) * 8 + (lane & 7), u = (k0 >> 3) + (j & 1);
+  ldsm_x4(smem_addr(tile) + swz_cb(r, u, rows), b00, b01, b10, b11);
+}
+
+// TMA 2-D load into this CTA's shared memory, completing on a local mbarrier
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_init_local(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_local(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// Bounded wait on phase `parity`; false if it did not complete within ~2 s.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (clock64() - t0 > 4000000000LL) return false;
+  }
+}
+
+}  // namespace mla
