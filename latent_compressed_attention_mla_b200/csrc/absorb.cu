@@ -8,12 +8,15 @@
 // The output is in the activation type, or f16 when the decode path reads
 // f16 queries (FP8 cache on the tensor cores).
 //
-// bf16 activations at DeepSeek-V3 dims (absorb_tc_kernel): one CTA per head
-// brings W^UK_h (d_nope x d_c, 128 KB) into shared memory with eight TMA
+// bf16 activations at DeepSeek-V3 dims (absorb_tc_kernel): one CTA per (head,
+// block of 32, 64 or 128 tokens; the largest block that still gives every SM a
+// CTA) brings W^UK_h (d_nope x d_c, 128 KB) into shared memory with eight TMA
 // boxes (issued before the programmatic-launch wait, so the fetch overlaps the
-// previous kernel), stages the head's q^C rows, and multiplies them with
+// previous kernel), stages the block's q^C rows, and multiplies them with
 // mma.sync m16n8k16 (fp32 accumulation); the eight warps split the d_c output
-// columns.  The kernel is bound by the 16.8 MB of W^UK read once from HBM.
+// columns, and the rows leave through a swizzled shared-memory stage as
+// 16-byte stores.  W^UK is read once from HBM (16.8 MB); the token blocks of
+// one head re-read it from L2.
 //
 // fp32 activations (absorb_kernel): one CTA per (head, 16-vector slice of d_c).  Thread (cg, dg) loads the
 // 16-byte vectors of W^UK_h for its column group cg and its rows d in group
@@ -229,49 +232,82 @@ __global__ void __launch_bounds__(128) absorb_kernel(const AbsorbArgs a) {
   }
 }
 
-// RoPE of q^R at the query's own position for head h (all tokens).
+// RoPE of q^R at the query's own position for head h, tokens [m0, m0 + mc).
+// Every thread first loads its items' positions and q^R pairs (four items at
+// a time), then rotates and stores them.
 template <typename T, typename TO>
-__device__ void rope_queries(const AbsorbArgs& a, int h) {
-  const int D = a.d_c + a.d_rope, M = a.batch * a.n_q, half = a.d_rope >> 1;
+__device__ void rope_query_rows(const AbsorbArgs& a, int h, int m0, int mc) {
+  const int D = a.d_c + a.d_rope, half = a.d_rope >> 1, n_items = mc * half;
   const T* qr = static_cast<const T*>(a.q_rope);
   TO* qa = static_cast<TO*>(a.q_abs);
-  for (int i = threadIdx.x; i < M * half; i += blockDim.x) {
-    const int m = i / half, k = i % half;
-    const int b = m / a.n_q, t = m % a.n_q;
-    const int p = a.seq_lens[b] - a.n_q + t;
-    float cs, sn;
-    rope_cos_sin(p, k, half, a.rope_base, &cs, &sn);
-    const T* src = qr + ((size_t)m * a.n_heads + h) * a.d_rope;
-    const float x1 = to_f(src[k]), x2 = to_f(src[half + k]);
-    TO* dst = qa + ((size_t)m * a.n_heads + h) * D + a.d_c;
-    dst[k] = from_f<TO>(x1 * cs - x2 * sn);
-    dst[half + k] = from_f<TO>(x2 * cs + x1 * sn);
+  int k_freq = -1;
+  double inv_freq = 0.0;
+  for (int i0 = 0; i0 < n_items; i0 += 4 * (int)blockDim.x) {
+    int pos[4];
+    float x1[4], x2[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * (int)blockDim.x + (int)threadIdx.x;
+      pos[u] = 0;
+      x1[u] = x2[u] = 0.f;
+      if (i < n_items) {
+        const int m = m0 + i / half, k = i % half, b = m / a.n_q, t = m % a.n_q;
+        pos[u] = a.seq_lens[b] - a.n_q + t;
+        const T* src = qr + ((size_t)m * a.n_heads + h) * a.d_rope;
+        x1[u] = to_f(src[k]);
+        x2[u] = to_f(src[half + k]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * (int)blockDim.x + (int)threadIdx.x;
+      if (i < n_items) {
+        const int m = m0 + i / half, k = i % half;
+        if (k != k_freq) {
+          k_freq = k;
+          inv_freq = rope_inv_freq(k, half, a.rope_base);
+        }
+        float cs, sn;
+        rope_cos_sin_at(pos[u], inv_freq, &cs, &sn);
+        TO* dst = qa + ((size_t)m * a.n_heads + h) * D + a.d_c;
+        dst[k] = from_f<TO>(x1[u] * cs - x2[u] * sn);
+        dst[half + k] = from_f<TO>(x2[u] * cs + x1[u] * sn);
+      }
+    }
   }
 }
 
 constexpr int kTcThreads = 256;
-constexpr int kTcMaxTok = 256;  // query rows staged per pass
-constexpr int kTcDn = 128, kTcDc = 512;  // DeepSeek-V3 shape of W^UK_h
+constexpr int kTcDn = 128, kTcDc = 512;             // DeepSeek-V3 shape of W^UK_h
 constexpr uint32_t kTcWBytes = kTcDn * kTcDc * 2;  // 128 KB
+constexpr int kTcStageRows = 32;                     // output rows staged per round
+constexpr uint32_t kTcStageBytes = kTcStageRows * kTcDc * 2;
+
+size_t absorb_tc_smem(int tok) { return kTcWBytes + (size_t)tok * kTcDn * 2 + kTcStageBytes + 1024; }
 
 struct AbsorbTcArgs {
   AbsorbArgs a;
   CUtensorMap map_w;  // W_uk as [n_heads * d_nope rows][d_c] bf16, box 64 x 128, 128-byte swizzle
 };
 
-__device__ __forceinline__ void store2(__nv_bfloat16* p, float x, float y) {
-  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(x, y);
+__device__ __forceinline__ uint32_t pack2(float x, float y, __nv_bfloat16*) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
-__device__ __forceinline__ void store2(__half* p, float x, float y) {
-  *reinterpret_cast<__half2*>(p) = __floats2half2_rn(x, y);
+__device__ __forceinline__ uint32_t pack2(float x, float y, __half*) {
+  const __half2 v = __floats2half2_rn(x, y);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 // q~[m, h, :] = q^C[m, h, :] . W^UK_h for bf16 activations at DeepSeek-V3
-// dims.  W^UK_h (d_nope rows x d_c columns) arrives by eight TMA boxes into
-// [8 column blocks][128 rows][128 B] with the 128-byte swizzle; the query rows
-// are staged by cp.async in the same layout.  Warp w owns columns [64w,
-// 64w + 64) and runs two 16-row query tiles at a time over them.
-template <typename TO>
+// dims; CTA (h, j) takes head h and tokens [j TOK, (j + 1) TOK).  W^UK_h
+// (d_nope rows x d_c columns) arrives by eight TMA boxes into [8 column
+// blocks][128 rows][128 B] with the 128-byte swizzle, issued before the
+// programmatic-launch wait; the query rows are staged by cp.async in the same
+// layout.  Warp w owns columns [64w, 64w + 64) and runs two 16-row query
+// tiles at a time; each 32-row result goes through a swizzled shared-memory
+// stage so that every output row leaves as 1 KB of 16-byte stores.
+template <typename TO, int TOK>
 __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_constant__ AbsorbTcArgs P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -279,8 +315,10 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_cons
   const AbsorbArgs& a = P.a;
   const int h = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int D = a.d_c + a.d_rope, M = a.batch * a.n_q;
-  uint8_t* Ws = smem;              // [8][128][128 B]
-  uint8_t* As = smem + kTcWBytes;  // [2][kTcMaxTok][128 B]
+  const int m0 = blockIdx.y * TOK, mc = min(TOK, M - m0), mpad = (mc + 31) & ~31;
+  uint8_t* Ws = smem;                    // [8][128][128 B]
+  uint8_t* As = smem + kTcWBytes;        // [2][TOK][128 B]
+  uint8_t* Os = As + TOK * kTcDn * 2;    // [32 rows][64 units of 16 B], unit u at u ^ (row & 7)
   const uint32_t bar = smem_addr(&wbar);
   if (tid == 0) mbar_init_local(bar, 1);
   __syncthreads();
@@ -291,69 +329,70 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_cons
       tma_load_2d(smem_addr(Ws) + cb * kTcDn * 128, &P.map_w, 64 * cb, h * kTcDn, bar);
   }
   pdl_wait();
-  if (h == 0) build_plan(a);
+  if (h == 0 && blockIdx.y == 0) build_plan(a);
   {
-    const size_t nblk = gridDim.x, bid = blockIdx.x;
+    const size_t nblk = (size_t)gridDim.x * gridDim.y, bid = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
     for (size_t i = bid * kTcThreads + tid; i < a.lse_count; i += nblk * kTcThreads) a.lse_part[i] = -INFINITY;
   }
   const __nv_bfloat16* qn = static_cast<const __nv_bfloat16*>(a.q_nope);
   TO* qa = static_cast<TO*>(a.q_abs);
-  bool w_ready = false;
-  for (int m0 = 0; m0 < M; m0 += kTcMaxTok) {
-    const int mc = min(kTcMaxTok, M - m0), mpad = (mc + 31) & ~31;
-    __syncthreads();  // previous pass done with As
-    for (int i = tid; i < mpad * (kTcDn / 8); i += kTcThreads) {
-      const int r = i / (kTcDn / 8), u = i % (kTcDn / 8);
-      const uint32_t off = swz_cb(r, u, kTcMaxTok);
-      if (r < mc)
-        cp_async16(smem_addr(As) + off, qn + ((size_t)(m0 + r) * a.n_heads + h) * kTcDn + u * 8);
-      else
-        *reinterpret_cast<uint4*>(As + off) = make_uint4(0, 0, 0, 0);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    if (!w_ready) {
-      if (!mbar_wait_bounded(bar, 0)) {
-        record_status(a.status, MLA_ERR_TIMEOUT);
-        return;
+  for (int i = tid; i < mpad * (kTcDn / 8); i += kTcThreads) {
+    const int r = i / (kTcDn / 8), u = i % (kTcDn / 8);
+    const uint32_t off = swz_cb(r, u, TOK);
+    if (r < mc)
+      cp_async16(smem_addr(As) + off, qn + ((size_t)(m0 + r) * a.n_heads + h) * kTcDn + u * 8);
+    else
+      *reinterpret_cast<uint4*>(As + off) = make_uint4(0, 0, 0, 0);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  const bool w_ok = mbar_wait_bounded(bar, 0);
+  if (__syncthreads_or(!w_ok)) {  // also publishes the staged query rows
+    if (tid == 0) record_status(a.status, MLA_ERR_TIMEOUT);
+    return;
+  }
+  const int g = lane >> 2, q = lane & 3;
+  for (int mt = 0; mt < mpad; mt += 32) {
+    float acc[2][8][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+#pragma unroll
+    for (int k0 = 0; k0 < kTcDn; k0 += 16) {
+      uint32_t a0[4], a1[4];
+      load_a_cb(As, TOK, mt, k0, lane, a0);
+      load_a_cb(As, TOK, mt + 16, k0, lane, a1);
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        uint32_t b00, b01, b10, b11;
+        load_b_kn_cb(Ws, kTcDn, k0, warp * 64 + np * 16, lane, b00, b01, b10, b11);
+        mma_bf16(acc[0][2 * np], a0, b00, b01);
+        mma_bf16(acc[0][2 * np + 1], a0, b10, b11);
+        mma_bf16(acc[1][2 * np], a1, b00, b01);
+        mma_bf16(acc[1][2 * np + 1], a1, b10, b11);
       }
-      w_ready = true;
     }
+    if (mt > 0) __syncthreads();  // the previous round's rows have left the stage
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int r0 = 16 * i + g, unit = warp * 8 + j;
+        *reinterpret_cast<uint32_t*>(Os + r0 * 1024 + ((unit ^ (r0 & 7)) << 4) + 4 * q) =
+            pack2(acc[i][j][0], acc[i][j][1], (TO*)nullptr);
+        *reinterpret_cast<uint32_t*>(Os + (r0 + 8) * 1024 + ((unit ^ (r0 & 7)) << 4) + 4 * q) =
+            pack2(acc[i][j][2], acc[i][j][3], (TO*)nullptr);
+      }
     __syncthreads();
-    const int g = lane >> 2, q = lane & 3;
-    for (int mt = 0; mt < mpad; mt += 32) {
-      float acc[2][8][4];
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
-#pragma unroll
-      for (int k0 = 0; k0 < kTcDn; k0 += 16) {
-        uint32_t a0[4], a1[4];
-        load_a_cb(As, kTcMaxTok, mt, k0, lane, a0);
-        load_a_cb(As, kTcMaxTok, mt + 16, k0, lane, a1);
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t b00, b01, b10, b11;
-          load_b_kn_cb(Ws, kTcDn, k0, warp * 64 + np * 16, lane, b00, b01, b10, b11);
-          mma_bf16(acc[0][2 * np], a0, b00, b01);
-          mma_bf16(acc[0][2 * np + 1], a0, b10, b11);
-          mma_bf16(acc[1][2 * np], a1, b00, b01);
-          mma_bf16(acc[1][2 * np + 1], a1, b10, b11);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = warp * 64 + j * 8 + 2 * q;
-          const int r0 = mt + 16 * i + g, r1 = r0 + 8;
-          if (r0 < mc) store2(qa + ((size_t)(m0 + r0) * a.n_heads + h) * D + col, acc[i][j][0], acc[i][j][1]);
-          if (r1 < mc) store2(qa + ((size_t)(m0 + r1) * a.n_heads + h) * D + col, acc[i][j][2], acc[i][j][3]);
-        }
+    const int rows = min(kTcStageRows, mc - mt);
+    for (int i = tid; i < rows * 64; i += kTcThreads) {
+      const int r = i >> 6, u = i & 63;
+      *reinterpret_cast<uint4*>(qa + ((size_t)(m0 + mt + r) * a.n_heads + h) * D + u * 8) =
+          *reinterpret_cast<const uint4*>(Os + r * 1024 + ((u ^ (r & 7)) << 4));
     }
   }
-  rope_queries<__nv_bfloat16, TO>(a, h);
+  rope_query_rows<__nv_bfloat16, TO>(a, h, m0, mc);
 }
 
 }  // namespace
@@ -388,24 +427,31 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
   a.lse_part = lse_part;
   a.lse_count = lse_count;
   a.status = status;
-  // the tensor-core kernel stages q^C with 16-byte copies
-  if (d.act_dtype == MLA_BF16 && absorb_tc_fits(d) && (reinterpret_cast<uintptr_t>(q_nope) & 15u) == 0) {
+  // the tensor-core kernel stages q^C with 16-byte copies and stores q~ rows
+  // (d_c + d_rope elements apart) with 16-byte stores
+  if (d.act_dtype == MLA_BF16 && absorb_tc_fits(d) && (reinterpret_cast<uintptr_t>(q_nope) & 15u) == 0 &&
+      (reinterpret_cast<uintptr_t>(q_abs) & 15u) == 0 && ((d.d_c + d.d_rope) * 2) % 16 == 0) {
     AbsorbTcArgs p;
     p.a = a;
     if (!make_tile_map_bf16(&p.map_w, W_uk, kTcDc, (uint64_t)d.n_heads * kTcDn, (uint64_t)kTcDc * 2, 64, kTcDn))
       return cudaErrorInvalidValue;
-    const size_t smem = kTcWBytes + (size_t)kTcMaxTok * kTcDn * 2 + 1024;
-    cudaError_t e;
-    if (q_abs_f16) {
-      e = cudaFuncSetAttribute(absorb_tc_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      e = launch_pdl(absorb_tc_kernel<__half>, dim3(d.n_heads), dim3(kTcThreads), smem, st, p);
-    } else {
-      e = cudaFuncSetAttribute(absorb_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
-      if (e != cudaSuccess) return e;
-      e = launch_pdl(absorb_tc_kernel<__nv_bfloat16>, dim3(d.n_heads), dim3(kTcThreads), smem, st, p);
-    }
+    // tokens per CTA: the largest block that still gives every SM a CTA
+    const int M = batch * n_q, sms = device_sm_count();
+    int tok = 32;
+    if ((long long)d.n_heads * ((M + 127) / 128) >= sms) tok = 128;
+    else if ((long long)d.n_heads * ((M + 63) / 64) >= sms) tok = 64;
+    const dim3 grid(d.n_heads, (M + tok - 1) / tok);
+    const size_t smem = absorb_tc_smem(tok);
+    auto pick = [&](auto k32, auto k64, auto k128) {
+      return tok == 128 ? k128 : tok == 64 ? k64 : k32;
+    };
+    auto kernel = q_abs_f16 ? pick(absorb_tc_kernel<__half, 32>, absorb_tc_kernel<__half, 64>,
+                                   absorb_tc_kernel<__half, 128>)
+                            : pick(absorb_tc_kernel<__nv_bfloat16, 32>, absorb_tc_kernel<__nv_bfloat16, 64>,
+                                   absorb_tc_kernel<__nv_bfloat16, 128>);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(kernel, grid, dim3(kTcThreads), smem, st, p);
     return e != cudaSuccess ? e : cudaGetLastError();
   }
   const int vec = d.act_dtype == MLA_F32 ? 4 : 8;

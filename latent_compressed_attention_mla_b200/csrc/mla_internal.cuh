@@ -112,14 +112,29 @@ __device__ __forceinline__ float e4m3_to_float(uint8_t code) {
   return float(v);
 }
 
-// RoPE angle cos/sin for rotation pair i of a d_rope-wide vector at position
-// pos: angle = pos * base^(-i/(d_rope/2)), evaluated in double precision and
-// rounded to float (positions reach 1.3e5, where a float angle loses ~1e-2 rad).
+// RoPE frequency of rotation pair i of a d_rope-wide vector: base^(-i/half),
+// in double precision.
+__device__ __forceinline__ double rope_inv_freq(int i, int half, float base) {
+  return exp(-log((double)base) * (double)i / (double)half);
+}
+
+// cos / sin of the RoPE angle pos * inv_freq.  The angle is formed in double
+// precision (positions reach 1.3e5, where a float angle is off by ~1e-2 rad),
+// brought into [-pi, pi] by Cody-Waite reduction against 2*pi held as the sum
+// of two doubles, and the reduced angle is evaluated in float (|error| of a
+// few 1e-7).
+__device__ __forceinline__ void rope_cos_sin_at(int pos, double inv_freq, float* c, float* s) {
+  constexpr double kTwoPiHi = 6.283185307179586232;    // 2*pi rounded to double
+  constexpr double kTwoPiLo = 2.4492935982947064e-16;  // 2*pi - kTwoPiHi
+  constexpr double kInvTwoPi = 0.15915494309189533577;
+  const double ang = (double)pos * inv_freq;
+  const double k = rint(ang * kInvTwoPi);
+  const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, ang));
+  sincosf((float)r, s, c);
+}
+
 __device__ __forceinline__ void rope_cos_sin(int pos, int i, int half, float base, float* c, float* s) {
-  double inv_freq = exp(-log((double)base) * (double)i / (double)half);
-  double ang = (double)pos * inv_freq;
-  *c = (float)cos(ang);
-  *s = (float)sin(ang);
+  rope_cos_sin_at(pos, rope_inv_freq(i, half, base), c, s);
 }
 
 // ----------------------------------------------------------------------------
@@ -217,6 +232,8 @@ cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t st);
 bool decode_tc_supported(const mla_dims& d, int n_q);
 // the tensor-core path for this cache reads the absorbed queries as f16
 bool decode_tc_wants_f16_queries(const mla_dims& d);
+// multiprocessor count of the current device (cached per device)
+int device_sm_count();
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st);
 int decode_tc_auto_splits(int num_sms, int n_q);
 

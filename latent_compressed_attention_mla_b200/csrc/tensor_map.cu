@@ -1,5 +1,6 @@
-// Host helper: 2-D TMA tensor maps through cuTensorMapEncodeTiled (reached via
-// the runtime's driver entry point, so the library does not link libcuda).
+// Host helpers: 2-D TMA tensor maps through cuTensorMapEncodeTiled (reached
+// via the runtime's driver entry point, so the library does not link
+// libcuda), and the device's multiprocessor count.
 #include <cuda.h>
 
 #include "mla_internal.cuh"
@@ -35,6 +36,18 @@ bool make_tile_map_bf16(void* map, const void* base, uint64_t cols, uint64_t row
   return enc(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+  constexpr int kMaxDev = 64;
+  static int cached[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < kMaxDev && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < kMaxDev) cached[dev] = n;
+  return n;
 }
 
 }  // namespace mla
