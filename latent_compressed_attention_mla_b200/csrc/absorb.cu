@@ -322,6 +322,7 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_cons
   const uint32_t bar = smem_addr(&wbar);
   if (tid == 0) mbar_init_local(bar, 1);
   __syncthreads();
+  MLA_STAMP(0);
   pdl_trigger();
   if (tid == 0) {
     mbar_expect_local(bar, kTcWBytes);
@@ -329,6 +330,7 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_cons
       tma_load_2d(smem_addr(Ws) + cb * kTcDn * 128, &P.map_w, 64 * cb, h * kTcDn, bar);
   }
   pdl_wait();
+  MLA_STAMP(1);
   if (h == 0 && blockIdx.y == 0) build_plan(a);
   {
     const size_t nblk = (size_t)gridDim.x * gridDim.y, bid = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
@@ -351,6 +353,7 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_cons
     if (tid == 0) record_status(a.status, MLA_ERR_TIMEOUT);
     return;
   }
+  MLA_STAMP(5);
   const int g = lane >> 2, q = lane & 3;
   for (int mt = 0; mt < mpad; mt += 32) {
     float acc[2][8][4];
@@ -392,7 +395,9 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_cons
           *reinterpret_cast<const uint4*>(Os + r * 1024 + ((u ^ (r & 7)) << 4));
     }
   }
+  MLA_STAMP(2);
   rope_query_rows<__nv_bfloat16, TO>(a, h, m0, mc);
+  MLA_STAMP(3);
 }
 
 }  // namespace
@@ -466,3 +471,5 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
 }
 
 }  // namespace mla
+
+MLA_STAMP_EXPORT(absorb)

@@ -199,6 +199,144 @@ __global__ void __launch_bounds__(256, 2) append_project_kernel(const AppendArgs
   }
 }
 
+// Small passes (at most kGvMaxTok tokens, bf16 activations): the projection
+// is a batched GEMV bound by reading the weights once; a cluster-free grid of
+// one wave starts every CTA at once (the tensor-core kernel's 8-CTA clusters
+// do not all fit on the GPCs together), which matters most for one token.  CTA j owns four output
+// columns: rows 4j..4j+3 of W^DKV, or for a k^R CTA the rotation pairs
+// (i0, i0 + 1) with their partners (i0 + half, i0 + 1 + half), i0 = 2 (j -
+// d_c/4), so RoPE stays inside the CTA.  Its 256 threads hold the four weight
+// rows in registers (16-byte vectors k = tid + 256 v), loaded before the
+// programmatic-launch wait; after it, each token's h row is dotted with them,
+// and the 4 x MT partial sums are reduced by a warp reduce-scatter and a
+// cross-warp sum in shared memory.  One wave of (d_c + d_rope) / 4 CTAs, no
+// clusters.
+constexpr int kGvThreads = 256;
+constexpr int kGvCols = 4;
+constexpr int kGvVec = 4;      // d_model <= kGvThreads * kGvVec * 8
+constexpr int kGvMaxTok = 4;
+
+template <int CACHE, int MT>
+__global__ void __launch_bounds__(kGvThreads) append_gemv_kernel(const AppendArgs a) {
+  constexpr int V = MT * kGvCols;  // partial sums per thread
+  static_assert(V <= 32 && (V & (V - 1)) == 0, "power-of-two partials per lane");
+  constexpr int kSteps = V == 1 ? 0 : V == 2 ? 1 : V == 4 ? 2 : V == 8 ? 3 : V == 16 ? 4 : 5;
+  __shared__ float red[kGvThreads / 32][V];
+  __shared__ float fin[V];
+  __shared__ int s_page[kGvMaxTok], s_row[kGvMaxTok], s_pos[kGvMaxTok];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int half = a.d_rope >> 1, c_ctas = a.d_c / kGvCols, nvec = a.d_model / 8;
+  const bool kr_cta = (int)blockIdx.x >= c_ctas;
+  const int i0 = ((int)blockIdx.x - c_ctas) * 2;
+  uint4 w[kGvCols][kGvVec];
+#pragma unroll
+  for (int r = 0; r < kGvCols; ++r) {
+    const __nv_bfloat16* wr =
+        !kr_cta ? static_cast<const __nv_bfloat16*>(a.W_dkv) + (size_t)(blockIdx.x * kGvCols + r) * a.d_model
+                : static_cast<const __nv_bfloat16*>(a.W_kr) + (size_t)(i0 + (r & 1) + (r >> 1) * half) * a.d_model;
+#pragma unroll
+    for (int v = 0; v < kGvVec; ++v) {
+      const int k = tid + kGvThreads * v;
+      w[r][v] = k < nvec ? *reinterpret_cast<const uint4*>(wr + 8 * k) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  pdl_trigger();
+  pdl_wait();
+  MLA_STAMP(1);
+  const int M = a.n_tokens;
+  if (tid < M) {
+    int prow = 0, position = 0;
+    s_page[tid] = token_slot(a, tid, &prow, &position);
+    s_row[tid] = prow;
+    s_pos[tid] = position;
+  }
+  const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(a.h);
+  for (int m0 = 0; m0 < M; m0 += MT) {
+    float x[V];
+#pragma unroll
+    for (int j = 0; j < MT; ++j) {
+#pragma unroll
+      for (int r = 0; r < kGvCols; ++r) x[j * kGvCols + r] = 0.f;
+      if (m0 + j < M) {
+        const __nv_bfloat16* hr = h + (size_t)(m0 + j) * a.d_model;
+#pragma unroll
+        for (int v = 0; v < kGvVec; ++v) {
+          const int k = tid + kGvThreads * v;
+          if (k < nvec) {
+            const uint4 hv = *reinterpret_cast<const uint4*>(hr + 8 * k);
+#pragma unroll
+            for (int r = 0; r < kGvCols; ++r) x[j * kGvCols + r] += dot_vec(w[r][v], hv, (__nv_bfloat16*)nullptr);
+          }
+        }
+      }
+    }
+    // reduce-scatter over the warp: at offset o a lane keeps the upper half of
+    // its values if (lane & o), the lower half otherwise, and adds the
+    // partner's copy of the half it keeps; after kSteps steps lane l holds
+    // value l >> (5 - kSteps), then the remaining offsets sum equal indices
+#pragma unroll
+    for (int st = 0; st < 5; ++st) {
+      const int o = 16 >> st;
+      if (st < kSteps) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < (V >> (st + 1)); ++i) {
+          const float send = up ? x[i] : x[i + (V >> (st + 1))];
+          const float keep = up ? x[i + (V >> (st + 1))] : x[i];
+          x[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      } else {
+        x[0] += __shfl_xor_sync(0xffffffffu, x[0], o);
+      }
+    }
+    if ((lane & ((1 << (5 - kSteps)) - 1)) == 0) red[warp][lane >> (5 - kSteps)] = x[0];
+    __syncthreads();
+    if (tid < V) {
+      float t = 0.f;
+#pragma unroll
+      for (int q = 0; q < kGvThreads / 32; ++q) t += red[q][tid];
+      fin[tid] = t;
+    }
+    __syncthreads();
+    // value j * 4 + r: token m0 + j, column r of this CTA
+    if (!kr_cta) {
+      if (tid < V && m0 + tid / kGvCols < M) {
+        const int j = tid / kGvCols, n_tok = m0 + j, page = s_page[n_tok];
+        const int col = blockIdx.x * kGvCols + tid % kGvCols;
+        if (page >= 0) {
+          if (CACHE == MLA_FP8_E4M3) {
+            a.raw[(size_t)n_tok * a.d_c + col] = fin[tid];
+          } else {
+            __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(a.pool + (size_t)page * a.page_bytes) +
+                                 (size_t)s_row[n_tok] * (a.d_c + a.d_rope);
+            row[col] = __float2bfloat16_rn(fin[tid]);
+          }
+        }
+      }
+    } else if (tid < 2 * MT && m0 + tid / 2 < M) {
+      const int j = tid / 2, pr = tid % 2, n_tok = m0 + j, page = s_page[n_tok];
+      if (page >= 0) {
+        const int i = i0 + pr;
+        const float x1 = fin[j * kGvCols + pr], x2 = fin[j * kGvCols + 2 + pr];
+        float cs, sn;
+        rope_cos_sin(s_pos[n_tok], i, half, a.rope_base, &cs, &sn);
+        uint8_t* pg = a.pool + (size_t)page * a.page_bytes;
+        __nv_bfloat16* kr;
+        if (CACHE == MLA_FP8_E4M3) {
+          const Fp8Page fp = fp8_page(a.page_size, a.d_c, a.d_rope);
+          kr = reinterpret_cast<__nv_bfloat16*>(pg + fp.kr_off) + (size_t)s_row[n_tok] * a.d_rope;
+        } else {
+          kr = reinterpret_cast<__nv_bfloat16*>(pg) + (size_t)s_row[n_tok] * (a.d_c + a.d_rope) + a.d_c;
+        }
+        kr[i] = __float2bfloat16_rn(x1 * cs - x2 * sn);
+        kr[i + half] = __float2bfloat16_rn(x2 * cs + x1 * sn);
+      }
+    }
+    __syncthreads();  // red and fin are rewritten by the next pass
+  }
+  MLA_STAMP(3);
+}
+
 // Block-wide max over 128 threads.
 __device__ __forceinline__ float block128_max(float v, float* sh) {
 #pragma unroll
@@ -280,6 +418,7 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
     mbar_init_local(hb, 1);
   }
   __syncthreads();
+  MLA_STAMP(0);
   pdl_trigger();
   if (tid == 0) {
     // weight slice: tile column j is W_dkv row tile*32 + j, or for a k^R tile
@@ -296,6 +435,7 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
     }
   }
   pdl_wait();
+  MLA_STAMP(1);
   const Fp8Page fp = fp8_page(a.page_size, a.d_c, a.d_rope);
   const int M = a.n_tokens, nk = ks / 16;
   uint32_t pass = 0;
@@ -313,6 +453,7 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
       record_status(a.status, MLA_ERR_TIMEOUT);
       return;
     }
+    MLA_STAMP(5);
     {
       const int combo = warp % combos, kp = warp / combos;
       if (kp < kparts) {
@@ -346,7 +487,9 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
         for (int kp = 1; kp < kparts; ++kp) v += Ps[(size_t)kp * kTcMb * kTcTile + i];
         Ps[i] = v;
       }
+    MLA_STAMP(6);
     cl.sync();  // every CTA's partial tile is complete (and this CTA is done reading Hs)
+    MLA_STAMP(7);
     // this CTA finishes rows [rank * rows, (rank + 1) * rows) of the tile
     const int rows = mpad / kTcCluster;
     const int per_row = is_kr ? kTcTile / 2 : kTcTile;
@@ -383,8 +526,10 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
         kr[i + half] = __float2bfloat16_rn(y2);
       }
     }
+    MLA_STAMP(2);
     cl.sync();  // peers are done reading this CTA's partials before the next pass
   }
+  MLA_STAMP(3);
 }
 
 }  // namespace
@@ -435,7 +580,24 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
 #define MLA_PROJ(T, K) append_project_kernel<T, K><<<grid, 256, 0, st>>>(a)
   const bool tc = d.act_dtype == MLA_BF16 && d.cache_dtype != MLA_F32 && d.d_model % (kTcCluster * 64) == 0 &&
                   d.d_c % kTcTile == 0 && d.d_rope % kTcTile == 0 && append_tc_smem(d) <= 227 * 1024;
-  if (tc) {
+  const bool gemv = d.act_dtype == MLA_BF16 && d.cache_dtype != MLA_F32 && n_tokens <= kGvMaxTok &&
+                    d.d_model % 8 == 0 && d.d_model <= kGvThreads * kGvVec * 8 && d.d_c % kGvCols == 0 &&
+                    d.d_rope % kGvCols == 0 && (reinterpret_cast<uintptr_t>(h) & 15u) == 0 &&
+                    (reinterpret_cast<uintptr_t>(W_dkv) & 15u) == 0 && (reinterpret_cast<uintptr_t>(W_kr) & 15u) == 0;
+  cudaError_t launch_err = cudaSuccess;
+  if (gemv) {
+    const dim3 ggrid((d.d_c + d.d_rope) / kGvCols);
+    const bool fp8 = d.cache_dtype == MLA_FP8_E4M3;
+    if (n_tokens == 1)
+      launch_err = fp8 ? launch_pdl(append_gemv_kernel<MLA_FP8_E4M3, 1>, ggrid, dim3(kGvThreads), 0, st, a)
+                       : launch_pdl(append_gemv_kernel<MLA_BF16, 1>, ggrid, dim3(kGvThreads), 0, st, a);
+    else if (n_tokens <= 2)
+      launch_err = fp8 ? launch_pdl(append_gemv_kernel<MLA_FP8_E4M3, 2>, ggrid, dim3(kGvThreads), 0, st, a)
+                       : launch_pdl(append_gemv_kernel<MLA_BF16, 2>, ggrid, dim3(kGvThreads), 0, st, a);
+    else
+      launch_err = fp8 ? launch_pdl(append_gemv_kernel<MLA_FP8_E4M3, 4>, ggrid, dim3(kGvThreads), 0, st, a)
+                       : launch_pdl(append_gemv_kernel<MLA_BF16, 4>, ggrid, dim3(kGvThreads), 0, st, a);
+  } else if (tc) {
     AppendTcArgs t;
     t.a = a;
     const uint64_t row_bytes = (uint64_t)d.d_model * 2;
@@ -447,11 +609,15 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
     const size_t smem = append_tc_smem(d);
     const int tgrid = (d.d_c / kTcTile + d.d_rope / kTcTile) * kTcCluster;
     if (d.cache_dtype == MLA_BF16) {
-      cudaFuncSetAttribute(append_tc_kernel<MLA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      launch_pdl(append_tc_kernel<MLA_BF16>, dim3(tgrid), dim3(kTcThreads), smem, st, t);
+      launch_err = cudaFuncSetAttribute(append_tc_kernel<MLA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)smem);
+      if (launch_err == cudaSuccess)
+        launch_err = launch_pdl(append_tc_kernel<MLA_BF16>, dim3(tgrid), dim3(kTcThreads), smem, st, t);
     } else {
-      cudaFuncSetAttribute(append_tc_kernel<MLA_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      launch_pdl(append_tc_kernel<MLA_FP8_E4M3>, dim3(tgrid), dim3(kTcThreads), smem, st, t);
+      launch_err = cudaFuncSetAttribute(append_tc_kernel<MLA_FP8_E4M3>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (launch_err == cudaSuccess)
+        launch_err = launch_pdl(append_tc_kernel<MLA_FP8_E4M3>, dim3(tgrid), dim3(kTcThreads), smem, st, t);
     }
   } else if (d.act_dtype == MLA_F32) {
     if (d.cache_dtype == MLA_F32) MLA_PROJ(float, MLA_F32);
@@ -463,7 +629,7 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
     else MLA_PROJ(__nv_bfloat16, MLA_FP8_E4M3);
   }
 #undef MLA_PROJ
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_err != cudaSuccess ? launch_err : cudaGetLastError();
   trace_record(MLA_TRACE_APPEND_PROJECT, true, st);
   if (e != cudaSuccess) return e;
   trace_record(MLA_TRACE_APPEND_FINALIZE, false, st);
@@ -478,3 +644,5 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
 }
 
 }  // namespace mla
+
+MLA_STAMP_EXPORT(append)

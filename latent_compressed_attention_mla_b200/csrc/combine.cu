@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
   const uint32_t bar = smem_addr(&wbar);
   if (tid == 0) mbar_init_local(bar, 1);
   __syncthreads();
+  MLA_STAMP(0);
   pdl_trigger();
   if (tid == 0) {
     mbar_expect_local(bar, kTcWBytes);
@@ -186,6 +187,7 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
       tma_load_2d(smem_addr(Ws) + cb * kTcDv * 128, &P.map_w, 64 * cb, h * kTcDv, bar);
   }
   pdl_wait();
+  MLA_STAMP(1);
   const int splits = plan[batch + 2];
   const int n_slots = batch + splits - 1;  // slot stride of the decode that wrote the partials
   // first slot row (t * n_slots + first split + b) and split count per token;
@@ -237,6 +239,7 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
     for (int i = tid; i < TOK * kTcDc / 4; i += kThreads) X[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   __syncthreads();
+  MLA_STAMP(4);
   auto weight = [&](int mi, int k) -> float {
     return k < kTcWCache ? s_w[mi][k]
                          : exp2f(P.lse_part[(size_t)(s_lo[mi] + k) * n_heads + h] - s_mx[mi]) * s_inv[mi];
@@ -354,11 +357,13 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
       }
     }
   }
+  MLA_STAMP(5);
   const bool w_ok = mbar_wait_bounded(bar, 0);
   if (__syncthreads_or(!w_ok)) {  // also publishes the u tile
     if (tid == 0) record_status(P.status, MLA_ERR_TIMEOUT);
     return;
   }
+  MLA_STAMP(6);
   // o[m, j] = sum_c u[m, c] W^UV_h[j, c]: warp w, columns [16w, 16w + 16)
   const int g = lane >> 2, q = lane & 3, n0 = warp * 16;
   float acc[TOK / 16][2][4];
@@ -378,6 +383,7 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
       mma_bf16(acc[i][1], af, b10, b11);
     }
   }
+  MLA_STAMP(2);
 #pragma unroll
   for (int i = 0; i < TOK / 16; ++i) {
     const int r0 = 16 * i + g, r1 = r0 + 8, col = n0 + 2 * q;
@@ -392,6 +398,7 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
       *reinterpret_cast<__nv_bfloat162*>(o1 + 8) = __floats2bfloat162_rn(acc[i][1][2], acc[i][1][3]);
     }
   }
+  MLA_STAMP(3);
 }
 
 }  // namespace
@@ -447,3 +454,5 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
 }
 
 }  // namespace mla
+
+MLA_STAMP_EXPORT(combine)

@@ -477,6 +477,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
 
   pdl_trigger();
   if (threadIdx.x == 0) TC_TRACE(12, 0);
+  MLA_STAMP(0);
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int i = 0; i < L::QKSlots; ++i) {
@@ -525,6 +526,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
   if (threadIdx.x == 0) TC_TRACE(13, 0);
   pdl_wait();
   if (threadIdx.x == 0) TC_TRACE(14, 0);
+  MLA_STAMP(1);
 
   auto page_of = [&](int b, int pg) -> int {
     int page = p.page_table[(size_t)b * p.max_pages + pg];
@@ -890,6 +892,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           if (!ok) break;
           tc_commit_pair(bar(L::S_FULL + (g & 1)));
           TC_TRACE(1, g);
+          if (g == 0) MLA_STAMP_ANY(4);
           if (it == n_tiles - 1) tc_commit_pair(bar(L::Q_EMPTY));
         }
         ++seg;
@@ -933,6 +936,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           if (!ok) break;
           tc_commit_pair(bar(L::O_DONE));
           TC_TRACE(3, g);
+          if (g == 0) MLA_STAMP_ANY(6);
         }
         ++seg;
       }
@@ -1067,6 +1071,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         fence_proxy_async();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (threadIdx.x == 0) TC_TRACE(6, g);
+        if (threadIdx.x == 0 && g == 0) MLA_STAMP_ANY(5);
         if (lane == 0) mbar_arrive_cluster(leader_bar(L::P_FULL));
       }
       if (!ok) break;
@@ -1119,6 +1124,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       }
       if (half == 0) p.lse_part[slot * kHeads + head] = l_tot > 0.f ? m_ref + __log2f(l_tot) : -INFINITY;
       if (threadIdx.x == 0) TC_TRACE(15, 0);
+      MLA_STAMP(2);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_bar(L::O_FREE));
@@ -1130,6 +1136,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
   __syncthreads();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   tc_fence_after();
+  MLA_STAMP(3);
   if (warp == L::QKWarp)
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
@@ -1264,3 +1271,5 @@ extern "C" int mla_tc_trace_read(void* host, size_t bytes) {
   return cudaMemcpyFromSymbol(host, mla::g_tc_trace, bytes) == cudaSuccess ? 0 : 8;
 }
 #endif
+
+MLA_STAMP_EXPORT(decode_tc)

@@ -234,6 +234,45 @@ bool decode_tc_supported(const mla_dims& d, int n_q);
 bool decode_tc_wants_f16_queries(const mla_dims& d);
 // multiprocessor count of the current device (cached per device)
 int device_sm_count();
+
+// Timeline stamps for latency studies, compiled in only with MLA_TC_TRACE:
+// per event slot, the earliest and latest %globaltimer over the CTAs whose
+// thread 0 reaches it.  Each translation unit keeps its own table and exports
+// mla_stamps_<unit>(host, reset) to read (and re-arm) it.
+#ifdef MLA_TC_TRACE
+namespace {
+__device__ unsigned long long g_stamps[16][2];
+}
+__device__ __forceinline__ void mla_stamp_now(int e) {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  atomicMin(&g_stamps[e][0], t);
+  atomicMax(&g_stamps[e][1], t);
+}
+#define MLA_STAMP(e)                          \
+  do {                                        \
+    if (threadIdx.x == 0) mla_stamp_now(e);   \
+  } while (0)
+#define MLA_STAMP_ANY(e) mla_stamp_now(e)
+#define MLA_STAMP_EXPORT(unit)                                                                  \
+  extern "C" int mla_stamps_##unit(unsigned long long* host, int reset) {                       \
+    if (host && cudaMemcpyFromSymbol(host, mla::g_stamps, sizeof(mla::g_stamps)) != cudaSuccess) \
+      return 1;                                                                                 \
+    if (reset) {                                                                                \
+      unsigned long long init[16][2];                                                           \
+      for (int i = 0; i < 16; ++i) {                                                            \
+        init[i][0] = ~0ull;                                                                     \
+        init[i][1] = 0ull;                                                                      \
+      }                                                                                         \
+      if (cudaMemcpyToSymbol(mla::g_stamps, init, sizeof(init)) != cudaSuccess) return 1;       \
+    }                                                                                           \
+    return 0;                                                                                   \
+  }
+#else
+#define MLA_STAMP(e) ((void)0)
+#define MLA_STAMP_ANY(e) ((void)0)
+#define MLA_STAMP_EXPORT(unit)
+#endif
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st);
 int decode_tc_auto_splits(int num_sms, int n_q);
 

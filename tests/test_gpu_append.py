@@ -22,6 +22,12 @@ CASES = [
     ("bf16-t1", dict(B=3, T=1, L=(0, 63, 700), cache_dtype="bf16")),
     ("bf16-t2", dict(B=5, T=2, L=(1, 64, 127, 128, 4000), cache_dtype="bf16")),
     ("fp8-t2", dict(B=5, T=2, L=(1, 64, 127, 128, 4000), cache_dtype="fp8")),
+    # passes of at most 4 tokens take the register-resident projection
+    ("bf16-1-token", dict(B=1, T=1, L=(4000,), cache_dtype="bf16")),
+    ("fp8-4-tokens", dict(B=2, T=2, L=(1, 1000), cache_dtype="fp8")),
+    # the smallest pass of the tensor-core projection, and one past a 16-row tile
+    ("bf16-5-tokens", dict(B=5, T=1, L=(0, 63, 64, 65, 511), cache_dtype="bf16")),
+    ("bf16-17-tokens", dict(B=17, T=1, L=tuple(int(x) for x in np.arange(17) * 29 % 250), cache_dtype="bf16")),
     # more tokens than one 64-token pass of the tensor-core projection
     ("bf16-70-tokens", dict(B=70, T=1, L=tuple(int(x) for x in np.arange(70) * 37 % 300), cache_dtype="bf16")),
     ("fp8-70-tokens", dict(B=35, T=2, L=tuple(int(x) for x in np.arange(35) * 53 % 400), cache_dtype="fp8")),
