@@ -386,6 +386,11 @@ struct SegmentWalker {
   }
 };
 
+// Bulk prefetch of [ptr, ptr + bytes) into L2 (16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
+
 // L2 prefetch of the pages of a CTA's first key tile, issued before the
 // grid-dependency wait by one warp (batch <= 32).  It reads only inputs of the
 // call (sequence lengths, page table), never the preceding kernel's output,
@@ -414,10 +419,7 @@ __device__ __noinline__ void prefetch_first_tile(const DecodeParams& p, int w, i
     const long long lp = g0 - e0 + 2 * (long long)rank + lane;  // page of sequence b0
     if (lp < min(g1, (long long)i0) - e0) {
       const int page = p.page_table[(size_t)b0 * p.max_pages + lp];
-      if (page >= 0 && page < p.num_pages)
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.pool + (size_t)page * p.page_bytes),
-                     "r"((uint32_t)p.page_bytes)
-                     : "memory");
+      if (page >= 0 && page < p.num_pages) prefetch_l2(p.pool + (size_t)page * p.page_bytes, (uint32_t)p.page_bytes);
     }
   }
 }
@@ -608,6 +610,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           int pg[2];
           for (int i = 0; i < 2; ++i) pg[i] = y_pages + i < npg ? page_of(s.b, pg0 + y_pages + i) : -1;
           if constexpr (kFp8) {
+            // this CTA's pages two tiles ahead (at a segment's start also one
+            // ahead) go to L2 now, so that the staging loads find them there.
+            // (Measured: a gain for the FP8 cache, whose converters bound the
+            // tile; a loss for bf16, whose ring loads wait behind the bulk
+            // prefetches in the TMA unit.)  Invalid entries are skipped here
+            // and reported when their tile is loaded.
+            if (pid == 0) {
+              for (int d = it == 0 ? 1 : 2; d <= 2 && it + d < n_tiles; ++d) {
+                const int pgp = s.page_lo + (it + d) * kTilePages + y_pages;
+                const int npgp = min(kTilePages, s.n_pages - (it + d) * kTilePages);
+                for (int i = 0; i < 2; ++i) {
+                  if (y_pages + i >= npgp) continue;
+                  const int page = p.page_table[(size_t)s.b * p.max_pages + pgp + i];
+                  if (page >= 0 && page < p.num_pages)
+                    prefetch_l2(p.pool + (size_t)page * p.page_bytes, (uint32_t)p.page_bytes);
+                }
+              }
+            }
             // scales of the tile's four pages (zero for pages past its end)
             if (pid == 0) {
               const uint32_t sb = gtile & 1;
@@ -912,14 +932,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         tc_fence_after();
         const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
         for (int it = 0; it < n_tiles && ok; ++it, ++g) {
+#ifdef MLA_TC_TRACE
+          const long long tq0 = clock64();
+          long long q_data = 0;
+#endif
           ok = mbar_wait(bar(L::S_FREE + (g & 1)), ((g >> 1) & 1) ^ 1, abort_flag, p.status);
+#ifdef MLA_TC_TRACE
+          if (!kFp8) TC_TRACE_VAL(11, g, clock64() - tq0);
+#endif
           if (!ok) break;
           tc_fence_after();
           const uint32_t sd = tmem + ((g & 1) ? kColS1 : kColS0);
           TC_TRACE(7, g);
 #pragma unroll 1
           for (int c = 0; c < kQKUnits; ++c) {
+#ifdef MLA_TC_TRACE
+            const long long tw = clock64();
+#endif
             ok = ring.wait_full(abort_flag, p.status);
+#ifdef MLA_TC_TRACE
+            q_data += clock64() - tw;
+#endif
             if (!ok) break;
             tc_fence_after();
             const uint64_t a = qdesc + 512 * c, bb = kdesc + 1024 * ring.pos.slot;
@@ -931,6 +964,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           if (!ok) break;
           tc_commit_pair(bar(L::S_FULL + (g & 1)));
           TC_TRACE(1, g);
+#ifdef MLA_TC_TRACE
+          if (!kFp8) TC_TRACE_VAL(8, g, q_data);
+#endif
           if (g == 0) MLA_STAMP_ANY(4);
           if (it == n_tiles - 1) tc_commit_pair(bar(L::Q_EMPTY));
         }
@@ -951,7 +987,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         if (s.n_pages == 0) continue;
         const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
         for (int it = 0; it < n_tiles && ok; ++it, ++g) {
+#ifdef MLA_TC_TRACE
+          const long long tp0 = clock64();
+          long long v_data = 0;
+#endif
           ok = mbar_wait(bar(L::P_FULL), g & 1, abort_flag, p.status);
+#ifdef MLA_TC_TRACE
+          if (!kFp8) TC_TRACE_VAL(10, g, clock64() - tp0);
+#endif
           if (!ok) break;
           if (it == 0 && seg > 0) {  // O of the previous segment must be read out first
             ok = mbar_wait(bar(L::O_FREE), (seg - 1) & 1, abort_flag, p.status);
@@ -963,7 +1006,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           for (int i = 0; i < kTilePages && ok; ++i)
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
+#ifdef MLA_TC_TRACE
+              const long long tw = clock64();
+#endif
               ok = ring.wait_full(abort_flag, p.status);
+#ifdef MLA_TC_TRACE
+              v_data += clock64() - tw;
+#endif
               if (!ok) break;
               tc_fence_after();
 #pragma unroll
@@ -975,6 +1024,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           if (!ok) break;
           tc_commit_pair(bar(L::O_DONE));
           TC_TRACE(3, g);
+#ifdef MLA_TC_TRACE
+          if (!kFp8) TC_TRACE_VAL(9, g, v_data);
+#endif
           if (g == 0) MLA_STAMP_ANY(6);
         }
         ++seg;
@@ -1051,39 +1103,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           alpha = fast_exp2(m_ref - tile_max);
           m_ref = tile_max;
         }
-        // the previous tile's PV MMAs read P and write O: wait for them
-        if (g >= 1) {
-          ok = mbar_wait(bar(L::O_DONE), (g - 1) & 1, abort_flag, p.status);
-          __syncwarp();
-          if (!ok) break;
-          tc_fence_after();
-        }
-        // tcgen05.ld/st are whole-warp instructions: rescale the warp's lanes
-        // together (alpha = 1 on lanes whose head keeps its reference max)
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-          for (int c = 0; c < 256; c += 32) {
-            const uint32_t col = (c < 128 ? kColO0 + c : kColO1 + (c - 128));
-            uint32_t orr[32];
-            tmem_ld32(tmem + lane_base + col, orr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
-            tmem_st32(tmem + lane_base + col, orr);
-          }
-          tmem_wait_st();
-        }
-        // pass 2: probabilities, written as P row hl of sub-tiles 2*half + q
-        // (64 keys, 128 B per row, 128-byte swizzle)
+        // pass 2: probabilities of page sub-tile 2*half + q, packed in pairs
         float psum = 0.f;
-#pragma unroll 1
-        for (int q = 0; q < 2; ++q) {
+        auto probs = [&](int q, uint32_t(&pk)[32]) {
           uint32_t sr[64];
           tmem_ld32(s_addr + 64 * q, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
           tmem_ld32(s_addr + 64 * q + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
           tmem_wait_ld();
           const int nvq = q ? nv[1] : nv[0];
-          uint32_t pk[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float e0 = 2 * j < nvq ? fast_exp2(__uint_as_float(sr[2 * j]) * p.scale_log2 - m_ref) : 0.f;
@@ -1100,17 +1127,84 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
             psum += f2.x + f2.y;
             pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
           }
+        };
+        // P row hl of sub-tile 2*half + q (64 keys, 128 B per row, 128-byte swizzle)
+        auto store_p = [&](int q, const uint32_t(&pk)[32]) {
           uint8_t* prow = smem + L::OffP + (2 * half + q) * 8192 + hl * 128;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             *reinterpret_cast<uint4*>(prow + ((u ^ (hl & 7)) * 16)) =
                 make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        };
+        // S of this tile is consumed: the QK MMAs two tiles on may overwrite it
+        auto release_s = [&]() {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(leader_bar(L::S_FREE + (g & 1)));
+        };
+        // the previous tile's PV MMAs read P and write O: wait for them, then
+        // rescale O if the reference max moved (tcgen05.ld/st are whole-warp
+        // instructions: the warp's lanes rescale together, alpha = 1 on lanes
+        // whose head keeps its reference)
+        auto wait_pv_rescale = [&]() -> bool {
+          if (g >= 1) {
+            if (!mbar_wait(bar(L::O_DONE), (g - 1) & 1, abort_flag, p.status)) return false;
+            __syncwarp();
+            tc_fence_after();
+          }
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+            for (int c = 0; c < 256; c += 32) {
+              const uint32_t col = (c < 128 ? kColO0 + c : kColO1 + (c - 128));
+              uint32_t orr[32];
+              tmem_ld32(tmem + lane_base + col, orr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
+              tmem_st32(tmem + lane_base + col, orr);
+            }
+            tmem_wait_st();
+          }
+          return true;
+        };
+        if constexpr (!kFp8) {
+          // the probabilities are formed while the previous PV runs; only
+          // their stores into P wait for it
+          uint32_t pk_lo[32], pk_hi[32];
+#pragma unroll 1
+          for (int q = 0; q < 2; ++q) {
+            uint32_t pk[32];
+            probs(q, pk);
+            if (q == 0) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) pk_lo[j] = pk[j];
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) pk_hi[j] = pk[j];
+            }
+          }
+          release_s();
+          ok = wait_pv_rescale();
+          __syncwarp();
+          if (!ok) break;
+          store_p(0, pk_lo);
+          store_p(1, pk_hi);
+        } else {
+          // 512 threads leave 128 registers each: no room to hold both
+          // sub-tiles' probabilities, so the wait comes first
+          ok = wait_pv_rescale();
+          __syncwarp();
+          if (!ok) break;
+#pragma unroll 1
+          for (int q = 0; q < 2; ++q) {
+            uint32_t pk[32];
+            probs(q, pk);
+            store_p(q, pk);
+          }
+          release_s();
         }
         l_part = l_part * alpha + psum;
-        // S of this tile is consumed
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_bar(L::S_FREE + (g & 1)));
+        tc_fence_before();  // rescaled O (tensor-memory stores) precedes the PV MMAs
         fence_proxy_async();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (threadIdx.x == 0) TC_TRACE(6, g);
