@@ -347,6 +347,9 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_cons
       *reinterpret_cast<uint4*>(As + off) = make_uint4(0, 0, 0, 0);
   }
   cp_async_commit();
+  // RoPE of q^R needs neither W^UK nor the product: it runs while the weights
+  // and query rows land
+  rope_query_rows<__nv_bfloat16, TO>(a, h, m0, mc);
   cp_async_wait<0>();
   const bool w_ok = mbar_wait_bounded(bar, 0);
   if (__syncthreads_or(!w_ok)) {  // also publishes the staged query rows
@@ -395,8 +398,6 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_cons
           *reinterpret_cast<const uint4*>(Os + r * 1024 + ((u ^ (r & 7)) << 4));
     }
   }
-  MLA_STAMP(2);
-  rope_query_rows<__nv_bfloat16, TO>(a, h, m0, mc);
   MLA_STAMP(3);
 }
 

@@ -247,31 +247,34 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
   if constexpr (TOK == 16) {
     // few tokens, many splits each: thread (column quad c, half r) takes
     // splits r, r + 2, ... of two tokens at a time, eight loads per token in
-    // flight, and adds its sums into the fp32 tile X
+    // flight (sixteen for a token without a partner), and adds its sums into
+    // the fp32 tile X
     float* X = reinterpret_cast<float*>(Us + TOK * kTcDc * 2);
     const int c0 = (tid & 127) * 4, r = tid >> 7;
 #pragma unroll 1
     for (int mi0 = 0; mi0 < mc; mi0 += 2) {
-      const int nmax = max(s_n[mi0], s_n[mi0 + 1]);
+      const bool single = s_n[mi0 + 1] == 0;  // the same for the whole CTA
+      const int nmax = max(s_n[mi0], s_n[mi0 + 1]), kstep = single ? 32 : 16;
       float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-      for (int k0 = r; k0 < nmax; k0 += 16) {
+      for (int k0 = r; k0 < nmax; k0 += kstep) {
         float4 v[2][8];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const int mi = mi0 + j, n = s_n[mi];
+          const int mi = single ? mi0 : mi0 + j, n = s_n[mi];
           const float* op = P.o_part + (size_t)s_lo[mi] * n_heads * kTcDc + (size_t)h * kTcDc + c0;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
+            const int k = k0 + 2 * (single ? 8 * j + u : u);
             v[j][u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (k0 + 2 * u < n) v[j][u] = *reinterpret_cast<const float4*>(op + (size_t)(k0 + 2 * u) * n_heads * kTcDc);
+            if (k < n) v[j][u] = *reinterpret_cast<const float4*>(op + (size_t)k * n_heads * kTcDc);
           }
         }
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const int mi = mi0 + j, n = s_n[mi];
+          const int mi = single ? mi0 : mi0 + j, n = s_n[mi];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int k = k0 + 2 * u;
+            const int k = k0 + 2 * (single ? 8 * j + u : u);
             const float wk = k < n ? weight(mi, k) : 0.f;
             // a zero weight marks a split with no key of the sequence, whose
             // partial was never written: its values are not read into u
@@ -283,6 +286,13 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
             }
           }
         }
+      }
+      if (single) {
+        acc[0].x += acc[1].x;
+        acc[0].y += acc[1].y;
+        acc[0].z += acc[1].z;
+        acc[0].w += acc[1].w;
+        acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int j = 0; j < 2; ++j) {

@@ -100,8 +100,8 @@ struct TcLayout {
   static constexpr int P_FULL = S_FREE + 2;             // leader: P written + O rescaled by both CTAs
   static constexpr int O_DONE = P_FULL + 1;             // each CTA: the tile's PV MMAs finished
   static constexpr int O_FREE = O_DONE + 1;             // leader: O read out by both CTAs' epilogues
-  static constexpr int Q_FULL = O_FREE + 1;             // leader: Q bytes of both CTAs
-  static constexpr int Q_EMPTY = Q_FULL + 1;            // each CTA: last QK of a segment finished
+  static constexpr int Q_FULL = O_FREE + 1;             // [kChunks] leader: Q chunk bytes of both CTAs
+  static constexpr int Q_EMPTY = Q_FULL + kChunks;      // each CTA: last QK of a segment finished
   static constexpr int QST_FULL = Q_EMPTY + 1;          // [QStSlots] local: staged bytes landed
   static constexpr int QST_EMPTY = QST_FULL + QStSlots; // [QStSlots] local: both converter warps done
   static constexpr int PST_FULL = QST_EMPTY + QStSlots; // [PStSlots]
@@ -533,7 +533,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
     mbar_init(bar(L::P_FULL), 8);
     mbar_init(bar(L::O_DONE), 1);
     mbar_init(bar(L::O_FREE), 8);
-    mbar_init(bar(L::Q_FULL), 1);
+    for (int c = 0; c < kChunks; ++c) mbar_init(bar(L::Q_FULL + c), 1);
     mbar_init(bar(L::Q_EMPTY), 1);
     for (int i = 0; i < L::QStSlots; ++i) {
       mbar_init(bar(L::QST_FULL + i), 1);
@@ -595,11 +595,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         if (pid == 0) {
           if (seg > 0) ok = mbar_wait(bar(L::Q_EMPTY), (seg - 1) & 1, abort_flag, p.status);
           if (!ok) break;
-          if (rank == 0) mbar_expect_tx(bar(L::Q_FULL), 2 * kQBytes);
+          // one barrier per 64-column chunk: the first tile's MMAs of unit c
+          // wait only for chunk c
+          if (rank == 0)
+            for (int c = 0; c < kChunks; ++c) mbar_expect_tx(bar(L::Q_FULL + c), 2 * 8192);
           const int qrow = ((s.b * p.n_q + t) * kHeads) + kHalfHeads * (int)rank;
-          const uint32_t qbar = leader_bar(L::Q_FULL);
           for (int c = 0; c < kChunks; ++c)
-            tma_load_2d_pair(sbase + L::OffQ + c * 8192, &P.map_q, 64 * c, qrow, qbar);
+            tma_load_2d_pair(sbase + L::OffQ + c * 8192, &P.map_q, 64 * c, qrow, leader_bar(L::Q_FULL + c));
         }
         const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
         for (int it = 0; it < n_tiles && ok; ++it) {
@@ -927,9 +929,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       const uint64_t kdesc = sdesc(sbase + L::OffQKRing, 16, 1024);  // slot: + 1024 slot
       while (ok && walk.next(s)) {
         if (s.n_pages == 0) continue;
-        ok = mbar_wait(bar(L::Q_FULL), seg & 1, abort_flag, p.status);
-        if (!ok) break;
-        tc_fence_after();
         const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
         for (int it = 0; it < n_tiles && ok; ++it, ++g) {
 #ifdef MLA_TC_TRACE
@@ -946,6 +945,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           TC_TRACE(7, g);
 #pragma unroll 1
           for (int c = 0; c < kQKUnits; ++c) {
+            if (it == 0) {  // the segment's queries, chunk c
+              ok = mbar_wait(bar(L::Q_FULL + c), seg & 1, abort_flag, p.status);
+              if (!ok) break;
+            }
 #ifdef MLA_TC_TRACE
             const long long tw = clock64();
 #endif
