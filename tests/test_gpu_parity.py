@@ -72,6 +72,12 @@ def test_two_query_tokens_causal(cache):
     check_step(cfg, heads=list(range(0, 128, 7)))
 
 
+def test_three_query_tokens_causal_f32():
+    # fp32 mode (CUDA-core path, 1e-5 bar), three causal tokens over a page edge
+    cfg = W.CONFIGS[0].with_(name="t3-f32", B=2, T=3, L=(62, 200), seed=13)
+    check_step(cfg)
+
+
 def test_split_count_invariance_f32():
     cfg = W.CONFIGS[0]
     outs = [GpuProblem(cfg, num_splits=s).run()[0].cpu() for s in (1, 3, 5)]

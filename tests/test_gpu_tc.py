@@ -1,7 +1,7 @@
 """GPU parity of the tcgen05 decode kernel (DeepSeek-V3 dims, bf16 and FP8
 caches): against the CPU oracle, against the CUDA-core kernel, and on the edge
 cases of its tiling (tails, single-token sequences, splits inside and across
-sequences, two causal query tokens, empty splits)."""
+sequences, two to four causal query tokens, empty splits)."""
 import numpy as np
 import pytest
 import torch
@@ -38,6 +38,10 @@ CASES = [
     ("more-splits-than-tiles", dict(B=1, L=(200,)), 16),
     ("t2-causal", dict(B=2, T=2, L=(62, 200)), 3),
     ("t2-page-edge", dict(B=2, T=2, L=(63, 127)), 2),
+    # wider multi-token (speculative-verify) steps: T = 3 and 4 causal tokens,
+    # the new tokens straddling a page boundary
+    ("t3-causal", dict(B=2, T=3, L=(62, 300)), 3),
+    ("t4-causal", dict(B=1, T=4, L=(190,)), 2),
 ]
 
 
