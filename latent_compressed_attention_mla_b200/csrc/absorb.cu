@@ -13,9 +13,10 @@
 // CTA) brings W^UK_h (d_nope x d_c, 128 KB) into shared memory with eight TMA
 // boxes (issued before the programmatic-launch wait, so the fetch overlaps the
 // previous kernel), stages the block's q^C rows, and multiplies them with
-// mma.sync m16n8k16 (fp32 accumulation); the eight warps split the d_c output
-// columns, and the rows leave through a swizzled shared-memory stage as
-// 16-byte stores.  W^UK is read once from HBM (16.8 MB); the token blocks of
+// mma.sync m16n8k16 (fp32 accumulation); the warps (eight, or four for
+// 32-token blocks, whose CTAs then fit beside the append kernel's) split the
+// d_c output columns, and the rows leave through a swizzled shared-memory
+// stage as 16-byte stores.  W^UK is read once from HBM (16.8 MB); the token blocks of
 // one head re-read it from L2.
 //
 // fp32 activations (absorb_kernel): one CTA per (head, 16-vector slice of d_c).  Thread (cg, dg) loads the
@@ -277,7 +278,6 @@ __device__ void rope_query_rows(const AbsorbArgs& a, int h, int m0, int mc) {
   }
 }
 
-constexpr int kTcThreads = 256;
 constexpr int kTcDn = 128, kTcDc = 512;             // DeepSeek-V3 shape of W^UK_h
 constexpr uint32_t kTcWBytes = kTcDn * kTcDc * 2;  // 128 KB
 constexpr int kTcStageRows = 32;                     // output rows staged per round
@@ -304,18 +304,24 @@ __device__ __forceinline__ uint32_t pack2(float x, float y, __half*) {
 // (d_nope rows x d_c columns) arrives by eight TMA boxes into [8 column
 // blocks][128 rows][128 B] with the 128-byte swizzle, issued before the
 // programmatic-launch wait; the query rows are staged by cp.async in the same
-// layout.  Warp w owns columns [64w, 64w + 64) and runs two 16-row query
-// tiles at a time; each 32-row result goes through a swizzled shared-memory
-// stage so that every output row leaves as 1 KB of 16-byte stores.
-template <typename TO, int TOK>
-__global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_constant__ AbsorbTcArgs P) {
+// layout.  With 256 threads warp w owns columns [64w, 64w + 64) and runs two
+// 16-row query tiles at a time; with 128 threads (small batches: few
+// registers, so the CTAs fit beside the preceding append kernel's and fetch
+// their weights while it runs) warp w owns [128w, 128w + 128) and one 16-row
+// tile at a time.  Each result goes through a swizzled shared-memory stage so
+// that every output row leaves as 1 KB of 16-byte stores.
+template <typename TO, int TOK, int THREADS>
+__global__ void __launch_bounds__(THREADS) absorb_tc_kernel(const __grid_constant__ AbsorbTcArgs P) {
+  constexpr int kWarps = THREADS / 32, kColsW = kTcDc / kWarps, kNP = kColsW / 16;
+  constexpr int kMT = THREADS == 256 ? 2 : 1, kRows = 16 * kMT;  // query rows per round
+  static_assert(kRows <= kTcStageRows && TOK % kRows == 0, "stage");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t wbar;
   const AbsorbArgs& a = P.a;
   const int h = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int D = a.d_c + a.d_rope, M = a.batch * a.n_q;
-  const int m0 = blockIdx.y * TOK, mc = min(TOK, M - m0), mpad = (mc + 31) & ~31;
+  const int m0 = blockIdx.y * TOK, mc = min(TOK, M - m0), mpad = (mc + kRows - 1) / kRows * kRows;
   uint8_t* Ws = smem;                    // [8][128][128 B]
   uint8_t* As = smem + kTcWBytes;        // [2][TOK][128 B]
   uint8_t* Os = As + TOK * kTcDn * 2;    // [32 rows][64 units of 16 B], unit u at u ^ (row & 7)
@@ -334,11 +340,11 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_cons
   if (h == 0 && blockIdx.y == 0) build_plan(a);
   {
     const size_t nblk = (size_t)gridDim.x * gridDim.y, bid = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
-    for (size_t i = bid * kTcThreads + tid; i < a.lse_count; i += nblk * kTcThreads) a.lse_part[i] = -INFINITY;
+    for (size_t i = bid * THREADS + tid; i < a.lse_count; i += nblk * THREADS) a.lse_part[i] = -INFINITY;
   }
   const __nv_bfloat16* qn = static_cast<const __nv_bfloat16*>(a.q_nope);
   TO* qa = static_cast<TO*>(a.q_abs);
-  for (int i = tid; i < mpad * (kTcDn / 8); i += kTcThreads) {
+  for (int i = tid; i < mpad * (kTcDn / 8); i += THREADS) {
     const int r = i / (kTcDn / 8), u = i % (kTcDn / 8);
     const uint32_t off = swz_cb(r, u, TOK);
     if (r < mc)
@@ -358,41 +364,42 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(const __grid_cons
   }
   MLA_STAMP(5);
   const int g = lane >> 2, q = lane & 3;
-  for (int mt = 0; mt < mpad; mt += 32) {
-    float acc[2][8][4];
+  for (int mt = 0; mt < mpad; mt += kRows) {
+    float acc[kMT][2 * kNP][4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < kMT; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+      for (int j = 0; j < 2 * kNP; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
 #pragma unroll
     for (int k0 = 0; k0 < kTcDn; k0 += 16) {
-      uint32_t a0[4], a1[4];
-      load_a_cb(As, TOK, mt, k0, lane, a0);
-      load_a_cb(As, TOK, mt + 16, k0, lane, a1);
+      uint32_t af[kMT][4];
 #pragma unroll
-      for (int np = 0; np < 4; ++np) {
+      for (int i = 0; i < kMT; ++i) load_a_cb(As, TOK, mt + 16 * i, k0, lane, af[i]);
+#pragma unroll
+      for (int np = 0; np < kNP; ++np) {
         uint32_t b00, b01, b10, b11;
-        load_b_kn_cb(Ws, kTcDn, k0, warp * 64 + np * 16, lane, b00, b01, b10, b11);
-        mma_bf16(acc[0][2 * np], a0, b00, b01);
-        mma_bf16(acc[0][2 * np + 1], a0, b10, b11);
-        mma_bf16(acc[1][2 * np], a1, b00, b01);
-        mma_bf16(acc[1][2 * np + 1], a1, b10, b11);
+        load_b_kn_cb(Ws, kTcDn, k0, warp * kColsW + np * 16, lane, b00, b01, b10, b11);
+#pragma unroll
+        for (int i = 0; i < kMT; ++i) {
+          mma_bf16(acc[i][2 * np], af[i], b00, b01);
+          mma_bf16(acc[i][2 * np + 1], af[i], b10, b11);
+        }
       }
     }
     if (mt > 0) __syncthreads();  // the previous round's rows have left the stage
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < kMT; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int r0 = 16 * i + g, unit = warp * 8 + j;
+      for (int j = 0; j < 2 * kNP; ++j) {
+        const int r0 = 16 * i + g, unit = warp * (kColsW / 8) + j;
         *reinterpret_cast<uint32_t*>(Os + r0 * 1024 + ((unit ^ (r0 & 7)) << 4) + 4 * q) =
             pack2(acc[i][j][0], acc[i][j][1], (TO*)nullptr);
         *reinterpret_cast<uint32_t*>(Os + (r0 + 8) * 1024 + ((unit ^ (r0 & 7)) << 4) + 4 * q) =
             pack2(acc[i][j][2], acc[i][j][3], (TO*)nullptr);
       }
     __syncthreads();
-    const int rows = min(kTcStageRows, mc - mt);
-    for (int i = tid; i < rows * 64; i += kTcThreads) {
+    const int rows = min(kRows, mc - mt);
+    for (int i = tid; i < rows * 64; i += THREADS) {
       const int r = i >> 6, u = i & 63;
       *reinterpret_cast<uint4*>(qa + ((size_t)(m0 + mt + r) * a.n_heads + h) * D + u * 8) =
           *reinterpret_cast<const uint4*>(Os + r * 1024 + ((u ^ (r & 7)) << 4));
@@ -448,16 +455,20 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
     else if ((long long)d.n_heads * ((M + 63) / 64) >= sms) tok = 64;
     const dim3 grid(d.n_heads, (M + tok - 1) / tok);
     const size_t smem = absorb_tc_smem(tok);
-    auto pick = [&](auto k32, auto k64, auto k128) {
-      return tok == 128 ? k128 : tok == 64 ? k64 : k32;
+    // a single 32-token block per head (at most 32 tokens) runs 128 threads,
+    // so that its CTAs fit beside the append kernel's; otherwise 256
+    const bool narrow = M <= 32;
+    const int threads = narrow ? 128 : 256;
+    auto pick = [&](auto k32n, auto k32, auto k64, auto k128) {
+      return tok == 128 ? k128 : tok == 64 ? k64 : narrow ? k32n : k32;
     };
-    auto kernel = q_abs_f16 ? pick(absorb_tc_kernel<__half, 32>, absorb_tc_kernel<__half, 64>,
-                                   absorb_tc_kernel<__half, 128>)
-                            : pick(absorb_tc_kernel<__nv_bfloat16, 32>, absorb_tc_kernel<__nv_bfloat16, 64>,
-                                   absorb_tc_kernel<__nv_bfloat16, 128>);
+    auto kernel = q_abs_f16 ? pick(absorb_tc_kernel<__half, 32, 128>, absorb_tc_kernel<__half, 32, 256>,
+                                   absorb_tc_kernel<__half, 64, 256>, absorb_tc_kernel<__half, 128, 256>)
+                            : pick(absorb_tc_kernel<__nv_bfloat16, 32, 128>, absorb_tc_kernel<__nv_bfloat16, 32, 256>,
+                                   absorb_tc_kernel<__nv_bfloat16, 64, 256>, absorb_tc_kernel<__nv_bfloat16, 128, 256>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(kernel, grid, dim3(kTcThreads), smem, st, p);
+    e = launch_pdl(kernel, grid, dim3(threads), smem, st, p);
     return e != cudaSuccess ? e : cudaGetLastError();
   }
   const int vec = d.act_dtype == MLA_F32 ? 4 : 8;
