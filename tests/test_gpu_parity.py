@@ -78,6 +78,27 @@ def test_three_query_tokens_causal_f32():
     check_step(cfg)
 
 
+# The full-size workloads in the launch configuration the bench times (the
+# whole step, automatic split count), checked on sampled outputs that the
+# oracle computes one by one: the ragged batch's shortest and longest
+# sequences, one long-context sequence, one FP8 sequence with its two causal
+# query tokens.
+FULL_SAMPLES = [
+    (2, "minmax", [1, 64, 127]),
+    (3, [0], [0, 77]),
+    (4, [5], [3, 100]),
+]
+
+
+@pytest.mark.parametrize("ci,seqs,heads", FULL_SAMPLES, ids=["ragged-b64", "long-b8", "fp8-b128-t2"])
+def test_full_size_sampled(ci, seqs, heads):
+    cfg = W.CONFIGS[ci]
+    if seqs == "minmax":
+        L = np.asarray(cfg.L)
+        seqs = [int(np.argmin(L)), int(np.argmax(L))]
+    check_step(cfg, heads=heads, seqs=seqs)
+
+
 def test_split_count_invariance_f32():
     cfg = W.CONFIGS[0]
     outs = [GpuProblem(cfg, num_splits=s).run()[0].cpu() for s in (1, 3, 5)]
