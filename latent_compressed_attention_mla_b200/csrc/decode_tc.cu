@@ -774,16 +774,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
 #endif
             if (!ok) break;
             const uint8_t* src = smem + L::OffQSt + stage.slot * kStageBytes;
+            constexpr int kG = 512 / kConvThreads;  // 16-byte groups per thread
+            // all of the thread's codes and scales are loaded before any store
+            uint4 v[kG];
+            float sc[kG];
 #pragma unroll
-            for (int k = 0; k < 512 / kConvThreads; ++k) {
+            for (int k = 0; k < kG; ++k) {
               const int gi = k * kConvThreads + ct, r = gi >> 2, q = gi & 3;  // r: unit row (page r/64)
-              const uint4 v = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
-              const __half2 s2 = __float2half2_rn(scl[r * 4 + (c >> 1)]);
+              v[k] = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
+              sc[k] = scl[r * 4 + (c >> 1)];
+            }
+#pragma unroll
+            for (int k = 0; k < kG; ++k) {
+              const int gi = k * kConvThreads + ct, r = gi >> 2, q = gi & 3;
+              const __half2 s2 = __float2half2_rn(sc[k]);
               uint32_t o[8];
-              e4m3x4_scaled(v.x, s2, o[0], o[1]);
-              e4m3x4_scaled(v.y, s2, o[2], o[3]);
-              e4m3x4_scaled(v.z, s2, o[4], o[5]);
-              e4m3x4_scaled(v.w, s2, o[6], o[7]);
+              e4m3x4_scaled(v[k].x, s2, o[0], o[1]);
+              e4m3x4_scaled(v[k].y, s2, o[2], o[3]);
+              e4m3x4_scaled(v[k].z, s2, o[4], o[5]);
+              e4m3x4_scaled(v[k].w, s2, o[6], o[7]);
               uint8_t* rp = dstu + r * 128;
               *reinterpret_cast<uint4*>(rp + (((2 * q) ^ (r & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
               *reinterpret_cast<uint4*>(rp + (((2 * q + 1) ^ (r & 7)) * 16)) = make_uint4(o[4], o[5], o[6], o[7]);
@@ -799,12 +808,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
               if (!ok) break;
               const uint8_t* src = smem + L::OffQSt + stage.slot * kStageBytes;
               uint8_t* dst = dstu + i * 8192;
+              constexpr int kG = 512 / kConvThreads;
+              uint4 v[kG];
 #pragma unroll
-              for (int k = 0; k < 512 / kConvThreads; ++k) {
+              for (int k = 0; k < kG; ++k) {
                 const int gi = k * kConvThreads + ct, row = gi >> 3, u = gi & 7;
-                const uint4 v = *reinterpret_cast<const uint4*>(src + row * 128 + u * 16);
+                v[k] = *reinterpret_cast<const uint4*>(src + row * 128 + u * 16);
+              }
+#pragma unroll
+              for (int k = 0; k < kG; ++k) {
+                const int gi = k * kConvThreads + ct, row = gi >> 3, u = gi & 7;
                 *reinterpret_cast<uint4*>(dst + row * 128 + ((u ^ (row & 7)) * 16)) =
-                    make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+                    make_uint4(bf16x2_to_f16x2(v[k].x), bf16x2_to_f16x2(v[k].y), bf16x2_to_f16x2(v[k].z),
+                               bf16x2_to_f16x2(v[k].w));
               }
               fence_proxy_async();
               __syncwarp();
@@ -873,17 +889,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
             uint8_t* dst = smem + L::OffPVRing + unit.slot * kUnitBytes;
             // 64 rows x 128 codes -> two 64-column atoms (8 KB apart); rows
             // past the visible keys are zero
+            constexpr int kG = 512 / kConvThreads;
+            // all of the thread's codes and scales are loaded before any store
+            uint4 v[kG];
+            float sc[kG];
 #pragma unroll
-            for (int k = 0; k < 512 / kConvThreads; ++k) {
+            for (int k = 0; k < kG; ++k) {
+              const int gi = k * kConvThreads + ct, row = gi >> 3, q = gi & 7;
+              v[k] = make_uint4(0, 0, 0, 0);
+              sc[k] = 0.f;
+              if (row < valid) {
+                v[k] = *reinterpret_cast<const uint4*>(src + row * 128 + q * 16);
+                sc[k] = scl[row * 4 + 2 * j + blk];
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < kG; ++k) {
               const int gi = k * kConvThreads + ct, row = gi >> 3, q = gi & 7;
               uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
               if (row < valid) {
-                const uint4 v = *reinterpret_cast<const uint4*>(src + row * 128 + q * 16);
-                const __half2 s2 = __float2half2_rn(scl[row * 4 + 2 * j + blk]);
-                e4m3x4_scaled(v.x, s2, o[0], o[1]);
-                e4m3x4_scaled(v.y, s2, o[2], o[3]);
-                e4m3x4_scaled(v.z, s2, o[4], o[5]);
-                e4m3x4_scaled(v.w, s2, o[6], o[7]);
+                const __half2 s2 = __float2half2_rn(sc[k]);
+                e4m3x4_scaled(v[k].x, s2, o[0], o[1]);
+                e4m3x4_scaled(v[k].y, s2, o[2], o[3]);
+                e4m3x4_scaled(v[k].z, s2, o[4], o[5]);
+                e4m3x4_scaled(v[k].w, s2, o[6], o[7]);
               }
               // the eight threads of a row cover both 64-column atoms; threads
               // of the second atom store their odd unit first, so the two
