@@ -292,7 +292,7 @@ def main():
         return run_reference(args, cfg)
 
     from latent_compressed_attention_mla_b200 import binding as B
-    from latent_compressed_attention_mla_b200.decoder import MlaDecodeSession
+    from latent_compressed_attention_mla_b200.decoder import MlaDecodeSession, packed_step_buffers
     from latent_compressed_attention_mla_b200.paged_cache import PagedLatentCache
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -449,12 +449,16 @@ def main():
                       "path": "tcgen05" if path == 1 else "simt", "splits": splits}
 
     # end to end through the public API: pinned host inputs -> device -> step -> host output
-    host_in = {k: v.cpu().pin_memory() for k, v in inputs0.items()}
+    # the step's inputs in one pinned block and one device block (one transfer)
+    host_in, dev_in = packed_step_buffers({k: (inputs0[k].shape, inputs0[k].dtype) for k in ("h", "q_nope", "q_rope")},
+                                          dev)
+    for k in host_in:
+        host_in[k].copy_(inputs0[k].cpu())
     host_out = torch.empty(sess.out.shape, dtype=sess.out.dtype).pin_memory()
-    dev_in = {k: torch.empty_like(v) for k, v in inputs0.items()}
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = host_out.numel() * host_out.element_size()
-    for i in range(min(args.warmup, 5)):
+    # untimed: every buffer set once (the session records its graph on first use)
+    for i in range(max(min(args.warmup, 5), copies)):
         w, _, pool = sets[i % copies]
         sess.step_from_host(host_in, dev_in, seq_idx, pos, seq_lens, w, pt, pool, host_out)
     torch.cuda.synchronize()

@@ -3,7 +3,11 @@
 The session owns the scratch workspaces; the caller owns weights, the paged
 cache and the page table.  `step` takes device tensors; `step_from_host`
 copies a step's inputs from (pinned) host memory, runs the step and copies the
-output back, the path a serving loop driven from the host takes.
+output back, the path a serving loop driven from the host takes.  By default
+it records that sequence (copies in, the library's launches, copy out) as a
+CUDA graph the first time it meets a set of buffers and replays the graph on
+later calls with the same buffers, so a step costs one graph launch on the
+host instead of several library calls and copies.
 """
 from __future__ import annotations
 
@@ -24,6 +28,7 @@ class MlaDecodeSession:
         act = torch.float32 if dims.act_dtype == B.MLA_F32 else torch.bfloat16
         self.out = torch.empty(batch, n_q, dims.n_heads, dims.d_v, dtype=act, device=self.device)
         self.lse = torch.empty(batch, n_q, dims.n_heads, dtype=torch.float32, device=self.device)
+        self._graphs = {}  # buffer addresses of a step_from_host call -> its recorded graph
 
     def append(self, h, seq_idx, pos, W_dkv, W_kr, page_table, cache_pool, stream=None):
         B.mla_append_latent(self.dims, h, seq_idx, pos, W_dkv, W_kr, page_table, cache_pool, self.append_ws, stream)
@@ -44,13 +49,99 @@ class MlaDecodeSession:
         return self.attend(q_nope, q_rope, weights["W_uk"], weights["W_uv"], cache_pool, page_table, seq_lens,
                            out, lse, stream)
 
-    def step_from_host(self, host_in: dict, dev_in: dict, seq_idx, pos, seq_lens, weights, page_table, cache_pool,
-                       host_out: torch.Tensor, stream=None):
-        """host_in: pinned h, q_nope, q_rope; dev_in: device buffers of the same
-        shapes.  Copies in, runs the step, copies `out` back into host_out."""
-        for k in ("h", "q_nope", "q_rope"):
-            dev_in[k].copy_(host_in[k], non_blocking=True)
+    @staticmethod
+    def _span(ts):
+        """The bytes of tensors that lie end to end, in this order, in one
+        storage, as one uint8 tensor; None otherwise."""
+        st = ts[0].untyped_storage()
+        pos = ts[0].data_ptr()
+        for t in ts:
+            if t.untyped_storage().data_ptr() != st.data_ptr() or not t.is_contiguous() or t.data_ptr() != pos:
+                return None
+            pos += t.numel() * t.element_size()
+        whole = torch.empty(0, dtype=torch.uint8, device=ts[0].device).set_(st)
+        off = ts[0].data_ptr() - st.data_ptr()
+        return whole[off:off + (pos - ts[0].data_ptr())]
+
+    def _step_from_host_eager(self, host_in, dev_in, seq_idx, pos, seq_lens, weights, page_table, cache_pool,
+                              host_out):
+        names = ("h", "q_nope", "q_rope")
+        src = self._span([host_in[k] for k in names])
+        dst = self._span([dev_in[k] for k in names])
+        if src is not None and dst is not None and src.numel() == dst.numel():
+            dst.copy_(src, non_blocking=True)  # inputs packed in one block each side: one transfer
+        else:
+            for k in names:
+                dev_in[k].copy_(host_in[k], non_blocking=True)
         out, _ = self.step(dev_in["h"], seq_idx, pos, dev_in["q_nope"], dev_in["q_rope"], seq_lens, weights,
-                           page_table, cache_pool, stream=stream)
+                           page_table, cache_pool)
         host_out.copy_(out, non_blocking=True)
+
+    def step_from_host(self, host_in: dict, dev_in: dict, seq_idx, pos, seq_lens, weights, page_table, cache_pool,
+                       host_out: torch.Tensor, stream=None, use_graph: bool = True):
+        """host_in: pinned h, q_nope, q_rope; dev_in: device buffers of the same
+        shapes.  Copies in, runs the step, copies `out` back into host_out
+        (asynchronously on the current stream).  When the three inputs lie end
+        to end in one block on each side (as `packed_step_buffers` makes them),
+        they move in one transfer.
+
+        With use_graph, the first call with a given set of buffers runs eagerly
+        and records the same work as a CUDA graph; later calls with those
+        buffers replay it.  The graph reads the host inputs and writes the
+        host output at replay time, so every call moves its own data; the
+        buffers (and the tensors the dims describe) must keep their addresses,
+        which the cache key checks."""
+        if stream is not None:
+            with torch.cuda.stream(stream):
+                return self.step_from_host(host_in, dev_in, seq_idx, pos, seq_lens, weights, page_table, cache_pool,
+                                           host_out, None, use_graph)
+        if not use_graph:
+            self._step_from_host_eager(host_in, dev_in, seq_idx, pos, seq_lens, weights, page_table, cache_pool,
+                                       host_out)
+            return host_out
+        key = (tuple(t.data_ptr() for t in (host_in["h"], host_in["q_nope"], host_in["q_rope"], dev_in["h"],
+                                             dev_in["q_nope"], dev_in["q_rope"], seq_idx, pos, seq_lens, page_table,
+                                             cache_pool, host_out)),
+               tuple(weights[k].data_ptr() for k in ("W_dkv", "W_kr", "W_uk", "W_uv")),
+               tuple(host_in[k].shape for k in ("h", "q_nope", "q_rope")), tuple(page_table.shape),
+               cache_pool.numel(), torch.cuda.current_stream().cuda_stream)
+        g = self._graphs.get(key)
+        if g is not None:
+            g.replay()
+            return host_out
+        # first use of these buffers: run eagerly (one-time library set-up
+        # happens outside capture), then record the graph for the next calls
+        self._step_from_host_eager(host_in, dev_in, seq_idx, pos, seq_lens, weights, page_table, cache_pool,
+                                   host_out)
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                self._step_from_host_eager(host_in, dev_in, seq_idx, pos, seq_lens, weights, page_table, cache_pool,
+                                           host_out)
+        torch.cuda.current_stream().wait_stream(side)
+        self._graphs[key] = g
         return host_out
+
+
+def packed_step_buffers(shapes_dtypes: dict, device) -> tuple[dict, dict]:
+    """Pinned host and device buffers for a step's inputs, each side one block
+    with the tensors laid end to end (16-byte aligned), so that
+    `step_from_host` moves them in one transfer.  shapes_dtypes: name ->
+    (shape, dtype), in the order h, q_nope, q_rope."""
+    sizes = []
+    for shape, dtype in shapes_dtypes.values():
+        n = int(torch.Size(shape).numel()) * torch.empty(0, dtype=dtype).element_size()
+        sizes.append(n)
+    if any(n % 16 for n in sizes[:-1]):
+        raise ValueError("packed step inputs must be 16-byte multiples")
+    total = sum(sizes)
+    host = torch.empty(total, dtype=torch.uint8).pin_memory()
+    dev = torch.empty(total, dtype=torch.uint8, device=device)
+    out_h, out_d, off = {}, {}, 0
+    for (name, (shape, dtype)), n in zip(shapes_dtypes.items(), sizes):
+        out_h[name] = host[off:off + n].view(dtype).view(shape)
+        out_d[name] = dev[off:off + n].view(dtype).view(shape)
+        off += n
+    return out_h, out_d
