@@ -161,11 +161,6 @@ __device__ __forceinline__ void tc_trace(int e, uint32_t g) {
     if (blockIdx.x < kTrCtas && (g) < kTrTiles)                                      \
       g_tc_trace[(blockIdx.x * kTrTiles + (g)) * kTrEvents + (e)] = (unsigned long long)(v); \
   } while (0)
-__device__ __forceinline__ unsigned long long tc_now() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 #else
 #define TC_TRACE(e, g) ((void)0)
 #define TC_TRACE_VAL(e, g, v) ((void)0)
@@ -865,7 +860,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         const int pg0 = s.page_lo + it * kTilePages;
         const int npg = min(kTilePages, s.n_pages - it * kTilePages);
 #ifdef MLA_TC_TRACE
-        long long w_unit = 0, w_stage = 0, t_tile = clock64();
+        long long w_unit = 0, w_stage = 0, w_conv = 0, w_fence = 0, t_tile = clock64();
 #endif
         for (int i = 0; i < kTilePages && ok; ++i) {
           const int valid = i < npg ? min(kPage, s.nvis - (pg0 + i) * kPage) : 0;
@@ -887,6 +882,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
 #endif
             const uint8_t* src = smem + L::OffPSt + stage.slot * kStageBytes;
             uint8_t* dst = smem + L::OffPVRing + unit.slot * kUnitBytes;
+#ifdef MLA_TC_TRACE
+            const long long tc0 = clock64();
+#endif
             // 64 rows x 128 codes -> two 64-column atoms (8 KB apart); rows
             // past the visible keys are zero
             constexpr int kG = 512 / kConvThreads;
@@ -923,12 +921,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
               *reinterpret_cast<uint4*>(rp + (((u0 + odd) ^ (row & 7)) * 16)) = odd ? od : ev;
               *reinterpret_cast<uint4*>(rp + (((u0 + 1 - odd) ^ (row & 7)) * 16)) = odd ? ev : od;
             }
+#ifdef MLA_TC_TRACE
+            const long long tc1 = clock64();
+            w_conv += tc1 - tc0;
+#endif
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) {
               mbar_arrive_local(bar(L::PST_EMPTY + stage.slot));
               mbar_arrive_cluster(leader_bar(L::PV_FULL + unit.slot));
             }
+#ifdef MLA_TC_TRACE
+            w_fence += clock64() - tc1;
+#endif
             stage.advance(L::PStSlots);
             unit.advance(L::PVSlots);
           }
@@ -939,6 +944,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           TC_TRACE_VAL(12, gt, w_unit);
           TC_TRACE_VAL(13, gt, w_stage);
           TC_TRACE_VAL(14, gt, clock64() - t_tile);
+          TC_TRACE_VAL(0, gt, w_conv);
+          TC_TRACE_VAL(5, gt, w_fence);
         }
 #endif
         __syncwarp();
