@@ -229,6 +229,22 @@ def cpu_baseline(cfg: WL.MlaConfig, budget_s: float = 15.0) -> dict:
             "sample": describe_sample(step) + f"; {n} calls in {dt:.1f} s"}
 
 
+def max_over_ranks(x: float, pg, device) -> float:
+    """The largest of the ranks' values, returned on every rank (x itself
+    without a process group).  Timing of a multi-GPU run is the slowest rank's."""
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, tokens_per_step: int, steps: int, ms: float) -> float:
+    """Tokens of all ranks (each runs the same per-rank workload: weak scaling)
+    over the slowest rank's time."""
+    return world * tokens_per_step * steps / (ms / 1e3)
+
+
 def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -381,11 +397,7 @@ def main():
     if pg:
         pg.barrier()
     clocks = sampler.stop(t_start_wall, t_end_wall)
-    ms = e0.elapsed_time(e1)
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
 
     # per-kernel durations: the same K steps again, launched eagerly with the
     # library recording a CUDA event before and after each kernel on the launch
@@ -412,7 +424,7 @@ def main():
     status = B.mla_get_status()
 
     tokens_per_step = cfg.B * cfg.T
-    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    value = whole_job_tokens_per_s(world, tokens_per_step, args.steps, ms)
     kms = {name: ksum[k] / args.steps for k, name in enumerate(B.TRACE_KERNELS)}  # ms per launch
     if cfg.cache_dtype != "fp8":
         kms.pop("append_finalize")  # only FP8 caches launch it; its events bracket nothing here
@@ -471,12 +483,8 @@ def main():
         sess.step_from_host(host_in, dev_in, seq_idx, pos, seq_lens, w, pt, pool, host_out)
     f1.record()
     torch.cuda.synchronize()
-    ms_e2e = f0.elapsed_time(f1)
-    if pg:
-        t = torch.tensor([ms_e2e], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e = {"value": world * tokens_per_step * args.steps / (ms_e2e / 1e3), "unit": "tokens/s",
+    ms_e2e = max_over_ranks(f0.elapsed_time(f1), pg, dev)
+    e2e = {"value": whole_job_tokens_per_s(world, tokens_per_step, args.steps, ms_e2e), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
