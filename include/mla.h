@@ -71,6 +71,13 @@ enum {
 
 /* mla_dims.flags */
 #define MLA_FLAG_FORCE_SIMT 1u /* use the CUDA-core kernels even where tcgen05 kernels exist */
+/* Self-test of failure detection: mla_combine's tensor-core kernel (bf16
+ * activations at DeepSeek-V3 dims) does not fetch its weights, so its bounded
+ * wait for them (~2 s) expires; the call then records MLA_ERR_TIMEOUT in the
+ * device status word and leaves out and lse_out unwritten.  No copy is in
+ * flight when the wait gives up, and the context stays usable.  Ignored by
+ * the other kernels. */
+#define MLA_FLAG_SELFTEST_STALL 2u
 
 typedef struct {
   int32_t n_heads;     /* n_h (128 for DeepSeek-V3) */

@@ -16,7 +16,10 @@ LIB_PATH = os.path.join(_PKG, "libmla.so")
 
 MLA_F32, MLA_BF16, MLA_FP8_E4M3 = 0, 1, 2
 MLA_FLAG_FORCE_SIMT = 1
+MLA_FLAG_SELFTEST_STALL = 2  # combine skips its weight fetch: its bounded wait expires (tests)
 
+(MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_ALIGNMENT, MLA_ERR_LAUNCH,
+ MLA_ERR_TIMEOUT, MLA_ERR_BOUNDS, MLA_ERR_CUDA) = range(9)
 ERRORS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_WORKSPACE",
           4: "MLA_ERR_ALIGNMENT", 5: "MLA_ERR_LAUNCH", 6: "MLA_ERR_TIMEOUT", 7: "MLA_ERR_BOUNDS",
           8: "MLA_ERR_CUDA"}

@@ -145,6 +145,7 @@ struct CombineTcArgs {
   float* lse_out;
   int* status;
   int n_heads, batch, n_q;
+  int stall;          // self-test: the weight fetch is not issued (its wait expires)
   CUtensorMap map_w;  // W_uv as [n_heads * d_v rows][d_c] bf16, box 64 x 128, 128-byte swizzle
 };
 
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
   __syncthreads();
   MLA_STAMP(0);
   pdl_trigger();
-  if (tid == 0) {
+  if (tid == 0 && !P.stall) {
     mbar_expect_local(bar, kTcWBytes);
     for (int cb = 0; cb < kTcDc / 64; ++cb)
       tma_load_2d(smem_addr(Ws) + cb * kTcDv * 128, &P.map_w, 64 * cb, h * kTcDv, bar);
@@ -439,6 +440,7 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
     p.n_heads = d.n_heads;
     p.batch = batch;
     p.n_q = n_q;
+    p.stall = (d.flags & MLA_FLAG_SELFTEST_STALL) ? 1 : 0;
     if (!make_tile_map_bf16(&p.map_w, W_uv, kTcDc, (uint64_t)d.n_heads * kTcDv, (uint64_t)kTcDc * 2, 64, kTcDv))
       return cudaErrorInvalidValue;
     // tokens per CTA: the largest block that still gives every SM a CTA

@@ -1,0 +1,59 @@
+"""GPU failure detection without a GPU fault: errors the kernels detect are
+reported through the device status word, and the context stays usable.
+
+* An out-of-range page-table entry is caught by the kernels' own range checks
+  (the access is redirected to page 0 and MLA_ERR_BOUNDS recorded); the other
+  sequences of the batch are unaffected.
+* A bounded wait that runs out (the self-test flag stops the combine from
+  fetching its weights, so nothing completes the barrier it waits on) records
+  MLA_ERR_TIMEOUT after about two seconds; the next step runs normally."""
+import numpy as np
+import pytest
+import torch
+
+from latent_compressed_attention_mla_b200 import binding as B
+from latent_compressed_attention_mla_b200 import workloads as W
+from tests.gpu_harness import GpuProblem, OracleProblem, rel_err, tolerance
+
+pytestmark = pytest.mark.gpu
+
+SMALL = W.CONFIGS[1].with_(name="fail", B=2, T=1, L=(300, 500), seed=31)
+
+
+@pytest.mark.parametrize("flags", [0, B.MLA_FLAG_FORCE_SIMT], ids=["tcgen05", "cuda-core"])
+@pytest.mark.parametrize("cache", ["bf16", "fp8"])
+def test_out_of_range_page_is_reported(cache, flags):
+    cfg = SMALL.with_(cache_dtype=cache)
+    assert B.mla_get_status() == 0
+    # the cache is written through the valid table; only the library calls see
+    # the bad entry (a page of sequence 1's history, past the pool's end)
+    g = GpuProblem(cfg, flags=flags)
+    bad = g.page_table.clone()
+    bad[1, 2] = cfg.num_pages + 5
+    g.page_table = bad
+    out, _ = g.run()
+    assert g.status() == B.MLA_ERR_BOUNDS
+    # sequence 0 never touches the bad entry
+    o = OracleProblem(cfg)
+    heads = list(range(0, 128, 9))
+    ref = o.expected(0, heads)[0]
+    assert rel_err(out[0][:, heads].float().cpu().numpy(), ref) <= tolerance(cfg)
+    # the status word was read and cleared; a clean step reports nothing
+    GpuProblem(cfg, flags=flags).run()
+    assert B.mla_get_status() == 0
+
+
+def test_expired_wait_is_reported_and_context_survives():
+    cfg = SMALL
+    if B.decode_path(B.dims_for(cfg), cfg.T) != 1:
+        pytest.skip("the tensor-core combine runs on sm_100 only")
+    g = GpuProblem(cfg, flags=B.MLA_FLAG_SELFTEST_STALL)
+    g.run()
+    assert g.status() == B.MLA_ERR_TIMEOUT
+    good = GpuProblem(cfg)
+    out, _ = good.run()
+    assert good.status() == 0
+    o = OracleProblem(cfg)
+    heads = list(range(0, 128, 9))
+    for b in range(cfg.B):
+        assert rel_err(out[b][:, heads].float().cpu().numpy(), o.expected(b, heads)[0]) <= tolerance(cfg)
