@@ -168,14 +168,19 @@ def ragged_lengths(seed: int, B: int, lo: int, hi: int) -> np.ndarray:
     return np.random.default_rng(seed).integers(lo, hi, size=B, endpoint=True)
 
 
-CONFIGS = [
-    MlaConfig(name="tiny-f32", seed=0, n_heads=4, d_c=64, d_rope=16, d_nope=32, d_v=32,
-              d_model=128, B=1, T=1, L=(256,), act_dtype="f32", cache_dtype="f32"),
-    _v3("v3-b1-l4096", 1, 1, 1, [4096], "bf16"),
-    _v3("v3-ragged-b64", 2, 64, 1, ragged_lengths(2, 64, 1024, 32768), "bf16"),
-    _v3("v3-long-b8-l131072", 3, 8, 1, [131072] * 8, "bf16"),
-    _v3("v3-fp8-b128-l16384-t2", 4, 128, 2, [16384] * 128, "fp8"),
-]
+# The workloads by what they are: a tiny fp32 problem; DeepSeek-V3 dims with
+# one sequence of 4096 tokens; a ragged batch of 64 (lengths 1024-32768); 8
+# sequences of 131072; an FP8 cache with 128 sequences of 16384 and two causal
+# query tokens each.
+TINY_F32 = MlaConfig(name="tiny-f32", seed=0, n_heads=4, d_c=64, d_rope=16, d_nope=32, d_v=32,
+                     d_model=128, B=1, T=1, L=(256,), act_dtype="f32", cache_dtype="f32")
+V3_B1_L4096 = _v3("v3-b1-l4096", 1, 1, 1, [4096], "bf16")
+V3_RAGGED_B64 = _v3("v3-ragged-b64", 2, 64, 1, ragged_lengths(2, 64, 1024, 32768), "bf16")
+V3_LONG_B8 = _v3("v3-long-b8-l131072", 3, 8, 1, [131072] * 8, "bf16")
+V3_FP8_B128_T2 = _v3("v3-fp8-b128-l16384-t2", 4, 128, 2, [16384] * 128, "fp8")
+
+# in this order for bench.py --config
+CONFIGS = [TINY_F32, V3_B1_L4096, V3_RAGGED_B64, V3_LONG_B8, V3_FP8_B128_T2]
 
 
 # ----------------------------------------------------------------------------

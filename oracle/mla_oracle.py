@@ -25,7 +25,7 @@ Notation: n_h heads, d_c latent rank, d_R decoupled-RoPE width, d_nope per-head
 content width, d_v per-head value width, d model width.  W_uk[h] and W_uv[h]
 are [d_nope, d_c] and [d_v, d_c] (the module's [n_heads, d_head, d_latent]).
 
-Readings where the pages are silent or garbled (each is listed in the design doc):
+Readings where the pages are silent or garbled:
   * RoPE is the rotate-half form of the decoding module's apply_rope; angles
     and their sine/cosine are taken in float64.
   * The cached k^R is rotated once, at its own position, when it is appended;

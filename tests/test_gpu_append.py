@@ -17,7 +17,7 @@ from tests.gpu_harness import GpuProblem, OracleProblem
 
 pytestmark = pytest.mark.gpu
 
-V3 = W.CONFIGS[1]
+V3 = W.V3_B1_L4096
 CASES = [
     ("bf16-t1", dict(B=3, T=1, L=(0, 63, 700), cache_dtype="bf16")),
     ("bf16-t2", dict(B=5, T=2, L=(1, 64, 127, 128, 4000), cache_dtype="bf16")),
@@ -101,7 +101,7 @@ def test_append_f32_cache_matches_oracle():
     """fp32 activations and cache (the tiny configuration): within fp32 rounding."""
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
-    cfg = W.CONFIGS[0].with_(name="append-f32", B=3, T=2, L=(0, 100, 255), seed=77)
+    cfg = W.TINY_F32.with_(name="append-f32", B=3, T=2, L=(0, 100, 255), seed=77)
     g = GpuProblem(cfg)
     g.session.append(g.inputs["h"], g.seq_idx, g.pos, g.weights["W_dkv"], g.weights["W_kr"], g.page_table,
                      g.cache.pool)

@@ -17,7 +17,7 @@ from tests.gpu_harness import GpuProblem, OracleProblem, rel_err, tolerance
 
 pytestmark = pytest.mark.gpu
 
-SMALL = W.CONFIGS[1].with_(name="fail", B=2, T=1, L=(300, 500), seed=31)
+SMALL = W.V3_B1_L4096.with_(name="fail", B=2, T=1, L=(300, 500), seed=31)
 
 
 @pytest.mark.parametrize("flags", [0, B.MLA_FLAG_FORCE_SIMT], ids=["tcgen05", "cuda-core"])

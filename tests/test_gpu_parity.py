@@ -13,7 +13,7 @@ from tests.gpu_harness import GpuProblem, OracleProblem, rel_err, tolerance
 
 pytestmark = pytest.mark.gpu
 
-SMALL_V3 = W.CONFIGS[1]
+SMALL_V3 = W.V3_B1_L4096
 
 
 def small(cfg, **kw):
@@ -43,20 +43,20 @@ def check_step(cfg, flags=0, num_splits=0, heads=None, seqs=None):
 
 
 def test_tiny_f32_full_step():
-    check_step(W.CONFIGS[0])
+    check_step(W.TINY_F32)
 
 
 @pytest.mark.parametrize("splits", [1, 2, 7, 64])
 def test_tiny_f32_split_counts(splits):
-    check_step(W.CONFIGS[0], num_splits=splits)
+    check_step(W.TINY_F32, num_splits=splits)
 
 
 def test_v3_b1_l4096_full_step():
-    check_step(W.CONFIGS[1])
+    check_step(W.V3_B1_L4096)
 
 
 def test_v3_b1_l4096_simt():
-    check_step(W.CONFIGS[1], flags=B.MLA_FLAG_FORCE_SIMT, heads=list(range(0, 128, 9)))
+    check_step(W.V3_B1_L4096, flags=B.MLA_FLAG_FORCE_SIMT, heads=list(range(0, 128, 9)))
 
 
 @pytest.mark.parametrize("cache", ["bf16", "fp8"])
@@ -74,7 +74,7 @@ def test_two_query_tokens_causal(cache):
 
 def test_three_query_tokens_causal_f32():
     # fp32 mode (CUDA-core path, 1e-5 bar), three causal tokens over a page edge
-    cfg = W.CONFIGS[0].with_(name="t3-f32", B=2, T=3, L=(62, 200), seed=13)
+    cfg = W.TINY_F32.with_(name="t3-f32", B=2, T=3, L=(62, 200), seed=13)
     check_step(cfg)
 
 
@@ -84,15 +84,14 @@ def test_three_query_tokens_causal_f32():
 # sequences, one long-context sequence, one FP8 sequence with its two causal
 # query tokens.
 FULL_SAMPLES = [
-    (2, "minmax", [1, 64, 127]),
-    (3, [0], [0, 77]),
-    (4, [5], [3, 100]),
+    (W.V3_RAGGED_B64, "minmax", [1, 64, 127]),
+    (W.V3_LONG_B8, [0], [0, 77]),
+    (W.V3_FP8_B128_T2, [5], [3, 100]),
 ]
 
 
-@pytest.mark.parametrize("ci,seqs,heads", FULL_SAMPLES, ids=["ragged-b64", "long-b8", "fp8-b128-t2"])
-def test_full_size_sampled(ci, seqs, heads):
-    cfg = W.CONFIGS[ci]
+@pytest.mark.parametrize("cfg,seqs,heads", FULL_SAMPLES, ids=["ragged-b64", "long-b8", "fp8-b128-t2"])
+def test_full_size_sampled(cfg, seqs, heads):
     if seqs == "minmax":
         L = np.asarray(cfg.L)
         seqs = [int(np.argmin(L)), int(np.argmax(L))]
@@ -100,7 +99,7 @@ def test_full_size_sampled(ci, seqs, heads):
 
 
 def test_split_count_invariance_f32():
-    cfg = W.CONFIGS[0]
+    cfg = W.TINY_F32
     outs = [GpuProblem(cfg, num_splits=s).run()[0].cpu() for s in (1, 3, 5)]
     for x in outs[1:]:
         assert torch.allclose(x, outs[0], rtol=0, atol=1e-6 * outs[0].abs().max().item())

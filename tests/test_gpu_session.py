@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("packed", [False, True], ids=["separate-inputs", "packed-inputs"])
 @pytest.mark.parametrize("cache", ["bf16", "fp8"])
 def test_step_from_host_replays_match_eager(cache, packed):
-    cfg = W.CONFIGS[1].with_(name="session", B=3, T=1, L=(100, 700, 64), cache_dtype=cache, seed=21)
+    cfg = W.V3_B1_L4096.with_(name="session", B=3, T=1, L=(100, 700, 64), cache_dtype=cache, seed=21)
     g = GpuProblem(cfg)
     sess = MlaDecodeSession(g.dims, cfg.B, cfg.T, 0, "cuda")
     if packed:

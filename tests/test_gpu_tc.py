@@ -12,7 +12,7 @@ from tests.gpu_harness import GpuProblem, OracleProblem, rel_err
 
 pytestmark = pytest.mark.gpu
 
-V3 = W.CONFIGS[1]
+V3 = W.V3_B1_L4096
 
 
 def tc_available():

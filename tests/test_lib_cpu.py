@@ -41,7 +41,7 @@ def test_page_bytes_match_accounting(cfg):
 
 
 def test_v3_row_is_576_scalars():
-    d = B.dims_for(W.CONFIGS[1])
+    d = B.dims_for(W.V3_B1_L4096)
     assert B.cache_page_bytes(d) == 64 * 576 * 2
 
 
@@ -49,17 +49,17 @@ def test_v3_row_is_576_scalars():
     ("d_c", 24, 1), ("d_rope", 3, 1), ("d_model", 100, 1), ("act_dtype", 7, 1), ("cache_dtype", 9, 1),
     ("softmax_scale", 0.0, 1), ("softmax_scale", float("inf"), 1), ("rope_base", -1.0, 1), ("n_heads", 0, 1)])
 def test_invalid_dims_rejected(field, value, code):
-    d = B.dims_for(W.CONFIGS[1])
+    d = B.dims_for(W.V3_B1_L4096)
     setattr(d, field, value)
     assert B.check_dims(d) == code
     assert B.cache_page_bytes(d) == 0
 
 
 def test_unsupported_combinations():
-    d = B.dims_for(W.CONFIGS[1])
+    d = B.dims_for(W.V3_B1_L4096)
     d.cache_dtype = B.MLA_F32  # fp32 cache needs fp32 activations
     assert B.check_dims(d) == 2
-    d = B.dims_for(W.CONFIGS[4])
+    d = B.dims_for(W.V3_FP8_B128_T2)
     d.d_c = 496  # FP8 tiles are 128 wide
     assert B.check_dims(d) == 2
 
@@ -75,7 +75,7 @@ def _p(x):
 
 
 def test_host_side_argument_errors_return_before_any_launch():
-    L, d = B.lib(), B.dims_for(W.CONFIGS[1])
+    L, d = B.lib(), B.dims_for(W.V3_B1_L4096)
     ref = ctypes.byref(d)
     fake = _p(0x10000)  # never dereferenced: validation fails first
     ws_need = B.decode_workspace_bytes(d, 1, 1, 4)
@@ -98,7 +98,7 @@ def test_host_side_argument_errors_return_before_any_launch():
     assert L.mla_append_latent(ref, _p(0x10002), 3, fake, fake, fake, fake, fake, 1, 1, fake, 1, None, 0,
                                None) == 4
     # FP8 caches keep fp32 c between the projection and the quantiser
-    d8 = B.dims_for(W.CONFIGS[4])
+    d8 = B.dims_for(W.V3_FP8_B128_T2)
     ref8 = ctypes.byref(d8)
     need = B.append_workspace_bytes(d8, 3)
     assert need >= 3 * 512 * 4
@@ -107,7 +107,7 @@ def test_host_side_argument_errors_return_before_any_launch():
 
 
 def test_workspace_layout_grows_with_splits():
-    d = B.dims_for(W.CONFIGS[3])
+    d = B.dims_for(W.V3_LONG_B8)
     a = B.decode_workspace_bytes(d, 8, 1, 10)
     b = B.decode_workspace_bytes(d, 8, 1, 20)
     # each extra split adds one slot of n_h * (d_c + 1) floats

@@ -69,6 +69,6 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     bench = _load_bench()
     monkeypatch.setenv("RANK", "1")
     args = argparse.Namespace(steps=1, warmup=0, gpus=2)
-    cfg = bench.WL.CONFIGS[0]
+    cfg = bench.WL.TINY_F32
     assert bench.run_reference(args, cfg) is None
     assert capsys.readouterr().out == ""

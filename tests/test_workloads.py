@@ -34,7 +34,7 @@ def test_configs():
 
 
 def test_page_table_is_a_permutation():
-    cfg = W.CONFIGS[2]
+    cfg = W.V3_RAGGED_B64
     pt = W.page_table(cfg)
     used = pt[pt >= 0]
     assert len(used) == cfg.num_pages and len(np.unique(used)) == cfg.num_pages
@@ -43,9 +43,9 @@ def test_page_table_is_a_permutation():
 
 
 def test_history_rows_slices_agree():
-    cfg = W.CONFIGS[0]
+    cfg = W.TINY_F32
     full = W.history_rows(cfg, 0, 0, 256)
     part = W.history_rows(cfg, 0, 100, 140)
     assert torch.equal(full["c"][100:140], part["c"]) and torch.equal(full["kr"][100:140], part["kr"])
-    f8 = W.history_rows(W.CONFIGS[4], 3, 10, 20)
+    f8 = W.history_rows(W.V3_FP8_B128_T2, 3, 10, 20)
     assert f8["codes"].dtype == torch.uint8 and f8["scales"].shape == (10, 4)

@@ -23,8 +23,8 @@ def _tokens(cfg, start, n, device):
     return (h, torch.from_numpy(seq.astype(np.int32)).to(device), torch.from_numpy(pos.astype(np.int32)).to(device))
 
 
-@pytest.mark.parametrize("cfg", [W.CONFIGS[0], W.CONFIGS[1].with_(name="noalloc-v3", B=3, L=(200, 200, 200)),
-                                 W.CONFIGS[1].with_(name="noalloc-fp8", B=2, L=(300, 300), cache_dtype="fp8")],
+@pytest.mark.parametrize("cfg", [W.TINY_F32, W.V3_B1_L4096.with_(name="noalloc-v3", B=3, L=(200, 200, 200)),
+                                 W.V3_B1_L4096.with_(name="noalloc-fp8", B=2, L=(300, 300), cache_dtype="fp8")],
                          ids=lambda c: c.name)
 def test_noalloc_append_matches_workspace_append(cfg):
     dev = "cuda"
@@ -46,7 +46,7 @@ def test_noalloc_append_matches_workspace_append(cfg):
 
 
 def test_noalloc_rejects_requests_beyond_its_array():
-    cfg = W.CONFIGS[1].with_(name="noalloc-big", B=1, L=(0,))
+    cfg = W.V3_B1_L4096.with_(name="noalloc-big", B=1, L=(0,))
     dims = B.dims_for(cfg)
     n = 65536 // (cfg.d_c + cfg.d_rope) + 1  # one token more than fits
     dev = "cuda"
