@@ -149,7 +149,8 @@ struct CombineTcArgs {
   CUtensorMap map_w;  // W_uv as [n_heads * d_v rows][d_c] bf16, box 64 x 128, 128-byte swizzle
 };
 
-// W^UV_h, the bf16 u tile and, for 16-token blocks, the fp32 u sums
+// W^UV_h, the bf16 u tile and, for 16-token blocks, the fp32 scratch of the
+// groups' sums
 size_t combine_tc_smem(int tok) {
   return kTcWBytes + (size_t)tok * kTcDc * 2 + (tok == 16 ? (size_t)tok * kTcDc * 4 : 0) + 1024;
 }
@@ -158,11 +159,48 @@ size_t combine_tc_smem(int tok) {
 // blocks][128 rows][128 B] (128-byte swizzle); the merged u tile is [8 column
 // blocks][TOK tokens][128 B] in the same layout; warp w then owns output
 // columns [16w, 16w + 16) for every 16-token tile.
-template <int TOK>
+// A 16-byte piece of a split partial row: eight bf16 or four fp32 columns.
+// Loads bring raw pieces into registers; the conversion to fp32 happens only
+// when they are used, so that all of a round's loads are in flight together.
+template <bool PB> struct PartUnit;
+template <> struct PartUnit<true> {
+  static constexpr int kCols = 8;
+  __device__ static uint4 load(const float* o_part, size_t row, int c0) {
+    return *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(o_part) + row * 512 + c0);
+  }
+  __device__ static void to_float(const uint4& x, float (&v)[8]) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+};
+template <> struct PartUnit<false> {
+  static constexpr int kCols = 4;
+  __device__ static uint4 load(const float* o_part, size_t row, int c0) {
+    return *reinterpret_cast<const uint4*>(o_part + row * 512 + c0);
+  }
+  __device__ static void to_float(const uint4& x, float (&v)[4]) {
+    v[0] = __uint_as_float(x.x);
+    v[1] = __uint_as_float(x.y);
+    v[2] = __uint_as_float(x.z);
+    v[3] = __uint_as_float(x.w);
+  }
+};
+
+// PB: the split partials are bf16 (written by the tensor-core decode), else fp32.
+template <int TOK, bool PB>
 __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_constant__ CombineTcArgs P) {
   static_assert(TOK % 16 == 0 && TOK <= 64, "token block");
+  using PU = PartUnit<PB>;
+  constexpr int kCU = PU::kCols;            // columns per 16-byte load
+  constexpr int kUnits = kTcDc / kCU;       // loads per partial row
+  constexpr int kGroups = kThreads / kUnits;  // threads per column unit (token groups / split groups)
   constexpr int kTPW = TOK / 8;             // tokens per warp in the weight pass
-  constexpr int kJ = TOK / 2;               // tokens per thread in the merge
+  constexpr int kJ = TOK / kGroups;         // tokens per thread in the merge
   constexpr int kJB = kJ < 8 ? kJ : 8;      // of which in flight together
   constexpr int kKU = 2;                    // splits per load round
   extern __shared__ uint8_t smem_tc[];
@@ -235,39 +273,52 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
       }
     }
   }
-  if constexpr (TOK == 16) {
-    float4* X = reinterpret_cast<float4*>(Us + TOK * kTcDc * 2);
-    for (int i = tid; i < TOK * kTcDc / 4; i += kThreads) X[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
   __syncthreads();
   MLA_STAMP(4);
   auto weight = [&](int mi, int k) -> float {
     return k < kTcWCache ? s_w[mi][k]
                          : exp2f(P.lse_part[(size_t)(s_lo[mi] + k) * n_heads + h] - s_mx[mi]) * s_inv[mi];
   };
+  // thread (column unit cu, group gr): columns [c0, c0 + kCU)
+  const int cu = tid % kUnits, gr = tid / kUnits, c0 = cu * kCU;
+  auto part_row = [&](int mi, int k) { return (size_t)(s_lo[mi] + k) * n_heads + h; };
+  auto store_u = [&](int mi, const float* a) {
+    // kCU columns of token mi as bf16 into the swizzled u tile
+#pragma unroll
+    for (int e = 0; e < kCU; e += 4) {
+      const __nv_bfloat162 lo2 = __floats2bfloat162_rn(a[e], a[e + 1]);
+      const __nv_bfloat162 hi2 = __floats2bfloat162_rn(a[e + 2], a[e + 3]);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
+      pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
+      *reinterpret_cast<uint2*>(Us + swz_cb(mi, (c0 + e) >> 3, TOK) + ((c0 + e) & 7) * 2) = pk;
+    }
+  };
   if constexpr (TOK == 16) {
-    // few tokens, many splits each: thread (column quad c, half r) takes
-    // splits r, r + 2, ... of two tokens at a time, eight loads per token in
-    // flight (sixteen for a token without a partner), and adds its sums into
-    // the fp32 tile X
-    float* X = reinterpret_cast<float*>(Us + TOK * kTcDc * 2);
-    const int c0 = (tid & 127) * 4, r = tid >> 7;
+    // few tokens, many splits each: the kGroups groups take splits gr,
+    // gr + kGroups, ... of two tokens at a time, eight loads per token in
+    // flight (sixteen for a token without a partner); the groups' sums meet
+    // in the fp32 scratch R and are added in group order (deterministic)
+    float* R = reinterpret_cast<float*>(Us + TOK * kTcDc * 2);  // [kGroups][2][d_c]
 #pragma unroll 1
     for (int mi0 = 0; mi0 < mc; mi0 += 2) {
       const bool single = s_n[mi0 + 1] == 0;  // the same for the whole CTA
-      const int nmax = max(s_n[mi0], s_n[mi0 + 1]), kstep = single ? 32 : 16;
-      float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-      for (int k0 = r; k0 < nmax; k0 += kstep) {
-        float4 v[2][8];
+      const int nmax = max(s_n[mi0], s_n[mi0 + 1]), kstep = (single ? 16 : 8) * kGroups;
+      float acc[2][kCU];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < kCU; ++e) acc[j][e] = 0.f;
+      for (int k0 = gr; k0 < nmax; k0 += kstep) {
+        uint4 raw[2][8];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int mi = single ? mi0 : mi0 + j, n = s_n[mi];
-          const float* op = P.o_part + (size_t)s_lo[mi] * n_heads * kTcDc + (size_t)h * kTcDc + c0;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int k = k0 + 2 * (single ? 8 * j + u : u);
-            v[j][u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (k < n) v[j][u] = *reinterpret_cast<const float4*>(op + (size_t)k * n_heads * kTcDc);
+            const int k = k0 + kGroups * (single ? 8 * j + u : u);
+            raw[j][u] = make_uint4(0, 0, 0, 0);
+            if (k < n) raw[j][u] = PU::load(P.o_part, part_row(mi, k), c0);
           }
         }
 #pragma unroll
@@ -275,72 +326,83 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
           const int mi = single ? mi0 : mi0 + j, n = s_n[mi];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int k = k0 + 2 * (single ? 8 * j + u : u);
+            const int k = k0 + kGroups * (single ? 8 * j + u : u);
             const float wk = k < n ? weight(mi, k) : 0.f;
             // a zero weight marks a split with no key of the sequence, whose
             // partial was never written: its values are not read into u
             if (wk != 0.f) {
-              acc[j].x = fmaf(wk, v[j][u].x, acc[j].x);
-              acc[j].y = fmaf(wk, v[j][u].y, acc[j].y);
-              acc[j].z = fmaf(wk, v[j][u].z, acc[j].z);
-              acc[j].w = fmaf(wk, v[j][u].w, acc[j].w);
+              float v[kCU];
+              PU::to_float(raw[j][u], v);
+#pragma unroll
+              for (int e = 0; e < kCU; ++e) acc[j][e] = fmaf(wk, v[e], acc[j][e]);
             }
           }
         }
       }
       if (single) {
-        acc[0].x += acc[1].x;
-        acc[0].y += acc[1].y;
-        acc[0].z += acc[1].z;
-        acc[0].w += acc[1].w;
-        acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < kCU; ++e) {
+          acc[0][e] += acc[1][e];
+          acc[1][e] = 0.f;
+        }
       }
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float* x = X + (mi0 + j) * kTcDc + c0;
-        atomicAdd(x, acc[j].x);
-        atomicAdd(x + 1, acc[j].y);
-        atomicAdd(x + 2, acc[j].z);
-        atomicAdd(x + 3, acc[j].w);
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < kCU; ++e) R[(gr * 2 + j) * kTcDc + c0 + e] = acc[j][e];
+      __syncthreads();
+      // thread t: token mi0 + t / 128, columns 4 (t % 128) .. + 3
+      {
+        const int j = tid >> 7, c = (tid & 127) * 4;
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < kGroups; ++q) {
+          const float4 x = *reinterpret_cast<const float4*>(R + (q * 2 + j) * kTcDc + c);
+          sum.x += x.x;
+          sum.y += x.y;
+          sum.z += x.z;
+          sum.w += x.w;
+        }
+        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(sum.x, sum.y);
+        const __nv_bfloat162 hi2 = __floats2bfloat162_rn(sum.z, sum.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
+        pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
+        *reinterpret_cast<uint2*>(Us + swz_cb(mi0 + j, c >> 3, TOK) + (c & 7) * 2) = pk;
       }
+      __syncthreads();  // R is rewritten by the next pair
     }
-    __syncthreads();
-    for (int i = tid; i < TOK * kTcDc / 4; i += kThreads) {
-      const int mi = i / (kTcDc / 4), c = (i % (kTcDc / 4)) * 4;
-      const float4 a = *reinterpret_cast<const float4*>(X + mi * kTcDc + c);
-      const __nv_bfloat162 lo2 = __floats2bfloat162_rn(a.x, a.y);
-      const __nv_bfloat162 hi2 = __floats2bfloat162_rn(a.z, a.w);
-      uint2 pk;
-      pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
-      pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
-      *reinterpret_cast<uint2*>(Us + swz_cb(mi, c >> 3, TOK) + (c & 7) * 2) = pk;
+    // rows of the tile past the last token stay zero
+    for (int i = tid; i < (TOK - ((mc + 1) & ~1)) * (kTcDc / 8); i += kThreads) {
+      const int mi = ((mc + 1) & ~1) + i / (kTcDc / 8), u = i % (kTcDc / 8);
+      *reinterpret_cast<uint4*>(Us + swz_cb(mi, u, TOK)) = make_uint4(0, 0, 0, 0);
     }
   } else {
-    // u[m, c0..c0+3] = sum_k w_k o_k[c0..c0+3] for tokens r, r + 2, ...
-    const int c0 = (tid & 127) * 4, r = tid >> 7;
+    // u[m, c0..c0+kCU) = sum_k w_k o_k[c0..c0+kCU) for tokens gr, gr + kGroups, ...
 #pragma unroll 1
     for (int j0 = 0; j0 < kJ; j0 += kJB) {
       int nmax = 0;
 #pragma unroll
-      for (int j = 0; j < kJB; ++j) nmax = max(nmax, s_n[r + 2 * (j0 + j)]);
-      float4 acc[kJB];
+      for (int j = 0; j < kJB; ++j) nmax = max(nmax, s_n[gr + kGroups * (j0 + j)]);
+      float acc[kJB][kCU];
 #pragma unroll
-      for (int j = 0; j < kJB; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < kJB; ++j)
+#pragma unroll
+        for (int e = 0; e < kCU; ++e) acc[j][e] = 0.f;
       for (int k0 = 0; k0 < nmax; k0 += kKU) {
-        float4 v[kJB][kKU];
+        uint4 raw[kJB][kKU];
 #pragma unroll
         for (int j = 0; j < kJB; ++j) {
-          const int mi = r + 2 * (j0 + j), n = s_n[mi];
-          const float* op = P.o_part + (size_t)s_lo[mi] * n_heads * kTcDc + (size_t)h * kTcDc + c0;
+          const int mi = gr + kGroups * (j0 + j), n = s_n[mi];
 #pragma unroll
           for (int u = 0; u < kKU; ++u) {
-            v[j][u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (k0 + u < n) v[j][u] = *reinterpret_cast<const float4*>(op + (size_t)(k0 + u) * n_heads * kTcDc);
+            raw[j][u] = make_uint4(0, 0, 0, 0);
+            if (k0 + u < n) raw[j][u] = PU::load(P.o_part, part_row(mi, k0 + u), c0);
           }
         }
 #pragma unroll
         for (int j = 0; j < kJB; ++j) {
-          const int mi = r + 2 * (j0 + j), n = s_n[mi];
+          const int mi = gr + kGroups * (j0 + j), n = s_n[mi];
 #pragma unroll
           for (int u = 0; u < kKU; ++u) {
             const int k = k0 + u;
@@ -348,24 +410,16 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
             // a zero weight marks a split with no key of the sequence, whose
             // partial was never written: its values are not read into u
             if (wk != 0.f) {
-              acc[j].x = fmaf(wk, v[j][u].x, acc[j].x);
-              acc[j].y = fmaf(wk, v[j][u].y, acc[j].y);
-              acc[j].z = fmaf(wk, v[j][u].z, acc[j].z);
-              acc[j].w = fmaf(wk, v[j][u].w, acc[j].w);
+              float v[kCU];
+              PU::to_float(raw[j][u], v);
+#pragma unroll
+              for (int e = 0; e < kCU; ++e) acc[j][e] = fmaf(wk, v[e], acc[j][e]);
             }
           }
         }
       }
 #pragma unroll
-      for (int j = 0; j < kJB; ++j) {
-        const int mi = r + 2 * (j0 + j);
-        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc[j].x, acc[j].y);
-        const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc[j].z, acc[j].w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
-        pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
-        *reinterpret_cast<uint2*>(Us + swz_cb(mi, c0 >> 3, TOK) + (c0 & 7) * 2) = pk;
-      }
+      for (int j = 0; j < kJB; ++j) store_u(gr + kGroups * (j0 + j), acc[j]);
     }
   }
   MLA_STAMP(5);
@@ -419,8 +473,8 @@ int combine_max_splits() { return kMaxSplits; }
 int combine_max_d_c(int act_dtype) { return kMaxVecPerLane * 32 * (act_dtype == MLA_F32 ? 4 : 8); }
 
 cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n_q, const int32_t* plan,
-                           const float* o_part, const float* lse_part, void* out, float* lse_out, int* status,
-                           cudaStream_t st) {
+                           const float* o_part, bool part_bf16, const float* lse_part, void* out, float* lse_out,
+                           int* status, cudaStream_t st) {
   const size_t smem = combine_smem_bytes(d);
   cudaError_t e;
   if (d.act_dtype == MLA_F32) {
@@ -448,7 +502,12 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
     int tok = 16;
     if ((long long)d.n_heads * ((M + 63) / 64) >= sms) tok = 64;
     else if ((long long)d.n_heads * ((M + 31) / 32) >= sms) tok = 32;
-    auto kernel = tok == 64 ? combine_tc_kernel<64> : tok == 32 ? combine_tc_kernel<32> : combine_tc_kernel<16>;
+    auto kernel = part_bf16 ? (tok == 64   ? combine_tc_kernel<64, true>
+                               : tok == 32 ? combine_tc_kernel<32, true>
+                                           : combine_tc_kernel<16, true>)
+                            : (tok == 64   ? combine_tc_kernel<64, false>
+                               : tok == 32 ? combine_tc_kernel<32, false>
+                                           : combine_tc_kernel<16, false>);
     const size_t tsm = combine_tc_smem(tok);
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e != cudaSuccess) return e;

@@ -1090,11 +1090,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
     bool ok = true;
     while (walk.next(s)) {
       const size_t slot = (size_t)t * p.n_slots + (w + s.b);
-      float* od = p.o_part + (slot * kHeads + head) * kDC;
+      // the split partials of this path are bf16 rows (the combine reads them so)
+      __nv_bfloat16* od = reinterpret_cast<__nv_bfloat16*>(p.o_part) + (slot * kHeads + head) * kDC;
       if (s.n_pages == 0 || !ok) {
         for (int j = 0; j < 2; ++j)
-          for (int c = 0; c < 128; c += 4)
-            *reinterpret_cast<float4*>(od + 256 * j + 128 * half + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int c = 0; c < 128; c += 8)
+            *reinterpret_cast<uint4*>(od + 256 * j + 128 * half + c) = make_uint4(0, 0, 0, 0);
         if (half == 0) p.lse_part[slot * kHeads + head] = -INFINITY;
         continue;
       }
@@ -1261,30 +1262,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       const float l_tot = l_part + red_l[(half ^ 1) * 64 + hl];
       asm volatile("bar.sync 1, 128;" ::: "memory");
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-      // O leaves through the (free) P buffer as 32-column x 64-head boxes,
-      // stored by TMA: lanes 0-63 hold dims [256j, 256j+128), lanes 64-127
-      // dims [256j+128, 256j+256).  Four 8 KB staging slots: two iterations
-      // of both halves in flight.
+      // O leaves, normalised and rounded to bf16, through the (free) P buffer
+      // as 64-column x 64-head boxes stored by TMA: lanes 0-63 hold dims
+      // [256j, 256j+128), lanes 64-127 dims [256j+128, 256j+256).  Four 8 KB
+      // staging slots: two iterations of both halves in flight.
       {
         const bool issuer = hl == 0;  // thread 0 of each half
         const int orow = (int)((((size_t)t * p.n_slots + w + s.b) * kHeads) + kHalfHeads * rank);
 #pragma unroll 1
-        for (int i = 0; i < 8; ++i) {
-          const int c = 32 * i;
+        for (int i = 0; i < 4; ++i) {
+          const int c = 64 * i;
           if (i >= 2) {
             if (issuer) bulk_wait_read<1>();
             asm volatile("bar.sync %0, 64;" ::"r"(2 + half) : "memory");
           }
           const uint32_t col = (c < 128 ? kColO0 + c : kColO1 + (c - 128));
-          uint32_t orr[32];
-          tmem_ld32(tmem + lane_base + col, orr);
+          uint32_t orr[64];
+          tmem_ld32(tmem + lane_base + col, *reinterpret_cast<uint32_t(*)[32]>(&orr[0]));
+          tmem_ld32(tmem + lane_base + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&orr[32]));
           tmem_wait_ld();
           uint8_t* box = smem + L::OffP + ((i & 1) * 2 + half) * 8192 + hl * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4*>(box + ((q ^ (hl & 7)) * 16)) =
-                make_float4(__uint_as_float(orr[4 * q]) * inv, __uint_as_float(orr[4 * q + 1]) * inv,
-                            __uint_as_float(orr[4 * q + 2]) * inv, __uint_as_float(orr[4 * q + 3]) * inv);
+          for (int q = 0; q < 8; ++q) {
+            uint32_t u[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[8 * q + 2 * e]) * inv,
+                                                              __uint_as_float(orr[8 * q + 2 * e + 1]) * inv);
+              u[e] = *reinterpret_cast<const uint32_t*>(&v2);
+            }
+            *reinterpret_cast<uint4*>(box + ((q ^ (hl & 7)) * 16)) = make_uint4(u[0], u[1], u[2], u[3]);
+          }
           fence_proxy_async();
           asm volatile("bar.sync %0, 64;" ::"r"(2 + half) : "memory");
           if (issuer) {
@@ -1378,10 +1386,10 @@ bool make_o_map(CUtensorMap* m, void* base, uint64_t rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)kDC, rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)kDC * 4};
-  const cuuint32_t box[2] = {32, (cuuint32_t)kHalfHeads};
+  const cuuint64_t strides[1] = {(cuuint64_t)kDC * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kHalfHeads};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }

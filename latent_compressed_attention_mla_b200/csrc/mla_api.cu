@@ -216,8 +216,10 @@ int mla_combine(const mla_dims* dims, const void* W_uv, int batch, int n_q, int 
   if (!aligned16(W_uv) || !aligned16(workspace)) return MLA_ERR_ALIGNMENT;
   const uint8_t* ws = static_cast<const uint8_t*>(workspace);
   trace_record(MLA_TRACE_COMBINE, false, (cudaStream_t)stream);
+  // the partials' row type follows the decode path that wrote them
+  const bool part_bf16 = mla_decode_path(dims, n_q) == 1;
   cudaError_t e = launch_combine(*dims, W_uv, batch, n_q, reinterpret_cast<const int32_t*>(ws + L.off_plan),
-                                 reinterpret_cast<const float*>(ws + L.off_o),
+                                 reinterpret_cast<const float*>(ws + L.off_o), part_bf16,
                                  reinterpret_cast<const float*>(ws + L.off_lse), out, lse_out, status_ptr(),
                                  (cudaStream_t)stream);
   trace_record(MLA_TRACE_COMBINE, true, (cudaStream_t)stream);

@@ -145,7 +145,9 @@ __device__ __forceinline__ void rope_cos_sin(int pos, int i, int half, float bas
 //           overlapping each sequence
 //   q_abs : [batch, n_q, n_heads, d_c + d_rope] act type (absorbed queries,
 //           rotated q^R appended)
-//   o_part: float32 [n_q, n_slots, n_heads, d_c] per-split normalised latent sums
+//   o_part: [n_q, n_slots, n_heads, d_c] per-split normalised latent sums,
+//           float32 rows from the CUDA-core decode, bf16 rows (in the first
+//           half of the region) from the tensor-core decode
 //   lse   : float32 [n_q, n_slots, n_heads] per-split log2-sum-exp2 of the scores
 //           scaled by softmax_scale*log2(e) (-inf for an empty split)
 // A split w covers global key tiles [w*TT/W, (w+1)*TT/W) of the concatenated
@@ -276,7 +278,10 @@ __device__ __forceinline__ void mla_stamp_now(int e) {
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st);
 int decode_tc_auto_splits(int num_sms, int n_q);
 
+// part_bf16: the split partials are bf16 rows (the tensor-core decode writes
+// them so), else fp32 (the CUDA-core decode)
 cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n_q, const int32_t* plan,
-                           const float* o_part, const float* lse_part, void* out, float* lse_out, int* status, cudaStream_t st);
+                           const float* o_part, bool part_bf16, const float* lse_part, void* out, float* lse_out,
+                           int* status, cudaStream_t st);
 
 }  // namespace mla
