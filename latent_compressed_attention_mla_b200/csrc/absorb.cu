@@ -278,6 +278,65 @@ __device__ void rope_query_rows(const AbsorbArgs& a, int h, int m0, int mc) {
   }
 }
 
+// RoPE of q^R for d_rope = 64 with 16-byte accesses: item (token, quarter
+// q) rotates pairs 8q .. 8q + 7 (both halves of each pair are one 16-byte
+// load and store each); a thread loads all of its items before rotating any,
+// so its loads form one round.  Pointers of q^R rows and q~ rows are 16-byte
+// aligned (checked by the launcher).
+template <typename TO, int kPer>
+__device__ void rope_query_rows_v8(const AbsorbArgs& a, int h, int m0, int mc) {
+  constexpr int kHalf = 32;
+  const int D = a.d_c + 2 * kHalf, n_items = mc * 4;
+  const int qt = threadIdx.x & 3;  // the same quarter for all of a thread's items
+  // base^(-i/32) for i = 8qt .. 8qt + 7: one power, then the constant ratio
+  // base^(-1/32) (relative error ~1e-15, far below the float rotation's)
+  double invf[8];
+  invf[0] = rope_inv_freq(8 * qt, kHalf, a.rope_base);
+  const double ratio = rope_inv_freq(1, kHalf, a.rope_base);
+#pragma unroll
+  for (int e = 1; e < 8; ++e) invf[e] = invf[e - 1] * ratio;
+  const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(a.q_rope);
+  TO* qa = static_cast<TO*>(a.q_abs);
+  for (int i0 = 0; i0 < n_items; i0 += kPer * (int)blockDim.x) {
+    uint4 x1[kPer], x2[kPer];
+    int pos[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = i0 + u * (int)blockDim.x + (int)threadIdx.x;
+      pos[u] = 0;
+      x1[u] = x2[u] = make_uint4(0, 0, 0, 0);
+      if (i < n_items) {
+        const int m = m0 + (i >> 2), b = m / a.n_q, t = m % a.n_q;
+        pos[u] = a.seq_lens[b] - a.n_q + t;
+        const __nv_bfloat16* src = qr + ((size_t)m * a.n_heads + h) * (2 * kHalf) + 8 * qt;
+        x1[u] = *reinterpret_cast<const uint4*>(src);
+        x2[u] = *reinterpret_cast<const uint4*>(src + kHalf);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = i0 + u * (int)blockDim.x + (int)threadIdx.x;
+      if (i < n_items) {
+        const int m = m0 + (i >> 2);
+        const __nv_bfloat16* v1 = reinterpret_cast<const __nv_bfloat16*>(&x1[u]);
+        const __nv_bfloat16* v2 = reinterpret_cast<const __nv_bfloat16*>(&x2[u]);
+        TO y1[8], y2[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float cs, sn;
+          rope_cos_sin_at(pos[u], invf[e], &cs, &sn);
+          const float a1 = __bfloat162float(v1[e]), a2 = __bfloat162float(v2[e]);
+          y1[e] = from_f<TO>(a1 * cs - a2 * sn);
+          y2[e] = from_f<TO>(a2 * cs + a1 * sn);
+        }
+        TO* dst = qa + ((size_t)m * a.n_heads + h) * D + a.d_c + 8 * qt;
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(y1);
+        *reinterpret_cast<uint4*>(dst + kHalf) = *reinterpret_cast<const uint4*>(y2);
+      }
+    }
+  }
+}
+
 constexpr int kTcDn = 128, kTcDc = 512;             // DeepSeek-V3 shape of W^UK_h
 constexpr uint32_t kTcWBytes = kTcDn * kTcDc * 2;  // 128 KB
 constexpr int kTcStageRows = 32;                     // output rows staged per round
@@ -287,6 +346,7 @@ size_t absorb_tc_smem(int tok) { return kTcWBytes + (size_t)tok * kTcDn * 2 + kT
 
 struct AbsorbTcArgs {
   AbsorbArgs a;
+  int rope_v8;        // q^R rows 16-byte aligned: vector RoPE (d_rope = 64)
   CUtensorMap map_w;  // W_uk as [n_heads * d_nope rows][d_c] bf16, box 64 x 128, 128-byte swizzle
 };
 
@@ -355,8 +415,13 @@ __global__ void __launch_bounds__(THREADS) absorb_tc_kernel(const __grid_constan
   cp_async_commit();
   // RoPE of q^R needs neither W^UK nor the product: it runs while the weights
   // and query rows land
-  rope_query_rows<__nv_bfloat16, TO>(a, h, m0, mc);
+  if (a.d_rope == 64 && P.rope_v8 && mc >= 8)
+    rope_query_rows_v8<TO, (TOK * 4 + THREADS - 1) / THREADS>(a, h, m0, mc);
+  else
+    rope_query_rows<__nv_bfloat16, TO>(a, h, m0, mc);
+  MLA_STAMP(4);
   cp_async_wait<0>();
+  MLA_STAMP(6);
   const bool w_ok = mbar_wait_bounded(bar, 0);
   if (__syncthreads_or(!w_ok)) {  // also publishes the staged query rows
     if (tid == 0) record_status(a.status, MLA_ERR_TIMEOUT);
@@ -446,6 +511,7 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
       (reinterpret_cast<uintptr_t>(q_abs) & 15u) == 0 && ((d.d_c + d.d_rope) * 2) % 16 == 0) {
     AbsorbTcArgs p;
     p.a = a;
+    p.rope_v8 = d.d_rope == 64 && (reinterpret_cast<uintptr_t>(q_rope) & 15u) == 0;
     if (!make_tile_map_bf16(&p.map_w, W_uk, kTcDc, (uint64_t)d.n_heads * kTcDn, (uint64_t)kTcDc * 2, 64, kTcDn))
       return cudaErrorInvalidValue;
     // tokens per CTA: the largest block that still gives every SM a CTA
