@@ -342,7 +342,11 @@ constexpr uint32_t kTcWBytes = kTcDn * kTcDc * 2;  // 128 KB
 constexpr int kTcStageRows = 32;                     // output rows staged per round
 constexpr uint32_t kTcStageBytes = kTcStageRows * kTcDc * 2;
 
-size_t absorb_tc_smem(int tok) { return kTcWBytes + (size_t)tok * kTcDn * 2 + kTcStageBytes + 1024; }
+// W^UK_h's columns of one CTA (d_c / nsplit), the staged query rows, the
+// output stage
+size_t absorb_tc_smem(int tok, int nsplit) {
+  return kTcWBytes / nsplit + (size_t)tok * kTcDn * 2 + kTcStageBytes / nsplit + 1024;
+}
 
 struct AbsorbTcArgs {
   AbsorbArgs a;
@@ -370,30 +374,33 @@ __device__ __forceinline__ uint32_t pack2(float x, float y, __half*) {
 // their weights while it runs) warp w owns [128w, 128w + 128) and one 16-row
 // tile at a time.  Each result goes through a swizzled shared-memory stage so
 // that every output row leaves as 1 KB of 16-byte stores.
-template <typename TO, int TOK, int THREADS>
+template <typename TO, int TOK, int THREADS, int NSPLIT>
 __global__ void __launch_bounds__(THREADS) absorb_tc_kernel(const __grid_constant__ AbsorbTcArgs P) {
-  constexpr int kWarps = THREADS / 32, kColsW = kTcDc / kWarps, kNP = kColsW / 16;
+  constexpr int kCols = kTcDc / NSPLIT;  // output columns of this CTA
+  constexpr int kWarps = THREADS / 32, kColsW = kCols / kWarps, kNP = kColsW / 16;
   constexpr int kMT = THREADS == 256 ? 2 : 1, kRows = 16 * kMT;  // query rows per round
-  static_assert(kRows <= kTcStageRows && TOK % kRows == 0, "stage");
+  constexpr int kRowUnits = kCols / 8;   // 16-byte units of a staged output row
+  static_assert(kRows <= kTcStageRows && TOK % kRows == 0 && kNP >= 1, "stage");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t wbar;
   const AbsorbArgs& a = P.a;
   const int h = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int part = (int)blockIdx.y % NSPLIT;  // column part: columns [part kCols, (part + 1) kCols)
   const int D = a.d_c + a.d_rope, M = a.batch * a.n_q;
-  const int m0 = blockIdx.y * TOK, mc = min(TOK, M - m0), mpad = (mc + kRows - 1) / kRows * kRows;
-  uint8_t* Ws = smem;                    // [8][128][128 B]
-  uint8_t* As = smem + kTcWBytes;        // [2][TOK][128 B]
-  uint8_t* Os = As + TOK * kTcDn * 2;    // [32 rows][64 units of 16 B], unit u at u ^ (row & 7)
+  const int m0 = (int)(blockIdx.y / NSPLIT) * TOK, mc = min(TOK, M - m0), mpad = (mc + kRows - 1) / kRows * kRows;
+  uint8_t* Ws = smem;                           // [kCols / 64][128][128 B]
+  uint8_t* As = smem + kTcWBytes / NSPLIT;      // [2][TOK][128 B]
+  uint8_t* Os = As + TOK * kTcDn * 2;           // [32 rows][kRowUnits units of 16 B], unit u at u ^ (row & 7)
   const uint32_t bar = smem_addr(&wbar);
   if (tid == 0) mbar_init_local(bar, 1);
   __syncthreads();
   MLA_STAMP(0);
   pdl_trigger();
   if (tid == 0) {
-    mbar_expect_local(bar, kTcWBytes);
-    for (int cb = 0; cb < kTcDc / 64; ++cb)
-      tma_load_2d(smem_addr(Ws) + cb * kTcDn * 128, &P.map_w, 64 * cb, h * kTcDn, bar);
+    mbar_expect_local(bar, kTcWBytes / NSPLIT);
+    for (int cb = 0; cb < kCols / 64; ++cb)
+      tma_load_2d(smem_addr(Ws) + cb * kTcDn * 128, &P.map_w, part * kCols + 64 * cb, h * kTcDn, bar);
   }
   pdl_wait();
   MLA_STAMP(1);
@@ -414,11 +421,13 @@ __global__ void __launch_bounds__(THREADS) absorb_tc_kernel(const __grid_constan
   }
   cp_async_commit();
   // RoPE of q^R needs neither W^UK nor the product: it runs while the weights
-  // and query rows land
-  if (a.d_rope == 64 && P.rope_v8 && mc >= 8)
-    rope_query_rows_v8<TO, (TOK * 4 + THREADS - 1) / THREADS>(a, h, m0, mc);
-  else
-    rope_query_rows<__nv_bfloat16, TO>(a, h, m0, mc);
+  // and query rows land (in the first column part's CTA)
+  if (part == 0) {
+    if (a.d_rope == 64 && P.rope_v8 && mc >= 8)
+      rope_query_rows_v8<TO, (TOK * 4 + THREADS - 1) / THREADS>(a, h, m0, mc);
+    else
+      rope_query_rows<__nv_bfloat16, TO>(a, h, m0, mc);
+  }
   MLA_STAMP(4);
   cp_async_wait<0>();
   MLA_STAMP(6);
@@ -457,17 +466,17 @@ __global__ void __launch_bounds__(THREADS) absorb_tc_kernel(const __grid_constan
 #pragma unroll
       for (int j = 0; j < 2 * kNP; ++j) {
         const int r0 = 16 * i + g, unit = warp * (kColsW / 8) + j;
-        *reinterpret_cast<uint32_t*>(Os + r0 * 1024 + ((unit ^ (r0 & 7)) << 4) + 4 * q) =
+        *reinterpret_cast<uint32_t*>(Os + r0 * (kRowUnits * 16) + ((unit ^ (r0 & 7)) << 4) + 4 * q) =
             pack2(acc[i][j][0], acc[i][j][1], (TO*)nullptr);
-        *reinterpret_cast<uint32_t*>(Os + (r0 + 8) * 1024 + ((unit ^ (r0 & 7)) << 4) + 4 * q) =
+        *reinterpret_cast<uint32_t*>(Os + (r0 + 8) * (kRowUnits * 16) + ((unit ^ (r0 & 7)) << 4) + 4 * q) =
             pack2(acc[i][j][2], acc[i][j][3], (TO*)nullptr);
       }
     __syncthreads();
     const int rows = min(kRows, mc - mt);
-    for (int i = tid; i < rows * 64; i += THREADS) {
-      const int r = i >> 6, u = i & 63;
-      *reinterpret_cast<uint4*>(qa + ((size_t)(m0 + mt + r) * a.n_heads + h) * D + u * 8) =
-          *reinterpret_cast<const uint4*>(Os + r * 1024 + ((u ^ (r & 7)) << 4));
+    for (int i = tid; i < rows * kRowUnits; i += THREADS) {
+      const int r = i / kRowUnits, u = i % kRowUnits;
+      *reinterpret_cast<uint4*>(qa + ((size_t)(m0 + mt + r) * a.n_heads + h) * D + part * kCols + u * 8) =
+          *reinterpret_cast<const uint4*>(Os + r * (kRowUnits * 16) + ((u ^ (r & 7)) << 4));
     }
   }
   MLA_STAMP(3);
@@ -519,8 +528,11 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
     int tok = 32;
     if ((long long)d.n_heads * ((M + 127) / 128) >= sms) tok = 128;
     else if ((long long)d.n_heads * ((M + 63) / 64) >= sms) tok = 64;
-    const dim3 grid(d.n_heads, (M + tok - 1) / tok);
-    const size_t smem = absorb_tc_smem(tok);
+    // small batches split each head's 512 columns over two CTAs: half the
+    // weight fetch per CTA, and two CTAs fit on an SM
+    const int nsplit = M <= 32 ? 2 : 1;
+    const dim3 grid(d.n_heads, (M + tok - 1) / tok * nsplit);
+    const size_t smem = absorb_tc_smem(tok, nsplit);
     // a single 32-token block per head (at most 32 tokens) runs 128 threads,
     // so that its CTAs fit beside the append kernel's; otherwise 256
     const bool narrow = M <= 32;
@@ -528,10 +540,12 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
     auto pick = [&](auto k32n, auto k32, auto k64, auto k128) {
       return tok == 128 ? k128 : tok == 64 ? k64 : narrow ? k32n : k32;
     };
-    auto kernel = q_abs_f16 ? pick(absorb_tc_kernel<__half, 32, 128>, absorb_tc_kernel<__half, 32, 256>,
-                                   absorb_tc_kernel<__half, 64, 256>, absorb_tc_kernel<__half, 128, 256>)
-                            : pick(absorb_tc_kernel<__nv_bfloat16, 32, 128>, absorb_tc_kernel<__nv_bfloat16, 32, 256>,
-                                   absorb_tc_kernel<__nv_bfloat16, 64, 256>, absorb_tc_kernel<__nv_bfloat16, 128, 256>);
+    auto kernel = q_abs_f16 ? pick(absorb_tc_kernel<__half, 32, 128, 2>, absorb_tc_kernel<__half, 32, 256, 1>,
+                                   absorb_tc_kernel<__half, 64, 256, 1>, absorb_tc_kernel<__half, 128, 256, 1>)
+                            : pick(absorb_tc_kernel<__nv_bfloat16, 32, 128, 2>,
+                                   absorb_tc_kernel<__nv_bfloat16, 32, 256, 1>,
+                                   absorb_tc_kernel<__nv_bfloat16, 64, 256, 1>,
+                                   absorb_tc_kernel<__nv_bfloat16, 128, 256, 1>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kernel, grid, dim3(threads), smem, st, p);
