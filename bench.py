@@ -348,7 +348,7 @@ def main():
                      cache0.pool.clone()))
     sess = MlaDecodeSession(dims, cfg.B, cfg.T, args.splits, dev)
     # the split count mla_decode uses: explicit, else the automatic count capped
-    # at one split per 4 key tiles of batch * max_pages
+    # at one split per 4 pages of batch * max_pages
     splits = args.splits or min(B.auto_splits(dims, cfg.B, cfg.T), max(1, -(-cfg.B * cfg.max_pages // 4)))
     path = B.decode_path(dims, cfg.T)
 

@@ -18,8 +18,10 @@
 //  * Per 256-key tile (four pages):
 //      QK : S[128 heads x 256 keys] = Q[128 x 576] . K^T   (M=128 pair, N=256, K=576)
 //      PV : O[128 heads x 512]     += P[128 x 256] . C[256 x 512]  (two N=256 MMAs)
-//    The leader CTA supplies pages 0-1 of the tile as its half of the QK B
-//    operand, the peer pages 2-3.  S (2 buffers) and O live in tensor memory
+//    The leader CTA supplies pages 0 and 2 of the tile as its half of the QK
+//    B operand, the peer pages 1 and 3 (so a two-page tile gives each CTA one
+//    page); the key positions of S and P follow that order (tile_page).  S (2
+//    buffers) and O live in tensor memory
 //    (TMEM), 2x2 layout: row m, column n < N/2 -> lane m, column n;
 //    n >= N/2 -> lane 64+m, column n-N/2.
 //  * Operands stream through two rings of 16 KB units (128-byte swizzle) in
@@ -381,6 +383,11 @@ struct SegmentWalker {
   }
 };
 
+// Page of a tile at key position pos (0..3; the order of the S columns and
+// the P sub-tiles: the leader's two pages, then the peer's): CTA r of the pair
+// holds pages r and r + 2, so a tile of two pages puts one page in each CTA.
+__device__ __forceinline__ int tile_page(int pos) { return (pos >> 1) + 2 * (pos & 1); }
+
 // Bulk prefetch of [ptr, ptr + bytes) into L2 (16-byte aligned, bytes % 16 == 0).
 __device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
@@ -391,7 +398,7 @@ __device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes) {
 // call (sequence lengths, page table), never the preceding kernel's output,
 // and a prefetch cannot change a result: at worst it fetches pages that go
 // unused.  The split of pages is the plan's rule; CTA `rank` of the pair
-// takes pages 2 rank and 2 rank + 1 of the tile.
+// takes pages rank and rank + 2 of the tile.
 __device__ __noinline__ void prefetch_first_tile(const DecodeParams& p, int w, int rank, int lane) {
   int pages = 0;
   if (lane < p.batch) {
@@ -411,7 +418,7 @@ __device__ __noinline__ void prefetch_first_tile(const DecodeParams& p, int w, i
   const int b0 = own ? __ffs(own) - 1 : 0;
   const int e0 = __shfl_sync(0xffffffffu, excl, b0), i0 = __shfl_sync(0xffffffffu, incl, b0);
   if (g0 < g1 && own && lane < 2) {
-    const long long lp = g0 - e0 + 2 * (long long)rank + lane;  // page of sequence b0
+    const long long lp = g0 - e0 + tile_page(2 * rank + lane);  // page of sequence b0
     if (lp < min(g1, (long long)i0) - e0) {
       const int page = p.page_table[(size_t)b0 * p.max_pages + lp];
       if (page >= 0 && page < p.num_pages) prefetch_l2(p.pool + (size_t)page * p.page_bytes, (uint32_t)p.page_bytes);
@@ -579,7 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       const int pid = warp - L::QKProdWarp;
       RingProducer ring{kFp8 ? L::QStSlots : L::QKSlots, L::Producers, pid};
       const uint32_t empty0 = kFp8 ? bar(L::QST_EMPTY) : bar(L::QK_EMPTY);
-      const int y_pages = 2 * (int)rank;  // this CTA's two pages of a tile
+      const int y_pages = 2 * (int)rank;  // this CTA's key positions of a tile (pages tile_page(...))
       SegmentWalker walk(p, w, t);
       Segment s;
       uint32_t seg = 0, gtile = 0;
@@ -605,7 +612,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           // this CTA's pages; pages past the tile's end come from outside the
           // tensor (zero fill)
           int pg[2];
-          for (int i = 0; i < 2; ++i) pg[i] = y_pages + i < npg ? page_of(s.b, pg0 + y_pages + i) : -1;
+          for (int i = 0; i < 2; ++i) {
+            const int tp = tile_page(y_pages + i);
+            pg[i] = tp < npg ? page_of(s.b, pg0 + tp) : -1;
+          }
           if constexpr (kFp8) {
             // this CTA's pages two tiles ahead (at a segment's start also one
             // ahead) go to L2 now, so that the staging loads find them there.
@@ -615,11 +625,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
             // and reported when their tile is loaded.
             if (pid == 0) {
               for (int d = it == 0 ? 1 : 2; d <= 2 && it + d < n_tiles; ++d) {
-                const int pgp = s.page_lo + (it + d) * kTilePages + y_pages;
+                const int pgp = s.page_lo + (it + d) * kTilePages;
                 const int npgp = min(kTilePages, s.n_pages - (it + d) * kTilePages);
                 for (int i = 0; i < 2; ++i) {
-                  if (y_pages + i >= npgp) continue;
-                  const int page = p.page_table[(size_t)s.b * p.max_pages + pgp + i];
+                  const int tp = tile_page(y_pages + i);
+                  if (tp >= npgp) continue;
+                  const int page = p.page_table[(size_t)s.b * p.max_pages + pgp + tp];
                   if (page >= 0 && page < p.num_pages)
                     prefetch_l2(p.pool + (size_t)page * p.page_bytes, (uint32_t)p.page_bytes);
                 }
@@ -683,10 +694,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         for (int it = 0; it < n_tiles && ok; ++it) {
           const int pg0 = s.page_lo + it * kTilePages;
           const int npg = min(kTilePages, s.n_pages - it * kTilePages);
-          // page i outer, N-half j inner
+          // key position i outer (page tile_page(i)), N-half j inner
           for (int i = 0; i < kTilePages; ++i) {
-            const int valid = i < npg ? min(kPage, s.nvis - (pg0 + i) * kPage) : 0;
-            const int page = valid > 0 ? page_of(s.b, pg0 + i) : 0;
+            const int tp = tile_page(i);
+            const int valid = tp < npg ? min(kPage, s.nvis - (pg0 + tp) * kPage) : 0;
+            const int page = valid > 0 ? page_of(s.b, pg0 + tp) : 0;
             for (int j = 0; j < 2; ++j) {
               uint32_t slot;
               if (!ring.claim(empty0, slot, ok, abort_flag, p.status)) continue;
@@ -746,7 +758,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       for (int it = 0; it < n_tiles && ok; ++it, ++gt) {
         ok = mbar_wait(bar(L::SCL_FULL + (gt & 1)), (gt >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
-        const float* scl = reinterpret_cast<const float*>(smem + L::OffScl + (gt & 1) * kSclBytes) + y_pages * 256;
+        // the tile's scales, [4 pages][64 rows][4 tiles of 128 columns]
+        const float* scl = reinterpret_cast<const float*>(smem + L::OffScl + (gt & 1) * kSclBytes);
 #ifdef MLA_TC_TRACE
         long long w_unit = 0, w_stage = 0, t_tile = clock64();
 #endif
@@ -775,9 +788,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
             float sc[kG];
 #pragma unroll
             for (int k = 0; k < kG; ++k) {
-              const int gi = k * kConvThreads + ct, r = gi >> 2, q = gi & 3;  // r: unit row (page r/64)
+              const int gi = k * kConvThreads + ct, r = gi >> 2, q = gi & 3;  // r: unit row (this CTA's page r/64)
               v[k] = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
-              sc[k] = scl[r * 4 + (c >> 1)];
+              sc[k] = scl[(tile_page(y_pages + (r >> 6)) * 64 + (r & 63)) * 4 + (c >> 1)];
             }
 #pragma unroll
             for (int k = 0; k < kG; ++k) {
@@ -863,8 +876,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         long long w_unit = 0, w_stage = 0, w_conv = 0, w_fence = 0, t_tile = clock64();
 #endif
         for (int i = 0; i < kTilePages && ok; ++i) {
-          const int valid = i < npg ? min(kPage, s.nvis - (pg0 + i) * kPage) : 0;
-          const float* scl = scl_t + i * 256;
+          const int tp = tile_page(i);
+          const int valid = tp < npg ? min(kPage, s.nvis - (pg0 + tp) * kPage) : 0;
+          const float* scl = scl_t + tp * 256;
           for (int j = 0; j < 2 && ok; ++j) {
 #ifdef MLA_TC_TRACE
             long long tw = clock64();
@@ -1074,9 +1088,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
   } else if (warp < 4) {
     // ------------------------------------------------------- softmax, epilogue
     // Thread L (TMEM lane) holds head hl of this CTA; lanes 0-63 see the
-    // keys of pages 0-1 of a tile, lanes 64-127 those of pages 2-3 (the QK B
-    // operand holds the leader's two pages in N columns [0,128), the peer's in
-    // [128,256); 2x2 layout).  S is read twice from TMEM: once for the max,
+    // keys of the leader's pages (0 and 2 of a tile), lanes 64-127 those of the
+    // peer's (1 and 3): the QK B operand holds the leader's two pages in N
+    // columns [0,128), the peer's in [128,256); 2x2 layout.  S is read twice from TMEM: once for the max,
     // once for the probabilities, so that few registers hold scores at a time.
     // The per-page loops stay rolled: the smaller code runs measurably faster
     // (the first tile of a step executes it from a cold instruction cache).
@@ -1108,12 +1122,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         if (threadIdx.x == 0) TC_TRACE(4, g);
         tc_fence_after();
         const uint32_t s_addr = tmem + lane_base + ((g & 1) ? kColS1 : kColS0);
-        // visible keys of this thread's two pages (page 2*half + q of the tile)
+        // visible keys of this thread's two key positions 2*half + q (pages tile_page(2*half + q))
         const int pg0 = s.page_lo + it * kTilePages;
         int nv[2];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          const int pg = pg0 + 2 * half + q;
+          const int pg = pg0 + tile_page(2 * half + q);
           nv[q] = pg < s.page_lo + s.n_pages ? max(0, min(kPage, s.nvis - pg * kPage)) : 0;
         }
         // pass 1: the tile's max (scale > 0 commutes with max)
