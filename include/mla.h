@@ -127,7 +127,7 @@ size_t mla_append_workspace_bytes(const mla_dims* dims, int n_tokens);
 /* mla_append_latent_noalloc: mla_append_latent for callers that cannot
  * allocate device memory at call time (a plugin or callback whose host
  * framework owns all device memory and offers no scratch buffer, or a loop in
- * which an allocation would synchronise the device).  The paper has no
+ * which an allocation would synchronise the device).  The source articles have no
  * counterpart: this is a deployment variant of the S1 append.
  * Same arguments and results as mla_append_latent, without the workspace: the
  * fp32 scratch lives in a fixed array inside the library, 65,536 floats
