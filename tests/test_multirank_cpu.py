@@ -5,6 +5,7 @@ data-path collective.)"""
 import argparse
 import datetime
 import importlib.util
+import json
 import multiprocessing as mp
 import os
 import socket
@@ -72,3 +73,25 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     cfg = bench.WL.TINY_F32
     assert bench.run_reference(args, cfg) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_one_contract_line(monkeypatch, capsys):
+    """Rank 0 of the reference arm times the oracle and prints the bench
+    contract's JSON line, with its CPU baseline and a zero-copy e2e."""
+    bench = _load_bench()
+    monkeypatch.setenv("RANK", "0")
+    args = argparse.Namespace(steps=1, warmup=1, gpus=1)
+    cfg = bench.WL.TINY_F32
+    bench.run_reference(args, cfg)
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert d["config"]["workload"] == cfg.name
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
