@@ -1,7 +1,7 @@
 """GPU parity of the tcgen05 decode kernel (DeepSeek-V3 dims, bf16 and FP8
 caches): against the CPU oracle, against the CUDA-core kernel, and on the edge
 cases of its tiling (tails, single-token sequences, splits inside and across
-sequences, two to four causal query tokens, empty splits)."""
+sequences, two to eight causal query tokens, empty splits)."""
 import numpy as np
 import pytest
 import torch
@@ -42,6 +42,8 @@ CASES = [
     # the new tokens straddling a page boundary
     ("t3-causal", dict(B=2, T=3, L=(62, 300)), 3),
     ("t4-causal", dict(B=1, T=4, L=(190,)), 2),
+    # the most query tokens the tensor-core kernel takes (8), straddling a page
+    ("t8-max", dict(B=2, T=8, L=(60, 250)), 3),
 ]
 
 
