@@ -16,6 +16,16 @@ def test_bf16_matches_torch_cast():
     np.testing.assert_array_equal(O.to_bf16(x32.astype(np.float64)), ref)
 
 
+def test_generic_rounding_at_fp32_matches_ieee_cast():
+    # the same rounding routine at fp32's parameters (24-bit significand,
+    # emin -126, gradual underflow) against the IEEE float32 conversion,
+    # over normal and subnormal binades
+    rng = np.random.default_rng(1)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-44, 38, 20000),
+                        [0.0, 1.0 + 2.0 ** -24, 1.0 + 3 * 2.0 ** -24, 2.0 ** -149, 1.5 * 2.0 ** -149, 2.0 ** -126]])
+    np.testing.assert_array_equal(O.round_to_format(x, 24, -126), x.astype(np.float32).astype(np.float64))
+
+
 def test_bf16_ties_to_even():
     # 1 + 2^-8 lies halfway between 1 and 1 + 2^-7: ties go to the even significand (1.0)
     assert O.to_bf16(1.0 + 2.0 ** -8) == 1.0
