@@ -6,10 +6,13 @@ W^UV (libmla's three C-ABI calls).  Prints ONE JSON line.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl ours|reference]
 
 --config indexes the workloads in latent_compressed_attention_mla_b200.workloads
-(default 1: DeepSeek-V3 dims, B=1, L=4096, bf16).  With N>1 (torchrun) every
-rank runs an independent replica of the workload (weak scaling); the time is
-the max over ranks.  `--impl reference` times the CPU oracle (float64 numpy)
-on this host instead, rank 0 only.
+(default 4: DeepSeek-V3 dims, FP8 latent cache, 128 sequences of 16384 tokens,
+two causal query tokens each: the largest workload).  On one GPU the line also
+carries, under "configs", the other DeepSeek-V3-shaped workloads (one sequence
+of 4096; a ragged batch of 64; 8 sequences of 131072) timed the same way.
+With N>1 (torchrun) every rank runs an independent replica of the workload
+(weak scaling); the time is the max over ranks.  `--impl reference` times the
+CPU oracle (float64 numpy) on this host instead, rank 0 only.
 """
 from __future__ import annotations
 
@@ -167,9 +170,9 @@ class OracleStep:
     """One step of the workload on the CPU oracle: the oracle's append of the
     step's tokens and its explicit-form decode.  `heads` bounds the sample."""
 
-    def __init__(self, cfg: WL.MlaConfig, seqs, heads):
+    def __init__(self, cfg: WL.MlaConfig, seqs, heads, form: str = "explicit"):
         from oracle import mla_oracle as O
-        self.O, self.cfg, self.seqs, self.heads = O, cfg, list(seqs), list(heads)
+        self.O, self.cfg, self.seqs, self.heads, self.form = O, cfg, list(seqs), list(heads), form
         self.w = {k: v.double().numpy() for k, v in WL.weights(cfg, "cpu").items()}
         self.inp = {k: v.double().numpy() for k, v in WL.step_inputs(cfg, "cpu").items()}
         self.seq_idx, self.pos = WL.new_token_index(cfg)
@@ -187,8 +190,13 @@ class OracleStep:
             C1, KR1 = O.decode_cache_rows(O.encode_cache_rows(c, kr, cfg.cache_dtype))
             C = np.concatenate([self.hist[b][0], C1])
             KR = np.concatenate([self.hist[b][1], KR1])
-            O.decode_explicit(self.inp["q_nope"][b], self.inp["q_rope"][b], C, KR, self.w["W_uk"], self.w["W_uv"],
-                              int(cfg.seq_lens[b]), cfg.softmax_scale, cfg.rope_base, self.heads)
+            if self.form == "absorbed":  # all heads
+                O.decode_absorbed(self.inp["q_nope"][b], self.inp["q_rope"][b], C, KR, self.w["W_uk"],
+                                  self.w["W_uv"], int(cfg.seq_lens[b]), cfg.softmax_scale, cfg.rope_base)
+            else:
+                O.decode_explicit(self.inp["q_nope"][b], self.inp["q_rope"][b], C, KR, self.w["W_uk"],
+                                  self.w["W_uv"], int(cfg.seq_lens[b]), cfg.softmax_scale, cfg.rope_base,
+                                  self.heads)
 
     def tokens_per_call(self) -> float:
         """Decode tokens the call covers, counting a head sample as that fraction of a token."""
@@ -211,22 +219,35 @@ def oracle_sample(cfg: WL.MlaConfig, budget_s: float):
 
 
 def describe_sample(s: OracleStep) -> str:
-    return (f"oracle append + explicit decode of sequence(s) {s.seqs} (L={[int(s.cfg.L[b]) for b in s.seqs]}), "
+    return (f"oracle append + {s.form} decode of sequence(s) {s.seqs} (L={[int(s.cfg.L[b]) for b in s.seqs]}), "
             f"{len(s.heads)} of {s.cfg.n_heads} heads, {s.cfg.T} query token(s) each; "
             f"tokens/s counts a head sample as that fraction of a token")
 
 
-def cpu_baseline(cfg: WL.MlaConfig, budget_s: float = 15.0) -> dict:
-    step, _ = oracle_sample(cfg, budget_s / 3)
+def _time_calls(step, budget_s: float, max_calls: int = 50):
     n, t0 = 0, time.perf_counter()
     while True:
         step()
         n += 1
-        if time.perf_counter() - t0 >= budget_s or n >= 50:
+        if time.perf_counter() - t0 >= budget_s or n >= max_calls:
             break
-    dt = time.perf_counter() - t0
-    return {"value": n * step.tokens_per_call() / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": describe_sample(step) + f"; {n} calls in {dt:.1f} s"}
+    return n, time.perf_counter() - t0
+
+
+def cpu_baseline(cfg: WL.MlaConfig, budget_s: float = 15.0) -> dict:
+    """The oracle as it stands on the host cores: its explicit form (the oracle
+    of record) on a bounded sample, and beside it its absorbed form (all heads
+    of whole sequences, the same mathematics the GPU path runs)."""
+    step, _ = oracle_sample(cfg, budget_s / 3)
+    n, dt = _time_calls(step, budget_s)
+    out = {"value": n * step.tokens_per_call() / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": describe_sample(step) + f"; {n} calls in {dt:.1f} s"}
+    seqs = [int(np.argmin(cfg.L))] if cfg.B > 1 else [0]
+    absorbed = OracleStep(cfg, seqs, range(cfg.n_heads), form="absorbed")
+    n, dt = _time_calls(absorbed, budget_s / 3)
+    out["absorbed_form"] = {"value": n * absorbed.tokens_per_call() / dt, "unit": "tokens/s",
+                            "sample": describe_sample(absorbed) + f"; {n} calls in {dt:.1f} s"}
+    return out
 
 
 def max_over_ranks(x: float, pg, device) -> float:
@@ -263,40 +284,250 @@ def run_reference(args, cfg):
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_dict(cfg, None), "impl": "reference",
+            "config": config_dict(cfg), "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": describe_sample(step)},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def config_dict(cfg, extra):
-    d = {"workload": cfg.name, "batch": cfg.B, "n_q": cfg.T,
-         "context_before_step": int(cfg.L[0]) if len(set(cfg.L)) == 1 else
-         {"min": int(min(cfg.L)), "max": int(max(cfg.L)), "sum": int(sum(cfg.L))},
-         "n_heads": cfg.n_heads, "d_c": cfg.d_c, "d_rope": cfg.d_rope, "d_nope": cfg.d_nope, "d_v": cfg.d_v,
-         "d_model": cfg.d_model, "page_size": cfg.page_size, "cache": cfg.cache_dtype, "act": cfg.act_dtype,
-         "seed": cfg.seed}
-    if extra:
-        d.update(extra)
-    return d
+def config_dict(cfg):
+    """The workload, by what it is (the same dict in both arms of the bench)."""
+    return {"workload": cfg.name, "batch": cfg.B, "n_q": cfg.T,
+            "context_before_step": int(cfg.L[0]) if len(set(cfg.L)) == 1 else
+            {"min": int(min(cfg.L)), "max": int(max(cfg.L)), "sum": int(sum(cfg.L))},
+            "n_heads": cfg.n_heads, "d_c": cfg.d_c, "d_rope": cfg.d_rope, "d_nope": cfg.d_nope, "d_v": cfg.d_v,
+            "d_model": cfg.d_model, "page_size": cfg.page_size, "cache": cfg.cache_dtype, "act": cfg.act_dtype,
+            "seed": cfg.seed}
+
+
+def roofline_times(work: dict, peaks: dict, tpeak: float) -> dict:
+    """Per kernel: (t_bytes, t_flops) at the measured HBM copy rate and the given tensor peak, seconds."""
+    return {k: (w["bytes"] / (peaks["hbm_gbs"] * 1e9), w["flops"] / (tpeak * 1e12)) for k, w in work.items()}
+
+
+def step_summary(cfg, work: dict, kms: dict, ms_step: float, peaks: dict, tpeak: float) -> dict:
+    """Per-kernel rows, the attend kernel's latent-cache figures and the
+    whole step's roofline fraction from per-kernel device times (ms)."""
+    rt = roofline_times(work, peaks, tpeak)
+    rows = {}
+    for name, t in kms.items():
+        t_s = t / 1e3
+        tb, tf = rt[name]
+        rows[name] = {"us": 1e3 * t, "bound": "tensor" if tf > tb else "hbm",
+                      "GBps": work[name]["bytes"] / t_s / 1e9 if t_s > 0 else None,
+                      "TFLOPs": work[name]["flops"] / t_s / 1e12 if t_s > 0 else None,
+                      "roofline_frac": max(tb, tf) / t_s if t_s > 0 else None}
+    att = work["attend"]
+    t_att = kms["attend"] / 1e3
+    t_core = max(att["cache_bytes"] / (peaks["hbm_gbs"] * 1e9), att["flops"] / (tpeak * 1e12))
+    t_roof_step = sum(max(rt[k]) for k in kms)
+    return {
+        "rows": rows,
+        "attend": {"us": 1e6 * t_att, "latent_cache_TBps": att["cache_bytes"] / t_att / 1e12,
+                   "TFLOPs": att["flops"] / t_att / 1e12, "core_roofline_us": 1e6 * t_core,
+                   "frac_of_core_roofline": t_core / t_att},
+        "full_step_roofline_us": 1e6 * t_roof_step,
+        "full_step_frac": t_roof_step / (ms_step / 1e3),
+    }
+
+
+class Workload:
+    """One workload resident on the device, with enough copies of everything a
+    step touches that consecutive steps do not find their inputs in L2, and a
+    decode session; `step(i)` runs the library's calls for step i."""
+
+    def __init__(self, cfg, dev, splits: int, flags: int):
+        from latent_compressed_attention_mla_b200 import binding as B
+        from latent_compressed_attention_mla_b200.decoder import MlaDecodeSession
+        from latent_compressed_attention_mla_b200.paged_cache import PagedLatentCache
+        self.B, self.cfg, self.dev = B, cfg, dev
+        self.dims = B.dims_for(cfg, flags)
+        self.page_bytes = B.cache_page_bytes(self.dims)
+        self.work = kernel_work(cfg, self.page_bytes)
+        weights0 = WL.weights(cfg, dev)
+        self.inputs0 = WL.step_inputs(cfg, dev)
+        self.pt = torch.from_numpy(WL.page_table(cfg)).to(dev)
+        self.seq_idx, self.pos = (torch.from_numpy(x).to(dev) for x in WL.new_token_index(cfg))
+        self.seq_lens = torch.from_numpy(cfg.seq_lens.astype(np.int32)).to(dev)
+        cache0 = PagedLatentCache(self.dims, cfg.num_pages, dev)
+        for b in range(cfg.B):
+            L = int(cfg.L[b])
+            for s0 in range(0, L, 1 << 18):
+                s1 = min(L, s0 + (1 << 18))
+                cache0.write_rows(self.pt[b], torch.arange(s0, s1, device=dev), WL.history_rows(cfg, b, s0, s1, dev))
+        per_copy = sum(t.numel() * t.element_size() for t in list(weights0.values()) + list(self.inputs0.values()))
+        per_copy += cache0.pool.numel()
+        self.copies = 1 if per_copy > 3 * L2_BYTES else int(math.ceil(3 * L2_BYTES / per_copy))
+        self.per_copy = per_copy
+        self.sets = [(weights0, self.inputs0, cache0.pool)]
+        for _ in range(self.copies - 1):
+            self.sets.append(({k: v.clone() for k, v in weights0.items()},
+                              {k: v.clone() for k, v in self.inputs0.items()}, cache0.pool.clone()))
+        self.sess = MlaDecodeSession(self.dims, cfg.B, cfg.T, splits, dev)
+        # the split count mla_decode uses: explicit, else the automatic count
+        # capped at one split per 4 pages of batch * max_pages
+        self.splits = splits or min(B.auto_splits(self.dims, cfg.B, cfg.T), max(1, -(-cfg.B * cfg.max_pages // 4)))
+        self.path = B.decode_path(self.dims, cfg.T)
+        # library kernels per step: append (+ the FP8 quantiser), absorb, attend, combine
+        self.launches_per_step = 4 + (1 if cfg.cache_dtype == "fp8" else 0)
+
+    def step(self, i):
+        w, x, pool = self.sets[i % self.copies]
+        self.sess.step(x["h"], self.seq_idx, self.pos, x["q_nope"], x["q_rope"], self.seq_lens, w, self.pt, pool)
+
+    def capture(self):
+        """One CUDA graph per buffer set (eager steps first: one-time set-up in
+        the library happens outside capture)."""
+        for i in range(min(2, self.copies)):
+            self.step(i)
+        torch.cuda.synchronize()
+        graphs = []
+        for r in range(self.copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.step(r)
+            graphs.append(g)
+        return graphs
+
+    def l2_note(self) -> str:
+        return (f"inputs rotate over {self.copies} copies ({self.copies * self.per_copy / 2**20:.0f} MiB > 126 MiB L2)"
+                if self.copies > 1 else f"inputs ({self.per_copy / 2**30:.2f} GiB) larger than L2")
+
+
+def time_graph_steps(wl: Workload, graphs, steps: int, warmup: int, pg, local: int):
+    """Device time of `steps` graph replays (CUDA events on the replay stream,
+    barrier + synchronize on both sides, max over ranks), with clocks sampled
+    during the timed region."""
+    B = wl.B
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    if B.mla_get_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    t_start_wall = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        graphs[(warmup + i) % len(graphs)].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t_end_wall = time.time()
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop(t_start_wall, t_end_wall)
+    return max_over_ranks(e0.elapsed_time(e1), pg, wl.dev), clocks
+
+
+def timeline_kernel_ms(wl: Workload, steps: int) -> dict:
+    """Per-kernel device spans (ms, mean over `steps` steps) from graph replays
+    whose kernels stamp %globaltimer into a device timeline (mla_set_timeline):
+    the same launches as the timed replays, with the grid-dependency chain
+    between the kernels intact."""
+    B = wl.B
+    nk = len(B.TRACE_KERNELS)
+    tl = torch.empty(2 * nk, dtype=torch.int64, device=wl.dev)
+    ring = torch.empty(steps, 2 * nk, dtype=torch.int64, device=wl.dev)
+    B.mla_set_timeline(tl)
+    try:
+        graphs = wl.capture()
+    finally:
+        B.mla_set_timeline(None)
+    for i in range(steps):
+        B.timeline_init(tl)
+        graphs[i % len(graphs)].replay()
+        ring[i].copy_(tl)
+    host = ring.cpu().numpy()
+    del graphs
+    sums = {}
+    for i in range(steps):
+        for k, v in B.timeline_spans_ns(host[i]).items():
+            sums[k] = sums.get(k, 0.0) + v
+    return {k: v / steps / 1e6 for k, v in sums.items()}
+
+
+def e2e_pass(wl: Workload, steps: int, warmup: int, pg):
+    """The same metric through the session's host-driven step: pinned host
+    inputs copied in, the step, the output copied back, every step."""
+    from latent_compressed_attention_mla_b200.decoder import packed_step_buffers
+    sess, inputs0 = wl.sess, wl.inputs0
+    host_in, dev_in = packed_step_buffers({k: (inputs0[k].shape, inputs0[k].dtype) for k in ("h", "q_nope", "q_rope")},
+                                          wl.dev)
+    for k in host_in:
+        host_in[k].copy_(inputs0[k].cpu())
+    host_out = torch.empty(sess.out.shape, dtype=sess.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+    # untimed: every buffer set once (the session records its graph on first use)
+    for i in range(max(min(warmup, 5), wl.copies)):
+        w, _, pool = wl.sets[i % wl.copies]
+        sess.step_from_host(host_in, dev_in, wl.seq_idx, wl.pos, wl.seq_lens, w, wl.pt, pool, host_out)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for i in range(steps):
+        w, _, pool = wl.sets[i % wl.copies]
+        sess.step_from_host(host_in, dev_in, wl.seq_idx, wl.pos, wl.seq_lens, w, wl.pt, pool, host_out)
+    f1.record()
+    torch.cuda.synchronize()
+    return max_over_ranks(f0.elapsed_time(f1), pg, wl.dev), h2d, d2h
+
+
+def measure(cfg, args, dev, pg, local: int, peaks: dict) -> dict:
+    """Time one workload: graph replays (the value), per-kernel spans from
+    timeline replays, and the roofline figures."""
+    wl = Workload(cfg, dev, args.splits, args.flags)
+    graphs = wl.capture()
+    ms, clocks = time_graph_steps(wl, graphs, args.steps, args.warmup, pg, local)
+    del graphs
+    kms = timeline_kernel_ms(wl, max(args.steps, 5))
+    if cfg.cache_dtype != "fp8":
+        kms.pop("append_finalize", None)
+    ms_step = ms / args.steps
+    # a kernel timed alone (or a short region) takes the burst tensor peak
+    tpeak = peaks["bf16_tflops_sustained"] if ms > 1000.0 else peaks["bf16_tflops"]
+    summ = step_summary(cfg, wl.work, kms, ms_step, peaks, tpeak)
+    return {"wl": wl, "ms": ms, "ms_step": ms_step, "clocks": clocks, "kms": kms, "tpeak": tpeak, **summ}
+
+
+def config_entry(cfg, m: dict, world: int) -> dict:
+    """A workload's figures for the per-config map of the JSON line."""
+    return {"ms_per_step": m["ms_step"], "tokens_per_s": whole_job_tokens_per_s(world, cfg.B * cfg.T, 1, m["ms_step"]),
+            "attend_us": round(m["attend"]["us"], 3),
+            "latent_cache_TBps": m["attend"]["latent_cache_TBps"], "attend_TFLOPs": m["attend"]["TFLOPs"],
+            "core_roofline_us": m["attend"]["core_roofline_us"],
+            "frac_of_core_roofline": m["attend"]["frac_of_core_roofline"],
+            "full_step_roofline_us": m["full_step_roofline_us"], "full_step_frac": m["full_step_frac"],
+            "kernels_us": {k: round(v["us"], 3) for k, v in m["rows"].items()},
+            "splits": m["wl"].splits, "path": "tcgen05" if m["wl"].path == 1 else "simt",
+            "l2": m["wl"].l2_note(), "clocks": m["clocks"]}
 
 
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
+EXTRA_CONFIGS = (1, 2, 3)  # the other DeepSeek-V3-shaped workloads, reported beside the headline
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--flags", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-graph", dest="graph", action="store_false",
-                    help="launch each step eagerly instead of replaying a captured CUDA graph")
+    ap.add_argument("--no-extra-configs", dest="extra", action="store_false",
+                    help="time only the headline workload (no per-config map)")
     ap.add_argument("--batch", type=int, default=0,
                     help="keep only the first N sequences of the workload (smaller case of the same kernels, "
                          "e.g. for profiler captures); the workload name records it")
@@ -306,10 +537,6 @@ def main():
         cfg = cfg.with_(name=f"{cfg.name}[:{args.batch}]", B=args.batch, L=tuple(cfg.L[:args.batch]))
     if args.impl == "reference":
         return run_reference(args, cfg)
-
-    from latent_compressed_attention_mla_b200 import binding as B
-    from latent_compressed_attention_mla_b200.decoder import MlaDecodeSession, packed_step_buffers
-    from latent_compressed_attention_mla_b200.paged_cache import PagedLatentCache
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -323,169 +550,45 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
         pg = dist
 
-    dims = B.dims_for(cfg, args.flags)
-    page_bytes = B.cache_page_bytes(dims)
-    work = kernel_work(cfg, page_bytes)
-
-    # one copy of everything a step touches; rotate copies when one fits in L2
-    weights0 = WL.weights(cfg, dev)
-    inputs0 = WL.step_inputs(cfg, dev)
-    pt = torch.from_numpy(WL.page_table(cfg)).to(dev)
-    seq_idx, pos = (torch.from_numpy(x).to(dev) for x in WL.new_token_index(cfg))
-    seq_lens = torch.from_numpy(cfg.seq_lens.astype(np.int32)).to(dev)
-    cache0 = PagedLatentCache(dims, cfg.num_pages, dev)
-    for b in range(cfg.B):
-        L = int(cfg.L[b])
-        for s0 in range(0, L, 1 << 18):
-            s1 = min(L, s0 + (1 << 18))
-            cache0.write_rows(pt[b], torch.arange(s0, s1, device=dev), WL.history_rows(cfg, b, s0, s1, dev))
-    per_copy = sum(t.numel() * t.element_size() for t in list(weights0.values()) + list(inputs0.values()))
-    per_copy += cache0.pool.numel()
-    copies = 1 if per_copy > 3 * L2_BYTES else int(math.ceil(3 * L2_BYTES / per_copy))
-    sets = [(weights0, inputs0, cache0.pool)]
-    for _ in range(copies - 1):
-        sets.append(({k: v.clone() for k, v in weights0.items()}, {k: v.clone() for k, v in inputs0.items()},
-                     cache0.pool.clone()))
-    sess = MlaDecodeSession(dims, cfg.B, cfg.T, args.splits, dev)
-    # the split count mla_decode uses: explicit, else the automatic count capped
-    # at one split per 4 pages of batch * max_pages
-    splits = args.splits or min(B.auto_splits(dims, cfg.B, cfg.T), max(1, -(-cfg.B * cfg.max_pages // 4)))
-    path = B.decode_path(dims, cfg.T)
-
-    def step(i):
-        w, x, pool = sets[i % copies]
-        sess.step(x["h"], seq_idx, pos, x["q_nope"], x["q_rope"], seq_lens, w, pt, pool)
-
-    # eager steps first: one-time set-up in the library happens outside capture
-    for i in range(min(2, copies) if args.graph else 0):
-        step(i)
-    torch.cuda.synchronize()
-    graphs = []
-    if args.graph:
-        for r in range(copies):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                step(r)
-            graphs.append(g)
-
-    def run_step(i):
-        if graphs:
-            graphs[i % copies].replay()
-        else:
-            step(i)
-
-    for i in range(args.warmup):
-        run_step(i)
-    torch.cuda.synchronize()
-    if B.mla_get_status() != 0:
-        raise RuntimeError("device status set during warm-up")
-
-    # timed region: K steps, nothing else on the stream
-    sampler = ClockSampler(local)
-    time.sleep(0.3)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    t_start_wall = time.time()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(args.steps):
-        run_step(args.warmup + i)
-    e1.record()
-    torch.cuda.synchronize()
-    t_end_wall = time.time()
-    if pg:
-        pg.barrier()
-    clocks = sampler.stop(t_start_wall, t_end_wall)
-    ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
-
-    # per-kernel durations: the same K steps again, launched eagerly with the
-    # library recording a CUDA event before and after each kernel on the launch
-    # stream (a ring of event sets, read back RING steps behind)
-    nk = len(B.TRACE_KERNELS)
-    RING = 32
-    ring = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(RING)]
-    ksum = np.zeros(nk)
-
-    def harvest(evs):
-        evs[-1].synchronize()
-        for k in range(nk):
-            ksum[k] += evs[2 * k].elapsed_time(evs[2 * k + 1])
-
-    for i in range(args.steps):
-        if i >= RING:
-            harvest(ring[i % RING])
-        B.mla_set_trace_events(ring[i % RING])
-        step(args.warmup + i)
-    torch.cuda.synchronize()
-    B.mla_set_trace_events(None)
-    for i in range(max(0, args.steps - RING), args.steps):
-        harvest(ring[i % RING])
-    status = B.mla_get_status()
-
-    tokens_per_step = cfg.B * cfg.T
-    value = whole_job_tokens_per_s(world, tokens_per_step, args.steps, ms)
-    kms = {name: ksum[k] / args.steps for k, name in enumerate(B.TRACE_KERNELS)}  # ms per launch
-    if cfg.cache_dtype != "fp8":
-        kms.pop("append_finalize")  # only FP8 caches launch it; its events bracket nothing here
-    launches_per_step = len(kms)
     peaks = load_peaks()
-    long_region = ms > 1000.0
-    tpeak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
-    rows = {}
-    for name, t in kms.items():
-        wk = work[name]
-        t_s = t / 1e3
-        t_bytes = wk["bytes"] / (peaks["hbm_gbs"] * 1e9)
-        t_flops = wk["flops"] / (tpeak * 1e12)
-        bound = "tensor" if t_flops > t_bytes else "hbm"
-        rows[name] = {"us": 1e3 * t, "GBps": wk["bytes"] / t_s / 1e9 if t_s > 0 else None,
-                      "TFLOPs": wk["flops"] / t_s / 1e12 if t_s > 0 else None, "bound": bound,
-                      "roofline_frac": (max(t_bytes, t_flops) / t_s) if t_s > 0 else None}
-    dom = max(kms, key=lambda k: kms[k])
-    wd, td = work[dom], kms[dom] / 1e3
+    m = measure(cfg, args, dev, pg, local, peaks)
+    wl = m["wl"]
+    ms_e2e, h2d, d2h = e2e_pass(wl, args.steps, args.warmup, pg)
+    status = wl.B.mla_get_status()
+    tokens_per_step = cfg.B * cfg.T
+    value = whole_job_tokens_per_s(world, tokens_per_step, args.steps, m["ms"])
+    e2e = {"value": whole_job_tokens_per_s(world, tokens_per_step, args.steps, ms_e2e), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    rows = m["rows"]
+    dom = max(m["kms"], key=lambda k: m["kms"][k])
+    wd, td = wl.work[dom], m["kms"][dom] / 1e3
     if rows[dom]["bound"] == "tensor":
-        roof = {"bound": "tensor", "achieved": wd["flops"] / td / 1e12, "peak": tpeak, "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": wd["flops"] / td / 1e12, "peak": m["tpeak"], "unit": "TFLOP/s"}
     else:
         roof = {"bound": "hbm", "achieved": wd["bytes"] / td / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = measured_traffic(cfg.name, dom)
     roof["kernel"] = dom
-    roof["peak_source"] = peaks["source"] + (" sustained" if (roof["bound"] == "tensor" and long_region) else
-                                             (" burst" if roof["bound"] == "tensor" else " copy"))
-    att = work["attend"]
-    t_att = kms["attend"] / 1e3
-    t_core = max(att["cache_bytes"] / (peaks["hbm_gbs"] * 1e9), att["flops"] / (tpeak * 1e12))
-    attend_summary = {"latent_cache_TBps": att["cache_bytes"] / t_att / 1e12, "TFLOPs": att["flops"] / t_att / 1e12,
-                      "core_roofline_us": 1e6 * t_core, "frac_of_core_roofline": t_core / t_att,
-                      "path": "tcgen05" if path == 1 else "simt", "splits": splits}
+    roof["peak_source"] = peaks["source"] + (
+        (" sustained" if m["tpeak"] == peaks["bf16_tflops_sustained"] else " burst") if roof["bound"] == "tensor"
+        else " copy")
+    setup = {"l2": wl.l2_note(), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+             "splits": wl.splits, "path": "tcgen05" if wl.path == 1 else "simt"}
+    launches = wl.launches_per_step * args.steps
+    # free the headline workload before the others are built
+    del m["wl"], wl
+    torch.cuda.empty_cache()
 
-    # end to end through the public API: pinned host inputs -> device -> step -> host output
-    # the step's inputs in one pinned block and one device block (one transfer)
-    host_in, dev_in = packed_step_buffers({k: (inputs0[k].shape, inputs0[k].dtype) for k in ("h", "q_nope", "q_rope")},
-                                          dev)
-    for k in host_in:
-        host_in[k].copy_(inputs0[k].cpu())
-    host_out = torch.empty(sess.out.shape, dtype=sess.out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = host_out.numel() * host_out.element_size()
-    # untimed: every buffer set once (the session records its graph on first use)
-    for i in range(max(min(args.warmup, 5), copies)):
-        w, _, pool = sets[i % copies]
-        sess.step_from_host(host_in, dev_in, seq_idx, pos, seq_lens, w, pt, pool, host_out)
-    torch.cuda.synchronize()
-    if pg:
-        pg.barrier()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record()
-    for i in range(args.steps):
-        w, _, pool = sets[i % copies]
-        sess.step_from_host(host_in, dev_in, seq_idx, pos, seq_lens, w, pt, pool, host_out)
-    f1.record()
-    torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(f0.elapsed_time(f1), pg, dev)
-    e2e = {"value": whole_job_tokens_per_s(world, tokens_per_step, args.steps, ms_e2e), "unit": "tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    extra = {}
+    if args.extra and world == 1 and args.batch == 0:
+        for ci in EXTRA_CONFIGS:
+            if ci == args.config:
+                continue
+            c = WL.CONFIGS[ci]
+            mc = measure(c, args, dev, None, local, peaks)
+            extra[c.name] = config_entry(c, mc, world)
+            del mc
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -496,21 +599,23 @@ def main():
         pg.destroy_process_group()
     if rank != 0:
         return
-    l2 = (f"inputs rotate over {copies} copies ({copies * per_copy / 2**20:.0f} MiB > 126 MiB L2)" if copies > 1
-          else f"inputs ({per_copy / 2**30:.2f} GiB) larger than L2")
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": m["ms_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.act_dtype if cfg.cache_dtype != "fp8" else "bf16+e4m3-cache",
         "data": "synthetic (seeded counter-based generator; random-init weights)",
-        "config": config_dict(cfg, {"l2": l2, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                                    "splits": splits}),
-        "roofline": roof, "attend": attend_summary, "kernels_us": {k: round(v["us"], 3) for k, v in rows.items()},
+        "config": config_dict(cfg), "setup": setup,
+        "roofline": roof,
+        "attend": {**{k: v for k, v in m["attend"].items() if k != "us"}, "us": round(m["attend"]["us"], 3)},
+        "kernels_us": {k: round(v["us"], 3) for k, v in rows.items()},
         "kernel_roofline_frac": {k: (round(v["roofline_frac"], 4) if v["roofline_frac"] else None)
                                  for k, v in rows.items()},
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
-        "timing": ("CUDA-graph replay of each step" if args.graph else "eager launches") +
-                  "; per-kernel times from a second, traced pass of the same steps",
+        "full_step_roofline_us": m["full_step_roofline_us"], "full_step_frac": m["full_step_frac"],
+        "configs": extra,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": m["clocks"],
+        "timing": ("CUDA-graph replay of each step (CUDA events around the replays); per-kernel spans from "
+                   "%globaltimer stamps the kernels write in a second series of replays of the same steps "
+                   "(mla_set_timeline)"),
         "device_status": status,
     }
     print(json.dumps(line), flush=True)

@@ -20,7 +20,9 @@
  * General conventions
  *   - Every pointer argument is a DEVICE pointer owned by the caller unless
  *     stated otherwise.  The library allocates no device memory: scratch is the
- *     caller's `workspace`, sized by the matching *_workspace_bytes() call.
+ *     caller's `workspace`, sized by the matching *_workspace_bytes() call,
+ *     except for mla_append_latent_noalloc, whose scratch is a fixed 256 KiB
+ *     array inside the library on every GPU that loads it (see its note).
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
  *     is the legacy default stream).  Nothing synchronises except
  *     mla_get_status().  Kernels run on the current CUDA device.
@@ -71,12 +73,18 @@ enum {
 
 /* mla_dims.flags */
 #define MLA_FLAG_FORCE_SIMT 1u /* use the CUDA-core kernels even where tcgen05 kernels exist */
-/* Self-test of failure detection: mla_combine's tensor-core kernel (bf16
- * activations at DeepSeek-V3 dims) does not fetch its weights, so its bounded
- * wait for them (~2 s) expires; the call then records MLA_ERR_TIMEOUT in the
- * device status word and leaves out and lse_out unwritten.  No copy is in
- * flight when the wait gives up, and the context stays usable.  Ignored by
- * the other kernels. */
+/* Self-test of failure detection, for the tensor-core kernels at DeepSeek-V3
+ * dims (bf16 activations):
+ *   - mla_decode: the attention kernel's load producers issue no loads, so the
+ *     MMA issuers' and softmax warps' bounded waits (~2 s) expire; the CTA
+ *     pair that gives up first tells its peer, every role stops, the kernel
+ *     waits (bounded) for the MMAs it issued and frees its tensor memory;
+ *     MLA_ERR_TIMEOUT is recorded and the split partials are not valid.
+ *   - mla_combine: the kernel does not fetch its weights, so its bounded wait
+ *     for them expires; MLA_ERR_TIMEOUT is recorded and out and lse_out are
+ *     left unwritten.
+ * No copy is in flight when a wait gives up, and the context stays usable.
+ * Ignored by the other kernels. */
 #define MLA_FLAG_SELFTEST_STALL 2u
 
 typedef struct {
@@ -132,8 +140,11 @@ size_t mla_append_workspace_bytes(const mla_dims* dims, int n_tokens);
  * Same arguments and results as mla_append_latent, without the workspace: the
  * fp32 scratch lives in a fixed array inside the library, 65,536 floats
  * (256 KiB) on every GPU that loads it, held until the process exits.
- *   - n_tokens * (d_c + d_rope) must be <= 65536 (113 tokens at DeepSeek-V3
- *     dims); larger requests return MLA_ERR_WORKSPACE and launch nothing.
+ *   - The scratch a call uses is what mla_append_workspace_bytes() reports:
+ *     n_tokens * d_c floats for an FP8 cache, none for bf16 and fp32 caches.
+ *     An FP8 request must fit the array (n_tokens * d_c <= 65536: 128 tokens
+ *     at DeepSeek-V3 dims); a larger one returns MLA_ERR_WORKSPACE and
+ *     launches nothing.  bf16 and fp32 caches have no size limit here.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
  *   - All calls share the array: calls whose kernels overlap on the GPU race.
@@ -219,6 +230,22 @@ enum {
  * table is process-wide host state read at launch time; it is not
  * thread-safe.  Returns MLA_OK or MLA_ERR_INVALID_ARG (n_events too small). */
 int mla_set_trace_events(void* const* events, int n_events);
+
+/* Device timeline of the kernels, for timing a step from CUDA-graph replays
+ * (where events recorded between kernels would break their programmatic
+ * dependent launch).  `device_buffer` is a DEVICE array of 2*MLA_TRACE_COUNT
+ * uint64 owned by the caller, or NULL to switch the timeline off.  Kernels
+ * launched while it is installed write, for each kernel k above:
+ *   [2k]   the earliest %globaltimer value (ns) at which one of its CTAs had
+ *          passed its wait for the preceding kernel (atomic minimum: the
+ *          caller initialises it to UINT64_MAX),
+ *   [2k+1] the latest value at which one of its CTAs finished (atomic
+ *          maximum: initialised to 0).
+ * So [2k+1] - [2k] is kernel k's span on the device with its dependency
+ * already met.  The pointer is read at launch time (a graph keeps the value it
+ * was captured with); it is process-wide host state and not thread-safe.
+ * Returns MLA_OK. */
+int mla_set_timeline(unsigned long long* device_buffer);
 
 /* Synchronise `stream`, then read and clear the device status word of the
  * current device into *status (MLA_OK or MLA_ERR_TIMEOUT / MLA_ERR_BOUNDS).

@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_PKG, "libmla.so")
 
 MLA_F32, MLA_BF16, MLA_FP8_E4M3 = 0, 1, 2
 MLA_FLAG_FORCE_SIMT = 1
-MLA_FLAG_SELFTEST_STALL = 2  # combine skips its weight fetch: its bounded wait expires (tests)
+MLA_FLAG_SELFTEST_STALL = 2  # decode issues no loads, combine no weight fetch: bounded waits expire (tests)
 
 (MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_ALIGNMENT, MLA_ERR_LAUNCH,
  MLA_ERR_TIMEOUT, MLA_ERR_BOUNDS, MLA_ERR_CUDA) = range(9)
@@ -28,7 +28,7 @@ ERRORS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "M
 EXPORTED = ("mla_cache_page_bytes", "mla_check_dims", "mla_append_workspace_bytes", "mla_append_latent",
             "mla_append_latent_noalloc",
             "mla_decode_workspace_bytes", "mla_decode", "mla_combine", "mla_decode_path", "mla_auto_splits",
-            "mla_set_trace_events", "mla_get_status", "mla_error_string")
+            "mla_set_trace_events", "mla_set_timeline", "mla_get_status", "mla_error_string")
 TRACE_KERNELS = ("append_project", "append_finalize", "absorb", "attend", "combine")
 
 
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
         L.mla_get_status.argtypes, L.mla_get_status.restype = [P, ctypes.POINTER(ctypes.c_int)], I
         L.mla_error_string.argtypes, L.mla_error_string.restype = [I], ctypes.c_char_p
         L.mla_set_trace_events.argtypes, L.mla_set_trace_events.restype = [ctypes.POINTER(P), I], I
+        L.mla_set_timeline.argtypes, L.mla_set_timeline.restype = [P], I
         _lib = L
     return _lib
 
@@ -154,8 +155,9 @@ def mla_append_latent(dims, h, seq_idx, pos, W_dkv, W_kr, page_table, cache_pool
 
 def mla_append_latent_noalloc(dims, h, seq_idx, pos, W_dkv, W_kr, page_table, cache_pool, stream=None):
     """S1 without a workspace, for callers that cannot allocate device memory
-    at call time: the library's fixed scratch array is used instead (at most
-    65,536 floats, i.e. n_tokens * (d_c + d_rope) <= 65536)."""
+    at call time: the library's fixed scratch array is used instead (65,536
+    floats; an FP8-cache call needs n_tokens * d_c of them, bf16 and fp32
+    caches none)."""
     _cuda(h, seq_idx, pos, W_dkv, W_kr, page_table, cache_pool)
     num_pages = cache_pool.numel() * cache_pool.element_size() // cache_page_bytes(dims)
     rc = lib().mla_append_latent_noalloc(ctypes.byref(dims), _ptr(h), h.shape[0], _ptr(seq_idx), _ptr(pos),
@@ -203,3 +205,36 @@ def mla_set_trace_events(events):
             e.record()
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check(lib().mla_set_trace_events(arr, len(events)), "mla_set_trace_events")
+
+
+def mla_set_timeline(buffer):
+    """Install a device int64 tensor of 2 * len(TRACE_KERNELS) elements as the
+    kernels' timeline (None switches it off).  Per kernel k, element 2k gets
+    the earliest ns time a CTA passed its dependency wait (initialise to -1,
+    i.e. all bits set) and 2k+1 the latest time a CTA finished (initialise to 0)."""
+    if buffer is None:
+        _check(lib().mla_set_timeline(None), "mla_set_timeline")
+        return
+    _cuda(buffer)
+    if buffer.dtype != torch.int64 or buffer.numel() < 2 * len(TRACE_KERNELS):
+        raise ValueError("timeline buffer: int64 tensor of 2 * len(TRACE_KERNELS) elements")
+    _check(lib().mla_set_timeline(_ptr(buffer)), "mla_set_timeline")
+
+
+def timeline_init(buffer):
+    """Reset a timeline buffer (on the current stream): begins to UINT64_MAX, ends to 0."""
+    v = buffer.view(-1, 2)
+    v[:, 0].fill_(-1)
+    v[:, 1].zero_()
+
+
+def timeline_spans_ns(host_values) -> dict:
+    """kernel name -> span (ns) from a timeline read back to the host
+    (int64 values; begins of kernels that did not run stay all-ones)."""
+    out = {}
+    for k, name in enumerate(TRACE_KERNELS):
+        b = int(host_values[2 * k]) & 0xFFFFFFFFFFFFFFFF
+        e = int(host_values[2 * k + 1])
+        if b != 0xFFFFFFFFFFFFFFFF and e > 0:
+            out[name] = e - b
+    return out

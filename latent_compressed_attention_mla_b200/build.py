@@ -1,4 +1,8 @@
-"""Build libmla.so in-tree with nvcc for sm_100a (B200)."""
+"""Build libmla.so in-tree with nvcc for sm_100a (B200).
+
+Each translation unit compiles to an object in parallel (objects under
+_build/, which is not part of the sources), then nvcc links the shared
+library next to this file."""
 from __future__ import annotations
 
 import glob
@@ -6,12 +10,14 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libmla.so")
-NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
-              "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
+OBJ_DIR = os.path.join(ROOT, "_build")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+NVCC_FLAGS = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
 
 
 def sources() -> list[str]:
@@ -34,16 +40,33 @@ def needs_build() -> bool:
 
 
 def build(verbose: bool = False, extra: list[str] | None = None) -> str:
-    cmd = [_nvcc(), *NVCC_FLAGS, *(extra or []), "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp",
-           *sources()]
+    nvcc = _nvcc()
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    inc = ["-I", os.path.join(ROOT, "include")]
+
+    def compile_one(src: str):
+        obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
+        cmd = [nvcc, *NVCC_FLAGS, *(extra or []), *inc, "-c", "-o", obj, src]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        return obj, subprocess.run(cmd, capture_output=True, text=True)
+
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        results = list(ex.map(compile_one, sources()))
+    failed = False
+    for _, r in results:
+        if r.stdout or r.stderr:
+            (sys.stderr if r.returncode else sys.stdout).write(r.stdout + r.stderr)
+        failed |= r.returncode != 0
+    if failed:
+        raise RuntimeError("nvcc failed building libmla.so")
+    link = [nvcc, *ARCH, "-shared", "-o", LIB + ".tmp", *[o for o, _ in results]]
     if verbose:
-        print(" ".join(cmd), flush=True)
-    r = subprocess.run(cmd, capture_output=True, text=True)
+        print(" ".join(link), flush=True)
+    r = subprocess.run(link, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building libmla.so")
-    if verbose and (r.stdout or r.stderr):
-        print(r.stdout + r.stderr)
+        raise RuntimeError("nvcc failed linking libmla.so")
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

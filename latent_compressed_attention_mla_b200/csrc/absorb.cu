@@ -55,6 +55,7 @@ struct AbsorbArgs {
   float* lse_part;
   size_t lse_count;
   int* status;
+  unsigned long long* timeline;  // device timeline (null: off)
 };
 
 template <typename T> struct VecN;
@@ -155,6 +156,7 @@ __global__ void __launch_bounds__(128) absorb_kernel(const AbsorbArgs a) {
   const int M = a.batch * a.n_q;
   const int rows = (a.d_nope + kDG - 1) / kDG;
   const bool col_ok = c0 < a.d_c;
+  tl_begin(a.timeline, MLA_TRACE_ABSORB);
 
   if (blockIdx.x == 0 && blockIdx.y == 0) build_plan(a);
   // every split's log-sum-exp slot starts empty
@@ -231,6 +233,7 @@ __global__ void __launch_bounds__(128) absorb_kernel(const AbsorbArgs a) {
       dst[half + k] = from_f<TO>(x2 * cs + x1 * sn);
     }
   }
+  tl_end(a.timeline, MLA_TRACE_ABSORB);
 }
 
 // RoPE of q^R at the query's own position for head h, tokens [m0, m0 + mc).
@@ -404,6 +407,7 @@ __global__ void __launch_bounds__(THREADS) absorb_tc_kernel(const __grid_constan
   }
   pdl_wait();
   MLA_STAMP(1);
+  tl_begin(a.timeline, MLA_TRACE_ABSORB);
   if (h == 0 && blockIdx.y == 0) build_plan(a);
   {
     const size_t nblk = (size_t)gridDim.x * gridDim.y, bid = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
@@ -480,6 +484,7 @@ __global__ void __launch_bounds__(THREADS) absorb_tc_kernel(const __grid_constan
     }
   }
   MLA_STAMP(3);
+  tl_end(a.timeline, MLA_TRACE_ABSORB);
 }
 
 }  // namespace
@@ -514,6 +519,7 @@ cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const 
   a.lse_part = lse_part;
   a.lse_count = lse_count;
   a.status = status;
+  a.timeline = timeline_ptr();
   // the tensor-core kernel stages q^C with 16-byte copies and stores q~ rows
   // (d_c + d_rope elements apart) with 16-byte stores
   if (d.act_dtype == MLA_BF16 && absorb_tc_fits(d) && (reinterpret_cast<uintptr_t>(q_nope) & 15u) == 0 &&

@@ -57,6 +57,7 @@ struct AppendArgs {
   float rope_base;
   float* raw;  // fp32 [n_tokens][d_c] scratch (FP8 caches only)
   int* status;
+  unsigned long long* timeline;  // device timeline (null: off)
 };
 
 // Physical (page, row) of token n, or page -1 (recorded) if out of range.
@@ -97,6 +98,7 @@ __device__ __forceinline__ float dot_vec(const uint4& w, const uint4& x, float*)
 template <typename T, int CACHE>
 __global__ void __launch_bounds__(256, 2) append_project_kernel(const AppendArgs a) {
   constexpr int VEC = Vec<T>::n;
+  tl_begin(a.timeline, MLA_TRACE_APPEND_PROJECT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rs = warp % kRows, kq = warp / kRows;
   const int half = a.d_rope >> 1;
@@ -197,6 +199,7 @@ __global__ void __launch_bounds__(256, 2) append_project_kernel(const AppendArgs
     }
     __syncthreads();
   }
+  tl_end_nosync(a.timeline, MLA_TRACE_APPEND_PROJECT);
 }
 
 // Small passes (at most kGvMaxTok tokens, bf16 activations): the projection
@@ -243,6 +246,7 @@ __global__ void __launch_bounds__(kGvThreads) append_gemv_kernel(const AppendArg
   pdl_trigger();
   pdl_wait();
   MLA_STAMP(1);
+  tl_begin(a.timeline, MLA_TRACE_APPEND_PROJECT);
   const int M = a.n_tokens;
   if (tid < M) {
     int prow = 0, position = 0;
@@ -335,6 +339,7 @@ __global__ void __launch_bounds__(kGvThreads) append_gemv_kernel(const AppendArg
     __syncthreads();  // red and fin are rewritten by the next pass
   }
   MLA_STAMP(3);
+  tl_end_nosync(a.timeline, MLA_TRACE_APPEND_PROJECT);
 }
 
 // Block-wide max over 128 threads.
@@ -353,6 +358,7 @@ __device__ __forceinline__ float block128_max(float v, float* sh) {
 __global__ void __launch_bounds__(128) append_fp8_finalize_kernel(const AppendArgs a) {
   pdl_trigger();
   pdl_wait();
+  tl_begin(a.timeline, MLA_TRACE_APPEND_FINALIZE);
   __shared__ float sh[4];
   const int n = blockIdx.x, tid = threadIdx.x;
   int prow, position;
@@ -370,6 +376,7 @@ __global__ void __launch_bounds__(128) append_fp8_finalize_kernel(const AppendAr
     codes[t0 + tid] = (uint8_t)__nv_cvt_float_to_fp8(v / scale, __NV_SATFINITE, __NV_E4M3);
     if (tid == 0) sc[t0 / 128] = scale;
   }
+  tl_end(a.timeline, MLA_TRACE_APPEND_FINALIZE);
 }
 
 constexpr int kTcCluster = 8;   // CTAs per output tile (d_model split)
@@ -436,6 +443,7 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
   }
   pdl_wait();
   MLA_STAMP(1);
+  tl_begin(a.timeline, MLA_TRACE_APPEND_PROJECT);
   const Fp8Page fp = fp8_page(a.page_size, a.d_c, a.d_rope);
   const int M = a.n_tokens, nk = ks / 16;
   uint32_t pass = 0;
@@ -530,6 +538,7 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
     cl.sync();  // peers are done reading this CTA's partials before the next pass
   }
   MLA_STAMP(3);
+  tl_end_nosync(a.timeline, MLA_TRACE_APPEND_PROJECT);
 }
 
 }  // namespace
@@ -575,6 +584,7 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
   a.rope_base = d.rope_base;
   a.raw = raw;
   a.status = status;
+  a.timeline = timeline_ptr();
   const int grid = (d.d_c + kRows - 1) / kRows + d.d_rope / 2;
   trace_record(MLA_TRACE_APPEND_PROJECT, false, st);
 #define MLA_PROJ(T, K) append_project_kernel<T, K><<<grid, 256, 0, st>>>(a)

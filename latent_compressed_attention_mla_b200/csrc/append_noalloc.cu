@@ -1,9 +1,10 @@
 // mla_append_latent_noalloc: the latent append for callers that cannot
 // allocate device memory when they call us (a plugin or callback whose host
 // framework owns all device memory and hands out no scratch buffer, or a loop
-// where an allocation would synchronise the device).  Its scratch -- the fp32
-// projections [n_tokens][d_c + d_rope] that the two append kernels pass
-// between them -- is a fixed array in this file instead of a caller workspace.
+// where an allocation would synchronise the device).  Its scratch -- for an
+// FP8 cache, the fp32 latent projections [n_tokens][d_c] that the projection
+// kernel hands to the quantiser; bf16 and fp32 caches need none -- is a fixed
+// array in this file instead of a caller workspace.
 //
 // The array lives in every GPU that loads the library, for as long as the
 // process runs.  Calls share it: two calls whose kernels overlap on the GPU
@@ -15,13 +16,15 @@
 namespace mla {
 int* device_status_word();
 size_t cache_page_bytes(const mla_dims& d);
+size_t append_scratch_floats(const mla_dims& d, int n_tokens);
 }  // namespace mla
 
 using namespace mla;
 
 namespace {
 
-// 65,536 floats (256 KiB): for DeepSeek-V3 dims (576 per token) up to 113 tokens.
+// 65,536 floats (256 KiB): an FP8-cache append at DeepSeek-V3 dims (d_c = 512
+// floats per token) of up to 128 tokens.
 constexpr size_t kNoAllocScratchFloats = 65536;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
@@ -55,8 +58,8 @@ extern "C" int mla_append_latent_noalloc(const mla_dims* dims, const void* h, in
   if (n_tokens < 0 || batch < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
   if (n_tokens == 0) return MLA_OK;
   if (!h || !seq_idx || !pos || !W_dkv || !W_kr || !page_table || !cache_pool) return MLA_ERR_INVALID_ARG;
-  // the request must fit the fixed array
-  if ((size_t)n_tokens * (size_t)(dims->d_c + dims->d_rope) > kNoAllocScratchFloats) return MLA_ERR_WORKSPACE;
+  // the scratch this request uses must fit the fixed array
+  if (append_scratch_floats(*dims, n_tokens) > kNoAllocScratchFloats) return MLA_ERR_WORKSPACE;
   if (!aligned16(h) || !aligned16(W_dkv) || !aligned16(W_kr) || !aligned16(cache_pool)) return MLA_ERR_ALIGNMENT;
   float* scratch = scratch_on_current_device();
   if (!scratch) return MLA_ERR_CUDA;

@@ -58,7 +58,8 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) combine_kernel(
     const T* __restrict__ W_uv, int n_heads, int d_c, int d_v, int batch, int n_q,
     const int32_t* __restrict__ plan, const float* __restrict__ o_part, const float* __restrict__ lse_part,
-    T* __restrict__ out, float* __restrict__ lse_out) {
+    T* __restrict__ out, float* __restrict__ lse_out, unsigned long long* timeline) {
+  tl_begin(timeline, MLA_TRACE_COMBINE);
   constexpr int VEC = CVec<T>::n;
   extern __shared__ float smem[];
   float* u_s = smem;                        // [kTok][d_c]
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(
       }
     }
   }
+  tl_end(timeline, MLA_TRACE_COMBINE);
 }
 
 constexpr int kTcDc = 512, kTcDv = 128;   // DeepSeek-V3 shape of W^UV_h
@@ -146,6 +148,7 @@ struct CombineTcArgs {
   int* status;
   int n_heads, batch, n_q;
   int stall;          // self-test: the weight fetch is not issued (its wait expires)
+  unsigned long long* timeline;  // device timeline (null: off)
   CUtensorMap map_w;  // W_uv as [n_heads * d_v rows][d_c] bf16, box 64 x 128, 128-byte swizzle
 };
 
@@ -227,6 +230,7 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
   }
   pdl_wait();
   MLA_STAMP(1);
+  tl_begin(P.timeline, MLA_TRACE_COMBINE);
   const int splits = plan[batch + 2];
   const int n_slots = batch + splits - 1;  // slot stride of the decode that wrote the partials
   // first slot row (t * n_slots + first split + b) and split count per token;
@@ -464,6 +468,7 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
     }
   }
   MLA_STAMP(3);
+  tl_end(P.timeline, MLA_TRACE_COMBINE);
 }
 
 }  // namespace
@@ -481,7 +486,8 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
     e = cudaFuncSetAttribute(combine_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     combine_kernel<float><<<d.n_heads, kThreads, smem, st>>>((const float*)W_uv, d.n_heads, d.d_c, d.d_v, batch, n_q,
-                                                              plan, o_part, lse_part, (float*)out, lse_out);
+                                                              plan, o_part, lse_part, (float*)out, lse_out,
+                                                              timeline_ptr());
   } else if (d.d_c == kTcDc && d.d_v == kTcDv && (reinterpret_cast<uintptr_t>(out) & 3u) == 0) {
     // paired bf16 stores; tile shapes are compile-time (DeepSeek-V3 dims)
     CombineTcArgs p;
@@ -495,6 +501,7 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
     p.batch = batch;
     p.n_q = n_q;
     p.stall = (d.flags & MLA_FLAG_SELFTEST_STALL) ? 1 : 0;
+    p.timeline = timeline_ptr();
     if (!make_tile_map_bf16(&p.map_w, W_uv, kTcDc, (uint64_t)d.n_heads * kTcDv, (uint64_t)kTcDc * 2, 64, kTcDv))
       return cudaErrorInvalidValue;
     // tokens per CTA: the largest block that still gives every SM a CTA
@@ -519,7 +526,7 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
     if (e != cudaSuccess) return e;
     combine_kernel<__nv_bfloat16><<<d.n_heads, kThreads, smem, st>>>(
         (const __nv_bfloat16*)W_uv, d.n_heads, d.d_c, d.d_v, batch, n_q, plan, o_part, lse_part,
-        (__nv_bfloat16*)out, lse_out);
+        (__nv_bfloat16*)out, lse_out, timeline_ptr());
   }
   return cudaGetLastError();
 }

@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
   const int32_t* tile_start = p.plan;
   const long long TT = tile_start[p.batch];
   const long long g0 = split_tile_begin(w, TT, p.splits), g1 = split_tile_begin(w + 1, TT, p.splits);
+  tl_begin(p.timeline, MLA_TRACE_ATTEND);
   if (g0 >= g1) return;
   const int P = p.d.page_size;
   int b = seq_of_tile(tile_start, p.batch, g0);
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
     if (kl == 0) p.lse_part[slot * p.d.n_heads + h] = l > 0.f ? m + log2f(l) : -INFINITY;
     g = seg_end;
   }
+  tl_end(p.timeline, MLA_TRACE_ATTEND);
 }
 
 template <int CACHE, typename QT>

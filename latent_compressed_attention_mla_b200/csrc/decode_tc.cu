@@ -110,7 +110,8 @@ struct TcLayout {
   static constexpr int PST_EMPTY = PST_FULL + PStSlots; // [PStSlots]
   static constexpr int SCL_FULL = PST_EMPTY + PStSlots;  // [SclBufs] local: a tile's scales landed
   static constexpr int SCL_EMPTY = SCL_FULL + SclBufs;   // [SclBufs] local: all converter warps done
-  static constexpr int NumBars = SCL_EMPTY + SclBufs;
+  static constexpr int DRAIN = SCL_EMPTY + SclBufs;      // each CTA: both MMA issuers' operations completed
+  static constexpr int NumBars = DRAIN + 1;
   static constexpr uint32_t OffMisc = OffBar + NumBars * 8;
   static constexpr uint32_t OffRedMax = OffMisc + 16;   // float [2][64]
   static constexpr uint32_t OffRedL = OffRedMax + 512;  // float [2][64]
@@ -135,6 +136,12 @@ constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s
+// after an abort: the bound on the wait for the issued MMAs, and the time
+// given to bulk copies whose completion this CTA cannot observe (its half of a
+// pair load completes on the leader's barrier); both far above the latency of
+// the operation
+constexpr long long kDrainLimitCycles = 20000000LL;   // ~10 ms
+constexpr unsigned long long kCopyGraceNs = 200000ull;  // 200 us
 
 // instruction descriptors (kind::f16, dense, f32 accumulator; operands bf16
 // or f16, the same for A and B)
@@ -211,8 +218,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Give up the CTA pair's work: set this CTA's abort flag and the peer's (a
+// distributed shared memory store), so that every role of both CTAs stops at
+// its next wait instead of running into its own limit.
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag) {
+  *abort_flag = 1;
+  const uint32_t peer = map_to_rank(smem_u32((const void*)abort_flag), cluster_rank() ^ 1u);
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer), "r"(1u) : "memory");
+}
+
 // Bounded wait.  Returns false (and records MLA_ERR_TIMEOUT) if the phase does
-// not complete within the limit or another role of this CTA already gave up.
+// not complete within the limit, or false at once if a role of this CTA or of
+// the peer CTA already gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -220,11 +237,36 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > kWaitLimitCycles) {
-      *abort_flag = 1;
+      raise_abort(abort_flag);
       record_status(status, MLA_ERR_TIMEOUT);
       return false;
     }
   }
+}
+
+// Bounded wait that ignores the abort flag (the teardown after an abort).
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, long long limit_cycles) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > limit_cycles) return false;
+  return true;
+}
+
+// The 128 softmax threads agree on a wait's outcome: true only if it succeeded
+// for all of them (a barrier with an AND reduction on named barrier 1), so
+// that they leave their loop together and never wait at a named barrier for a
+// warp that has gone.
+__device__ __forceinline__ bool softmax_all_ok(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)__all_sync(0xffffffffu, ok))
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -549,6 +591,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       mbar_init(bar(L::SCL_FULL + i), 1);
       mbar_init(bar(L::SCL_EMPTY + i), 2 * L::ConvWarps);
     }
+    mbar_init(bar(L::DRAIN), 2);  // the QK and the PV issuer's final commit
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == L::QKWarp) {
@@ -570,6 +613,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
   pdl_wait();
   if (threadIdx.x == 0) TC_TRACE(14, 0);
   MLA_STAMP(1);
+  tl_begin(p.timeline, MLA_TRACE_ATTEND);
 
   auto page_of = [&](int b, int pg) -> int {
     int page = p.page_table[(size_t)b * p.max_pages + pg];
@@ -580,9 +624,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
     return page;
   };
 
+  // Self-test of failure detection: no producer issues a load, so the MMA
+  // issuers' and softmax warps' bounded waits expire with no copy in flight.
+  const bool stall = (p.d.flags & MLA_FLAG_SELFTEST_STALL) != 0;
   if (warp >= L::QKProdWarp && warp < L::QKProdWarp + L::Producers) {
     // -------------------------------------------------------------- TMA: Q, QK
-    if (lane == 0) {
+    if (lane == 0 && !stall) {
       const int pid = warp - L::QKProdWarp;
       RingProducer ring{kFp8 ? L::QStSlots : L::QKSlots, L::Producers, pid};
       const uint32_t empty0 = kFp8 ? bar(L::QST_EMPTY) : bar(L::QK_EMPTY);
@@ -681,7 +728,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
     }
   } else if (warp >= L::PVProdWarp && warp < L::PVProdWarp + L::Producers) {
     // ------------------------------------------------------------------ TMA: PV
-    if (lane == 0) {
+    if (lane == 0 && !stall) {
       RingProducer ring{kFp8 ? L::PStSlots : L::PVSlots, L::Producers, warp - L::PVProdWarp};
       const uint32_t empty0 = kFp8 ? bar(L::PST_EMPTY) : bar(L::PV_EMPTY);
       const int x_pv = 128 * (int)rank;  // this CTA's 128 columns of an N=256 half
@@ -757,6 +804,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
       for (int it = 0; it < n_tiles && ok; ++it, ++gt) {
         ok = mbar_wait(bar(L::SCL_FULL + (gt & 1)), (gt >> 1) & 1, abort_flag, p.status);
+        ok = __all_sync(0xffffffffu, ok);  // the warp leaves together
         if (!ok) break;
         // the tile's scales, [4 pages][64 rows][4 tiles of 128 columns]
         const float* scl = reinterpret_cast<const float*>(smem + L::OffScl + (gt & 1) * kSclBytes);
@@ -768,6 +816,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           long long tw = clock64();
 #endif
           ok = mbar_wait(bar(L::QK_EMPTY + unit.slot), unit.phase ^ 1, abort_flag, p.status);
+          ok = __all_sync(0xffffffffu, ok);  // the warp leaves together
 #ifdef MLA_TC_TRACE
           w_unit += clock64() - tw;
           tw = clock64();
@@ -777,6 +826,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           if (c < kChunks - 1) {
             // [2 pages][64 rows][64 codes]; the scale of columns [64c, 64c+64) is tile c/2
             ok = mbar_wait(bar(L::QST_FULL + stage.slot), stage.phase, abort_flag, p.status);
+            ok = __all_sync(0xffffffffu, ok);  // the warp leaves together
 #ifdef MLA_TC_TRACE
             w_stage += clock64() - tw;
 #endif
@@ -813,6 +863,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
             // k^R: one staged page (64 rows x 64 bf16) per half of the unit
             for (int i = 0; i < 2 && ok; ++i) {
               ok = mbar_wait(bar(L::QST_FULL + stage.slot), stage.phase, abort_flag, p.status);
+              ok = __all_sync(0xffffffffu, ok);  // the warp leaves together
               if (!ok) break;
               const uint8_t* src = smem + L::OffQSt + stage.slot * kStageBytes;
               uint8_t* dst = dstu + i * 8192;
@@ -868,6 +919,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
       for (int it = 0; it < n_tiles && ok; ++it, ++gt) {
         ok = mbar_wait(bar(L::SCL_FULL + (gt & 1)), (gt >> 1) & 1, abort_flag, p.status);
+        ok = __all_sync(0xffffffffu, ok);  // the warp leaves together
         if (!ok) break;
         const float* scl_t = reinterpret_cast<const float*>(smem + L::OffScl + (gt & 1) * kSclBytes);
         const int pg0 = s.page_lo + it * kTilePages;
@@ -884,12 +936,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
             long long tw = clock64();
 #endif
             ok = mbar_wait(bar(L::PV_EMPTY + unit.slot), unit.phase ^ 1, abort_flag, p.status);
+            ok = __all_sync(0xffffffffu, ok);  // the warp leaves together
             if (!ok) break;
 #ifdef MLA_TC_TRACE
             w_unit += clock64() - tw;
             tw = clock64();
 #endif
             ok = mbar_wait(bar(L::PST_FULL + stage.slot), stage.phase, abort_flag, p.status);
+            ok = __all_sync(0xffffffffu, ok);  // the warp leaves together
             if (!ok) break;
 #ifdef MLA_TC_TRACE
             w_stage += clock64() - tw;
@@ -1025,6 +1079,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         }
         ++seg;
       }
+      // completes, in both CTAs, once every MMA this thread issued has finished
+      tc_commit_pair(bar(L::DRAIN));
     }
   } else if (warp == L::PVWarp) {
     // ---------------------------------------------------------- MMA: O += P C
@@ -1084,6 +1140,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         }
         ++seg;
       }
+      tc_commit_pair(bar(L::DRAIN));
     }
   } else if (warp < 4) {
     // ------------------------------------------------------- softmax, epilogue
@@ -1116,8 +1173,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       float m_ref = -INFINITY, l_part = 0.f;
       const int n_tiles = (s.n_pages + kTilePages - 1) / kTilePages;
       for (int it = 0; it < n_tiles; ++it, ++g) {
-        ok = mbar_wait(bar(L::S_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.status);
-        __syncwarp();
+        ok = softmax_all_ok(mbar_wait(bar(L::S_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.status));
         if (!ok) break;
         if (threadIdx.x == 0) TC_TRACE(4, g);
         tc_fence_after();
@@ -1202,8 +1258,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
         // whose head keeps its reference)
         auto wait_pv_rescale = [&]() -> bool {
           if (g >= 1) {
-            if (!mbar_wait(bar(L::O_DONE), (g - 1) & 1, abort_flag, p.status)) return false;
-            __syncwarp();
+            // warp-uniform outcome: the TMEM accesses below are whole-warp
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::O_DONE), (g - 1) & 1, abort_flag, p.status)))
+              return false;
             tc_fence_after();
           }
           if (__any_sync(0xffffffffu, rescale)) {
@@ -1238,16 +1295,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
             }
           }
           release_s();
-          ok = wait_pv_rescale();
-          __syncwarp();
+          ok = softmax_all_ok(wait_pv_rescale());
           if (!ok) break;
           store_p(0, pk_lo);
           store_p(1, pk_hi);
         } else {
           // 512 threads leave 128 registers each: no room to hold both
           // sub-tiles' probabilities, so the wait comes first
-          ok = wait_pv_rescale();
-          __syncwarp();
+          ok = softmax_all_ok(wait_pv_rescale());
           if (!ok) break;
 #pragma unroll 1
           for (int q = 0; q < 2; ++q) {
@@ -1267,8 +1322,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
       }
       if (!ok) break;
       // epilogue: wait for the last PV, normalise, write the split's partial
-      ok = mbar_wait(bar(L::O_DONE), (g - 1) & 1, abort_flag, p.status);
-      __syncwarp();
+      ok = softmax_all_ok(mbar_wait(bar(L::O_DONE), (g - 1) & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
       red_l[half * 64 + hl] = l_part;
@@ -1334,9 +1388,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
   __syncthreads();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   tc_fence_after();
+  // After an abort by either CTA (whichever gave up set both flags before its
+  // cluster arrival, so both CTAs read the same value here): wait, bounded,
+  // for the MMAs issued so far, give bulk copies in flight time to land, and
+  // meet the peer again, so that neither CTA's shared memory or tensor memory
+  // goes while an operation of the pair may still use it.
+  if (*abort_flag) {
+    if (threadIdx.x == 0) {
+      mbar_wait_for(bar(L::DRAIN), 0, kDrainLimitCycles);
+      const unsigned long long t0 = global_ns();
+      while (global_ns() - t0 < kCopyGraceNs) {
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    tc_fence_after();
+  }
   MLA_STAMP(3);
-  if (warp == L::QKWarp)
+  tl_end_nosync(p.timeline, MLA_TRACE_ATTEND);
+  if (warp == L::QKWarp) {
+    // every MMA of the pair has completed (the issuers' final commits; already
+    // so on the normal path, where the softmax warps waited for the last ones)
+    if (lane == 0) mbar_wait_for(bar(L::DRAIN), 0, kDrainLimitCycles);
+    __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -21,6 +21,8 @@ using namespace mla;
 namespace mla {
 static cudaEvent_t g_trace[2 * MLA_TRACE_COUNT];
 static bool g_trace_on = false;
+static unsigned long long* g_timeline = nullptr;
+unsigned long long* timeline_ptr() { return g_timeline; }
 // Called only where no launch error is pending; a failed record is dropped
 // (and cleared) so that it is never reported as a kernel launch failure.
 void trace_record(int kernel, bool end, cudaStream_t st) {
@@ -198,6 +200,7 @@ int mla_decode(const mla_dims* dims, const void* q_nope, const void* q_rope, con
   p.n_slots = n_slots;
   p.scale_log2 = dims->softmax_scale * kLog2e;
   p.status = status;
+  p.timeline = timeline_ptr();
   trace_record(MLA_TRACE_ATTEND, false, st);
   e = path == 1 ? launch_decode_tc(p, st) : launch_decode_simt(p, st);
   trace_record(MLA_TRACE_ATTEND, true, st);
@@ -234,6 +237,11 @@ int mla_set_trace_events(void* const* events, int n_events) {
   if (n_events < 2 * MLA_TRACE_COUNT) return MLA_ERR_INVALID_ARG;
   for (int i = 0; i < 2 * MLA_TRACE_COUNT; ++i) g_trace[i] = (cudaEvent_t)events[i];
   g_trace_on = true;
+  return MLA_OK;
+}
+
+int mla_set_timeline(unsigned long long* device_buffer) {
+  g_timeline = device_buffer;
   return MLA_OK;
 }
 

@@ -209,10 +209,39 @@ struct DecodeParams {
   int batch, n_q, splits, n_slots;
   float scale_log2;        // softmax_scale * log2(e)
   int* status;
+  unsigned long long* timeline;  // device timeline (null: off)
 };
 
 // Tracing hook: events installed by mla_set_trace_events (may be null).
 void trace_record(int kernel, bool end, cudaStream_t st);
+
+// Device timeline installed by mla_set_timeline (null when off): the
+// launchers copy it into each kernel's arguments.  Per kernel k (MLA_TRACE_*),
+// thread 0 of every CTA keeps in [2k] the earliest %globaltimer at which a CTA
+// passed its grid-dependency wait and in [2k + 1] the latest at which one
+// finished, so a graph replay of a step gives each kernel's span on the device.
+unsigned long long* timeline_ptr();
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void tl_begin(unsigned long long* tl, int k) {
+  if (tl && threadIdx.x == 0) atomicMin(tl + 2 * k, global_ns());
+}
+// at the end of a CTA: the CTA's other threads are done first (tl is uniform
+// over the grid, so the barrier is taken by all threads or none)
+__device__ __forceinline__ void tl_end(unsigned long long* tl, int k) {
+  if (tl) {
+    __syncthreads();
+    if (threadIdx.x == 0) atomicMax(tl + 2 * k + 1, global_ns());
+  }
+}
+// at the end of a CTA whose threads have already synchronised
+__device__ __forceinline__ void tl_end_nosync(unsigned long long* tl, int k) {
+  if (tl && threadIdx.x == 0) atomicMax(tl + 2 * k + 1, global_ns());
+}
 
 // ----------------------------------------------------------------------------
 // Launchers (host side), each returning cudaError_t of the launch.

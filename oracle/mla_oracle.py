@@ -72,6 +72,12 @@ def to_f32(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
 
 
+def to_f16(x) -> np.ndarray:
+    """IEEE binary16 rounding (11-bit significand, minimum normal exponent
+    -14), as float64; no overflow handling (values here stay far below 65504)."""
+    return round_to_format(x, 11, -14)
+
+
 # OCP FP8 E4M3 ("fn": no infinities, S.1111.111 is NaN): bias 7, 3 mantissa
 # bits, largest finite 448, smallest subnormal 2**-9.
 E4M3_MAX = 448.0
@@ -253,14 +259,22 @@ def decode_explicit(q_nope, q_rope, C, KR, W_uk, W_uv, seq_len: int, scale: floa
 
 
 def decode_absorbed(q_nope, q_rope, C, KR, W_uk, W_uv, seq_len: int, scale: float,
-                    base: float = 10000.0):
+                    base: float = 10000.0, q_round=None):
     """Same contract as decode_explicit (all heads); also returns the latent
-    aggregate u [T, n_h, d_c]."""
+    aggregate u [T, n_h, d_c].
+
+    q_round: None, or a rounding (e.g. to_bf16) applied to the absorbed query
+    q~ and the rotated q^R before they are scored.  The pages fix no precision
+    for the query; a tensor-core kernel must hold it in its operand format, and
+    this option gives the attention of exactly such a rounded query (everything
+    else in float64), to tell the format's own error from a kernel's."""
     C = np.asarray(C, np.float64)[:seq_len]
     KR = np.asarray(KR, np.float64)[:seq_len]
     T = np.asarray(q_nope).shape[0]
     pos = query_positions(seq_len, T)
     q_t, q_r = absorb_query(q_nope, q_rope, W_uk, pos, base)  # [T, n_h, d_c], [T, n_h, d_R]
+    if q_round is not None:
+        q_t, q_r = q_round(q_t), q_round(q_r)
     W_uv = np.asarray(W_uv, np.float64)
     n_h = q_t.shape[1]
     o = np.zeros((T, n_h, W_uv.shape[1]))

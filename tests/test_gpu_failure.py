@@ -6,7 +6,14 @@ reported through the device status word, and the context stays usable.
   sequences of the batch are unaffected.
 * A bounded wait that runs out (the self-test flag stops the combine from
   fetching its weights, so nothing completes the barrier it waits on) records
-  MLA_ERR_TIMEOUT after about two seconds; the next step runs normally."""
+  MLA_ERR_TIMEOUT after about two seconds; the next step runs normally.
+* The same for the tensor-core attention kernel: under the self-test flag its
+  load producers issue nothing, the waits of the MMA issuers and softmax warps
+  expire, the CTA pair unwinds together (the one that gives up tells its
+  peer) and frees its tensor memory; the status reads MLA_ERR_TIMEOUT and the
+  next step on the same context matches the oracle."""
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -53,6 +60,29 @@ def test_expired_wait_is_reported_and_context_survives():
     good = GpuProblem(cfg)
     out, _ = good.run()
     assert good.status() == 0
+    o = OracleProblem(cfg)
+    heads = list(range(0, 128, 9))
+    for b in range(cfg.B):
+        assert rel_err(out[b][:, heads].float().cpu().numpy(), o.expected(b, heads)[0]) <= tolerance(cfg)
+
+
+@pytest.mark.parametrize("cache", ["bf16", "fp8"])
+def test_decode_expired_wait_is_reported_and_context_survives(cache):
+    cfg = SMALL.with_(cache_dtype=cache, T=2, L=(300, 900))
+    if B.decode_path(B.dims_for(cfg), cfg.T) != 1:
+        pytest.skip("the tensor-core decode runs on sm_100 only")
+    g = GpuProblem(cfg)
+    i = g.inputs
+    g.session.append(i["h"], g.seq_idx, g.pos, g.weights["W_dkv"], g.weights["W_kr"], g.page_table, g.cache.pool)
+    assert g.status() == 0
+    stall = B.dims_for(cfg, B.MLA_FLAG_SELFTEST_STALL)
+    ws = torch.empty(B.decode_workspace_bytes(stall, cfg.B, cfg.T, 0), dtype=torch.uint8, device="cuda")
+    t0 = time.time()
+    B.mla_decode(stall, i["q_nope"], i["q_rope"], g.weights["W_uk"], g.cache.pool, g.page_table, g.seq_lens, ws)
+    assert B.mla_get_status() == B.MLA_ERR_TIMEOUT
+    assert time.time() - t0 < 30.0  # the pairs unwound after their limit, not at the test's timeout
+    out, _ = g.run()
+    assert g.status() == 0
     o = OracleProblem(cfg)
     heads = list(range(0, 128, 9))
     for b in range(cfg.B):

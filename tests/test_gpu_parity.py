@@ -79,23 +79,47 @@ def test_three_query_tokens_causal_f32():
 
 
 # The full-size workloads in the launch configuration the bench times (the
-# whole step, automatic split count), checked on sampled outputs that the
-# oracle computes one by one: the ragged batch's shortest and longest
-# sequences, one long-context sequence, one FP8 sequence with its two causal
-# query tokens.
-FULL_SAMPLES = [
-    (W.V3_RAGGED_B64, "minmax", [1, 64, 127]),
-    (W.V3_LONG_B8, [0], [0, 77]),
-    (W.V3_FP8_B128_T2, [5], [3, 100]),
-]
+# whole step, automatic split count), checked element by element on sampled
+# sequences: the shortest and the longest, and two more drawn with a fixed
+# seed; every head and every query token against the oracle's absorbed form
+# (itself pinned to the explicit form), and the explicit form of record on a
+# few heads of the same sequences.
+FULL_SIZE = [(W.V3_RAGGED_B64, [1, 64, 127]), (W.V3_LONG_B8, [0, 77]), (W.V3_FP8_B128_T2, [3, 100])]
 
 
-@pytest.mark.parametrize("cfg,seqs,heads", FULL_SAMPLES, ids=["ragged-b64", "long-b8", "fp8-b128-t2"])
-def test_full_size_sampled(cfg, seqs, heads):
-    if seqs == "minmax":
-        L = np.asarray(cfg.L)
-        seqs = [int(np.argmin(L)), int(np.argmax(L))]
-    check_step(cfg, heads=heads, seqs=seqs)
+def sampled_sequences(cfg, n_random=2, seed=2026):
+    L = np.asarray(cfg.L)
+    picked = [int(np.argmin(L)), int(np.argmax(L))]
+    if picked[0] == picked[1]:  # all lengths equal: the first and the last sequence
+        picked = [0, cfg.B - 1]
+    rest = [b for b in range(cfg.B) if b not in picked]
+    picked += sorted(np.random.default_rng(seed).choice(rest, n_random, replace=False).tolist())
+    return picked
+
+
+@pytest.mark.parametrize("cfg,heads_x", FULL_SIZE, ids=["ragged-b64", "long-b8", "fp8-b128-t2"])
+def test_full_size_sampled(cfg, heads_x):
+    g = GpuProblem(cfg)
+    out, lse = g.run()
+    assert g.status() == 0
+    o = OracleProblem(cfg)
+    seqs = sampled_sequences(cfg)
+    got_o, ref_o, got_l, ref_l, got_x, ref_x = [], [], [], [], [], []
+    for b in seqs:
+        cache = o.cache_values(b)
+        ro, rl = o.expected_absorbed(b, cache=cache)
+        got_o.append(out[b].float().cpu().numpy())
+        ref_o.append(ro)
+        got_l.append(lse[b].cpu().numpy())
+        ref_l.append(rl)
+        got_x.append(out[b][:, heads_x].float().cpu().numpy())
+        ref_x.append(o.expected(b, heads_x, cache=cache)[0])
+    e_o = rel_err(np.stack(got_o), np.stack(ref_o))
+    e_l = rel_err(np.stack(got_l), np.stack(ref_l))
+    e_x = rel_err(np.stack(got_x), np.stack(ref_x))
+    assert e_o <= 1e-2, f"sequences {seqs}, all heads: output rel err {e_o:.3e}"
+    assert e_l <= 1e-2, f"sequences {seqs}, all heads: lse rel err {e_l:.3e}"
+    assert e_x <= 1e-2, f"sequences {seqs}, heads {heads_x}: explicit-form rel err {e_x:.3e}"
 
 
 def test_split_count_invariance_f32():

@@ -39,6 +39,34 @@ def closed_form_rotate(x, p, base=10000.0):
     return out
 
 
+@pytest.mark.parametrize("fmt", ["bf16", "f16"])
+def test_query_rounding_option_matches_sdpa_on_a_rounded_query(fmt):
+    """decode_absorbed(q_round=...) is the attention of the query rounded to
+    that format: in the textbook reduction (n_h = 1, W_uk = W_uv = I) it equals
+    torch's attention on a query cast to the format by torch itself."""
+    rng = np.random.default_rng(31)
+    d_c, d_r, S, T = 16, 8, 40, 2
+    P = rand_problem(rng, n_h=1, d_c=d_c, d_r=d_r, d_nope=d_c, d_v=d_c, S=S, T=T)
+    P["q_nope"] = P["q_nope"] * 7.0  # wide logits, so that the rounding shows
+    P["W_uk"] = np.eye(d_c)[None]
+    P["W_uv"] = np.eye(d_c)[None]
+    rnd = O.to_bf16 if fmt == "bf16" else O.to_f16
+    tdt = torch.bfloat16 if fmt == "bf16" else torch.float16
+    o, _, _ = O.decode_absorbed(**P, q_round=rnd)
+    o_exact, _, _ = O.decode_absorbed(**P)
+    pos = S - T + np.arange(T)
+    Q = np.stack([np.concatenate([P["q_nope"][t, 0], closed_form_rotate(P["q_rope"][t, 0], pos[t])])
+                  for t in range(T)])
+    Q = torch.from_numpy(Q.astype(np.float32)).to(tdt).to(torch.float64)
+    K = np.concatenate([P["C"], P["KR"]], axis=1)
+    mask = np.arange(S)[None, :] <= pos[:, None]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q[None], torch.from_numpy(K)[None], torch.from_numpy(P["C"])[None],
+        attn_mask=torch.from_numpy(mask)[None])[0].numpy()
+    np.testing.assert_allclose(o[:, 0], ref, rtol=1e-12, atol=1e-13)
+    assert np.abs(o - o_exact).max() > 0  # the option does round
+
+
 @pytest.mark.parametrize("T", [1, 2])
 def test_textbook_reduction_matches_torch_sdpa(T):
     """n_h = 1, d_nope = d_c, W_uk = W_uv = I: MLA is single-head attention with

@@ -16,6 +16,15 @@ def test_bf16_matches_torch_cast():
     np.testing.assert_array_equal(O.to_bf16(x32.astype(np.float64)), ref)
 
 
+def test_f16_matches_torch_cast():
+    rng = np.random.default_rng(2)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-9, 4, 20000),
+                        [0.0, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 2.0 ** -24, 2.0 ** -14, 3e-8]])
+    x = x[np.abs(x) < 65504.0]
+    ref = torch.from_numpy(x).to(torch.float16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.to_f16(x), ref)
+
+
 def test_generic_rounding_at_fp32_matches_ieee_cast():
     # the same rounding routine at fp32's parameters (24-bit significand,
     # emin -126, gradual underflow) against the IEEE float32 conversion,

@@ -46,16 +46,42 @@ def test_noalloc_append_matches_workspace_append(cfg):
 
 
 def test_noalloc_rejects_requests_beyond_its_array():
-    cfg = W.V3_B1_L4096.with_(name="noalloc-big", B=1, L=(0,))
+    """An FP8-cache append needs n_tokens * d_c floats of scratch: one token
+    more than the 65,536-float array holds is refused before any launch."""
+    cfg = W.V3_B1_L4096.with_(name="noalloc-big", B=1, L=(0,), cache_dtype="fp8")
     dims = B.dims_for(cfg)
-    n = 65536 // (cfg.d_c + cfg.d_rope) + 1  # one token more than fits
+    n = 65536 // cfg.d_c + 1  # one token more than fits
     dev = "cuda"
     w = W.weights(cfg, dev)
     h = torch.zeros(n, cfg.d_model, dtype=torch.bfloat16, device=dev)
     seq = torch.zeros(n, dtype=torch.int32, device=dev)
-    pos = torch.zeros(n, dtype=torch.int32, device=dev)
-    pt = torch.zeros(1, 4, dtype=torch.int32, device=dev)
+    pos = torch.arange(n, dtype=torch.int32, device=dev)
+    pt = torch.arange(4, dtype=torch.int32, device=dev).view(1, 4)
     pool = torch.zeros(4 * B.cache_page_bytes(dims), dtype=torch.uint8, device=dev)
     with pytest.raises(B.MlaError) as e:
         B.mla_append_latent_noalloc(dims, h, seq, pos, w["W_dkv"], w["W_kr"], pt, pool)
     assert e.value.code == 3
+    assert int(pool.ne(0).sum()) == 0  # nothing was launched
+
+
+def test_noalloc_bf16_needs_no_scratch():
+    """A bf16-cache append uses no scratch, so a pass larger than the array
+    could hold for an FP8 cache is accepted and matches the workspace append."""
+    cfg = W.V3_B1_L4096.with_(name="noalloc-bf16-big", B=1, L=(0,))
+    dims = B.dims_for(cfg)
+    n = 65536 // cfg.d_c + 1
+    dev = "cuda"
+    w = W.weights(cfg, dev)
+    h = W.normal(cfg.seed + 7, W.S_H, n * cfg.d_model, dev).view(n, cfg.d_model).to(torch.bfloat16)
+    seq = torch.zeros(n, dtype=torch.int32, device=dev)
+    pos = torch.arange(n, dtype=torch.int32, device=dev)
+    pages = (n + 63) // 64
+    pt = torch.arange(pages, dtype=torch.int32, device=dev).view(1, pages)
+    ref = torch.zeros(pages * B.cache_page_bytes(dims), dtype=torch.uint8, device=dev)
+    got = torch.zeros_like(ref)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    B.mla_append_latent(dims, h, seq, pos, w["W_dkv"], w["W_kr"], pt, ref, ws)
+    B.mla_append_latent_noalloc(dims, h, seq, pos, w["W_dkv"], w["W_kr"], pt, got)
+    assert B.mla_get_status() == 0
+    assert torch.equal(ref, got)
+    assert int(got.ne(0).sum()) > 0
