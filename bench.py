@@ -531,10 +531,15 @@ def main():
     ap.add_argument("--batch", type=int, default=0,
                     help="keep only the first N sequences of the workload (smaller case of the same kernels, "
                          "e.g. for profiler captures); the workload name records it")
+    ap.add_argument("--context", type=int, default=0,
+                    help="cache every sequence with this many tokens before the step instead (a smaller case of "
+                         "the same batch and kernels, e.g. for profiler captures); the workload name records it")
     args = ap.parse_args()
     cfg = WL.CONFIGS[args.config]
     if 0 < args.batch < cfg.B:
         cfg = cfg.with_(name=f"{cfg.name}[:{args.batch}]", B=args.batch, L=tuple(cfg.L[:args.batch]))
+    if args.context > 0:
+        cfg = cfg.with_(name=f"{cfg.name}[L={args.context}]", L=args.context)
     if args.impl == "reference":
         return run_reference(args, cfg)
 
@@ -580,7 +585,7 @@ def main():
     torch.cuda.empty_cache()
 
     extra = {}
-    if args.extra and world == 1 and args.batch == 0:
+    if args.extra and world == 1 and args.batch == 0 and args.context == 0:
         for ci in EXTRA_CONFIGS:
             if ci == args.config:
                 continue
