@@ -6,11 +6,12 @@
 // Cache by 93%", "3. Decoupled RoPE and Matrix Absorption"; decoding module
 // step 5).
 //
-// bf16 activations at DeepSeek-V3 dims (combine_tc_kernel): one CTA per
-// (head, block of 16, 32 or 64 tokens; the largest block that still gives
-// every SM a CTA).  Eight TMA boxes bring W^UV_h (d_v x d_c, 128 KB) into
-// swizzled shared memory, issued before the programmatic-launch wait, while
-// the CTA merges the splits of its tokens into a bf16 u tile: a warp per token
+// bf16 activations at DeepSeek-V3 dims (combine_tc_kernel): one CTA per head,
+// looping over blocks of 16, 32 or 64 tokens (by batch size).  Eight TMA boxes
+// bring W^UV_h (d_v x d_c, 128 KB) into swizzled shared memory once, issued
+// before the programmatic-launch wait (so every head's fetch overlaps the
+// decode's tail), while the CTA merges the splits of a block's tokens into a
+// bf16 u tile: a warp per token
 // forms the split weights (the loads of all its tokens in flight together),
 // then thread (column quad c, parity r) accumulates the weighted partials of
 // tokens r, r + 2, ..., eight tokens' loads in flight at a time.  mma.sync
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
   const int32_t* plan = P.plan;
   uint8_t* Ws = smem;              // [8][d_v][128 B]
   uint8_t* Us = smem + kTcWBytes;  // [8][TOK][128 B]
-  const int M = batch * n_q, m0 = blockIdx.y * TOK, mc = min(TOK, M - m0);
+  const int M = batch * n_q;
   const uint32_t bar = smem_addr(&wbar);
   if (tid == 0) mbar_init_local(bar, 1);
   __syncthreads();
@@ -233,239 +234,245 @@ __global__ void __launch_bounds__(kThreads) combine_tc_kernel(const __grid_const
   tl_begin(P.timeline, MLA_TRACE_COMBINE);
   const int splits = plan[batch + 2];
   const int n_slots = batch + splits - 1;  // slot stride of the decode that wrote the partials
-  // first slot row (t * n_slots + first split + b) and split count per token;
-  // tokens past the end take no split
-  if (tid < TOK) {
-    int row = 0, n = 0;
-    if (tid < mc) {
-      const int m = m0 + tid, b = m / n_q, t = m % n_q;
-      row = t * n_slots + plan[batch + 5 + 2 * b] + b;
-      n = min(plan[batch + 6 + 2 * b], kMaxSplits);
-    }
-    s_lo[tid] = row;
-    s_n[tid] = n;
-  }
-  __syncthreads();
-  // merge weights: warp w takes tokens w, w + 8, ...; lane k holds split k
-  {
-    float lv[kTPW];
-#pragma unroll
-    for (int j = 0; j < kTPW; ++j) {
-      const int mi = warp + 8 * j;
-      lv[j] = lane < s_n[mi] ? P.lse_part[(size_t)(s_lo[mi] + lane) * n_heads + h] : -INFINITY;
-    }
-#pragma unroll
-    for (int j = 0; j < kTPW; ++j) {
-      const int mi = warp + 8 * j, n = s_n[mi];
-      const float* lse = P.lse_part + (size_t)s_lo[mi] * n_heads + h;
-      float mx = lv[j];
-      for (int k = lane + 32; k < n; k += 32) mx = fmaxf(mx, lse[(size_t)k * n_heads]);
-#pragma unroll
-      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      // a split holding no key of the sequence has lse = -inf: weight 0
-      const float e = mx > -INFINITY ? exp2f(lv[j] - mx) : 0.f;
-      float sum = e;
-      for (int k = lane + 32; k < n; k += 32) sum += exp2f(lse[(size_t)k * n_heads] - mx);
-#pragma unroll
-      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      const float inv = sum > 0.f ? 1.f / sum : 0.f;
-      s_w[mi][lane] = e * inv;
-      if (lane == 0) {
-        s_mx[mi] = mx;
-        s_inv[mi] = inv;
-        if (P.lse_out && mi < mc) P.lse_out[(size_t)(m0 + mi) * n_heads + h] = sum > 0.f ? (mx + log2f(sum)) * kLn2 : -INFINITY;
+  // token blocks blockIdx.y, blockIdx.y + gridDim.y, ... of TOK tokens; W^UV_h
+  // stays in shared memory for all of them
+  for (int m0 = blockIdx.y * TOK; m0 < M; m0 += gridDim.y * TOK) {
+    const int mc = min(TOK, M - m0);
+    // first slot row (t * n_slots + first split + b) and split count per token;
+    // tokens past the end take no split
+    if (tid < TOK) {
+      int row = 0, n = 0;
+      if (tid < mc) {
+        const int m = m0 + tid, b = m / n_q, t = m % n_q;
+        row = t * n_slots + plan[batch + 5 + 2 * b] + b;
+        n = min(plan[batch + 6 + 2 * b], kMaxSplits);
       }
+      s_lo[tid] = row;
+      s_n[tid] = n;
     }
-  }
-  __syncthreads();
-  MLA_STAMP(4);
-  auto weight = [&](int mi, int k) -> float {
-    return k < kTcWCache ? s_w[mi][k]
-                         : exp2f(P.lse_part[(size_t)(s_lo[mi] + k) * n_heads + h] - s_mx[mi]) * s_inv[mi];
-  };
-  // thread (column unit cu, group gr): columns [c0, c0 + kCU)
-  const int cu = tid % kUnits, gr = tid / kUnits, c0 = cu * kCU;
-  auto part_row = [&](int mi, int k) { return (size_t)(s_lo[mi] + k) * n_heads + h; };
-  auto store_u = [&](int mi, const float* a) {
-    // kCU columns of token mi as bf16 into the swizzled u tile
+    __syncthreads();
+    // merge weights: warp w takes tokens w, w + 8, ...; lane k holds split k
+    {
+      float lv[kTPW];
 #pragma unroll
-    for (int e = 0; e < kCU; e += 4) {
-      const __nv_bfloat162 lo2 = __floats2bfloat162_rn(a[e], a[e + 1]);
-      const __nv_bfloat162 hi2 = __floats2bfloat162_rn(a[e + 2], a[e + 3]);
-      uint2 pk;
-      pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
-      pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
-      *reinterpret_cast<uint2*>(Us + swz_cb(mi, (c0 + e) >> 3, TOK) + ((c0 + e) & 7) * 2) = pk;
-    }
-  };
-  if constexpr (TOK == 16) {
-    // few tokens, many splits each: the kGroups groups take splits gr,
-    // gr + kGroups, ... of two tokens at a time, eight loads per token in
-    // flight (sixteen for a token without a partner); the groups' sums meet
-    // in the fp32 scratch R and are added in group order (deterministic)
-    float* R = reinterpret_cast<float*>(Us + TOK * kTcDc * 2);  // [kGroups][2][d_c]
-#pragma unroll 1
-    for (int mi0 = 0; mi0 < mc; mi0 += 2) {
-      const bool single = s_n[mi0 + 1] == 0;  // the same for the whole CTA
-      const int nmax = max(s_n[mi0], s_n[mi0 + 1]), kstep = (single ? 16 : 8) * kGroups;
-      float acc[2][kCU];
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int e = 0; e < kCU; ++e) acc[j][e] = 0.f;
-      for (int k0 = gr; k0 < nmax; k0 += kstep) {
-        uint4 raw[2][8];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int mi = single ? mi0 : mi0 + j, n = s_n[mi];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int k = k0 + kGroups * (single ? 8 * j + u : u);
-            raw[j][u] = make_uint4(0, 0, 0, 0);
-            if (k < n) raw[j][u] = PU::load(P.o_part, part_row(mi, k), c0);
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int mi = single ? mi0 : mi0 + j, n = s_n[mi];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int k = k0 + kGroups * (single ? 8 * j + u : u);
-            const float wk = k < n ? weight(mi, k) : 0.f;
-            // a zero weight marks a split with no key of the sequence, whose
-            // partial was never written: its values are not read into u
-            if (wk != 0.f) {
-              float v[kCU];
-              PU::to_float(raw[j][u], v);
-#pragma unroll
-              for (int e = 0; e < kCU; ++e) acc[j][e] = fmaf(wk, v[e], acc[j][e]);
-            }
-          }
-        }
-      }
-      if (single) {
-#pragma unroll
-        for (int e = 0; e < kCU; ++e) {
-          acc[0][e] += acc[1][e];
-          acc[1][e] = 0.f;
-        }
+      for (int j = 0; j < kTPW; ++j) {
+        const int mi = warp + 8 * j;
+        lv[j] = lane < s_n[mi] ? P.lse_part[(size_t)(s_lo[mi] + lane) * n_heads + h] : -INFINITY;
       }
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
+      for (int j = 0; j < kTPW; ++j) {
+        const int mi = warp + 8 * j, n = s_n[mi];
+        const float* lse = P.lse_part + (size_t)s_lo[mi] * n_heads + h;
+        float mx = lv[j];
+        for (int k = lane + 32; k < n; k += 32) mx = fmaxf(mx, lse[(size_t)k * n_heads]);
 #pragma unroll
-        for (int e = 0; e < kCU; ++e) R[(gr * 2 + j) * kTcDc + c0 + e] = acc[j][e];
-      __syncthreads();
-      // thread t: token mi0 + t / 128, columns 4 (t % 128) .. + 3
-      {
-        const int j = tid >> 7, c = (tid & 127) * 4;
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        // a split holding no key of the sequence has lse = -inf: weight 0
+        const float e = mx > -INFINITY ? exp2f(lv[j] - mx) : 0.f;
+        float sum = e;
+        for (int k = lane + 32; k < n; k += 32) sum += exp2f(lse[(size_t)k * n_heads] - mx);
 #pragma unroll
-        for (int q = 0; q < kGroups; ++q) {
-          const float4 x = *reinterpret_cast<const float4*>(R + (q * 2 + j) * kTcDc + c);
-          sum.x += x.x;
-          sum.y += x.y;
-          sum.z += x.z;
-          sum.w += x.w;
+        for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float inv = sum > 0.f ? 1.f / sum : 0.f;
+        s_w[mi][lane] = e * inv;
+        if (lane == 0) {
+          s_mx[mi] = mx;
+          s_inv[mi] = inv;
+          if (P.lse_out && mi < mc) P.lse_out[(size_t)(m0 + mi) * n_heads + h] = sum > 0.f ? (mx + log2f(sum)) * kLn2 : -INFINITY;
         }
-        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(sum.x, sum.y);
-        const __nv_bfloat162 hi2 = __floats2bfloat162_rn(sum.z, sum.w);
+      }
+    }
+    __syncthreads();
+    MLA_STAMP(4);
+    auto weight = [&](int mi, int k) -> float {
+      return k < kTcWCache ? s_w[mi][k]
+                           : exp2f(P.lse_part[(size_t)(s_lo[mi] + k) * n_heads + h] - s_mx[mi]) * s_inv[mi];
+    };
+    // thread (column unit cu, group gr): columns [c0, c0 + kCU)
+    const int cu = tid % kUnits, gr = tid / kUnits, c0 = cu * kCU;
+    auto part_row = [&](int mi, int k) { return (size_t)(s_lo[mi] + k) * n_heads + h; };
+    auto store_u = [&](int mi, const float* a) {
+      // kCU columns of token mi as bf16 into the swizzled u tile
+#pragma unroll
+      for (int e = 0; e < kCU; e += 4) {
+        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(a[e], a[e + 1]);
+        const __nv_bfloat162 hi2 = __floats2bfloat162_rn(a[e + 2], a[e + 3]);
         uint2 pk;
         pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
         pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
-        *reinterpret_cast<uint2*>(Us + swz_cb(mi0 + j, c >> 3, TOK) + (c & 7) * 2) = pk;
+        *reinterpret_cast<uint2*>(Us + swz_cb(mi, (c0 + e) >> 3, TOK) + ((c0 + e) & 7) * 2) = pk;
       }
-      __syncthreads();  // R is rewritten by the next pair
-    }
-    // rows of the tile past the last token stay zero
-    for (int i = tid; i < (TOK - ((mc + 1) & ~1)) * (kTcDc / 8); i += kThreads) {
-      const int mi = ((mc + 1) & ~1) + i / (kTcDc / 8), u = i % (kTcDc / 8);
-      *reinterpret_cast<uint4*>(Us + swz_cb(mi, u, TOK)) = make_uint4(0, 0, 0, 0);
-    }
-  } else {
-    // u[m, c0..c0+kCU) = sum_k w_k o_k[c0..c0+kCU) for tokens gr, gr + kGroups, ...
+    };
+    if constexpr (TOK == 16) {
+      // few tokens, many splits each: the kGroups groups take splits gr,
+      // gr + kGroups, ... of two tokens at a time, eight loads per token in
+      // flight (sixteen for a token without a partner); the groups' sums meet
+      // in the fp32 scratch R and are added in group order (deterministic)
+      float* R = reinterpret_cast<float*>(Us + TOK * kTcDc * 2);  // [kGroups][2][d_c]
 #pragma unroll 1
-    for (int j0 = 0; j0 < kJ; j0 += kJB) {
-      int nmax = 0;
+      for (int mi0 = 0; mi0 < mc; mi0 += 2) {
+        const bool single = s_n[mi0 + 1] == 0;  // the same for the whole CTA
+        const int nmax = max(s_n[mi0], s_n[mi0 + 1]), kstep = (single ? 16 : 8) * kGroups;
+        float acc[2][kCU];
 #pragma unroll
-      for (int j = 0; j < kJB; ++j) nmax = max(nmax, s_n[gr + kGroups * (j0 + j)]);
-      float acc[kJB][kCU];
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
-      for (int j = 0; j < kJB; ++j)
+          for (int e = 0; e < kCU; ++e) acc[j][e] = 0.f;
+        for (int k0 = gr; k0 < nmax; k0 += kstep) {
+          uint4 raw[2][8];
 #pragma unroll
-        for (int e = 0; e < kCU; ++e) acc[j][e] = 0.f;
-      for (int k0 = 0; k0 < nmax; k0 += kKU) {
-        uint4 raw[kJB][kKU];
+          for (int j = 0; j < 2; ++j) {
+            const int mi = single ? mi0 : mi0 + j, n = s_n[mi];
 #pragma unroll
-        for (int j = 0; j < kJB; ++j) {
-          const int mi = gr + kGroups * (j0 + j), n = s_n[mi];
-#pragma unroll
-          for (int u = 0; u < kKU; ++u) {
-            raw[j][u] = make_uint4(0, 0, 0, 0);
-            if (k0 + u < n) raw[j][u] = PU::load(P.o_part, part_row(mi, k0 + u), c0);
+            for (int u = 0; u < 8; ++u) {
+              const int k = k0 + kGroups * (single ? 8 * j + u : u);
+              raw[j][u] = make_uint4(0, 0, 0, 0);
+              if (k < n) raw[j][u] = PU::load(P.o_part, part_row(mi, k), c0);
+            }
           }
-        }
 #pragma unroll
-        for (int j = 0; j < kJB; ++j) {
-          const int mi = gr + kGroups * (j0 + j), n = s_n[mi];
+          for (int j = 0; j < 2; ++j) {
+            const int mi = single ? mi0 : mi0 + j, n = s_n[mi];
 #pragma unroll
-          for (int u = 0; u < kKU; ++u) {
-            const int k = k0 + u;
-            const float wk = k < n ? weight(mi, k) : 0.f;
-            // a zero weight marks a split with no key of the sequence, whose
-            // partial was never written: its values are not read into u
-            if (wk != 0.f) {
-              float v[kCU];
-              PU::to_float(raw[j][u], v);
+            for (int u = 0; u < 8; ++u) {
+              const int k = k0 + kGroups * (single ? 8 * j + u : u);
+              const float wk = k < n ? weight(mi, k) : 0.f;
+              // a zero weight marks a split with no key of the sequence, whose
+              // partial was never written: its values are not read into u
+              if (wk != 0.f) {
+                float v[kCU];
+                PU::to_float(raw[j][u], v);
 #pragma unroll
-              for (int e = 0; e < kCU; ++e) acc[j][e] = fmaf(wk, v[e], acc[j][e]);
+                for (int e = 0; e < kCU; ++e) acc[j][e] = fmaf(wk, v[e], acc[j][e]);
+              }
             }
           }
         }
+        if (single) {
+#pragma unroll
+          for (int e = 0; e < kCU; ++e) {
+            acc[0][e] += acc[1][e];
+            acc[1][e] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < kCU; ++e) R[(gr * 2 + j) * kTcDc + c0 + e] = acc[j][e];
+        __syncthreads();
+        // thread t: token mi0 + t / 128, columns 4 (t % 128) .. + 3
+        {
+          const int j = tid >> 7, c = (tid & 127) * 4;
+          float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int q = 0; q < kGroups; ++q) {
+            const float4 x = *reinterpret_cast<const float4*>(R + (q * 2 + j) * kTcDc + c);
+            sum.x += x.x;
+            sum.y += x.y;
+            sum.z += x.z;
+            sum.w += x.w;
+          }
+          const __nv_bfloat162 lo2 = __floats2bfloat162_rn(sum.x, sum.y);
+          const __nv_bfloat162 hi2 = __floats2bfloat162_rn(sum.z, sum.w);
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
+          pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
+          *reinterpret_cast<uint2*>(Us + swz_cb(mi0 + j, c >> 3, TOK) + (c & 7) * 2) = pk;
+        }
+        __syncthreads();  // R is rewritten by the next pair
       }
+      // rows of the tile past the last token stay zero
+      for (int i = tid; i < (TOK - ((mc + 1) & ~1)) * (kTcDc / 8); i += kThreads) {
+        const int mi = ((mc + 1) & ~1) + i / (kTcDc / 8), u = i % (kTcDc / 8);
+        *reinterpret_cast<uint4*>(Us + swz_cb(mi, u, TOK)) = make_uint4(0, 0, 0, 0);
+      }
+    } else {
+      // u[m, c0..c0+kCU) = sum_k w_k o_k[c0..c0+kCU) for tokens gr, gr + kGroups, ...
+#pragma unroll 1
+      for (int j0 = 0; j0 < kJ; j0 += kJB) {
+        int nmax = 0;
 #pragma unroll
-      for (int j = 0; j < kJB; ++j) store_u(gr + kGroups * (j0 + j), acc[j]);
+        for (int j = 0; j < kJB; ++j) nmax = max(nmax, s_n[gr + kGroups * (j0 + j)]);
+        float acc[kJB][kCU];
+#pragma unroll
+        for (int j = 0; j < kJB; ++j)
+#pragma unroll
+          for (int e = 0; e < kCU; ++e) acc[j][e] = 0.f;
+        for (int k0 = 0; k0 < nmax; k0 += kKU) {
+          uint4 raw[kJB][kKU];
+#pragma unroll
+          for (int j = 0; j < kJB; ++j) {
+            const int mi = gr + kGroups * (j0 + j), n = s_n[mi];
+#pragma unroll
+            for (int u = 0; u < kKU; ++u) {
+              raw[j][u] = make_uint4(0, 0, 0, 0);
+              if (k0 + u < n) raw[j][u] = PU::load(P.o_part, part_row(mi, k0 + u), c0);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < kJB; ++j) {
+            const int mi = gr + kGroups * (j0 + j), n = s_n[mi];
+#pragma unroll
+            for (int u = 0; u < kKU; ++u) {
+              const int k = k0 + u;
+              const float wk = k < n ? weight(mi, k) : 0.f;
+              // a zero weight marks a split with no key of the sequence, whose
+              // partial was never written: its values are not read into u
+              if (wk != 0.f) {
+                float v[kCU];
+                PU::to_float(raw[j][u], v);
+#pragma unroll
+                for (int e = 0; e < kCU; ++e) acc[j][e] = fmaf(wk, v[e], acc[j][e]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < kJB; ++j) store_u(gr + kGroups * (j0 + j), acc[j]);
+      }
     }
-  }
-  MLA_STAMP(5);
-  const bool w_ok = mbar_wait_bounded(bar, 0);
-  if (__syncthreads_or(!w_ok)) {  // also publishes the u tile
-    if (tid == 0) record_status(P.status, MLA_ERR_TIMEOUT);
-    return;
-  }
-  MLA_STAMP(6);
-  // o[m, j] = sum_c u[m, c] W^UV_h[j, c]: warp w, columns [16w, 16w + 16)
-  const int g = lane >> 2, q = lane & 3, n0 = warp * 16;
-  float acc[TOK / 16][2][4];
+    MLA_STAMP(5);
+    const bool w_ok = mbar_wait_bounded(bar, 0);
+    if (__syncthreads_or(!w_ok)) {  // also publishes the u tile
+      if (tid == 0) record_status(P.status, MLA_ERR_TIMEOUT);
+      return;
+    }
+    MLA_STAMP(6);
+    // o[m, j] = sum_c u[m, c] W^UV_h[j, c]: warp w, columns [16w, 16w + 16)
+    const int g = lane >> 2, q = lane & 3, n0 = warp * 16;
+    float acc[TOK / 16][2][4];
 #pragma unroll
-  for (int i = 0; i < TOK / 16; ++i)
+    for (int i = 0; i < TOK / 16; ++i)
 #pragma unroll
-    for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+      for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
 #pragma unroll 4
-  for (int k0 = 0; k0 < kTcDc; k0 += 16) {
-    uint32_t b00, b01, b10, b11;
-    load_b_nk_cb(Ws, kTcDv, k0, n0, lane, b00, b01, b10, b11);
+    for (int k0 = 0; k0 < kTcDc; k0 += 16) {
+      uint32_t b00, b01, b10, b11;
+      load_b_nk_cb(Ws, kTcDv, k0, n0, lane, b00, b01, b10, b11);
+#pragma unroll
+      for (int i = 0; i < TOK / 16; ++i) {
+        uint32_t af[4];
+        load_a_cb(Us, TOK, 16 * i, k0, lane, af);
+        mma_bf16(acc[i][0], af, b00, b01);
+        mma_bf16(acc[i][1], af, b10, b11);
+      }
+    }
+    MLA_STAMP(2);
 #pragma unroll
     for (int i = 0; i < TOK / 16; ++i) {
-      uint32_t af[4];
-      load_a_cb(Us, TOK, 16 * i, k0, lane, af);
-      mma_bf16(acc[i][0], af, b00, b01);
-      mma_bf16(acc[i][1], af, b10, b11);
+      const int r0 = 16 * i + g, r1 = r0 + 8, col = n0 + 2 * q;
+      __nv_bfloat16* o0 = P.out + ((size_t)(m0 + r0) * n_heads + h) * kTcDv + col;
+      __nv_bfloat16* o1 = P.out + ((size_t)(m0 + r1) * n_heads + h) * kTcDv + col;
+      if (r0 < mc) {
+        *reinterpret_cast<__nv_bfloat162*>(o0) = __floats2bfloat162_rn(acc[i][0][0], acc[i][0][1]);
+        *reinterpret_cast<__nv_bfloat162*>(o0 + 8) = __floats2bfloat162_rn(acc[i][1][0], acc[i][1][1]);
+      }
+      if (r1 < mc) {
+        *reinterpret_cast<__nv_bfloat162*>(o1) = __floats2bfloat162_rn(acc[i][0][2], acc[i][0][3]);
+        *reinterpret_cast<__nv_bfloat162*>(o1 + 8) = __floats2bfloat162_rn(acc[i][1][2], acc[i][1][3]);
+      }
     }
-  }
-  MLA_STAMP(2);
-#pragma unroll
-  for (int i = 0; i < TOK / 16; ++i) {
-    const int r0 = 16 * i + g, r1 = r0 + 8, col = n0 + 2 * q;
-    __nv_bfloat16* o0 = P.out + ((size_t)(m0 + r0) * n_heads + h) * kTcDv + col;
-    __nv_bfloat16* o1 = P.out + ((size_t)(m0 + r1) * n_heads + h) * kTcDv + col;
-    if (r0 < mc) {
-      *reinterpret_cast<__nv_bfloat162*>(o0) = __floats2bfloat162_rn(acc[i][0][0], acc[i][0][1]);
-      *reinterpret_cast<__nv_bfloat162*>(o0 + 8) = __floats2bfloat162_rn(acc[i][1][0], acc[i][1][1]);
-    }
-    if (r1 < mc) {
-      *reinterpret_cast<__nv_bfloat162*>(o1) = __floats2bfloat162_rn(acc[i][0][2], acc[i][0][3]);
-      *reinterpret_cast<__nv_bfloat162*>(o1 + 8) = __floats2bfloat162_rn(acc[i][1][2], acc[i][1][3]);
-    }
+    __syncthreads();  // the u tile and the block's split tables are rewritten next
   }
   MLA_STAMP(3);
   tl_end(P.timeline, MLA_TRACE_COMBINE);
@@ -504,11 +511,10 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
     p.timeline = timeline_ptr();
     if (!make_tile_map_bf16(&p.map_w, W_uv, kTcDc, (uint64_t)d.n_heads * kTcDv, (uint64_t)kTcDc * 2, 64, kTcDv))
       return cudaErrorInvalidValue;
-    // tokens per CTA: the largest block that still gives every SM a CTA
-    const int M = batch * n_q, sms = device_sm_count();
-    int tok = 16;
-    if ((long long)d.n_heads * ((M + 63) / 64) >= sms) tok = 64;
-    else if ((long long)d.n_heads * ((M + 31) / 32) >= sms) tok = 32;
+    // one CTA per head (W^UV_h fetched once, before the grid-dependency wait,
+    // by every CTA at once) looping over blocks of 16, 32 or 64 tokens
+    const int M = batch * n_q;
+    const int tok = M > 32 ? 64 : M > 16 ? 32 : 16;
     auto kernel = part_bf16 ? (tok == 64   ? combine_tc_kernel<64, true>
                                : tok == 32 ? combine_tc_kernel<32, true>
                                            : combine_tc_kernel<16, true>)
@@ -518,7 +524,7 @@ cudaError_t launch_combine(const mla_dims& d, const void* W_uv, int batch, int n
     const size_t tsm = combine_tc_smem(tok);
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(kernel, dim3(d.n_heads, (M + tok - 1) / tok), dim3(kThreads), tsm, st, p);
+    e = launch_pdl(kernel, dim3(d.n_heads, 1), dim3(kThreads), tsm, st, p);
     if (e != cudaSuccess) return e;
   } else {
     e = cudaFuncSetAttribute(combine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -31,6 +31,12 @@ CASES = [
     # more tokens than one 64-token pass of the tensor-core projection
     ("bf16-70-tokens", dict(B=70, T=1, L=tuple(int(x) for x in np.arange(70) * 37 % 300), cache_dtype="bf16")),
     ("fp8-70-tokens", dict(B=35, T=2, L=tuple(int(x) for x in np.arange(35) * 53 % 400), cache_dtype="fp8")),
+    # a last pass of 48 tokens (two of the eight warps idle), four full passes
+    # in one 256-token round, two rounds, and a one-token last pass
+    ("bf16-48-tokens", dict(B=48, T=1, L=tuple(int(x) for x in np.arange(48) * 41 % 300), cache_dtype="bf16")),
+    ("fp8-256-tokens", dict(B=128, T=2, L=tuple(int(x) for x in np.arange(128) * 67 % 500), cache_dtype="fp8")),
+    ("bf16-300-tokens", dict(B=150, T=2, L=tuple(int(x) for x in np.arange(150) * 31 % 200), cache_dtype="bf16")),
+    ("bf16-129-tokens", dict(B=129, T=1, L=tuple(int(x) for x in np.arange(129) * 43 % 260), cache_dtype="bf16")),
 ]
 
 
