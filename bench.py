@@ -497,6 +497,58 @@ def measure(cfg, args, dev, pg, local: int, peaks: dict) -> dict:
     return {"wl": wl, "ms": ms, "ms_step": ms_step, "clocks": clocks, "kms": kms, "tpeak": tpeak, **summ}
 
 
+def prefill_work(cfg) -> dict:
+    """Algorithmic FLOPs of a prefill step in the non-absorbed form: the
+    up-projection of every key's latent to per-head keys and values, and the
+    causal attention (query/key width d_nope + d_rope, value width d_v)."""
+    H, dc, dn, dr, dv = cfg.n_heads, cfg.d_c, cfg.d_nope, cfg.d_rope, cfg.d_v
+    keys = int(cfg.seq_lens.sum())
+    pairs = int(sum(int(L) * cfg.T + cfg.T * (cfg.T + 1) // 2 for L in cfg.L))
+    return {"upproj_flops": 2 * keys * H * (dn + dv) * dc, "attention_flops": 2 * pairs * H * (dn + dr + dv),
+            "absorbed_attention_flops": 2 * pairs * H * (dc + dr + dc), "pairs": pairs, "keys": keys}
+
+
+def measure_prefill(cfg, args, dev, peaks: dict) -> dict:
+    """A chunked-prefill step (append the chunk, then prefill attention over
+    the cache) timed by graph replays like the decode workloads; the
+    prefill call alone timed the same way."""
+    from latent_compressed_attention_mla_b200 import binding as B
+    wl = Workload(cfg, dev, 0, 0)
+    max_len = int(cfg.seq_lens.max())
+    out = torch.empty(cfg.B, cfg.T, cfg.n_heads, cfg.d_v, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(cfg.B, cfg.T, cfg.n_heads, dtype=torch.float32, device=dev)
+
+    def prefill(i, with_append=True):
+        w, x, pool = wl.sets[i % wl.copies]
+        if with_append:
+            wl.sess.append(x["h"], wl.seq_idx, wl.pos, w["W_dkv"], w["W_kr"], wl.pt, pool)
+        wl.sess.prefill(x["q_nope"], x["q_rope"], w["W_uk"], w["W_uv"], pool, wl.pt, wl.seq_lens, max_len, out, lse)
+
+    res = {}
+    for name, app in (("step", True), ("prefill", False)):
+        for i in range(2):
+            prefill(i, app)
+        torch.cuda.synchronize()
+        graphs = []
+        for r in range(wl.copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                prefill(r, app)
+            graphs.append(g)
+        ms, clocks = time_graph_steps(wl, graphs, args.steps, args.warmup, None, 0)
+        res[name] = (ms / args.steps, clocks)
+        del graphs
+    wk = prefill_work(cfg)
+    t_pf = res["prefill"][0] / 1e3
+    tpeak = peaks["bf16_tflops"]
+    flops = wk["upproj_flops"] + wk["attention_flops"]
+    return {"ms_per_step": res["step"][0], "tokens_per_s": cfg.B * cfg.T / (res["step"][0] / 1e3),
+            "prefill_us": 1e6 * t_pf, "prefill_TFLOPs": flops / t_pf / 1e12,
+            "frac_of_tensor_peak": flops / t_pf / 1e12 / tpeak,
+            "flops": {k: v for k, v in wk.items()}, "clocks": res["step"][1], "l2": wl.l2_note(),
+            "form": "non-absorbed (per-head keys and values from the latent), causal"}
+
+
 def config_entry(cfg, m: dict, world: int) -> dict:
     """A workload's figures for the per-config map of the JSON line."""
     return {"ms_per_step": m["ms_step"], "tokens_per_s": whole_job_tokens_per_s(world, cfg.B * cfg.T, 1, m["ms_step"]),
@@ -594,6 +646,8 @@ def main():
             extra[c.name] = config_entry(c, mc, world)
             del mc
             torch.cuda.empty_cache()
+        extra[WL.V3_PREFILL_CHUNK.name] = measure_prefill(WL.V3_PREFILL_CHUNK, args, dev, peaks)
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

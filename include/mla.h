@@ -207,6 +207,39 @@ int mla_combine(const mla_dims* dims, const void* W_uv, int batch, int n_q, int 
                 const void* workspace, size_t ws_bytes, void* out, float* lse_out,
                 void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Prefill (many new tokens per sequence)  mla_prefill: the non-absorbed form.
+ * A prefill step is compute-bound, and there reconstructing each head's keys
+ * and values from the latent is cheaper than the absorbed form ("DeepSeek MLA
+ * Architecture: How Multi-Head Latent Attention Cuts KV Cache by 93%",
+ * opening section on the prefill and decode phases; "1. Low-Rank Key-Value
+ * Compression"; "3. Decoupled RoPE and Matrix Absorption").  For sequence b,
+ * query j (position p = seq_lens[b] - n_q + j), head h, keys s = 0 .. p:
+ *   k_{s,h} = [W_uk[h] c_s ; k^R_s],  v_{s,h} = W_uv[h] c_s,
+ *   o_h = softmax(softmax_scale * [q_nope ; RoPE(q_rope, p)] . k_{s,h}) v_{s,h}
+ * which is the same result mla_decode + mla_combine give (causal among the
+ * n_q new tokens, which must already be in the cache).
+ *   q_nope, q_rope, W_uk, cache_pool, num_pages, page_table, max_pages,
+ *   seq_lens, batch, n_q as for mla_decode; W_uv as for mla_combine
+ *   max_seq_len  host-side upper bound of seq_lens[b] (sizes the grids and the
+ *                workspace); a longer sequence is skipped and MLA_ERR_BOUNDS
+ *                recorded
+ *   workspace    >= mla_prefill_workspace_bytes(dims, max_seq_len): one
+ *                sequence's gathered latent rows and its per-head keys and
+ *                values (about 65 KB per key at DeepSeek-V3 dims); sequences
+ *                run one after another
+ *   out [batch, n_q, n_heads, d_v] act, lse_out [batch, n_q, n_heads] float32
+ *   natural-log softmax denominators (may be NULL)
+ * DeepSeek-V3 dims only (d_c 512, d_rope 64, d_nope = d_v = 128, 64-token
+ * pages), bf16 activations, bf16 or FP8 cache; MLA_ERR_UNSUPPORTED otherwise.
+ * ------------------------------------------------------------------------- */
+size_t mla_prefill_workspace_bytes(const mla_dims* dims, int max_seq_len);
+int mla_prefill(const mla_dims* dims, const void* q_nope, const void* q_rope,
+                const void* W_uk, const void* W_uv, const void* cache_pool, int num_pages,
+                const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                int batch, int n_q, int max_seq_len, void* workspace, size_t ws_bytes,
+                void* out, float* lse_out, void* stream);
+
 /* Which decode kernel mla_decode would launch for these dims on the current
  * device: 0 = CUDA-core (SIMT) kernel, 1 = tcgen05 kernel; <0 = error code. */
 int mla_decode_path(const mla_dims* dims, int n_q);

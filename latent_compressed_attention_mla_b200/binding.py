@@ -27,7 +27,8 @@ ERRORS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "M
 # Every entry point declared in include/mla.h.
 EXPORTED = ("mla_cache_page_bytes", "mla_check_dims", "mla_append_workspace_bytes", "mla_append_latent",
             "mla_append_latent_noalloc",
-            "mla_decode_workspace_bytes", "mla_decode", "mla_combine", "mla_decode_path", "mla_auto_splits",
+            "mla_decode_workspace_bytes", "mla_decode", "mla_combine", "mla_prefill_workspace_bytes",
+            "mla_prefill", "mla_decode_path", "mla_auto_splits",
             "mla_set_trace_events", "mla_set_timeline", "mla_get_status", "mla_error_string")
 TRACE_KERNELS = ("append_project", "append_finalize", "absorb", "attend", "combine")
 
@@ -67,6 +68,9 @@ def lib() -> ctypes.CDLL:
         L.mla_decode.restype = I
         L.mla_combine.argtypes = [S, P, I, I, I, P, Z, P, P, P]
         L.mla_combine.restype = I
+        L.mla_prefill_workspace_bytes.argtypes, L.mla_prefill_workspace_bytes.restype = [S, I], Z
+        L.mla_prefill.argtypes = [S, P, P, P, P, P, I, P, I, P, I, I, I, P, Z, P, P, P]
+        L.mla_prefill.restype = I
         L.mla_decode_path.argtypes, L.mla_decode_path.restype = [S, I], I
         L.mla_auto_splits.argtypes, L.mla_auto_splits.restype = [S, I, I], I
         L.mla_get_status.argtypes, L.mla_get_status.restype = [P, ctypes.POINTER(ctypes.c_int)], I
@@ -185,6 +189,24 @@ def mla_combine(dims, W_uv, batch, n_q, workspace, out, lse_out=None, num_splits
                            workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse_out),
                            _stream(stream))
     _check(rc, "mla_combine")
+
+
+def prefill_workspace_bytes(dims: MlaDims, max_seq_len: int) -> int:
+    return int(lib().mla_prefill_workspace_bytes(ctypes.byref(dims), max_seq_len))
+
+
+def mla_prefill(dims, q_nope, q_rope, W_uk, W_uv, cache_pool, page_table, seq_lens, max_seq_len, workspace, out,
+                lse_out=None, stream=None):
+    """Prefill attention (non-absorbed form) of the n_q new tokens of each
+    sequence, already appended: writes out [B, n_q, n_h, d_v] and lse_out."""
+    _cuda(q_nope, q_rope, W_uk, W_uv, cache_pool, page_table, seq_lens, workspace, out, lse_out)
+    B, T = q_nope.shape[0], q_nope.shape[1]
+    num_pages = cache_pool.numel() * cache_pool.element_size() // cache_page_bytes(dims)
+    rc = lib().mla_prefill(ctypes.byref(dims), _ptr(q_nope), _ptr(q_rope), _ptr(W_uk), _ptr(W_uv), _ptr(cache_pool),
+                           num_pages, _ptr(page_table), page_table.shape[1], _ptr(seq_lens), B, T, max_seq_len,
+                           _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse_out),
+                           _stream(stream))
+    _check(rc, "mla_prefill")
 
 
 def mla_get_status(stream=None) -> int:

@@ -41,6 +41,21 @@ class MlaDecodeSession:
         B.mla_combine(self.dims, W_uv, self.batch, self.n_q, self.decode_ws, out, lse, self.num_splits, stream)
         return out, lse
 
+    def prefill(self, q_nope, q_rope, W_uk, W_uv, cache_pool, page_table, seq_lens, max_seq_len: int, out=None,
+                lse=None, stream=None):
+        """Prefill attention (the non-absorbed form) of the session's n_q new
+        tokens per sequence, already appended; max_seq_len bounds seq_lens.
+        The prefill workspace is allocated on first use for that bound."""
+        if getattr(self, "_prefill_ws_len", 0) < max_seq_len:
+            self._prefill_ws = torch.empty(B.prefill_workspace_bytes(self.dims, max_seq_len), dtype=torch.uint8,
+                                           device=self.device)
+            self._prefill_ws_len = max_seq_len
+        out = self.out if out is None else out
+        lse = self.lse if lse is None else lse
+        B.mla_prefill(self.dims, q_nope, q_rope, W_uk, W_uv, cache_pool, page_table, seq_lens, max_seq_len,
+                      self._prefill_ws, out, lse, stream)
+        return out, lse
+
     def step(self, h, seq_idx, pos, q_nope, q_rope, seq_lens, weights: dict, page_table, cache_pool, out=None,
              lse=None, stream=None):
         """Append the step's tokens, then attend (the page's order: the new token

@@ -182,6 +182,10 @@ V3_FP8_B128_T2 = _v3("v3-fp8-b128-l16384-t2", 4, 128, 2, [16384] * 128, "fp8")
 # in this order for bench.py --config
 CONFIGS = [TINY_F32, V3_B1_L4096, V3_RAGGED_B64, V3_LONG_B8, V3_FP8_B128_T2]
 
+# A chunked-prefill step: one sequence with 4096 cached tokens takes a chunk
+# of 4096 new tokens (appended, then attending causally over all 8192).
+V3_PREFILL_CHUNK = _v3("v3-prefill-l4096-t4096", 5, 1, 4096, [4096], "bf16")
+
 
 # ----------------------------------------------------------------------------
 # Generated tensors

@@ -112,3 +112,12 @@ def test_workspace_layout_grows_with_splits():
     b = B.decode_workspace_bytes(d, 8, 1, 20)
     # each extra split adds one slot of n_h * (d_c + 1) floats
     assert b - a >= 10 * 128 * 513 * 4 - 512
+
+
+def test_prefill_workspace_query():
+    d = B.dims_for(W.V3_B1_L4096)
+    n = B.prefill_workspace_bytes(d, 4096)
+    # latent rows and k^R (1152 B per key) plus keys and values of 128 heads (64 KB per key)
+    assert n >= 4096 * (1152 + 2 * 128 * 128 * 2)
+    assert B.prefill_workspace_bytes(d, 0) == 0
+    assert B.prefill_workspace_bytes(B.dims_for(W.TINY_F32), 256) == 0  # fp32 / other dims: no prefill kernel
