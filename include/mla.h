@@ -225,9 +225,11 @@ int mla_combine(const mla_dims* dims, const void* W_uv, int batch, int n_q, int 
  *                workspace); a longer sequence is skipped and MLA_ERR_BOUNDS
  *                recorded
  *   workspace    >= mla_prefill_workspace_bytes(dims, max_seq_len): one
- *                sequence's gathered latent rows and its per-head keys and
- *                values (about 65 KB per key at DeepSeek-V3 dims); sequences
- *                run one after another
+ *                sequence's gathered latent rows, its per-head keys and
+ *                values and its rotated queries (about 113 KB per token of
+ *                max_seq_len at DeepSeek-V3 dims); sequences run one after
+ *                another
+ *   out          16-byte aligned (MLA_ERR_ALIGNMENT otherwise)
  *   out [batch, n_q, n_heads, d_v] act, lse_out [batch, n_q, n_heads] float32
  *   natural-log softmax denominators (may be NULL)
  * DeepSeek-V3 dims only (d_c 512, d_rope 64, d_nope = d_v = 128, 64-token

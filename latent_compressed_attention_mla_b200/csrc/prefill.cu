@@ -15,16 +15,18 @@
 // 2 * (576 + 512) for the absorbed form, plus the up-projection's
 // 2 * 512 * 2 * 128 per (key, head) once per step.
 //
-// Per sequence, three kernels:
+// Per sequence, four kernels:
 //   1. gather: the sequence's latent rows c_s (dequantised for an FP8 cache)
-//      and k^R_s, from the paged cache into contiguous bf16 rows;
+//      and k^R_s, from the paged cache into contiguous bf16 rows, zero up to
+//      the next multiple of 128 keys;
 //   2. up-projection: K^C = C W_uk^T and V = C W_uv^T, mma.sync GEMMs whose
 //      128 x 128 output tiles are one head's keys, written head-major
 //      [head][key][128] so that an attention tile is one contiguous block;
-//   3. attention: one CTA per (head, block of 64 queries), four warps of 16
-//      queries, key tiles of 64 double-buffered by cp.async, online softmax
-//      in base 2 with the probabilities kept in registers (the score
-//      accumulators become the next MMA's A fragments), fp32 accumulation.
+//   3. queries: [q_nope ; RoPE(q_rope, p)] per (head, token), head-major;
+//   4. attention on the tensor cores (tcgen05, accumulators in tensor memory),
+//      one CTA per (head, block of 128 queries); see below.
+#include <cuda.h>
+
 #include "mla_internal.cuh"
 #include "mma_tile.cuh"
 
@@ -51,10 +53,11 @@ struct PrefillArgs {
   const int32_t* seq_lens;
   int n_heads, n_q, max_seq_len, fp8;
   float rope_base, scale_log2;
-  __nv_bfloat16* C;   // [max_seq_len, 512]
-  __nv_bfloat16* KR;  // [max_seq_len, 64]
-  __nv_bfloat16* Kc;  // [H, max_seq_len, 128]
-  __nv_bfloat16* V;   // [H, max_seq_len, 128]
+  int max_rows;       // max_seq_len rounded up to a whole 128-key tile
+  __nv_bfloat16* C;   // [max_rows, 512]
+  __nv_bfloat16* KR;  // [max_rows, 64]
+  __nv_bfloat16* Kc;  // [H, max_rows, 128]
+  __nv_bfloat16* V;   // [H, max_rows, 128]
   __nv_bfloat16* out; // [B, T, H, 128]
   float* lse_out;     // [B, T, H] or null
   int* status;
@@ -77,12 +80,14 @@ __global__ void __launch_bounds__(256) prefill_gather_kernel(const PrefillArgs a
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = seq_keys(a, b);
   const int s = blockIdx.x * 8 + warp;
-  if (S < 0 || s >= S) return;
-  int page = a.page_table[(size_t)b * a.max_pages + s / kPPage];
+  if (S < 0 || s >= (S + 127) / 128 * 128) return;
   uint4* c_dst = reinterpret_cast<uint4*>(a.C + (size_t)s * kPDc);
   uint4* kr_dst = reinterpret_cast<uint4*>(a.KR + (size_t)s * kPDr);
+  // rows past the sequence, up to its last 128-key tile, are zero: their
+  // keys and values come out zero (masked scores, zero probabilities)
+  const int page = s < S ? a.page_table[(size_t)b * a.max_pages + s / kPPage] : -1;
   if (page < 0 || page >= a.num_pages) {
-    record_status(a.status, MLA_ERR_BOUNDS);
+    if (s < S) record_status(a.status, MLA_ERR_BOUNDS);
     for (int u = lane; u < kPDc / 8; u += 32) c_dst[u] = make_uint4(0, 0, 0, 0);
     if (lane < kPDr / 8) kr_dst[lane] = make_uint4(0, 0, 0, 0);
     return;
@@ -132,10 +137,11 @@ __global__ void __launch_bounds__(kGThreads) prefill_upproj_kernel(const Prefill
   extern __shared__ __align__(128) uint8_t smem_g[];
   const int S = seq_keys(a, b);
   const int h = blockIdx.x, m0 = blockIdx.y * kGBm;
-  if (S < 0 || m0 >= S) return;
+  const int rows = (S + kGBm - 1) / kGBm * kGBm;  // whole 128-key tiles (zero rows past the sequence)
+  if (S < 0 || m0 >= rows) return;
   const bool is_v = blockIdx.z == 1;
   const __nv_bfloat16* W = (is_v ? a.W_uv : a.W_uk) + (size_t)h * kPDn * kPDc;
-  __nv_bfloat16* out = (is_v ? a.V : a.Kc) + (size_t)h * a.max_seq_len * kPDn;
+  __nv_bfloat16* out = (is_v ? a.V : a.Kc) + (size_t)h * a.max_rows * kPDn;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wm = warp >> 2, wn = warp & 3;  // warp tile: rows 64 wm .. +64, columns 32 wn .. +32
   auto stage_a = [&](int st) { return smem_g + st * kGStageBytes; };
@@ -145,8 +151,7 @@ __global__ void __launch_bounds__(kGThreads) prefill_upproj_kernel(const Prefill
     uint8_t* Bs = stage_b(st);
     for (int i = tid; i < kGBm * kGRowUnits; i += kGThreads) {
       const int r = i / kGRowUnits, u = i % kGRowUnits;
-      const int s = min(m0 + r, S - 1);  // rows past the sequence repeat its last key (never stored)
-      cp_async16(smem_addr(As) + swz(r, u, kGRowUnits), a.C + (size_t)s * kPDc + k0 + u * 8);
+      cp_async16(smem_addr(As) + swz(r, u, kGRowUnits), a.C + (size_t)(m0 + r) * kPDc + k0 + u * 8);
     }
     for (int i = tid; i < kGBn * kGRowUnits; i += kGThreads) {
       const int r = i / kGRowUnits, u = i % kGRowUnits;
@@ -197,210 +202,429 @@ __global__ void __launch_bounds__(kGThreads) prefill_upproj_kernel(const Prefill
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int c = 32 * wn + 8 * j + 2 * q;
-      if (r0 < S)
-        *reinterpret_cast<__nv_bfloat162*>(out + (size_t)r0 * kPDn + c) =
-            __floats2bfloat162_rn(acc[i][j][0], acc[i][j][1]);
-      if (r0 + 8 < S)
-        *reinterpret_cast<__nv_bfloat162*>(out + (size_t)(r0 + 8) * kPDn + c) =
-            __floats2bfloat162_rn(acc[i][j][2], acc[i][j][3]);
+      *reinterpret_cast<__nv_bfloat162*>(out + (size_t)r0 * kPDn + c) =
+          __floats2bfloat162_rn(acc[i][j][0], acc[i][j][1]);
+      *reinterpret_cast<__nv_bfloat162*>(out + (size_t)(r0 + 8) * kPDn + c) =
+          __floats2bfloat162_rn(acc[i][j][2], acc[i][j][3]);
     }
   }
 }
 
 // ----------------------------------------------------------------------------
-// 3. attention: one CTA per (head, block of 64 queries), four warps
+// 3. attention on the 5th-generation tensor cores: one CTA per (head, block of
+//    128 queries).  The 128 queries are the M dimension of tcgen05 MMAs with
+//    accumulators in tensor memory (query i in TMEM lane i):
+//      S[128 x 128 keys] = Q[128 x 192] . K^T     (12 MMAs of K = 16)
+//      O[128 x 128]     += P[128 x 128 keys] . V  (8 MMAs of K = 16)
+//    S is double-buffered (columns 0 and 128), O sits in columns 256-383.
+//    Warps 0-3 run the softmax (one query row per thread, a lazily updated
+//    reference max as in the decode: O is rescaled only when a row's tile
+//    maximum exceeds its reference by more than 2^8), write P as bf16 into
+//    shared memory and finish; warp 4 allocates tensor memory and one thread
+//    issues every MMA; warps 5 and 6 bring K and V tiles by TMA (128-byte
+//    swizzle).  Every wait is bounded; a CTA that gives up records
+//    MLA_ERR_TIMEOUT, waits (bounded) for the MMAs it issued and frees its
+//    tensor memory.
 // ----------------------------------------------------------------------------
-constexpr int kABq = 64, kABk = 64, kAThreads = 128;
-constexpr int kAKUnits = kPDk / 8;  // 24 units of a key row (192 wide)
-constexpr int kAVUnits = kPDv / 8;  // 16 units of a value row
-constexpr uint32_t kAQBytes = kABq * kPDk * 2;                          // 24 KB
-constexpr uint32_t kAKVBytes = kABk * kPDk * 2 + kABk * kPDv * 2;       // 40 KB per stage
-constexpr size_t kASmem = kAQBytes + 2 * kAKVBytes;
+constexpr int kTq = 128, kTk = 128;
+constexpr int kTThreads = 224;
+constexpr int kTMmaWarp = 4, kTKWarp = 5, kTVWarp = 6;
+constexpr uint32_t kTChunk = 128 * 128;            // one 64-column block of 128 rows (16 KB)
+constexpr uint32_t kTOffQ = 0;                     // [3][128 queries][128 B]
+constexpr uint32_t kTOffK = kTOffQ + 3 * kTChunk;  // [2 stages][3][128 keys][128 B]
+constexpr uint32_t kTOffV = kTOffK + 6 * kTChunk;  // [2 column halves][128 keys][128 B]
+constexpr uint32_t kTOffP = kTOffV + 2 * kTChunk;  // [2 key blocks][128 queries][128 B]
+constexpr uint32_t kTOffBar = kTOffP + 2 * kTChunk;
+enum { TQ_FULL = 0, TK_FULL = 1, TK_EMPTY = 3, TV_FULL = 5, TV_EMPTY = 6, TS_FULL = 7, TS_FREE = 9, TP_FULL = 11,
+       TO_DONE = 12, TDRAIN = 13, TNumBars = 14 };
+constexpr uint32_t kTOffMisc = kTOffBar + 8 * TNumBars;
+constexpr size_t kTSmem = kTOffMisc + 16 + 1024;   // + alignment slack
+constexpr uint32_t kTColS = 0, kTColO = 256, kTTmemCols = 512;
+constexpr long long kTWaitLimit = 4000000000LL;    // ~2 s
+constexpr float kTRescale = 8.0f;                  // log2 units
 
-__global__ void __launch_bounds__(kAThreads) prefill_attn_kernel(const PrefillArgs a, int b) {
-  extern __shared__ __align__(128) uint8_t smem_a[];
+struct TcAttnParams {
+  PrefillArgs a;
+  int b, max_rows;       // sequence; rows of one head's key / value block (max_seq_len rounded up to 128)
+  CUtensorMap map_q;     // Qr [H * T rows][192], box 64 x 128
+  CUtensorMap map_kc;    // Kc [H * max_rows][128], box 64 x 128
+  CUtensorMap map_kr;    // KR [max_rows][64], box 64 x 128
+  CUtensorMap map_v;     // V  [H * max_rows][128], box 64 x 128
+};
+
+__device__ __forceinline__ bool tc_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false (MLA_ERR_TIMEOUT recorded once) on expiry, or at once
+// when another role of the CTA already gave up.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
+  if (tc_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (tc_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kTWaitLimit) {
+      *abort_flag = 1;
+      record_status(status, MLA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tc_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_mma1(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// arrive on a barrier of this CTA once the MMAs this thread issued so far complete
+__device__ __forceinline__ void tc_commit1(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+// shared-memory matrix descriptor, 128-byte swizzle (sm_100 version field)
+__device__ __forceinline__ uint64_t tc_sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// instruction descriptor: kind::f16 with bf16 operands, f32 accumulator, dense
+constexpr uint32_t tc_idesc_bf16(int M, int N, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __grid_constant__ TcAttnParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const PrefillArgs& a = P.a;
+  const int b = P.b;
   const int S = seq_keys(a, b);
-  if (S < 0) return;
+  if (S < 0) return;  // the whole CTA, before any barrier or tensor memory
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = a.n_q, H = a.n_heads;
-  // heavier (later) query blocks first
-  const int qb = (int)(gridDim.x - 1 - blockIdx.x), h = blockIdx.y;
-  const int t0 = qb * kABq;
-  if (t0 >= T) return;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, qd = lane & 3;
-  uint8_t* Qs = smem_a;
-  auto Ks = [&](int st) { return smem_a + kAQBytes + st * kAKVBytes; };
-  auto Vs = [&](int st) { return smem_a + kAQBytes + st * kAKVBytes + kABk * kPDk * 2; };
-  const int p0 = S - T;  // position of query 0
-  const __nv_bfloat16* Kh = a.Kc + (size_t)h * a.max_seq_len * kPDn;
-  const __nv_bfloat16* Vh = a.V + (size_t)h * a.max_seq_len * kPDv;
-  auto load_kv = [&](int st, int s0) {
-    for (int i = tid; i < kABk * kAKUnits; i += kAThreads) {
-      const int r = i / kAKUnits, u = i % kAKUnits;
-      const int s = min(s0 + r, S - 1);  // rows past the sequence: masked scores, zero probabilities
-      const __nv_bfloat16* src = u < kPDn / 8 ? Kh + (size_t)s * kPDn + u * 8 : a.KR + (size_t)s * kPDr + (u - kPDn / 8) * 8;
-      cp_async16(smem_addr(Ks(st)) + swz(r, u, kAKUnits), src);
+  const int qb = (int)(gridDim.x - 1 - blockIdx.x), h = blockIdx.y;  // heavier (later) query blocks first
+  const int t0 = qb * kTq, p0 = S - T;
+  const int n_tiles = (p0 + min(T, t0 + kTq) + kTk - 1) / kTk;  // keys up to the block's last query
+  auto bar = [&](int i) -> uint32_t { return sbase + kTOffBar + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kTOffMisc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTOffMisc + 4);
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init_local(bar(TQ_FULL), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init_local(bar(TK_FULL + i), 1);
+      mbar_init_local(bar(TK_EMPTY + i), 1);
+      mbar_init_local(bar(TS_FULL + i), 1);
+      mbar_init_local(bar(TS_FREE + i), 4);
     }
-    for (int i = tid; i < kABk * kAVUnits; i += kAThreads) {
-      const int r = i / kAVUnits, u = i % kAVUnits;
-      const int s = min(s0 + r, S - 1);
-      cp_async16(smem_addr(Vs(st)) + swz(r, u, kAVUnits), Vh + (size_t)s * kPDv + u * 8);
-    }
-  };
-  // keys this block needs: up to the position of its last query
-  const int t_last = min(T, t0 + kABq) - 1;
-  const int n_keys = p0 + t_last + 1;
-  const int n_kb = (n_keys + kABk - 1) / kABk;
-  load_kv(0, 0);
-  cp_async_commit();
-  // Q tile: q_nope rows as they are, q^R rotated at each query's position
-  for (int i = tid; i < kABq * (kPDn / 8); i += kAThreads) {
-    const int r = i / (kPDn / 8), u = i % (kPDn / 8);
-    const int t = min(t0 + r, T - 1);
-    *reinterpret_cast<uint4*>(Qs + swz(r, u, kAKUnits)) =
-        *reinterpret_cast<const uint4*>(a.q_nope + (((size_t)b * T + t) * H + h) * kPDn + u * 8);
+    mbar_init_local(bar(TV_FULL), 1);
+    mbar_init_local(bar(TV_EMPTY), 1);
+    mbar_init_local(bar(TP_FULL), 4);
+    mbar_init_local(bar(TO_DONE), 1);
+    mbar_init_local(bar(TDRAIN), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int i = tid; i < kABq * (kPDr / 2); i += kAThreads) {
-    const int r = i / (kPDr / 2), k = i % (kPDr / 2);
-    const int t = min(t0 + r, T - 1);
-    const __nv_bfloat16* src = a.q_rope + (((size_t)b * T + t) * H + h) * kPDr;
-    float cs, sn;
-    rope_cos_sin(p0 + t, k, kPDr / 2, a.rope_base, &cs, &sn);
-    const float x1 = __bfloat162float(src[k]), x2 = __bfloat162float(src[k + kPDr / 2]);
-    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(Qs);
-    const int c1 = kPDn + k, c2 = kPDn + k + kPDr / 2;
-    dst[(swz(r, c1 >> 3, kAKUnits) >> 1) + (c1 & 7)] = __float2bfloat16_rn(x1 * cs - x2 * sn);
-    dst[(swz(r, c2 >> 3, kAKUnits) >> 1) + (c2 & 7)] = __float2bfloat16_rn(x2 * cs + x1 * sn);
+  if (warp == kTMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                 "r"(kTTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  tc_fence_before();
   __syncthreads();
-  uint32_t qf[kPDk / 16][4];
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int krow0 = h * P.max_rows;  // this head's first row in Kc and V
+
+  if (warp == kTKWarp) {
+    // ------------------------------------------------------------ TMA: Q, K
+    if (lane == 0) {
+      bool ok = true;
+      mbar_expect_local(bar(TQ_FULL), 3 * kTChunk);
+      for (int c = 0; c < 3; ++c) tma_load_2d(sbase + kTOffQ + c * kTChunk, &P.map_q, 64 * c, h * T + t0, bar(TQ_FULL));
+      for (int g = 0; g < n_tiles && ok; ++g) {
+        const int st = g & 1;
+        ok = tc_wait(bar(TK_EMPTY + st), ((g >> 1) & 1) ^ 1, abort_flag, a.status);
+        if (!ok) break;
+        const uint32_t fb = bar(TK_FULL + st), dst = sbase + kTOffK + st * 3 * kTChunk;
+        mbar_expect_local(fb, 3 * kTChunk);
+        tma_load_2d(dst, &P.map_kc, 0, krow0 + kTk * g, fb);
+        tma_load_2d(dst + kTChunk, &P.map_kc, 64, krow0 + kTk * g, fb);
+        tma_load_2d(dst + 2 * kTChunk, &P.map_kr, 0, kTk * g, fb);
+      }
+    }
+  } else if (warp == kTVWarp) {
+    // --------------------------------------------------------------- TMA: V
+    if (lane == 0) {
+      bool ok = true;
+      for (int g = 0; g < n_tiles && ok; ++g) {
+        ok = tc_wait(bar(TV_EMPTY), (g & 1) ^ 1, abort_flag, a.status);
+        if (!ok) break;
+        mbar_expect_local(bar(TV_FULL), 2 * kTChunk);
+        for (int c = 0; c < 2; ++c)
+          tma_load_2d(sbase + kTOffV + c * kTChunk, &P.map_v, 64 * c, krow0 + kTk * g, bar(TV_FULL));
+      }
+    }
+  } else if (warp == kTMmaWarp) {
+    // ---------------------------------------------------------------- MMAs
+    if (lane == 0) {
+      constexpr uint32_t kIdQK = tc_idesc_bf16(128, 128, false), kIdPV = tc_idesc_bf16(128, 128, true);
+      const uint64_t qdesc = tc_sdesc(sbase + kTOffQ, 16, 1024);   // chunk c: + 1024 c; K step: + 2
+      const uint64_t kdesc = tc_sdesc(sbase + kTOffK, 16, 1024);   // stage: + 3072; chunk: + 1024
+      const uint64_t pdesc = tc_sdesc(sbase + kTOffP, 16, 1024);   // key block: + 1024; K step: + 2
+      const uint64_t vdesc = tc_sdesc(sbase + kTOffV, kTChunk, 1024);  // 16 keys: + 128
+      bool ok = tc_wait(bar(TQ_FULL), 0, abort_flag, a.status);
+      for (int g = 0; g <= n_tiles && ok; ++g) {
+        if (g < n_tiles) {  // S(g) = Q K(g)^T
+          const int st = g & 1;
+          ok = tc_wait(bar(TS_FREE + st), ((g >> 1) & 1) ^ 1, abort_flag, a.status) &&
+               tc_wait(bar(TK_FULL + st), (g >> 1) & 1, abort_flag, a.status);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-  for (int kk = 0; kk < kPDk / 16; ++kk) load_a(Qs, kAKUnits, 16 * warp, 16 * kk, lane, qf[kk]);
-  // this thread's two query rows
-  const int ta = t0 + 16 * warp + g, tb = ta + 8;
-  const int pa = p0 + ta, pb = p0 + tb;
-  float o[kPDv / 8][4];
+          for (int c = 0; c < 3; ++c)
 #pragma unroll
-  for (int j = 0; j < kPDv / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+            for (int k = 0; k < 4; ++k)
+              tc_mma1(tmem + kTColS + 128 * st, qdesc + 1024 * c + 2 * k, kdesc + 3072 * st + 1024 * c + 2 * k, kIdQK,
+                      (c | k) ? 1u : 0u);
+          tc_commit1(bar(TK_EMPTY + st));
+          tc_commit1(bar(TS_FULL + st));
+        }
+        if (g >= 1) {  // O += P(g-1) V(g-1)
+          const int gp = g - 1;
+          ok = tc_wait(bar(TP_FULL), gp & 1, abort_flag, a.status) &&
+               tc_wait(bar(TV_FULL), gp & 1, abort_flag, a.status);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc_mma1(tmem + kTColO, pdesc + 1024 * kc + 2 * k, vdesc + 128 * (4 * kc + k), kIdPV,
+                      (gp | kc | k) ? 1u : 0u);
+          tc_commit1(bar(TV_EMPTY));
+          tc_commit1(bar(TO_DONE));
+        }
+      }
+      tc_commit1(bar(TDRAIN));  // completes once every MMA issued here has finished
+    }
+  } else {
+    // ------------------------------------------- softmax and epilogue, warps 0-3
+    const int i = 32 * warp + lane, t = t0 + i;
+    const int p = p0 + min(t, T - 1);  // rows past the last query repeat its position (not stored)
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int g = 0; g < n_tiles; ++g) {
+      const int st = g & 1;
+      ok = __all_sync(0xffffffffu, tc_wait(bar(TS_FULL + st), (g >> 1) & 1, abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t s_addr = tmem + lane_base + kTColS + 128 * st;
+      const int key0 = kTk * g;
+      // pass 1: the row's tile maximum (log2 units), keys past the query masked
+      float mx = -INFINITY;
 #pragma unroll 1
-  for (int kb = 0; kb < n_kb; ++kb) {
-    if (kb + 1 < n_kb) load_kv((kb + 1) & 1, (kb + 1) * kABk);
-    cp_async_commit();
-    cp_async_wait<1>();
+      for (int q = 0; q < 4; ++q) {
+        uint32_t r[32];
+        tc_ld32(s_addr + 32 * q, r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (key0 + 32 * q + j <= p) mx = fmaxf(mx, __uint_as_float(r[j]));
+      }
+      mx *= a.scale_log2;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (g == 0) {
+        m_ref = mx;  // key 0 is visible to every row
+      } else if (mx > m_ref + kTRescale) {
+        alpha = exp2f(m_ref - mx);
+        m_ref = mx;
+        rescale = true;
+      }
+      // pass 2: probabilities as bf16 pairs
+      uint32_t pk[64];
+      float psum = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t r[32];
+        tc_ld32(s_addr + 32 * q, r);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int k0 = key0 + 32 * q + 2 * j;
+          const float e0 = k0 <= p ? exp2f(__uint_as_float(r[2 * j]) * a.scale_log2 - m_ref) : 0.f;
+          const float e1 = k0 + 1 <= p ? exp2f(__uint_as_float(r[2 * j + 1]) * a.scale_log2 - m_ref) : 0.f;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+          const float2 f2 = __bfloat1622float2(h2);
+          psum += f2.x + f2.y;
+          pk[16 * q + j] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+      }
+      // S(g) is read: the QK MMAs two tiles on may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc_arrive(bar(TS_FREE + st));
+      // P(g-1) and O are in use by PV(g-1) until it completes
+      if (g >= 1) {
+        ok = __all_sync(0xffffffffu, tc_wait(bar(TO_DONE), (g - 1) & 1, abort_flag, a.status));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tc_ld32(tmem + lane_base + kTColO + 32 * c, r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+          tc_st32(tmem + lane_base + kTColO + 32 * c, r);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      }
+      l = l * alpha + psum;
+      // P row i: [2 key blocks][128 rows][128 B], 16-byte units XOR-swizzled by (row & 7)
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(smem + kTOffP + kc * kTChunk + i * 128 + ((u ^ (i & 7)) * 16)) =
+              make_uint4(pk[32 * kc + 4 * u], pk[32 * kc + 4 * u + 1], pk[32 * kc + 4 * u + 2],
+                         pk[32 * kc + 4 * u + 3]);
+      tc_fence_before();    // the rescaled O precedes the next PV MMAs
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P is read by the tensor cores
+      __syncwarp();
+      if (lane == 0) tc_arrive(bar(TP_FULL));
+    }
+    if (ok) {
+      ok = __all_sync(0xffffffffu, tc_wait(bar(TO_DONE), (n_tiles - 1) & 1, abort_flag, a.status));
+      if (ok) {
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16* orow = a.out + (((size_t)b * T + t) * H + h) * kPDv;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tc_ld32(tmem + lane_base + kTColO + 32 * c, r);
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const __nv_bfloat162 v2 =
+                __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * inv, __uint_as_float(r[2 * j + 1]) * inv);
+            w[j] = *reinterpret_cast<const uint32_t*>(&v2);
+          }
+          if (t < T)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              *reinterpret_cast<uint4*>(orow + 32 * c + 8 * u) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
+        if (a.lse_out && t < T) a.lse_out[((size_t)b * T + t) * H + h] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+
+  // teardown: every tensor-memory access finished before deallocation; after
+  // an abort, the MMAs issued so far are waited for (bounded) and copies in
+  // flight are given time to land
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort_flag) {
+    if (threadIdx.x == 0) {
+      const long long c0 = clock64();
+      while (!tc_try_wait(bar(TDRAIN), 0) && clock64() - c0 < 20000000LL) {
+      }
+      const unsigned long long n0 = global_ns();
+      while (global_ns() - n0 < 200000ull) {
+      }
+    }
     __syncthreads();
-    const uint8_t* K = Ks(kb & 1);
-    const uint8_t* Vt = Vs(kb & 1);
-    // scores [16 x 64] of this warp
-    float sc[kABk / 8][4];
-#pragma unroll
-    for (int j = 0; j < kABk / 8; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < kPDk / 16; ++kk)
-#pragma unroll
-      for (int jp = 0; jp < kABk / 16; ++jp) {
-        uint32_t b00, b01, b10, b11;
-        load_b_nk(K, kAKUnits, 16 * kk, 16 * jp, lane, b00, b01, b10, b11);
-        mma_bf16(sc[2 * jp], qf[kk], b00, b01);
-        mma_bf16(sc[2 * jp + 1], qf[kk], b10, b11);
+  }
+  if (warp == kTMmaWarp) {
+    if (lane == 0) {
+      const long long c0 = clock64();
+      while (!tc_try_wait(bar(TDRAIN), 0) && clock64() - c0 < 20000000LL) {
       }
-    // scale to log2 units, causal mask, online softmax (rows ta and tb)
-    const int s0 = kb * kABk;
-    float mxa = -INFINITY, mxb = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < kABk / 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int s = s0 + 8 * j + 2 * qd + e;
-        sc[j][e] = s <= pa && s < S ? sc[j][e] * a.scale_log2 : -INFINITY;
-        sc[j][2 + e] = s <= pb && s < S ? sc[j][2 + e] * a.scale_log2 : -INFINITY;
-        mxa = fmaxf(mxa, sc[j][e]);
-        mxb = fmaxf(mxb, sc[j][2 + e]);
-      }
-#pragma unroll
-    for (int off = 1; off <= 2; off <<= 1) {
-      mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, off));
-      mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, off));
     }
-    const float na = fmaxf(ma, mxa), nb = fmaxf(mb, mxb);
-    // rows with no visible key yet keep a -inf reference: their factors stay 0 / 1
-    const float ra = na == -INFINITY ? 0.f : na, rb = nb == -INFINITY ? 0.f : nb;
-    const float alpha_a = exp2f(ma - ra), alpha_b = exp2f(mb - rb);
-    ma = na;
-    mb = nb;
-    float sa = 0.f, sb = 0.f;
-    uint32_t pf[kABk / 16][4];
-#pragma unroll
-    for (int j = 0; j < kABk / 8; ++j) {
-      const float e0 = exp2f(sc[j][0] - ra), e1 = exp2f(sc[j][1] - ra);
-      const float e2 = exp2f(sc[j][2] - rb), e3 = exp2f(sc[j][3] - rb);
-      const __nv_bfloat162 pa2 = __floats2bfloat162_rn(e0, e1), pb2 = __floats2bfloat162_rn(e2, e3);
-      const float2 fa = __bfloat1622float2(pa2), fb = __bfloat1622float2(pb2);
-      sa += fa.x + fa.y;
-      sb += fb.x + fb.y;
-      // C fragments of n8 tiles 2k and 2k+1 form the A fragment of k16 block k
-      pf[j >> 1][(j & 1) * 2] = *reinterpret_cast<const uint32_t*>(&pa2);
-      pf[j >> 1][(j & 1) * 2 + 1] = *reinterpret_cast<const uint32_t*>(&pb2);
-    }
-    la = la * alpha_a + sa;
-    lb = lb * alpha_b + sb;
-#pragma unroll
-    for (int j = 0; j < kPDv / 8; ++j) {
-      o[j][0] *= alpha_a;
-      o[j][1] *= alpha_a;
-      o[j][2] *= alpha_b;
-      o[j][3] *= alpha_b;
-    }
-    // o += P V: P [16 x 64] (registers) times the value tile [64 x 128]
-#pragma unroll
-    for (int kk = 0; kk < kABk / 16; ++kk)
-#pragma unroll
-      for (int jp = 0; jp < kPDv / 16; ++jp) {
-        uint32_t b00, b01, b10, b11;
-        load_b_kn(Vt, kAVUnits, 16 * kk, 16 * jp, lane, b00, b01, b10, b11);
-        mma_bf16(o[2 * jp], pf[kk], b00, b01);
-        mma_bf16(o[2 * jp + 1], pf[kk], b10, b11);
-      }
-    __syncthreads();  // every warp is done with this stage before it is reloaded
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTTmemCols) : "memory");
   }
-  // the four threads of a row hold disjoint columns: reduce the row sums
-#pragma unroll
-  for (int off = 1; off <= 2; off <<= 1) {
-    la += __shfl_xor_sync(0xffffffffu, la, off);
-    lb += __shfl_xor_sync(0xffffffffu, lb, off);
-  }
-  const float ia = la > 0.f ? 1.f / la : 0.f, ib = lb > 0.f ? 1.f / lb : 0.f;
-#pragma unroll
-  for (int j = 0; j < kPDv / 8; ++j) {
-    const int c = 8 * j + 2 * qd;
-    if (ta < T)
-      *reinterpret_cast<__nv_bfloat162*>(a.out + (((size_t)b * T + ta) * H + h) * kPDv + c) =
-          __floats2bfloat162_rn(o[j][0] * ia, o[j][1] * ia);
-    if (tb < T)
-      *reinterpret_cast<__nv_bfloat162*>(a.out + (((size_t)b * T + tb) * H + h) * kPDv + c) =
-          __floats2bfloat162_rn(o[j][2] * ib, o[j][3] * ib);
-  }
-  if (a.lse_out && qd == 0) {
-    if (ta < T) a.lse_out[((size_t)b * T + ta) * H + h] = la > 0.f ? (ma + log2f(la)) * kLn2 : -INFINITY;
-    if (tb < T) a.lse_out[((size_t)b * T + tb) * H + h] = lb > 0.f ? (mb + log2f(lb)) * kLn2 : -INFINITY;
-  }
+}
+
+// Queries for the tensor-core attention: Qr[h][t] = [q_nope ; RoPE(q_rope, p)]
+// (192 bf16), one warp per (token, head).
+__global__ void __launch_bounds__(256) prefill_q_kernel(const PrefillArgs a, int b, __nv_bfloat16* Qr) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = seq_keys(a, b);
+  const int T = a.n_q, H = a.n_heads;
+  const int row = blockIdx.x * 8 + warp;  // t * H + h
+  if (S < 0 || row >= T * H) return;
+  const int t = row / H, h = row % H;
+  const size_t src = ((size_t)b * T + t) * H + h;
+  __nv_bfloat16* dst = Qr + ((size_t)h * T + t) * kPDk;
+  if (lane < kPDn / 8)
+    reinterpret_cast<uint4*>(dst)[lane] = reinterpret_cast<const uint4*>(a.q_nope + src * kPDn)[lane];
+  const int k = lane;  // rotation pair (k, k + 32)
+  float cs, sn;
+  rope_cos_sin(S - T + t, k, kPDr / 2, a.rope_base, &cs, &sn);
+  const float x1 = __bfloat162float(a.q_rope[src * kPDr + k]), x2 = __bfloat162float(a.q_rope[src * kPDr + k + kPDr / 2]);
+  dst[kPDn + k] = __float2bfloat16_rn(x1 * cs - x2 * sn);
+  dst[kPDn + k + kPDr / 2] = __float2bfloat16_rn(x2 * cs + x1 * sn);
 }
 
 struct PrefillLayout {
-  size_t off_c, off_kr, off_k, off_v, total;
+  size_t off_c, off_kr, off_k, off_v, off_q, total;
+  int max_rows;
 };
 
+// one sequence's latent rows, k^R, per-head keys and values (rows rounded up
+// to whole 128-key tiles) and its rotated queries [H][n_q][192]
 PrefillLayout prefill_layout(const mla_dims& d, int max_seq_len) {
   PrefillLayout L;
+  L.max_rows = (max_seq_len + 127) / 128 * 128;
+  const size_t R = (size_t)L.max_rows;
   size_t off = 0;
   L.off_c = off;
-  off = align_up(off + (size_t)max_seq_len * kPDc * 2, 256);
+  off = align_up(off + R * kPDc * 2, 256);
   L.off_kr = off;
-  off = align_up(off + (size_t)max_seq_len * kPDr * 2, 256);
+  off = align_up(off + R * kPDr * 2, 256);
   L.off_k = off;
-  off = align_up(off + (size_t)d.n_heads * max_seq_len * kPDn * 2, 256);
+  off = align_up(off + (size_t)d.n_heads * R * kPDn * 2, 256);
   L.off_v = off;
-  off = align_up(off + (size_t)d.n_heads * max_seq_len * kPDv * 2, 256);
+  off = align_up(off + (size_t)d.n_heads * R * kPDv * 2, 256);
+  L.off_q = off;
+  off = align_up(off + (size_t)d.n_heads * max_seq_len * kPDk * 2, 256);  // n_q <= max_seq_len
   L.total = off;
   return L;
 }
@@ -435,7 +659,7 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   const PrefillLayout L = prefill_layout(*dims, max_seq_len);
   if (!workspace || ws_bytes < L.total) return MLA_ERR_WORKSPACE;
   if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(W_uk) || !aligned16(W_uv) || !aligned16(cache_pool) ||
-      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(out) & 3u))
+      !aligned16(workspace) || !aligned16(out))
     return MLA_ERR_ALIGNMENT;
   PrefillArgs a;
   a.q_nope = static_cast<const __nv_bfloat16*>(q_nope);
@@ -462,18 +686,32 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse_out = lse_out;
   a.status = device_status_word();
+  a.max_rows = L.max_rows;
+  __nv_bfloat16* Qr = reinterpret_cast<__nv_bfloat16*>(ws + L.off_q);
   cudaStream_t st = (cudaStream_t)stream;
   const size_t gsmem = (size_t)kGStages * kGStageBytes;
   if (cudaFuncSetAttribute(prefill_upproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem) !=
           cudaSuccess ||
-      cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kASmem) !=
+      cudaFuncSetAttribute(prefill_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTSmem) !=
           cudaSuccess)
+    return MLA_ERR_LAUNCH;
+  TcAttnParams tp;
+  memset(&tp, 0, sizeof(tp));
+  tp.a = a;
+  tp.max_rows = L.max_rows;
+  const uint64_t H = (uint64_t)dims->n_heads, R = (uint64_t)L.max_rows;
+  if (!make_tile_map_bf16(&tp.map_q, Qr, kPDk, H * n_q, kPDk * 2, 64, kTq) ||
+      !make_tile_map_bf16(&tp.map_kc, a.Kc, kPDn, H * R, kPDn * 2, 64, kTk) ||
+      !make_tile_map_bf16(&tp.map_kr, a.KR, kPDr, R, kPDr * 2, 64, kTk) ||
+      !make_tile_map_bf16(&tp.map_v, a.V, kPDv, H * R, kPDv * 2, 64, kTk))
     return MLA_ERR_LAUNCH;
   // one sequence at a time: the workspace holds one sequence's keys and values
   for (int b = 0; b < batch; ++b) {
-    prefill_gather_kernel<<<(max_seq_len + 7) / 8, 256, 0, st>>>(a, b);
-    prefill_upproj_kernel<<<dim3(dims->n_heads, (max_seq_len + kGBm - 1) / kGBm, 2), kGThreads, gsmem, st>>>(a, b);
-    prefill_attn_kernel<<<dim3((n_q + kABq - 1) / kABq, dims->n_heads), kAThreads, kASmem, st>>>(a, b);
+    tp.b = b;
+    prefill_gather_kernel<<<L.max_rows / 8, 256, 0, st>>>(a, b);
+    prefill_upproj_kernel<<<dim3(dims->n_heads, L.max_rows / kGBm, 2), kGThreads, gsmem, st>>>(a, b);
+    prefill_q_kernel<<<(n_q * dims->n_heads + 7) / 8, 256, 0, st>>>(a, b, Qr);
+    prefill_attn_tc_kernel<<<dim3((n_q + kTq - 1) / kTq, dims->n_heads), kTThreads, kTSmem, st>>>(tp);
   }
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_LAUNCH;
 }
