@@ -424,18 +424,19 @@ def time_graph_steps(wl: Workload, graphs, steps: int, warmup: int, pg, local: i
     return max_over_ranks(e0.elapsed_time(e1), pg, wl.dev), clocks
 
 
-def timeline_kernel_ms(wl: Workload, steps: int) -> dict:
+def timeline_kernel_ms(wl: Workload, steps: int, capture=None) -> dict:
     """Per-kernel device spans (ms, mean over `steps` steps) from graph replays
     whose kernels stamp %globaltimer into a device timeline (mla_set_timeline):
     the same launches as the timed replays, with the grid-dependency chain
-    between the kernels intact."""
+    between the kernels intact.  `capture` returns the graphs (default: the
+    workload's decode step)."""
     B = wl.B
     nk = len(B.TRACE_KERNELS)
     tl = torch.empty(2 * nk, dtype=torch.int64, device=wl.dev)
     ring = torch.empty(steps, 2 * nk, dtype=torch.int64, device=wl.dev)
     B.mla_set_timeline(tl)
     try:
-        graphs = wl.capture()
+        graphs = (capture or wl.capture)()
     finally:
         B.mla_set_timeline(None)
     for i in range(steps):
@@ -524,8 +525,7 @@ def measure_prefill(cfg, args, dev, peaks: dict) -> dict:
             wl.sess.append(x["h"], wl.seq_idx, wl.pos, w["W_dkv"], w["W_kr"], wl.pt, pool)
         wl.sess.prefill(x["q_nope"], x["q_rope"], w["W_uk"], w["W_uv"], pool, wl.pt, wl.seq_lens, max_len, out, lse)
 
-    res = {}
-    for name, app in (("step", True), ("prefill", False)):
+    def capture(app):
         for i in range(2):
             prefill(i, app)
         torch.cuda.synchronize()
@@ -535,9 +535,15 @@ def measure_prefill(cfg, args, dev, peaks: dict) -> dict:
             with torch.cuda.graph(g):
                 prefill(r, app)
             graphs.append(g)
+        return graphs
+
+    res = {}
+    for name, app in (("step", True), ("prefill", False)):
+        graphs = capture(app)
         ms, clocks = time_graph_steps(wl, graphs, args.steps, args.warmup, None, 0)
         res[name] = (ms / args.steps, clocks)
         del graphs
+    kms = timeline_kernel_ms(wl, max(args.steps, 4), lambda: capture(True))
     wk = prefill_work(cfg)
     t_pf = res["prefill"][0] / 1e3
     tpeak = peaks["bf16_tflops"]
@@ -545,6 +551,9 @@ def measure_prefill(cfg, args, dev, peaks: dict) -> dict:
     return {"ms_per_step": res["step"][0], "tokens_per_s": cfg.B * cfg.T / (res["step"][0] / 1e3),
             "prefill_us": 1e6 * t_pf, "prefill_TFLOPs": flops / t_pf / 1e12,
             "frac_of_tensor_peak": flops / t_pf / 1e12 / tpeak,
+            "kernels_us": {k: round(1e3 * v, 3) for k, v in kms.items()},
+            "upproj_TFLOPs": wk["upproj_flops"] / (kms["prefill_upproj"] / 1e3) / 1e12,
+            "attention_TFLOPs": wk["attention_flops"] / (kms["prefill_attend"] / 1e3) / 1e12,
             "flops": {k: v for k, v in wk.items()}, "clocks": res["step"][1], "l2": wl.l2_note(),
             "form": "non-absorbed (per-head keys and values from the latent), causal"}
 

@@ -256,7 +256,10 @@ enum {
   MLA_TRACE_ABSORB = 2,         /* mla_decode: q~ = W_uk^T q_nope, RoPE(q_rope), split plan */
   MLA_TRACE_ATTEND = 3,         /* mla_decode: split-KV attention over the cache */
   MLA_TRACE_COMBINE = 4,        /* mla_combine: split merge and W_uv */
-  MLA_TRACE_COUNT = 5
+  MLA_TRACE_PREFILL_PREP = 5,   /* mla_prefill: query assembly (RoPE) and latent gather */
+  MLA_TRACE_PREFILL_UPPROJ = 6, /* mla_prefill: per-head keys and values from the latent */
+  MLA_TRACE_PREFILL_ATTEND = 7, /* mla_prefill: causal attention */
+  MLA_TRACE_COUNT = 8
 };
 /* Install a table of 2*MLA_TRACE_COUNT cudaEvent_t (passed as void*, created
  * by the caller with timing enabled): later calls record events[2k] before and

@@ -30,7 +30,8 @@ EXPORTED = ("mla_cache_page_bytes", "mla_check_dims", "mla_append_workspace_byte
             "mla_decode_workspace_bytes", "mla_decode", "mla_combine", "mla_prefill_workspace_bytes",
             "mla_prefill", "mla_decode_path", "mla_auto_splits",
             "mla_set_trace_events", "mla_set_timeline", "mla_get_status", "mla_error_string")
-TRACE_KERNELS = ("append_project", "append_finalize", "absorb", "attend", "combine")
+TRACE_KERNELS = ("append_project", "append_finalize", "absorb", "attend", "combine",
+                 "prefill_prep", "prefill_upproj", "prefill_attend")
 
 
 class MlaDims(ctypes.Structure):

@@ -61,6 +61,7 @@ struct PrefillArgs {
   __nv_bfloat16* out; // [B, T, H, 128]
   float* lse_out;     // [B, T, H] or null
   int* status;
+  unsigned long long* timeline;  // device timeline or null
 };
 
 // Keys of sequence b, or -1 (recorded) when its length is out of range.
@@ -76,10 +77,7 @@ __device__ __forceinline__ int seq_keys(const PrefillArgs& a, int b) {
 // ----------------------------------------------------------------------------
 // 1. gather: one warp per key
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) prefill_gather_kernel(const PrefillArgs a, int b) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = seq_keys(a, b);
-  const int s = blockIdx.x * 8 + warp;
+__device__ __forceinline__ void gather_row(const PrefillArgs& a, int b, int S, int s, int lane) {
   if (S < 0 || s >= (S + 127) / 128 * 128) return;
   uint4* c_dst = reinterpret_cast<uint4*>(a.C + (size_t)s * kPDc);
   uint4* kr_dst = reinterpret_cast<uint4*>(a.KR + (size_t)s * kPDr);
@@ -125,6 +123,12 @@ __global__ void __launch_bounds__(256) prefill_gather_kernel(const PrefillArgs a
     kr_dst[lane] = reinterpret_cast<const uint4*>(pg + fp.kr_off + (size_t)row * kPDr * 2)[lane];
 }
 
+__global__ void __launch_bounds__(256) prefill_gather_kernel(const PrefillArgs a, int b) {
+  tl_begin(a.timeline, MLA_TRACE_PREFILL_PREP);
+  gather_row(a, b, seq_keys(a, b), blockIdx.x * 8 + (threadIdx.x >> 5), threadIdx.x & 31);
+  tl_end(a.timeline, MLA_TRACE_PREFILL_PREP);
+}
+
 // ----------------------------------------------------------------------------
 // 2. up-projection: out[h][s][i] = sum_k C[s][k] W[h][i][k], one head per
 //    128-column tile; blockIdx.z picks W_uk -> Kc or W_uv -> V
@@ -135,6 +139,7 @@ constexpr uint32_t kGStageBytes = (kGBm + kGBn) * kGBk * 2;
 
 __global__ void __launch_bounds__(kGThreads) prefill_upproj_kernel(const PrefillArgs a, int b) {
   extern __shared__ __align__(128) uint8_t smem_g[];
+  tl_begin(a.timeline, MLA_TRACE_PREFILL_UPPROJ);
   const int S = seq_keys(a, b);
   const int h = blockIdx.x, m0 = blockIdx.y * kGBm;
   const int rows = (S + kGBm - 1) / kGBm * kGBm;  // whole 128-key tiles (zero rows past the sequence)
@@ -208,6 +213,7 @@ __global__ void __launch_bounds__(kGThreads) prefill_upproj_kernel(const Prefill
           __floats2bfloat162_rn(acc[i][j][2], acc[i][j][3]);
     }
   }
+  tl_end(a.timeline, MLA_TRACE_PREFILL_UPPROJ);  // CTAs that returned early did so as a whole
 }
 
 // ----------------------------------------------------------------------------
@@ -217,18 +223,20 @@ __global__ void __launch_bounds__(kGThreads) prefill_upproj_kernel(const Prefill
 //      S[128 x 128 keys] = Q[128 x 192] . K^T     (12 MMAs of K = 16)
 //      O[128 x 128]     += P[128 x 128 keys] . V  (8 MMAs of K = 16)
 //    S is double-buffered (columns 0 and 128), O sits in columns 256-383.
-//    Warps 0-3 run the softmax (one query row per thread, a lazily updated
-//    reference max as in the decode: O is rescaled only when a row's tile
-//    maximum exceeds its reference by more than 2^8), write P as bf16 into
-//    shared memory and finish; warp 4 allocates tensor memory and one thread
-//    issues every MMA; warps 5 and 6 bring K and V tiles by TMA (128-byte
+//    Warps 0-7 run the softmax (two threads per query row, each with half
+//    of the tile's keys and half of O's columns; a lazily updated reference
+//    max as in the decode: O is rescaled only when a row's tile maximum
+//    exceeds its reference by more than 2^8), write P as bf16 into shared
+//    memory and finish; warp 8 allocates tensor memory and one thread issues
+//    every MMA; warps 9 and 10 bring K and V tiles by TMA (128-byte
 //    swizzle).  Every wait is bounded; a CTA that gives up records
 //    MLA_ERR_TIMEOUT, waits (bounded) for the MMAs it issued and frees its
 //    tensor memory.
 // ----------------------------------------------------------------------------
 constexpr int kTq = 128, kTk = 128;
-constexpr int kTThreads = 224;
-constexpr int kTMmaWarp = 4, kTKWarp = 5, kTVWarp = 6;
+constexpr int kTSoftThreads = 256;                 // warps 0-7
+constexpr int kTThreads = kTSoftThreads + 96;
+constexpr int kTMmaWarp = 8, kTKWarp = 9, kTVWarp = 10;
 constexpr uint32_t kTChunk = 128 * 128;            // one 64-column block of 128 rows (16 KB)
 constexpr uint32_t kTOffQ = 0;                     // [3][128 queries][128 B]
 constexpr uint32_t kTOffK = kTOffQ + 3 * kTChunk;  // [2 stages][3][128 keys][128 B]
@@ -238,7 +246,8 @@ constexpr uint32_t kTOffBar = kTOffP + 2 * kTChunk;
 enum { TQ_FULL = 0, TK_FULL = 1, TK_EMPTY = 3, TV_FULL = 5, TV_EMPTY = 6, TS_FULL = 7, TS_FREE = 9, TP_FULL = 11,
        TO_DONE = 12, TDRAIN = 13, TNumBars = 14 };
 constexpr uint32_t kTOffMisc = kTOffBar + 8 * TNumBars;
-constexpr size_t kTSmem = kTOffMisc + 16 + 1024;   // + alignment slack
+constexpr uint32_t kTOffRed = kTOffMisc + 16;      // float [2 tiles][2 halves][128 rows] maxima, [2][128] sums
+constexpr size_t kTSmem = kTOffRed + 6 * 128 * 4 + 1024;  // + alignment slack
 constexpr uint32_t kTColS = 0, kTColO = 256, kTTmemCols = 512;
 constexpr long long kTWaitLimit = 4000000000LL;    // ~2 s
 constexpr float kTRescale = 8.0f;                  // log2 units
@@ -303,6 +312,35 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// 32 columns of this warp's 32 lanes, no wait: tc_wait_ld() before reading r
+__device__ __forceinline__ void tc_ld32_nw(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+// 2^x by the MUFU approximation (flushes subnormal results to zero; 2^-inf = 0)
+__device__ __forceinline__ float tc_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Barrier of the softmax warps (named barrier 1) that also ANDs a flag over them.
+__device__ __forceinline__ bool softmax_sync_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kTSoftThreads)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
@@ -332,6 +370,7 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
   const int b = P.b;
   const int S = seq_keys(a, b);
   if (S < 0) return;  // the whole CTA, before any barrier or tensor memory
+  tl_begin(a.timeline, MLA_TRACE_PREFILL_ATTEND);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = a.n_q, H = a.n_heads;
   const int qb = (int)(gridDim.x - 1 - blockIdx.x), h = blockIdx.y;  // heavier (later) query blocks first
@@ -347,11 +386,11 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
       mbar_init_local(bar(TK_FULL + i), 1);
       mbar_init_local(bar(TK_EMPTY + i), 1);
       mbar_init_local(bar(TS_FULL + i), 1);
-      mbar_init_local(bar(TS_FREE + i), 4);
+      mbar_init_local(bar(TS_FREE + i), kTSoftThreads / 32);
     }
     mbar_init_local(bar(TV_FULL), 1);
     mbar_init_local(bar(TV_EMPTY), 1);
-    mbar_init_local(bar(TP_FULL), 4);
+    mbar_init_local(bar(TP_FULL), kTSoftThreads / 32);
     mbar_init_local(bar(TO_DONE), 1);
     mbar_init_local(bar(TDRAIN), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -441,56 +480,66 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
       tc_commit1(bar(TDRAIN));  // completes once every MMA issued here has finished
     }
   } else {
-    // ------------------------------------------- softmax and epilogue, warps 0-3
-    const int i = 32 * warp + lane, t = t0 + i;
+    // --------------------------------------- softmax and epilogue, warps 0-7
+    // Thread (row i, half) owns keys [64 half, 64 half + 64) of every tile and
+    // columns [64 half, 64 half + 64) of O; the two halves of a row share their
+    // maxima and sums through shared memory.  Every exit from the loop passes
+    // the barrier that ANDs the warps' flags, so all 256 threads leave together.
+    const int i = 32 * (warp & 3) + lane, half = warp >> 2, t = t0 + i;
     const int p = p0 + min(t, T - 1);  // rows past the last query repeat its position (not stored)
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    float* red_max = reinterpret_cast<float*>(smem + kTOffRed);  // [2][2][128]
+    float* red_l = red_max + 512;                                // [2][128]
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int g = 0; g < n_tiles; ++g) {
       const int st = g & 1;
-      ok = __all_sync(0xffffffffu, tc_wait(bar(TS_FULL + st), (g >> 1) & 1, abort_flag, a.status));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t s_addr = tmem + lane_base + kTColS + 128 * st;
-      const int key0 = kTk * g;
-      // pass 1: the row's tile maximum (log2 units), keys past the query masked
+      bool okw = ok && __all_sync(0xffffffffu, tc_wait(bar(TS_FULL + st), (g >> 1) & 1, abort_flag, a.status));
+      uint32_t r[64];
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        uint32_t r[32];
-        tc_ld32(s_addr + 32 * q, r);
+      const int kb = kTk * g + 64 * half;  // key of r[0]
+      if (okw) {
+        tc_fence_after();
+        const uint32_t s_addr = tmem + lane_base + kTColS + 128 * st + 64 * half;
+        tc_ld32_nw(s_addr, r);
+        tc_ld32_nw(s_addr + 32, r + 32);
+        tc_wait_ld();
+        if (!__all_sync(0xffffffffu, kb + 63 <= p)) {  // the causal edge: keys past the query score -inf
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (key0 + 32 * q + j <= p) mx = fmaxf(mx, __uint_as_float(r[j]));
+          for (int j = 0; j < 64; ++j)
+            if (kb + j > p) r[j] = 0xFF800000u;
+        }
+        float m8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m8[j] = __uint_as_float(r[j]);
+#pragma unroll
+        for (int j = 8; j < 64; ++j) m8[j & 7] = fmaxf(m8[j & 7], __uint_as_float(r[j]));
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        mx *= a.scale_log2;
       }
-      mx *= a.scale_log2;
+      red_max[(2 * st + half) * 128 + i] = mx;
+      ok = softmax_sync_and(okw);
+      if (!ok) break;
+      const float tile_max = fmaxf(mx, red_max[(2 * st + (half ^ 1)) * 128 + i]);
       float alpha = 1.f;
       bool rescale = false;
       if (g == 0) {
-        m_ref = mx;  // key 0 is visible to every row
-      } else if (mx > m_ref + kTRescale) {
-        alpha = exp2f(m_ref - mx);
-        m_ref = mx;
+        m_ref = tile_max;  // key 0 is visible to every row
+      } else if (tile_max > m_ref + kTRescale) {
+        alpha = tc_exp2(m_ref - tile_max);
+        m_ref = tile_max;
         rescale = true;
       }
-      // pass 2: probabilities as bf16 pairs
-      uint32_t pk[64];
-      float psum = 0.f;
+      // probabilities as bf16 pairs; the row sum in fp32
+      uint32_t pk[32];
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t r[32];
-        tc_ld32(s_addr + 32 * q, r);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int k0 = key0 + 32 * q + 2 * j;
-          const float e0 = k0 <= p ? exp2f(__uint_as_float(r[2 * j]) * a.scale_log2 - m_ref) : 0.f;
-          const float e1 = k0 + 1 <= p ? exp2f(__uint_as_float(r[2 * j + 1]) * a.scale_log2 - m_ref) : 0.f;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-          const float2 f2 = __bfloat1622float2(h2);
-          psum += f2.x + f2.y;
-          pk[16 * q + j] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
+      for (int j = 0; j < 32; ++j) {
+        const float e0 = tc_exp2(fmaf(__uint_as_float(r[2 * j]), a.scale_log2, -m_ref));
+        const float e1 = tc_exp2(fmaf(__uint_as_float(r[2 * j + 1]), a.scale_log2, -m_ref));
+        s4[j & 3] += e0 + e1;
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+        pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
       }
       // S(g) is read: the QK MMAs two tiles on may overwrite it
       tc_fence_before();
@@ -498,59 +547,61 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
       if (lane == 0) tc_arrive(bar(TS_FREE + st));
       // P(g-1) and O are in use by PV(g-1) until it completes
       if (g >= 1) {
-        ok = __all_sync(0xffffffffu, tc_wait(bar(TO_DONE), (g - 1) & 1, abort_flag, a.status));
-        if (!ok) break;
+        if (!__all_sync(0xffffffffu, tc_wait(bar(TO_DONE), (g - 1) & 1, abort_flag, a.status))) {
+          ok = false;  // the next tile's barrier takes every warp out
+          continue;
+        }
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tc_ld32(tmem + lane_base + kTColO + 32 * c, r);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t o[32];
+          const uint32_t o_addr = tmem + lane_base + kTColO + 64 * half + 32 * c;
+          tc_ld32(o_addr, o);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-          tc_st32(tmem + lane_base + kTColO + 32 * c, r);
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tc_st32(o_addr, o);
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       }
-      l = l * alpha + psum;
-      // P row i: [2 key blocks][128 rows][128 B], 16-byte units XOR-swizzled by (row & 7)
+      l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+      // P row i, key block `half`: [2 key blocks][128 rows][128 B], 16-byte units XOR-swizzled by (row & 7)
 #pragma unroll
-      for (int kc = 0; kc < 2; ++kc)
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<uint4*>(smem + kTOffP + kc * kTChunk + i * 128 + ((u ^ (i & 7)) * 16)) =
-              make_uint4(pk[32 * kc + 4 * u], pk[32 * kc + 4 * u + 1], pk[32 * kc + 4 * u + 2],
-                         pk[32 * kc + 4 * u + 3]);
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4*>(smem + kTOffP + half * kTChunk + i * 128 + ((u ^ (i & 7)) * 16)) =
+            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       tc_fence_before();    // the rescaled O precedes the next PV MMAs
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P is read by the tensor cores
       __syncwarp();
       if (lane == 0) tc_arrive(bar(TP_FULL));
     }
-    if (ok) {
-      ok = __all_sync(0xffffffffu, tc_wait(bar(TO_DONE), (n_tiles - 1) & 1, abort_flag, a.status));
-      if (ok) {
-        tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16* orow = a.out + (((size_t)b * T + t) * H + h) * kPDv;
+    bool okf = ok && __all_sync(0xffffffffu, tc_wait(bar(TO_DONE), (n_tiles - 1) & 1, abort_flag, a.status));
+    red_l[half * 128 + i] = l;
+    okf = softmax_sync_and(okf);
+    if (okf) {
+      tc_fence_after();
+      const float lt = l + red_l[(half ^ 1) * 128 + i];
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      __nv_bfloat16* orow = a.out + (((size_t)b * T + t) * H + h) * kPDv + 64 * half;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tc_ld32(tmem + lane_base + kTColO + 32 * c, r);
-          uint32_t w[16];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o[32];
+        tc_ld32(tmem + lane_base + kTColO + 64 * half + 32 * c, o);
+        uint32_t w[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const __nv_bfloat162 v2 =
-                __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * inv, __uint_as_float(r[2 * j + 1]) * inv);
-            w[j] = *reinterpret_cast<const uint32_t*>(&v2);
-          }
-          if (t < T)
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              *reinterpret_cast<uint4*>(orow + 32 * c + 8 * u) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        for (int j = 0; j < 16; ++j) {
+          const __nv_bfloat162 v2 =
+              __floats2bfloat162_rn(__uint_as_float(o[2 * j]) * inv, __uint_as_float(o[2 * j + 1]) * inv);
+          w[j] = *reinterpret_cast<const uint32_t*>(&v2);
         }
-        if (a.lse_out && t < T) a.lse_out[((size_t)b * T + t) * H + h] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+        if (t < T)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * u) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
       }
+      if (half == 0 && a.lse_out && t < T)
+        a.lse_out[((size_t)b * T + t) * H + h] = lt > 0.f ? (m_ref + log2f(lt)) * kLn2 : -INFINITY;
     }
   }
 
@@ -560,6 +611,7 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  tl_end_nosync(a.timeline, MLA_TRACE_PREFILL_ATTEND);
   if (*abort_flag) {
     if (threadIdx.x == 0) {
       const long long c0 = clock64();
@@ -584,12 +636,9 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
 
 // Queries for the tensor-core attention: Qr[h][t] = [q_nope ; RoPE(q_rope, p)]
 // (192 bf16), one warp per (token, head).
-__global__ void __launch_bounds__(256) prefill_q_kernel(const PrefillArgs a, int b, __nv_bfloat16* Qr) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = seq_keys(a, b);
+__device__ __forceinline__ void q_row(const PrefillArgs& a, int b, __nv_bfloat16* Qr, int S, int row, int lane) {
   const int T = a.n_q, H = a.n_heads;
-  const int row = blockIdx.x * 8 + warp;  // t * H + h
-  if (S < 0 || row >= T * H) return;
+  if (S < 0 || row >= T * H) return;  // row = t * H + h
   const int t = row / H, h = row % H;
   const size_t src = ((size_t)b * T + t) * H + h;
   __nv_bfloat16* dst = Qr + ((size_t)h * T + t) * kPDk;
@@ -601,6 +650,12 @@ __global__ void __launch_bounds__(256) prefill_q_kernel(const PrefillArgs a, int
   const float x1 = __bfloat162float(a.q_rope[src * kPDr + k]), x2 = __bfloat162float(a.q_rope[src * kPDr + k + kPDr / 2]);
   dst[kPDn + k] = __float2bfloat16_rn(x1 * cs - x2 * sn);
   dst[kPDn + k + kPDr / 2] = __float2bfloat16_rn(x2 * cs + x1 * sn);
+}
+
+__global__ void __launch_bounds__(256) prefill_q_kernel(const PrefillArgs a, int b, __nv_bfloat16* Qr) {
+  tl_begin(a.timeline, MLA_TRACE_PREFILL_PREP);
+  q_row(a, b, Qr, seq_keys(a, b), blockIdx.x * 8 + (threadIdx.x >> 5), threadIdx.x & 31);
+  tl_end(a.timeline, MLA_TRACE_PREFILL_PREP);
 }
 
 struct PrefillLayout {
@@ -687,6 +742,7 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   a.lse_out = lse_out;
   a.status = device_status_word();
   a.max_rows = L.max_rows;
+  a.timeline = timeline_ptr();
   __nv_bfloat16* Qr = reinterpret_cast<__nv_bfloat16*>(ws + L.off_q);
   cudaStream_t st = (cudaStream_t)stream;
   const size_t gsmem = (size_t)kGStages * kGStageBytes;
@@ -708,10 +764,16 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   // one sequence at a time: the workspace holds one sequence's keys and values
   for (int b = 0; b < batch; ++b) {
     tp.b = b;
-    prefill_gather_kernel<<<L.max_rows / 8, 256, 0, st>>>(a, b);
-    prefill_upproj_kernel<<<dim3(dims->n_heads, L.max_rows / kGBm, 2), kGThreads, gsmem, st>>>(a, b);
+    trace_record(MLA_TRACE_PREFILL_PREP, false, st);
     prefill_q_kernel<<<(n_q * dims->n_heads + 7) / 8, 256, 0, st>>>(a, b, Qr);
+    prefill_gather_kernel<<<L.max_rows / 8, 256, 0, st>>>(a, b);
+    trace_record(MLA_TRACE_PREFILL_PREP, true, st);
+    trace_record(MLA_TRACE_PREFILL_UPPROJ, false, st);
+    prefill_upproj_kernel<<<dim3(dims->n_heads, L.max_rows / kGBm, 2), kGThreads, gsmem, st>>>(a, b);
+    trace_record(MLA_TRACE_PREFILL_UPPROJ, true, st);
+    trace_record(MLA_TRACE_PREFILL_ATTEND, false, st);
     prefill_attn_tc_kernel<<<dim3((n_q + kTq - 1) / kTq, dims->n_heads), kTThreads, kTSmem, st>>>(tp);
+    trace_record(MLA_TRACE_PREFILL_ATTEND, true, st);
   }
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_LAUNCH;
 }
