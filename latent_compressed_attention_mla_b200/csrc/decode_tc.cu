@@ -332,6 +332,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Scores of keys at or past `nvis` (a sub-tile's visible count) set to -inf,
+// so that they drop out of the max and their exponentials are 0.
+__device__ __forceinline__ void mask_scores(uint32_t (&sr)[64], int nvis) {
+  if (nvis < 64) {
+#pragma unroll
+    for (int j = 0; j < 64; ++j)
+      if (j >= nvis) sr[j] = 0xFF800000u;
+  }
+}
+// max of 64 scores in eight independent chains
+__device__ __forceinline__ float max64(const uint32_t (&sr)[64]) {
+  float m8[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m8[j] = __uint_as_float(sr[j]);
+#pragma unroll
+  for (int j = 8; j < 64; ++j) m8[j & 7] = fmaxf(m8[j & 7], __uint_as_float(sr[j]));
+  return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
@@ -1194,10 +1213,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           tmem_ld32(s_addr + 64 * q, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
           tmem_ld32(s_addr + 64 * q + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
           tmem_wait_ld();
-          const int nvq = q ? nv[1] : nv[0];
-#pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (j < nvq) mx = fmaxf(mx, __uint_as_float(sr[j]));
+          mask_scores(sr, q ? nv[1] : nv[0]);
+          mx = fmaxf(mx, max64(sr));
         }
         mx = mx * p.scale_log2;
         red_max[half * 64 + hl] = mx;
@@ -1220,23 +1237,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcLayout<kFp8>::Thre
           tmem_ld32(s_addr + 64 * q, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
           tmem_ld32(s_addr + 64 * q + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
           tmem_wait_ld();
-          const int nvq = q ? nv[1] : nv[0];
+          mask_scores(sr, q ? nv[1] : nv[0]);
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float e0 = 2 * j < nvq ? fast_exp2(__uint_as_float(sr[2 * j]) * p.scale_log2 - m_ref) : 0.f;
-            const float e1 = 2 * j + 1 < nvq ? fast_exp2(__uint_as_float(sr[2 * j + 1]) * p.scale_log2 - m_ref) : 0.f;
+            const float e0 = fast_exp2(__uint_as_float(sr[2 * j]) * p.scale_log2 - m_ref);
+            const float e1 = fast_exp2(__uint_as_float(sr[2 * j + 1]) * p.scale_log2 - m_ref);
             PT h2;
-            float2 f2;
-            if constexpr (kFp8) {
-              h2 = __floats2half2_rn(e0, e1);
-              f2 = __half22float2(h2);
-            } else {
-              h2 = __floats2bfloat162_rn(e0, e1);
-              f2 = __bfloat1622float2(h2);
-            }
-            psum += f2.x + f2.y;
+            if constexpr (kFp8) h2 = __floats2half2_rn(e0, e1);
+            else h2 = __floats2bfloat162_rn(e0, e1);
+            s4[j & 1] += e0;
+            s4[2 + (j & 1)] += e1;
             pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
           }
+          psum += (s4[0] + s4[1]) + (s4[2] + s4[3]);
         };
         // P row hl of sub-tile 2*half + q (64 keys, 128 B per row, 128-byte swizzle)
         auto store_p = [&](int q, const uint32_t(&pk)[32]) {
