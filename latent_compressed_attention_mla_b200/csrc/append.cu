@@ -30,6 +30,7 @@
 
 #include "mla_internal.cuh"
 #include "mma_tile.cuh"
+#include "tc_sm100.cuh"
 
 namespace mla {
 
@@ -73,6 +74,89 @@ __device__ __forceinline__ int token_slot(const AppendArgs& a, int n, int* row, 
   *position = p;
   return page;
 }
+
+// ----------------------------------------------------------------------------
+// Long chunks (hundreds of tokens and more): the projection is a GEMM with
+// M = tokens, [c ; k^R] = h [W_dkv ; W_kr]^T, run on the tcgen05 tensor cores
+// (tc_gemm_kernel) in 128-token x 192-output tiles: outputs [0,192),
+// [192,384) and [384,576), the last holding c 384-511 and all 64 k^R
+// outputs, so that the epilogue rotates each pair (i, i + 32) in registers.
+// d_c = 512, d_rope = 64, bf16 activations, bf16 or FP8 cache.
+// ----------------------------------------------------------------------------
+constexpr int kAgN = 192;
+constexpr int kAgMinTokens = 512;
+
+struct AppendGemm {
+  static constexpr int N = kAgN, Stages = 5;
+  int tiles, k_chunks;
+  int* status;
+  unsigned long long* timeline;
+  int trace;
+  AppendArgs a;
+  int fp8;
+  CUtensorMap map_h;   // h [n_tokens][d_model], box 64 x 128 (rows past n_tokens read as zero)
+  CUtensorMap map_wd;  // W_dkv [512][d_model], box 64 x 64
+  CUtensorMap map_wk;  // W_kr [64][d_model], box 64 x 64
+
+  __device__ bool skip(int) const { return false; }
+  __device__ const CUtensorMap* a_box(int t, int* row) const {
+    *row = 128 * (t / 3);
+    return &map_h;
+  }
+  __device__ const CUtensorMap* b_box(int t, int j, int* row) const {
+    const int r = kAgN * (t % 3) + 64 * j;
+    *row = r < 512 ? r : r - 512;
+    return r < 512 ? &map_wd : &map_wk;
+  }
+  __device__ void epilogue(int t, int r, uint32_t taddr) const {
+    const int n = 128 * (t / 3) + r, nt = t % 3;
+    const bool live = n < a.n_tokens;
+    int prow = 0, position = 0;
+    const int page = live ? token_slot(a, n, &prow, &position) : -1;
+    uint8_t* pg = page >= 0 ? a.pool + (size_t)page * a.page_bytes : nullptr;
+    const int n_c = nt < 2 ? 6 : 4;  // 32-column chunks of c in this tile
+#pragma unroll 1
+    for (int c4 = 0; c4 < n_c; ++c4) {
+      uint32_t v[32];
+      tc_ld32(taddr + 32 * c4, v);  // whole-warp: every lane loads, live or not
+      if (!pg) continue;
+      const int col = kAgN * nt + 32 * c4;
+      if (fp8) {
+        float4* dst = reinterpret_cast<float4*>(a.raw + (size_t)n * 512 + col);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          dst[u] = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]), __uint_as_float(v[4 * u + 2]),
+                               __uint_as_float(v[4 * u + 3]));
+      } else {
+        uint32_t w[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+          w[j] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(pg + ((size_t)prow * 576 + col) * 2);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      }
+    }
+    if (nt != 2) return;
+    // k^R: pair (i, i + 32) rotated by the angle of the token's position; one
+    // TMEM column of each at a time keeps the rolled loop in registers
+    const Fp8Page fp = fp8_page(a.page_size, 512, 64);
+    __nv_bfloat16* kr = !pg ? nullptr
+                        : fp8 ? reinterpret_cast<__nv_bfloat16*>(pg + fp.kr_off) + (size_t)prow * 64
+                              : reinterpret_cast<__nv_bfloat16*>(pg) + (size_t)prow * 576 + 512;
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+      const float x1 = __uint_as_float(tc_ld1(taddr + 128 + i)), x2 = __uint_as_float(tc_ld1(taddr + 160 + i));
+      if (!kr) continue;
+      float cs, sn;
+      rope_cos_sin(position, i, 32, a.rope_base, &cs, &sn);
+      kr[i] = __float2bfloat16_rn(x1 * cs - x2 * sn);
+      kr[i + 32] = __float2bfloat16_rn(x2 * cs + x1 * sn);
+    }
+  }
+};
 
 template <typename T> struct Vec;
 template <> struct Vec<__nv_bfloat16> { static constexpr int n = 8; };
@@ -594,8 +678,33 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
                     d.d_model % 8 == 0 && d.d_model <= kGvThreads * kGvVec * 8 && d.d_c % kGvCols == 0 &&
                     d.d_rope % kGvCols == 0 && (reinterpret_cast<uintptr_t>(h) & 15u) == 0 &&
                     (reinterpret_cast<uintptr_t>(W_dkv) & 15u) == 0 && (reinterpret_cast<uintptr_t>(W_kr) & 15u) == 0;
+  const bool big = d.act_dtype == MLA_BF16 && (d.cache_dtype == MLA_BF16 || d.cache_dtype == MLA_FP8_E4M3) &&
+                   d.d_c == 512 && d.d_rope == 64 && d.d_model % 64 == 0 && n_tokens >= kAgMinTokens &&
+                   (reinterpret_cast<uintptr_t>(h) & 15u) == 0 && (reinterpret_cast<uintptr_t>(W_dkv) & 15u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(W_kr) & 15u) == 0;
   cudaError_t launch_err = cudaSuccess;
-  if (gemv) {
+  if (big) {
+    AppendGemm g;
+    memset(&g, 0, sizeof(g));
+    g.a = a;
+    g.fp8 = d.cache_dtype == MLA_FP8_E4M3;
+    g.tiles = (n_tokens + 127) / 128 * 3;
+    g.k_chunks = d.d_model / 64;
+    g.status = status;
+    g.timeline = a.timeline;
+    g.trace = MLA_TRACE_APPEND_PROJECT;
+    const uint64_t row_bytes = (uint64_t)d.d_model * 2;
+    if (!make_tile_map_bf16(&g.map_h, h, d.d_model, n_tokens, row_bytes, 64, 128) ||
+        !make_tile_map_bf16(&g.map_wd, W_dkv, d.d_model, 512, row_bytes, 64, 64) ||
+        !make_tile_map_bf16(&g.map_wk, W_kr, d.d_model, 64, row_bytes, 64, 64))
+      return cudaErrorInvalidValue;
+    constexpr size_t smem = tc_gemm_smem<AppendGemm>();
+    launch_err = cudaFuncSetAttribute(tc_gemm_kernel<AppendGemm>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem);
+    if (launch_err == cudaSuccess)
+      launch_err = launch_pdl(tc_gemm_kernel<AppendGemm>, dim3(g.tiles < device_sm_count() ? g.tiles : device_sm_count()),
+                              dim3(kGemmThreads), smem, st, g);
+  } else if (gemv) {
     const dim3 ggrid((d.d_c + d.d_rope) / kGvCols);
     const bool fp8 = d.cache_dtype == MLA_FP8_E4M3;
     if (n_tokens == 1)

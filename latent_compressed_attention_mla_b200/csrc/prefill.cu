@@ -19,9 +19,10 @@
 //   1. gather: the sequence's latent rows c_s (dequantised for an FP8 cache)
 //      and k^R_s, from the paged cache into contiguous bf16 rows, zero up to
 //      the next multiple of 128 keys;
-//   2. up-projection: K^C = C W_uk^T and V = C W_uv^T, mma.sync GEMMs whose
-//      128 x 128 output tiles are one head's keys, written head-major
-//      [head][key][128] so that an attention tile is one contiguous block;
+//   2. up-projection: K^C = C W_uk^T and V = C W_uv^T, a tcgen05 GEMM whose
+//      128 x 256 output tiles are one head's keys and values, written
+//      head-major [head][key][128] so that an attention tile is one
+//      contiguous block;
 //   3. queries: [q_nope ; RoPE(q_rope, p)] per (head, token), head-major;
 //   4. attention on the tensor cores (tcgen05, accumulators in tensor memory),
 //      one CTA per (head, block of 128 queries); see below.
@@ -29,6 +30,7 @@
 
 #include "mla_internal.cuh"
 #include "mma_tile.cuh"
+#include "tc_sm100.cuh"
 
 namespace mla {
 
@@ -130,91 +132,56 @@ __global__ void __launch_bounds__(256) prefill_gather_kernel(const PrefillArgs a
 }
 
 // ----------------------------------------------------------------------------
-// 2. up-projection: out[h][s][i] = sum_k C[s][k] W[h][i][k], one head per
-//    128-column tile; blockIdx.z picks W_uk -> Kc or W_uv -> V
+// 2. up-projection on the tcgen05 tensor cores (tc_gemm_kernel): per 128-key
+//    row block m and head h, one 128 x 256 tile [K^C | V] = C [W_uk[h]; W_uv[h]]^T
+//    (K = 512), written head-major [head][key][128] so that an attention tile
+//    is one contiguous block.  Row blocks past the sequence's last 128-key
+//    tile are left out.
 // ----------------------------------------------------------------------------
-constexpr int kGBm = 128, kGBn = 128, kGBk = 64, kGStages = 3, kGThreads = 256;
-constexpr int kGRowUnits = kGBk / 8;  // 16-byte units per staged row
-constexpr uint32_t kGStageBytes = (kGBm + kGBn) * kGBk * 2;
+struct UpProjGemm {
+  static constexpr int N = 256, Stages = 4;
+  int tiles, k_chunks;
+  int* status;
+  unsigned long long* timeline;
+  int trace;
+  PrefillArgs a;
+  int b;
+  CUtensorMap map_c;   // C [max_rows][512], box 64 x 128
+  CUtensorMap map_wk;  // W_uk [H * 128][512], box 64 x 64
+  CUtensorMap map_wv;  // W_uv [H * 128][512], box 64 x 64
 
-__global__ void __launch_bounds__(kGThreads) prefill_upproj_kernel(const PrefillArgs a, int b) {
-  extern __shared__ __align__(128) uint8_t smem_g[];
-  tl_begin(a.timeline, MLA_TRACE_PREFILL_UPPROJ);
-  const int S = seq_keys(a, b);
-  const int h = blockIdx.x, m0 = blockIdx.y * kGBm;
-  const int rows = (S + kGBm - 1) / kGBm * kGBm;  // whole 128-key tiles (zero rows past the sequence)
-  if (S < 0 || m0 >= rows) return;
-  const bool is_v = blockIdx.z == 1;
-  const __nv_bfloat16* W = (is_v ? a.W_uv : a.W_uk) + (size_t)h * kPDn * kPDc;
-  __nv_bfloat16* out = (is_v ? a.V : a.Kc) + (size_t)h * a.max_rows * kPDn;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wm = warp >> 2, wn = warp & 3;  // warp tile: rows 64 wm .. +64, columns 32 wn .. +32
-  auto stage_a = [&](int st) { return smem_g + st * kGStageBytes; };
-  auto stage_b = [&](int st) { return smem_g + st * kGStageBytes + kGBm * kGBk * 2; };
-  auto load_stage = [&](int st, int k0) {
-    uint8_t* As = stage_a(st);
-    uint8_t* Bs = stage_b(st);
-    for (int i = tid; i < kGBm * kGRowUnits; i += kGThreads) {
-      const int r = i / kGRowUnits, u = i % kGRowUnits;
-      cp_async16(smem_addr(As) + swz(r, u, kGRowUnits), a.C + (size_t)(m0 + r) * kPDc + k0 + u * 8);
-    }
-    for (int i = tid; i < kGBn * kGRowUnits; i += kGThreads) {
-      const int r = i / kGRowUnits, u = i % kGRowUnits;
-      cp_async16(smem_addr(Bs) + swz(r, u, kGRowUnits), W + (size_t)r * kPDc + k0 + u * 8);
-    }
-  };
-  float acc[4][4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
-  constexpr int nk = kPDc / kGBk;  // 8
-#pragma unroll
-  for (int st = 0; st < kGStages - 1; ++st) {
-    load_stage(st, st * kGBk);
-    cp_async_commit();
+  __device__ bool skip(int t) const {
+    const int S = a.seq_lens[b];
+    const bool ok = S >= a.n_q && S <= a.max_seq_len && (long long)S <= (long long)a.max_pages * kPPage;
+    return !ok || 128 * (t / a.n_heads) >= S;  // the gather records a bad length
   }
+  __device__ const CUtensorMap* a_box(int t, int* row) const {
+    *row = 128 * (t / a.n_heads);
+    return &map_c;
+  }
+  __device__ const CUtensorMap* b_box(int t, int j, int* row) const {
+    *row = 128 * (t % a.n_heads) + 64 * (j & 1);
+    return j < 2 ? &map_wk : &map_wv;
+  }
+  __device__ void epilogue(int t, int r, uint32_t taddr) const {
+    const int h = t % a.n_heads, s = 128 * (t / a.n_heads) + r;
 #pragma unroll 1
-  for (int kt = 0; kt < nk; ++kt) {
-    cp_async_wait<kGStages - 2>();
-    __syncthreads();  // stage kt landed; every warp is done with stage kt - 1
-    if (kt + kGStages - 1 < nk) load_stage((kt + kGStages - 1) % kGStages, (kt + kGStages - 1) * kGBk);
-    cp_async_commit();
-    const uint8_t* As = stage_a(kt % kGStages);
-    const uint8_t* Bs = stage_b(kt % kGStages);
+    for (int c = 0; c < 8; ++c) {  // 32-column chunks: 0-3 K^C, 4-7 V
+      uint32_t v[32];
+      tc_ld32(taddr + 32 * c, v);
+      uint32_t w[16];
 #pragma unroll
-    for (int kk = 0; kk < kGBk; kk += 16) {
-      uint32_t af[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) load_a(As, kGRowUnits, 64 * wm + 16 * i, kk, lane, af[i]);
-#pragma unroll
-      for (int jp = 0; jp < 2; ++jp) {
-        uint32_t b00, b01, b10, b11;
-        load_b_nk(Bs, kGRowUnits, kk, 32 * wn + 16 * jp, lane, b00, b01, b10, b11);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          mma_bf16(acc[i][2 * jp], af[i], b00, b01);
-          mma_bf16(acc[i][2 * jp + 1], af[i], b10, b11);
-        }
+      for (int j = 0; j < 16; ++j) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+        w[j] = *reinterpret_cast<const uint32_t*>(&b2);
       }
+      __nv_bfloat16* out = (c < 4 ? a.Kc : a.V) + ((size_t)h * a.max_rows + s) * kPDn + 32 * (c & 3);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        reinterpret_cast<uint4*>(out)[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
     }
   }
-  // bf16 rows [h][s][128]
-  const int g = lane >> 2, q = lane & 3;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r0 = m0 + 64 * wm + 16 * i + g;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = 32 * wn + 8 * j + 2 * q;
-      *reinterpret_cast<__nv_bfloat162*>(out + (size_t)r0 * kPDn + c) =
-          __floats2bfloat162_rn(acc[i][j][0], acc[i][j][1]);
-      *reinterpret_cast<__nv_bfloat162*>(out + (size_t)(r0 + 8) * kPDn + c) =
-          __floats2bfloat162_rn(acc[i][j][2], acc[i][j][3]);
-    }
-  }
-  tl_end(a.timeline, MLA_TRACE_PREFILL_UPPROJ);  // CTAs that returned early did so as a whole
-}
+};
 
 // ----------------------------------------------------------------------------
 // 3. attention on the 5th-generation tensor cores: one CTA per (head, block of
@@ -249,7 +216,6 @@ constexpr uint32_t kTOffMisc = kTOffBar + 8 * TNumBars;
 constexpr uint32_t kTOffRed = kTOffMisc + 16;      // float [2 tiles][2 halves][128 rows] maxima, [2][128] sums
 constexpr size_t kTSmem = kTOffRed + 6 * 128 * 4 + 1024;  // + alignment slack
 constexpr uint32_t kTColS = 0, kTColO = 256, kTTmemCols = 512;
-constexpr long long kTWaitLimit = 4000000000LL;    // ~2 s
 constexpr float kTRescale = 8.0f;                  // log2 units
 
 struct TcAttnParams {
@@ -261,76 +227,6 @@ struct TcAttnParams {
   CUtensorMap map_v;     // V  [H * max_rows][128], box 64 x 128
 };
 
-__device__ __forceinline__ bool tc_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: false (MLA_ERR_TIMEOUT recorded once) on expiry, or at once
-// when another role of the CTA already gave up.
-__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
-  if (tc_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (tc_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kTWaitLimit) {
-      *abort_flag = 1;
-      record_status(status, MLA_ERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-__device__ __forceinline__ void tc_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_mma1(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
-      : "memory");
-}
-// arrive on a barrier of this CTA once the MMAs this thread issued so far complete
-__device__ __forceinline__ void tc_commit1(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-// 32 columns of this warp's 32 lanes, no wait: tc_wait_ld() before reading r
-__device__ __forceinline__ void tc_ld32_nw(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-}
-// 2^x by the MUFU approximation (flushes subnormal results to zero; 2^-inf = 0)
-__device__ __forceinline__ float tc_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 // Barrier of the softmax warps (named barrier 1) that also ANDs a flag over them.
 __device__ __forceinline__ bool softmax_sync_and(bool v) {
   uint32_t r;
@@ -341,27 +237,6 @@ __device__ __forceinline__ bool softmax_sync_and(bool v) {
       : "memory");
   return r != 0;
 }
-__device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
-      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
-      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-// shared-memory matrix descriptor, 128-byte swizzle (sm_100 version field)
-__device__ __forceinline__ uint64_t tc_sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// instruction descriptor: kind::f16 with bf16 operands, f32 accumulator, dense
-constexpr uint32_t tc_idesc_bf16(int M, int N, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
 __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __grid_constant__ TcAttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -745,8 +620,8 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   a.timeline = timeline_ptr();
   __nv_bfloat16* Qr = reinterpret_cast<__nv_bfloat16*>(ws + L.off_q);
   cudaStream_t st = (cudaStream_t)stream;
-  const size_t gsmem = (size_t)kGStages * kGStageBytes;
-  if (cudaFuncSetAttribute(prefill_upproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem) !=
+  constexpr size_t gsmem = tc_gemm_smem<UpProjGemm>();
+  if (cudaFuncSetAttribute(tc_gemm_kernel<UpProjGemm>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem) !=
           cudaSuccess ||
       cudaFuncSetAttribute(prefill_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTSmem) !=
           cudaSuccess)
@@ -756,6 +631,19 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   tp.a = a;
   tp.max_rows = L.max_rows;
   const uint64_t H = (uint64_t)dims->n_heads, R = (uint64_t)L.max_rows;
+  UpProjGemm up;
+  memset(&up, 0, sizeof(up));
+  up.a = a;
+  up.tiles = L.max_rows / 128 * dims->n_heads;
+  up.k_chunks = kPDc / 64;
+  up.status = a.status;
+  up.timeline = a.timeline;
+  up.trace = MLA_TRACE_PREFILL_UPPROJ;
+  if (!make_tile_map_bf16(&up.map_c, a.C, kPDc, R, kPDc * 2, 64, 128) ||
+      !make_tile_map_bf16(&up.map_wk, a.W_uk, kPDc, H * kPDn, kPDc * 2, 64, 64) ||
+      !make_tile_map_bf16(&up.map_wv, a.W_uv, kPDc, H * kPDv, kPDc * 2, 64, 64))
+    return MLA_ERR_LAUNCH;
+  const int up_grid = up.tiles < device_sm_count() ? up.tiles : device_sm_count();
   if (!make_tile_map_bf16(&tp.map_q, Qr, kPDk, H * n_q, kPDk * 2, 64, kTq) ||
       !make_tile_map_bf16(&tp.map_kc, a.Kc, kPDn, H * R, kPDn * 2, 64, kTk) ||
       !make_tile_map_bf16(&tp.map_kr, a.KR, kPDr, R, kPDr * 2, 64, kTk) ||
@@ -769,7 +657,8 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
     prefill_gather_kernel<<<L.max_rows / 8, 256, 0, st>>>(a, b);
     trace_record(MLA_TRACE_PREFILL_PREP, true, st);
     trace_record(MLA_TRACE_PREFILL_UPPROJ, false, st);
-    prefill_upproj_kernel<<<dim3(dims->n_heads, L.max_rows / kGBm, 2), kGThreads, gsmem, st>>>(a, b);
+    up.b = b;
+    tc_gemm_kernel<UpProjGemm><<<up_grid, kGemmThreads, gsmem, st>>>(up);
     trace_record(MLA_TRACE_PREFILL_UPPROJ, true, st);
     trace_record(MLA_TRACE_PREFILL_ATTEND, false, st);
     prefill_attn_tc_kernel<<<dim3((n_q + kTq - 1) / kTq, dims->n_heads), kTThreads, kTSmem, st>>>(tp);
