@@ -571,6 +571,15 @@ def config_entry(cfg, m: dict, world: int) -> dict:
             "l2": m["wl"].l2_note(), "clocks": m["clocks"]}
 
 
+def prefill_only(args):
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    n = args.prefill
+    cfg = WL.V3_PREFILL_CHUNK.with_(name=f"v3-prefill-l{n}-t{n}", T=n, L=(n,))
+    res = measure_prefill(cfg, args, dev, load_peaks())
+    print(json.dumps({"workload": cfg.name, **res}), flush=True)
+
+
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
@@ -595,7 +604,12 @@ def main():
     ap.add_argument("--context", type=int, default=0,
                     help="cache every sequence with this many tokens before the step instead (a smaller case of "
                          "the same batch and kernels, e.g. for profiler captures); the workload name records it")
+    ap.add_argument("--prefill", type=int, default=0,
+                    help="time only a prefill chunk of N new tokens over N cached tokens (a smaller case of the "
+                         "prefill kernels, e.g. for profiler captures) and print that measurement alone")
     args = ap.parse_args()
+    if args.prefill > 0:
+        return prefill_only(args)
     cfg = WL.CONFIGS[args.config]
     if 0 < args.batch < cfg.B:
         cfg = cfg.with_(name=f"{cfg.name}[:{args.batch}]", B=args.batch, L=tuple(cfg.L[:args.batch]))

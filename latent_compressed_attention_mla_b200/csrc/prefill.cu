@@ -510,26 +510,33 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
 }
 
 // Queries for the tensor-core attention: Qr[h][t] = [q_nope ; RoPE(q_rope, p)]
-// (192 bf16), one warp per (token, head).
-__device__ __forceinline__ void q_row(const PrefillArgs& a, int b, __nv_bfloat16* Qr, int S, int row, int lane) {
-  const int T = a.n_q, H = a.n_heads;
-  if (S < 0 || row >= T * H) return;  // row = t * H + h
-  const int t = row / H, h = row % H;
-  const size_t src = ((size_t)b * T + t) * H + h;
-  __nv_bfloat16* dst = Qr + ((size_t)h * T + t) * kPDk;
-  if (lane < kPDn / 8)
-    reinterpret_cast<uint4*>(dst)[lane] = reinterpret_cast<const uint4*>(a.q_nope + src * kPDn)[lane];
-  const int k = lane;  // rotation pair (k, k + 32)
-  float cs, sn;
-  rope_cos_sin(S - T + t, k, kPDr / 2, a.rope_base, &cs, &sn);
-  const float x1 = __bfloat162float(a.q_rope[src * kPDr + k]), x2 = __bfloat162float(a.q_rope[src * kPDr + k + kPDr / 2]);
-  dst[kPDn + k] = __float2bfloat16_rn(x1 * cs - x2 * sn);
-  dst[kPDn + k + kPDr / 2] = __float2bfloat16_rn(x2 * cs + x1 * sn);
-}
-
+// (192 bf16).  One CTA per new token t: the 32 RoPE angles of its position are
+// formed once (warp 0) and applied to every head (warp w takes heads w, w + 8, ...).
 __global__ void __launch_bounds__(256) prefill_q_kernel(const PrefillArgs a, int b, __nv_bfloat16* Qr) {
   tl_begin(a.timeline, MLA_TRACE_PREFILL_PREP);
-  q_row(a, b, Qr, seq_keys(a, b), blockIdx.x * 8 + (threadIdx.x >> 5), threadIdx.x & 31);
+  __shared__ float2 cs_sn[kPDr / 2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = seq_keys(a, b);
+  const int T = a.n_q, H = a.n_heads, t = blockIdx.x;
+  if (S >= 0 && warp == 0) {
+    float cs, sn;
+    rope_cos_sin(S - T + t, lane, kPDr / 2, a.rope_base, &cs, &sn);  // pair (lane, lane + 32)
+    cs_sn[lane] = make_float2(cs, sn);
+  }
+  __syncthreads();
+  if (S >= 0) {
+    const float2 r = cs_sn[lane];
+    for (int h = warp; h < H; h += 8) {
+      const size_t src = ((size_t)b * T + t) * H + h;
+      __nv_bfloat16* dst = Qr + ((size_t)h * T + t) * kPDk;
+      if (lane < kPDn / 8)
+        reinterpret_cast<uint4*>(dst)[lane] = reinterpret_cast<const uint4*>(a.q_nope + src * kPDn)[lane];
+      const float x1 = __bfloat162float(a.q_rope[src * kPDr + lane]);
+      const float x2 = __bfloat162float(a.q_rope[src * kPDr + lane + kPDr / 2]);
+      dst[kPDn + lane] = __float2bfloat16_rn(x1 * r.x - x2 * r.y);
+      dst[kPDn + lane + kPDr / 2] = __float2bfloat16_rn(x2 * r.x + x1 * r.y);
+    }
+  }
   tl_end(a.timeline, MLA_TRACE_PREFILL_PREP);
 }
 
@@ -653,7 +660,7 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   for (int b = 0; b < batch; ++b) {
     tp.b = b;
     trace_record(MLA_TRACE_PREFILL_PREP, false, st);
-    prefill_q_kernel<<<(n_q * dims->n_heads + 7) / 8, 256, 0, st>>>(a, b, Qr);
+    prefill_q_kernel<<<n_q, 256, 0, st>>>(a, b, Qr);
     prefill_gather_kernel<<<L.max_rows / 8, 256, 0, st>>>(a, b);
     trace_record(MLA_TRACE_PREFILL_PREP, true, st);
     trace_record(MLA_TRACE_PREFILL_UPPROJ, false, st);
