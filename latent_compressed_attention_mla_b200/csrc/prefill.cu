@@ -194,28 +194,29 @@ struct UpProjGemm {
 //    of the tile's keys and half of O's columns; a lazily updated reference
 //    max as in the decode: O is rescaled only when a row's tile maximum
 //    exceeds its reference by more than 2^8), write P as bf16 into shared
-//    memory and finish; warp 8 allocates tensor memory and one thread issues
-//    every MMA; warps 9 and 10 bring K and V tiles by TMA (128-byte
-//    swizzle).  Every wait is bounded; a CTA that gives up records
+//    memory and finish; warp 8 allocates tensor memory and one of its
+//    threads issues the QK MMAs, one thread of warp 11 the PV MMAs; warps 9
+//    and 10 bring K and V tiles by TMA (128-byte swizzle).  Every wait is bounded; a CTA that gives up records
 //    MLA_ERR_TIMEOUT, waits (bounded) for the MMAs it issued and frees its
 //    tensor memory.
 // ----------------------------------------------------------------------------
 constexpr int kTq = 128, kTk = 128;
 constexpr int kTSoftThreads = 256;                 // warps 0-7
-constexpr int kTThreads = kTSoftThreads + 96;
-constexpr int kTMmaWarp = 8, kTKWarp = 9, kTVWarp = 10;
+constexpr int kTThreads = kTSoftThreads + 128;
+constexpr int kTMmaWarp = 8, kTKWarp = 9, kTVWarp = 10, kTPvWarp = 11;  // kTMmaWarp: TMEM + QK MMAs
 constexpr uint32_t kTChunk = 128 * 128;            // one 64-column block of 128 rows (16 KB)
 constexpr uint32_t kTOffQ = 0;                     // [3][128 queries][128 B]
 constexpr uint32_t kTOffK = kTOffQ + 3 * kTChunk;  // [2 stages][3][128 keys][128 B]
 constexpr uint32_t kTOffV = kTOffK + 6 * kTChunk;  // [2 column halves][128 keys][128 B]
 constexpr uint32_t kTOffP = kTOffV + 2 * kTChunk;  // [2 key blocks][128 queries][128 B]
 constexpr uint32_t kTOffBar = kTOffP + 2 * kTChunk;
+// TP_FULL / TO_DONE: one per key half (the half's P written / its PV MMAs done)
 enum { TQ_FULL = 0, TK_FULL = 1, TK_EMPTY = 3, TV_FULL = 5, TV_EMPTY = 6, TS_FULL = 7, TS_FREE = 9, TP_FULL = 11,
-       TO_DONE = 12, TDRAIN = 13, TNumBars = 14 };
+       TO_DONE = 13, TDRAIN = 15, TNumBars = 16 };
 constexpr uint32_t kTOffMisc = kTOffBar + 8 * TNumBars;
-constexpr uint32_t kTOffRed = kTOffMisc + 16;      // float [2 tiles][2 halves][128 rows] maxima, [2][128] sums
-constexpr size_t kTSmem = kTOffRed + 6 * 128 * 4 + 1024;  // + alignment slack
-constexpr uint32_t kTColS = 0, kTColO = 256, kTTmemCols = 512;
+constexpr uint32_t kTOffRed = kTOffMisc + 16;      // float [2 halves][128 rows] maxima, then sums
+constexpr size_t kTSmem = kTOffRed + 4 * 128 * 4 + 1024;  // + alignment slack
+constexpr uint32_t kTColS = 0, kTColO = 256, kTTmemCols = 512;  // S: 0 and 128; O of key half h: 256 + 128 h
 constexpr float kTRescale = 8.0f;                  // log2 units
 
 struct TcAttnParams {
@@ -265,9 +266,11 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
     }
     mbar_init_local(bar(TV_FULL), 1);
     mbar_init_local(bar(TV_EMPTY), 1);
-    mbar_init_local(bar(TP_FULL), kTSoftThreads / 32);
-    mbar_init_local(bar(TO_DONE), 1);
-    mbar_init_local(bar(TDRAIN), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init_local(bar(TP_FULL + i), kTSoftThreads / 64);
+      mbar_init_local(bar(TO_DONE + i), 1);
+    }
+    mbar_init_local(bar(TDRAIN), 2);  // one final commit per MMA issuer
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kTMmaWarp) {
@@ -312,106 +315,113 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
       }
     }
   } else if (warp == kTMmaWarp) {
-    // ---------------------------------------------------------------- MMAs
+    // ------------------------------------------------------ QK MMAs: S = Q K^T
+    // Two issuing threads (QK here, PV in warp 11): an issue holds its thread
+    // until the tensor pipe takes the MMA, and each issuer's barrier waits,
+    // fences and commits overlap the other's MMAs.
     if (lane == 0) {
-      constexpr uint32_t kIdQK = tc_idesc_bf16(128, 128, false), kIdPV = tc_idesc_bf16(128, 128, true);
+      constexpr uint32_t kIdQK = tc_idesc_bf16(128, 128, false);
       const uint64_t qdesc = tc_sdesc(sbase + kTOffQ, 16, 1024);   // chunk c: + 1024 c; K step: + 2
       const uint64_t kdesc = tc_sdesc(sbase + kTOffK, 16, 1024);   // stage: + 3072; chunk: + 1024
-      const uint64_t pdesc = tc_sdesc(sbase + kTOffP, 16, 1024);   // key block: + 1024; K step: + 2
-      const uint64_t vdesc = tc_sdesc(sbase + kTOffV, kTChunk, 1024);  // 16 keys: + 128
       bool ok = tc_wait(bar(TQ_FULL), 0, abort_flag, a.status);
-      for (int g = 0; g <= n_tiles && ok; ++g) {
-        if (g < n_tiles) {  // S(g) = Q K(g)^T
-          const int st = g & 1;
-          ok = tc_wait(bar(TS_FREE + st), ((g >> 1) & 1) ^ 1, abort_flag, a.status) &&
-               tc_wait(bar(TK_FULL + st), (g >> 1) & 1, abort_flag, a.status);
-          if (!ok) break;
-          tc_fence_after();
+      for (int g = 0; g < n_tiles && ok; ++g) {
+        const int st = g & 1;
+        ok = tc_wait(bar(TS_FREE + st), ((g >> 1) & 1) ^ 1, abort_flag, a.status) &&
+             tc_wait(bar(TK_FULL + st), (g >> 1) & 1, abort_flag, a.status);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 3; ++c)
+        for (int c = 0; c < 3; ++c)
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              tc_mma1(tmem + kTColS + 128 * st, qdesc + 1024 * c + 2 * k, kdesc + 3072 * st + 1024 * c + 2 * k, kIdQK,
-                      (c | k) ? 1u : 0u);
-          tc_commit1(bar(TK_EMPTY + st));
-          tc_commit1(bar(TS_FULL + st));
-        }
-        if (g >= 1) {  // O += P(g-1) V(g-1)
-          const int gp = g - 1;
-          ok = tc_wait(bar(TP_FULL), gp & 1, abort_flag, a.status) &&
-               tc_wait(bar(TV_FULL), gp & 1, abort_flag, a.status);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kc = 0; kc < 2; ++kc)
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              tc_mma1(tmem + kTColO, pdesc + 1024 * kc + 2 * k, vdesc + 128 * (4 * kc + k), kIdPV,
-                      (gp | kc | k) ? 1u : 0u);
-          tc_commit1(bar(TV_EMPTY));
-          tc_commit1(bar(TO_DONE));
-        }
+          for (int k = 0; k < 4; ++k)
+            tc_mma1(tmem + kTColS + 128 * st, qdesc + 1024 * c + 2 * k, kdesc + 3072 * st + 1024 * c + 2 * k, kIdQK,
+                    (c | k) ? 1u : 0u);
+        tc_commit1(bar(TK_EMPTY + st));
+        tc_commit1(bar(TS_FULL + st));
       }
       tc_commit1(bar(TDRAIN));  // completes once every MMA issued here has finished
     }
+  } else if (warp == kTPvWarp) {
+    // ---------------------------------- PV MMAs: O_h += P_h V_h, key halves h
+    if (lane == 0) {
+      constexpr uint32_t kIdPV = tc_idesc_bf16(128, 128, true);
+      const uint64_t pdesc = tc_sdesc(sbase + kTOffP, 16, 1024);      // key block: + 1024; K step: + 2
+      const uint64_t vdesc = tc_sdesc(sbase + kTOffV, kTChunk, 1024);  // 16 keys: + 128
+      bool ok = true;
+      for (int g = 0; g < n_tiles && ok; ++g) {
+        ok = tc_wait(bar(TV_FULL), g & 1, abort_flag, a.status);
+        for (int hh = 0; hh < 2 && ok; ++hh) {
+          ok = tc_wait(bar(TP_FULL + hh), g & 1, abort_flag, a.status);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma1(tmem + kTColO + 128 * hh, pdesc + 1024 * hh + 2 * k, vdesc + 128 * (4 * hh + k), kIdPV,
+                    (g | k) ? 1u : 0u);
+          tc_commit1(bar(TO_DONE + hh));
+        }
+        if (!ok) break;
+        tc_commit1(bar(TV_EMPTY));
+      }
+      tc_commit1(bar(TDRAIN));
+    }
   } else {
     // --------------------------------------- softmax and epilogue, warps 0-7
-    // Thread (row i, half) owns keys [64 half, 64 half + 64) of every tile and
-    // columns [64 half, 64 half + 64) of O; the two halves of a row share their
-    // maxima and sums through shared memory.  Every exit from the loop passes
-    // the barrier that ANDs the warps' flags, so all 256 threads leave together.
+    // Thread (row i, half) owns keys [64 half, 64 half + 64) of every tile,
+    // with its own running max and sum and its own accumulator O_half (TMEM
+    // columns 256 + 128 half), so the two halves of a row never wait for each
+    // other inside the loop.  The epilogue merges them: thread (i, half)
+    // writes output columns [64 half, 64 half + 64) of
+    // (2^(m_0 - m) O_0 + 2^(m_1 - m) O_1) / (2^(m_0 - m) l_0 + 2^(m_1 - m) l_1).
+    // Every exit from the loop reaches the epilogue's barrier, which ANDs the
+    // warps' flags, so all 256 threads leave together.
     const int i = 32 * (warp & 3) + lane, half = warp >> 2, t = t0 + i;
     const int p = p0 + min(t, T - 1);  // rows past the last query repeat its position (not stored)
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    float* red_max = reinterpret_cast<float*>(smem + kTOffRed);  // [2][2][128]
-    float* red_l = red_max + 512;                                // [2][128]
-    float m_ref = -INFINITY, l = 0.f;
+    const uint32_t o_own = tmem + lane_base + kTColO + 128 * half;
+    float* red_m = reinterpret_cast<float*>(smem + kTOffRed);  // [2][128]
+    float* red_l = red_m + 256;                                // [2][128]
+    float m_ref = -INFINITY, l = 0.f;  // m_ref = -inf: no visible key of this half yet (O_half is 0)
     bool ok = true;
-    for (int g = 0; g < n_tiles; ++g) {
+    for (int g = 0; g < n_tiles && ok; ++g) {
       const int st = g & 1;
-      bool okw = ok && __all_sync(0xffffffffu, tc_wait(bar(TS_FULL + st), (g >> 1) & 1, abort_flag, a.status));
-      uint32_t r[64];
-      float mx = -INFINITY;
-      const int kb = kTk * g + 64 * half;  // key of r[0]
-      if (okw) {
-        tc_fence_after();
-        const uint32_t s_addr = tmem + lane_base + kTColS + 128 * st + 64 * half;
-        tc_ld32_nw(s_addr, r);
-        tc_ld32_nw(s_addr + 32, r + 32);
-        tc_wait_ld();
-        if (!__all_sync(0xffffffffu, kb + 63 <= p)) {  // the causal edge: keys past the query score -inf
-#pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (kb + j > p) r[j] = 0xFF800000u;
-        }
-        float m8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) m8[j] = __uint_as_float(r[j]);
-#pragma unroll
-        for (int j = 8; j < 64; ++j) m8[j & 7] = fmaxf(m8[j & 7], __uint_as_float(r[j]));
-        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        mx *= a.scale_log2;
-      }
-      red_max[(2 * st + half) * 128 + i] = mx;
-      ok = softmax_sync_and(okw);
+      ok = __all_sync(0xffffffffu, tc_wait(bar(TS_FULL + st), (g >> 1) & 1, abort_flag, a.status));
       if (!ok) break;
-      const float tile_max = fmaxf(mx, red_max[(2 * st + (half ^ 1)) * 128 + i]);
+      tc_fence_after();
+      uint32_t r[64];
+      const int kb = kTk * g + 64 * half;  // key of r[0]
+      const uint32_t s_addr = tmem + lane_base + kTColS + 128 * st + 64 * half;
+      tc_ld32_nw(s_addr, r);
+      tc_ld32_nw(s_addr + 32, r + 32);
+      tc_wait_ld();
+      if (!__all_sync(0xffffffffu, kb + 63 <= p)) {  // the causal edge: keys past the query score -inf
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+          if (kb + j > p) r[j] = 0xFF800000u;
+      }
+      float m8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m8[j] = __uint_as_float(r[j]);
+#pragma unroll
+      for (int j = 8; j < 64; ++j) m8[j & 7] = fmaxf(m8[j & 7], __uint_as_float(r[j]));
+      const float mx =
+          a.scale_log2 *
+          fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       float alpha = 1.f;
       bool rescale = false;
-      if (g == 0) {
-        m_ref = tile_max;  // key 0 is visible to every row
-      } else if (tile_max > m_ref + kTRescale) {
-        alpha = tc_exp2(m_ref - tile_max);
-        m_ref = tile_max;
-        rescale = true;
+      if (mx > m_ref + kTRescale) {  // also the first visible key (m_ref = -inf: O_half is 0, no rescale)
+        rescale = m_ref != -INFINITY;
+        alpha = rescale ? tc_exp2(m_ref - mx) : 0.f;
+        m_ref = mx;
       }
+      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // all masked so far: exponentials of -inf are 0
       // probabilities as bf16 pairs; the row sum in fp32
       uint32_t pk[32];
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float e0 = tc_exp2(fmaf(__uint_as_float(r[2 * j]), a.scale_log2, -m_ref));
-        const float e1 = tc_exp2(fmaf(__uint_as_float(r[2 * j + 1]), a.scale_log2, -m_ref));
+        const float e0 = tc_exp2(fmaf(__uint_as_float(r[2 * j]), a.scale_log2, -m_use));
+        const float e1 = tc_exp2(fmaf(__uint_as_float(r[2 * j + 1]), a.scale_log2, -m_use));
         s4[j & 3] += e0 + e1;
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
         pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
@@ -420,23 +430,20 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
       tc_fence_before();
       __syncwarp();
       if (lane == 0) tc_arrive(bar(TS_FREE + st));
-      // P(g-1) and O are in use by PV(g-1) until it completes
+      // P_half(g-1) and O_half are in use by the half's PV(g-1) until it completes
       if (g >= 1) {
-        if (!__all_sync(0xffffffffu, tc_wait(bar(TO_DONE), (g - 1) & 1, abort_flag, a.status))) {
-          ok = false;  // the next tile's barrier takes every warp out
-          continue;
-        }
+        ok = __all_sync(0xffffffffu, tc_wait(bar(TO_DONE + half), (g - 1) & 1, abort_flag, a.status));
+        if (!ok) break;
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          const uint32_t o_addr = tmem + lane_base + kTColO + 64 * half + 32 * c;
-          tc_ld32(o_addr, o);
+          tc_ld32(o_own + 32 * c, o);
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tc_st32(o_addr, o);
+          tc_st32(o_own + 32 * c, o);
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       }
@@ -446,28 +453,40 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
       for (int u = 0; u < 8; ++u)
         *reinterpret_cast<uint4*>(smem + kTOffP + half * kTChunk + i * 128 + ((u ^ (i & 7)) * 16)) =
             make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-      tc_fence_before();    // the rescaled O precedes the next PV MMAs
+      tc_fence_before();    // the rescaled O_half precedes the half's next PV MMAs
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P is read by the tensor cores
       __syncwarp();
-      if (lane == 0) tc_arrive(bar(TP_FULL));
+      if (lane == 0) tc_arrive(bar(TP_FULL + half));
     }
-    bool okf = ok && __all_sync(0xffffffffu, tc_wait(bar(TO_DONE), (n_tiles - 1) & 1, abort_flag, a.status));
+    // epilogue: both halves' last PV MMAs, then the merge
+    bool okf = ok;
+    for (int hh = 0; hh < 2 && okf; ++hh)
+      okf = __all_sync(0xffffffffu, tc_wait(bar(TO_DONE + hh), (n_tiles - 1) & 1, abort_flag, a.status));
+    red_m[half * 128 + i] = m_ref;
     red_l[half * 128 + i] = l;
     okf = softmax_sync_and(okf);
     if (okf) {
       tc_fence_after();
-      const float lt = l + red_l[(half ^ 1) * 128 + i];
+      const float m0 = red_m[i], m1 = red_m[128 + i];
+      const float m = fmaxf(m0, m1);  // finite: key 0 is visible to every row
+      const float a0 = m0 == -INFINITY ? 0.f : tc_exp2(m0 - m), a1 = m1 == -INFINITY ? 0.f : tc_exp2(m1 - m);
+      const float lt = a0 * red_l[i] + a1 * red_l[128 + i];
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float w0 = a0 * inv, w1 = a1 * inv;
       __nv_bfloat16* orow = a.out + (((size_t)b * T + t) * H + h) * kPDv + 64 * half;
+      const uint32_t o0 = tmem + lane_base + kTColO + 64 * half;  // O_0 columns [64 half, +64)
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
-        uint32_t o[32];
-        tc_ld32(tmem + lane_base + kTColO + 64 * half + 32 * c, o);
+        uint32_t x0[32], x1[32];
+        tc_ld32_nw(o0 + 32 * c, x0);
+        tc_ld32_nw(o0 + 128 + 32 * c, x1);
+        tc_wait_ld();
         uint32_t w[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const __nv_bfloat162 v2 =
-              __floats2bfloat162_rn(__uint_as_float(o[2 * j]) * inv, __uint_as_float(o[2 * j + 1]) * inv);
+          const float v0 = fmaf(__uint_as_float(x0[2 * j]), w0, __uint_as_float(x1[2 * j]) * w1);
+          const float v1 = fmaf(__uint_as_float(x0[2 * j + 1]), w0, __uint_as_float(x1[2 * j + 1]) * w1);
+          const __nv_bfloat162 v2 = __floats2bfloat162_rn(v0, v1);
           w[j] = *reinterpret_cast<const uint32_t*>(&v2);
         }
         if (t < T)
@@ -476,7 +495,7 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
             *reinterpret_cast<uint4*>(orow + 32 * c + 8 * u) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
       }
       if (half == 0 && a.lse_out && t < T)
-        a.lse_out[((size_t)b * T + t) * H + h] = lt > 0.f ? (m_ref + log2f(lt)) * kLn2 : -INFINITY;
+        a.lse_out[((size_t)b * T + t) * H + h] = lt > 0.f ? (m + log2f(lt)) * kLn2 : -INFINITY;
     }
   }
 
