@@ -3,7 +3,9 @@
 The session owns the scratch workspaces; the caller owns weights, the paged
 cache and the page table.  `step` takes device tensors; `step_from_host`
 copies a step's inputs from (pinned) host memory, runs the step and copies the
-output back, the path a serving loop driven from the host takes.  By default
+output back, the path a serving loop driven from the host takes; a
+`HostPipeline` does the same for a stream of steps with the copies of one
+step overlapped with the compute of its neighbours.  By default
 it records that sequence (copies in, the library's launches, copy out) as a
 CUDA graph the first time it meets a set of buffers and replays the graph on
 later calls with the same buffers, so a step costs one graph launch on the
@@ -140,23 +142,117 @@ class MlaDecodeSession:
         return host_out
 
 
+def _packed_block(shapes_dtypes: dict, device, pinned: bool) -> dict:
+    """Tensors of these shapes laid end to end (16-byte aligned) in one block:
+    pinned host memory, or device memory."""
+    sizes = []
+    for shape, dtype in shapes_dtypes.values():
+        sizes.append(int(torch.Size(shape).numel()) * torch.empty(0, dtype=dtype).element_size())
+    if any(n % 16 for n in sizes[:-1]):
+        raise ValueError("packed step inputs must be 16-byte multiples")
+    total = sum(sizes)
+    block = (torch.empty(total, dtype=torch.uint8).pin_memory() if pinned
+             else torch.empty(total, dtype=torch.uint8, device=device))
+    out, off = {}, 0
+    for (name, (shape, dtype)), n in zip(shapes_dtypes.items(), sizes):
+        out[name] = block[off:off + n].view(dtype).view(shape)
+        off += n
+    return out
+
+
 def packed_step_buffers(shapes_dtypes: dict, device) -> tuple[dict, dict]:
     """Pinned host and device buffers for a step's inputs, each side one block
     with the tensors laid end to end (16-byte aligned), so that
     `step_from_host` moves them in one transfer.  shapes_dtypes: name ->
     (shape, dtype), in the order h, q_nope, q_rope."""
-    sizes = []
-    for shape, dtype in shapes_dtypes.values():
-        n = int(torch.Size(shape).numel()) * torch.empty(0, dtype=dtype).element_size()
-        sizes.append(n)
-    if any(n % 16 for n in sizes[:-1]):
-        raise ValueError("packed step inputs must be 16-byte multiples")
-    total = sum(sizes)
-    host = torch.empty(total, dtype=torch.uint8).pin_memory()
-    dev = torch.empty(total, dtype=torch.uint8, device=device)
-    out_h, out_d, off = {}, {}, 0
-    for (name, (shape, dtype)), n in zip(shapes_dtypes.items(), sizes):
-        out_h[name] = host[off:off + n].view(dtype).view(shape)
-        out_d[name] = dev[off:off + n].view(dtype).view(shape)
-        off += n
-    return out_h, out_d
+    return _packed_block(shapes_dtypes, device, pinned=True), _packed_block(shapes_dtypes, device, pinned=False)
+
+
+class HostPipeline:
+    """Host-driven decode steps with the copies overlapped with the compute.
+
+    `submit` enqueues one step: its inputs are copied from pinned host memory
+    into one of two device input blocks on a copy-in stream, the step (append
+    -> decode -> combine, recorded as a CUDA graph per buffer set on first use)
+    runs on the current stream into one of two device outputs, and the output
+    is copied into the caller's pinned host buffer on a copy-out stream.  So
+    the inputs of step i+1 move in while step i runs, and the output of step i
+    moves out while step i+1 runs; every step still moves its own inputs and
+    its own output.  Events order each buffer's reuse: an input block is
+    overwritten only after the step two back has read it, and an output only
+    after its previous copy-out.  `finish` makes the current stream wait for
+    the last copy-out (host buffers hold their results once that stream
+    reaches it).  Steps run in submission order on the device, so a step sees
+    the cache rows every earlier step appended.  A step's host inputs must
+    stay unchanged until its copy-in has run, and its host output must not be
+    read before `finish` (or a later synchronisation) covers it."""
+
+    def __init__(self, sess: MlaDecodeSession, shapes_dtypes: dict):
+        self.sess = sess
+        dev = sess.device
+        self.names = tuple(shapes_dtypes)
+        # device inputs laid end to end as packed_step_buffers lays them out, so
+        # that packed host inputs move in one transfer
+        self.dev_in = [_packed_block(shapes_dtypes, dev, pinned=False) for _ in range(2)]
+        self.out = [torch.empty_like(sess.out) for _ in range(2)]
+        self.lse = [torch.empty_like(sess.lse) for _ in range(2)]
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        self.in_ready = [torch.cuda.Event() for _ in range(2)]
+        self.step_done = [torch.cuda.Event() for _ in range(2)]
+        self.out_read = [torch.cuda.Event() for _ in range(2)]
+        self.n = 0
+        self._graphs = {}
+
+    def _compute(self, k, seq_idx, pos, seq_lens, weights, page_table, cache_pool):
+        d = self.dev_in[k]
+        self.sess.step(d["h"], seq_idx, pos, d["q_nope"], d["q_rope"], seq_lens, weights, page_table, cache_pool,
+                       self.out[k], self.lse[k])
+
+    def submit(self, host_in: dict, seq_idx, pos, seq_lens, weights, page_table, cache_pool,
+               host_out: torch.Tensor, use_graph: bool = True):
+        k = self.n & 1
+        comp = torch.cuda.current_stream()
+        # inputs of this step: after the step two back has read block k
+        self.s_in.wait_event(self.step_done[k])
+        with torch.cuda.stream(self.s_in):
+            src = MlaDecodeSession._span([host_in[name] for name in self.names])
+            dst = MlaDecodeSession._span([self.dev_in[k][name] for name in self.names])
+            if src is not None and dst is not None and src.numel() == dst.numel():
+                dst.copy_(src, non_blocking=True)
+            else:
+                for name in self.names:
+                    self.dev_in[k][name].copy_(host_in[name], non_blocking=True)
+            self.in_ready[k].record(self.s_in)
+        comp.wait_event(self.in_ready[k])
+        comp.wait_event(self.out_read[k])  # output k has been copied out
+        args = (seq_idx, pos, seq_lens, weights, page_table, cache_pool)
+        if not use_graph:
+            self._compute(k, *args)
+        else:
+            key = (k, tuple(t.data_ptr() for t in (seq_idx, pos, seq_lens, page_table, cache_pool)),
+                   tuple(weights[w].data_ptr() for w in ("W_dkv", "W_kr", "W_uk", "W_uv")), comp.cuda_stream)
+            g = self._graphs.get(key)
+            if g is None:
+                self._compute(k, *args)  # first use: eager (one-time library set-up), then record
+                g = torch.cuda.CUDAGraph()
+                side = torch.cuda.Stream(device=self.sess.device)
+                side.wait_stream(comp)
+                with torch.cuda.stream(side):
+                    with torch.cuda.graph(g, stream=side):
+                        self._compute(k, *args)
+                comp.wait_stream(side)
+                self._graphs[key] = g
+            g.replay()
+        self.step_done[k].record(comp)
+        self.s_out.wait_event(self.step_done[k])
+        with torch.cuda.stream(self.s_out):
+            host_out.copy_(self.out[k], non_blocking=True)
+            self.out_read[k].record(self.s_out)
+        self.n += 1
+        return host_out
+
+    def finish(self):
+        comp = torch.cuda.current_stream()
+        for k in range(2):
+            comp.wait_event(self.out_read[k])
