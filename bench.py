@@ -504,9 +504,7 @@ def measure(cfg, args, dev, pg, local: int, peaks: dict) -> dict:
     graphs = wl.capture()
     ms, clocks = time_graph_steps(wl, graphs, args.steps, args.warmup, pg, local)
     del graphs
-    kms = timeline_kernel_ms(wl, max(args.steps, 5))
-    if cfg.cache_dtype != "fp8":
-        kms.pop("append_finalize", None)
+    kms = timeline_kernel_ms(wl, max(args.steps, 5))  # only the kernels that ran
     ms_step = ms / args.steps
     # a kernel timed alone (or a short region) takes the burst tensor peak
     tpeak = peaks["bf16_tflops_sustained"] if ms > 1000.0 else peaks["bf16_tflops"]

@@ -124,7 +124,13 @@ int mla_check_dims(const mla_dims* dims);
  *   cache_pool num_pages pages (layout above), written
  *   workspace  >= mla_append_workspace_bytes(dims, n_tokens) bytes of scratch
  *              (fp32 c values between the projection and the FP8 quantiser;
- *              0 bytes, and workspace may be NULL, for fp32/bf16 caches)
+ *              0 bytes, and workspace may be NULL, for fp32/bf16 caches).
+ *              With >= mla_append_workspace_bytes_fast(dims, n_tokens) bytes
+ *              (16-byte aligned), a step of 16 to 511 tokens at DeepSeek-V3
+ *              dims with bf16 activations takes the split-K tensor-core
+ *              projection, whose fp32 partial tiles live there; with less it
+ *              takes the cluster kernel.  Same results up to fp32 summation
+ *              order.
  * d_model must be a multiple of 32 and <= 8192 (bf16) / 4096 (fp32): the
  * projection keeps a lane's slice of each weight row in registers
  * (MLA_ERR_UNSUPPORTED otherwise).
@@ -132,6 +138,9 @@ int mla_check_dims(const mla_dims* dims);
  * MLA_ERR_BOUNDS is recorded in the device status word.  n_tokens == 0 is a no-op.
  * ------------------------------------------------------------------------- */
 size_t mla_append_workspace_bytes(const mla_dims* dims, int n_tokens);
+/* The workspace that enables the fastest append path for this request (never
+ * less than mla_append_workspace_bytes); 0 on invalid dims. */
+size_t mla_append_workspace_bytes_fast(const mla_dims* dims, int n_tokens);
 /* mla_append_latent_noalloc: mla_append_latent for callers that cannot
  * allocate device memory at call time (a plugin or callback whose host
  * framework owns all device memory and offers no scratch buffer, or a loop in

@@ -25,7 +25,8 @@ ERRORS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "M
           8: "MLA_ERR_CUDA"}
 
 # Every entry point declared in include/mla.h.
-EXPORTED = ("mla_cache_page_bytes", "mla_check_dims", "mla_append_workspace_bytes", "mla_append_latent",
+EXPORTED = ("mla_cache_page_bytes", "mla_check_dims", "mla_append_workspace_bytes",
+            "mla_append_workspace_bytes_fast", "mla_append_latent",
             "mla_append_latent_noalloc",
             "mla_decode_workspace_bytes", "mla_decode", "mla_combine", "mla_prefill_workspace_bytes",
             "mla_prefill", "mla_decode_path", "mla_auto_splits",
@@ -60,6 +61,7 @@ def lib() -> ctypes.CDLL:
         L.mla_cache_page_bytes.argtypes, L.mla_cache_page_bytes.restype = [S], Z
         L.mla_check_dims.argtypes, L.mla_check_dims.restype = [S], I
         L.mla_append_workspace_bytes.argtypes, L.mla_append_workspace_bytes.restype = [S, I], Z
+        L.mla_append_workspace_bytes_fast.argtypes, L.mla_append_workspace_bytes_fast.restype = [S, I], Z
         L.mla_append_latent.argtypes = [S, P, I, P, P, P, P, P, I, I, P, I, P, Z, P]
         L.mla_append_latent.restype = I
         L.mla_append_latent_noalloc.argtypes = [S, P, I, P, P, P, P, P, I, I, P, I, P]
@@ -132,6 +134,10 @@ def check_dims(dims: MlaDims) -> int:
 
 def append_workspace_bytes(dims: MlaDims, n_tokens: int) -> int:
     return int(lib().mla_append_workspace_bytes(ctypes.byref(dims), n_tokens))
+
+
+def append_workspace_bytes_fast(dims: MlaDims, n_tokens: int) -> int:
+    return int(lib().mla_append_workspace_bytes_fast(ctypes.byref(dims), n_tokens))
 
 
 def decode_workspace_bytes(dims: MlaDims, batch: int, n_q: int, num_splits: int = 0) -> int:

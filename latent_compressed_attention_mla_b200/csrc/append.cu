@@ -98,6 +98,10 @@ struct AppendGemm {
   CUtensorMap map_wd;  // W_dkv [512][d_model], box 64 x 64
   CUtensorMap map_wk;  // W_kr [64][d_model], box 64 x 64
 
+  __device__ int chunks(int, int* first) const {
+    *first = 0;
+    return k_chunks;
+  }
   __device__ bool skip(int) const { return false; }
   __device__ const CUtensorMap* a_box(int t, int* row) const {
     *row = 128 * (t / 3);
@@ -177,6 +181,143 @@ __device__ __forceinline__ float dot_vec(const uint4& w, const uint4& x, __nv_bf
 __device__ __forceinline__ float dot_vec(const uint4& w, const uint4& x, float*) {
   const float4 a = *reinterpret_cast<const float4*>(&w), b = *reinterpret_cast<const float4*>(&x);
   return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+
+// ----------------------------------------------------------------------------
+// Steps of 16 to 511 tokens: the same GEMM split along d_model (split-K), so
+// that about one wave of CTAs streams the weights: CTA tile (m, n, s) covers
+// 128 tokens, outputs [192 n, 192 n + 192) and the s-th of `splits` slices of
+// d_model, and writes its fp32 partial tile.  append_splitk_finish then sums a
+// token's partials in split order (deterministic), rotates k^R and stores the
+// row rounded to bf16, or quantises c for an FP8 cache (the quantiser of
+// append_fp8_finalize, so no second pass is needed).
+// ----------------------------------------------------------------------------
+constexpr int kAsMinTokens = 16;
+constexpr int kAsTilesPerWave = 144;  // split count: this many tiles or fewer,
+constexpr int kAsMaxSplits = 16;      // and at most this many partials per output (measured: 48 splits
+                                      // of a 64-token step cost 7 us more than 16, in the partials' sum)
+
+// Splits of a split-K append of n tokens at these dims, or 0 when that path
+// does not apply.
+int append_splitk_splits(const mla_dims& d, int n_tokens) {
+  if (d.act_dtype != MLA_BF16 || (d.cache_dtype != MLA_BF16 && d.cache_dtype != MLA_FP8_E4M3) || d.d_c != 512 ||
+      d.d_rope != 64 || d.d_model % 64 != 0 || n_tokens < kAsMinTokens || n_tokens >= kAgMinTokens)
+    return 0;
+  const int m_tiles = (n_tokens + 127) / 128, k_chunks = d.d_model / 64;
+  int s = kAsTilesPerWave / (3 * m_tiles);
+  s = s < kAsMaxSplits ? s : kAsMaxSplits;
+  return s < 1 ? 1 : (s > k_chunks ? k_chunks : s);
+}
+
+struct AppendSplitGemm {
+  static constexpr int N = kAgN, Stages = 5;
+  int tiles, m_tiles, splits, k_chunks;
+  int* status;
+  unsigned long long* timeline;
+  int trace;
+  float* part;  // [splits][m_tiles * 128][576] fp32
+  CUtensorMap map_h;   // h [n_tokens][d_model], box 64 x 128 (rows past n_tokens read as zero)
+  CUtensorMap map_wd;  // W_dkv [512][d_model], box 64 x 64
+  CUtensorMap map_wk;  // W_kr [64][d_model], box 64 x 64
+
+  // tile t: m = t % m_tiles, n = (t / m_tiles) % 3, s = t / (3 m_tiles)
+  __device__ bool skip(int) const { return false; }
+  __device__ int chunks(int t, int* first) const {
+    const int s = t / (3 * m_tiles);
+    const int c0 = s * k_chunks / splits, c1 = (s + 1) * k_chunks / splits;
+    *first = c0;
+    return c1 - c0;
+  }
+  __device__ const CUtensorMap* a_box(int t, int* row) const {
+    *row = 128 * (t % m_tiles);
+    return &map_h;
+  }
+  __device__ const CUtensorMap* b_box(int t, int j, int* row) const {
+    const int r = kAgN * ((t / m_tiles) % 3) + 64 * j;
+    *row = r < 512 ? r : r - 512;
+    return r < 512 ? &map_wd : &map_wk;
+  }
+  __device__ void epilogue(int t, int r, uint32_t taddr) const {
+    const int m = t % m_tiles, n = (t / m_tiles) % 3, s = t / (3 * m_tiles);
+    float4* dst = reinterpret_cast<float4*>(part + ((size_t)s * m_tiles * 128 + 128 * m + r) * 576 + kAgN * n);
+#pragma unroll 1
+    for (int c = 0; c < kAgN / 32; ++c) {
+      uint32_t v[32];
+      tc_ld32(taddr + 32 * c, v);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        dst[8 * c + u] = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                                     __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
+    }
+  }
+};
+
+// One CTA of 288 threads per token: threads 0-255 own c columns (2 t, 2 t + 1),
+// threads 256-287 the k^R pair (i, i + 32).
+template <int CACHE>
+__global__ void __launch_bounds__(288) append_splitk_finish_kernel(const AppendArgs a, const float* part, int splits,
+                                                                   int rows_pad) {
+  pdl_trigger();
+  pdl_wait();
+  tl_begin(a.timeline, MLA_TRACE_APPEND_FINALIZE);
+  __shared__ int s_slot[3];
+  __shared__ float s_max[8];
+  const int n = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    int prow = 0, position = 0;
+    s_slot[0] = token_slot(a, n, &prow, &position);
+    s_slot[1] = prow;
+    s_slot[2] = position;
+  }
+  __syncthreads();
+  const int page = s_slot[0], prow = s_slot[1], position = s_slot[2];
+  uint8_t* pg = page >= 0 ? a.pool + (size_t)page * a.page_bytes : nullptr;
+  const float* src = part + (size_t)n * 576;
+  const size_t stride = (size_t)rows_pad * 576;
+  // sums in split order: c columns (2 tid, 2 tid + 1), or the k^R pair (i, i + 32)
+  const int i = tid - 256;
+  const int c0 = tid < 256 ? 2 * tid : 512 + i, c1 = tid < 256 ? 2 * tid + 1 : 544 + i;
+  float x0 = 0.f, x1 = 0.f;
+#pragma unroll 8
+  for (int s = 0; s < splits; ++s) {
+    x0 += src[s * stride + c0];
+    x1 += src[s * stride + c1];
+  }
+  const Fp8Page fp = fp8_page(a.page_size, 512, 64);
+  float scale = 1.f;
+  if (CACHE == MLA_FP8_E4M3) {
+    // per 128-column tile of c (threads 64 t .. 64 t + 63: warps 2 t, 2 t + 1):
+    // scale = amax / 448 (IEEE fp32 division; 1 for an all-zero tile)
+    float m = tid < 256 ? fmaxf(fabsf(x0), fabsf(x1)) : 0.f;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0 && warp < 8) s_max[warp] = m;
+    __syncthreads();
+    if (tid < 256) {
+      const float amax = fmaxf(s_max[2 * (tid >> 6)], s_max[2 * (tid >> 6) + 1]);
+      scale = amax > 0.f ? amax / kE4M3Max : 1.0f;
+    }
+  }
+  if (pg) {
+    if (tid < 256) {
+      if (CACHE == MLA_FP8_E4M3) {
+        const uint32_t lo = __nv_cvt_float_to_fp8(x0 / scale, __NV_SATFINITE, __NV_E4M3);
+        const uint32_t hi = __nv_cvt_float_to_fp8(x1 / scale, __NV_SATFINITE, __NV_E4M3);
+        *reinterpret_cast<uint16_t*>(pg + (size_t)prow * 512 + 2 * tid) = (uint16_t)(lo | (hi << 8));
+        if ((tid & 63) == 0) reinterpret_cast<float*>(pg + fp.sc_off)[(size_t)prow * 4 + (tid >> 6)] = scale;
+      } else {
+        *reinterpret_cast<__nv_bfloat162*>(pg + ((size_t)prow * 576 + 2 * tid) * 2) = __floats2bfloat162_rn(x0, x1);
+      }
+    } else {
+      float cs, sn;
+      rope_cos_sin(position, i, 32, a.rope_base, &cs, &sn);
+      __nv_bfloat16* kr = CACHE == MLA_FP8_E4M3 ? reinterpret_cast<__nv_bfloat16*>(pg + fp.kr_off) + (size_t)prow * 64
+                                                : reinterpret_cast<__nv_bfloat16*>(pg) + (size_t)prow * 576 + 512;
+      kr[i] = __float2bfloat16_rn(x0 * cs - x1 * sn);
+      kr[i + 32] = __float2bfloat16_rn(x1 * cs + x0 * sn);
+    }
+  }
+  tl_end(a.timeline, MLA_TRACE_APPEND_FINALIZE);
 }
 
 template <typename T, int CACHE>
@@ -639,6 +780,11 @@ size_t cache_page_bytes(const mla_dims& d) {
 // kMaxVec 16-byte vectors per lane).
 int append_max_d_model(int act_dtype) { return kSplitK * kMaxVec * 32 * (act_dtype == MLA_F32 ? 4 : 8); }
 
+size_t append_splitk_floats(const mla_dims& d, int n_tokens) {
+  const int s = append_splitk_splits(d, n_tokens);
+  return s ? (size_t)s * ((n_tokens + 127) / 128) * 128 * 576 : 0;
+}
+
 size_t append_scratch_floats(const mla_dims& d, int n_tokens) {
   return d.cache_dtype == MLA_FP8_E4M3 ? (size_t)n_tokens * d.d_c : 0;
 }
@@ -646,7 +792,7 @@ size_t append_scratch_floats(const mla_dims& d, int n_tokens) {
 cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const int32_t* seq_idx,
                           const int32_t* pos, const void* W_dkv, const void* W_kr,
                           const int32_t* page_table, int batch, int max_pages, void* pool,
-                          int num_pages, size_t page_bytes, float* raw, int* status,
+                          int num_pages, size_t page_bytes, float* raw, size_t raw_floats, int* status,
                           cudaStream_t st) {
   AppendArgs a;
   a.h = h;
@@ -682,8 +828,49 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
                    d.d_c == 512 && d.d_rope == 64 && d.d_model % 64 == 0 && n_tokens >= kAgMinTokens &&
                    (reinterpret_cast<uintptr_t>(h) & 15u) == 0 && (reinterpret_cast<uintptr_t>(W_dkv) & 15u) == 0 &&
                    (reinterpret_cast<uintptr_t>(W_kr) & 15u) == 0;
+  const size_t sk_floats = append_splitk_floats(d, n_tokens);
+  const bool splitk = sk_floats > 0 && raw && raw_floats >= sk_floats && (reinterpret_cast<uintptr_t>(raw) & 15u) == 0 &&
+                      (reinterpret_cast<uintptr_t>(h) & 15u) == 0 && (reinterpret_cast<uintptr_t>(W_dkv) & 15u) == 0 &&
+                      (reinterpret_cast<uintptr_t>(W_kr) & 15u) == 0;
   cudaError_t launch_err = cudaSuccess;
-  if (big) {
+  if (splitk) {
+    AppendSplitGemm g;
+    memset(&g, 0, sizeof(g));
+    g.m_tiles = (n_tokens + 127) / 128;
+    g.splits = append_splitk_splits(d, n_tokens);
+    g.k_chunks = d.d_model / 64;
+    g.tiles = 3 * g.m_tiles * g.splits;
+    g.status = status;
+    g.timeline = a.timeline;
+    g.trace = MLA_TRACE_APPEND_PROJECT;
+    g.part = raw;
+    const uint64_t row_bytes = (uint64_t)d.d_model * 2;
+    if (!make_tile_map_bf16(&g.map_h, h, d.d_model, n_tokens, row_bytes, 64, 128) ||
+        !make_tile_map_bf16(&g.map_wd, W_dkv, d.d_model, 512, row_bytes, 64, 64) ||
+        !make_tile_map_bf16(&g.map_wk, W_kr, d.d_model, 64, row_bytes, 64, 64))
+      return cudaErrorInvalidValue;
+    constexpr size_t smem = tc_gemm_smem<AppendSplitGemm>();
+    launch_err = cudaFuncSetAttribute(tc_gemm_kernel<AppendSplitGemm>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem);
+    if (launch_err == cudaSuccess)
+      launch_err = launch_pdl(tc_gemm_kernel<AppendSplitGemm>,
+                              dim3(g.tiles < device_sm_count() ? g.tiles : device_sm_count()), dim3(kGemmThreads), smem,
+                              st, g);
+    if (launch_err == cudaSuccess) launch_err = cudaGetLastError();
+    trace_record(MLA_TRACE_APPEND_PROJECT, true, st);
+    if (launch_err != cudaSuccess) return launch_err;
+    // the partials -> the cache rows (bf16, or the FP8 quantiser)
+    trace_record(MLA_TRACE_APPEND_FINALIZE, false, st);
+    const int rows_pad = 128 * g.m_tiles;
+    launch_err = d.cache_dtype == MLA_FP8_E4M3
+                     ? launch_pdl(append_splitk_finish_kernel<MLA_FP8_E4M3>, dim3(n_tokens), dim3(288), 0, st, a,
+                                  (const float*)raw, g.splits, rows_pad)
+                     : launch_pdl(append_splitk_finish_kernel<MLA_BF16>, dim3(n_tokens), dim3(288), 0, st, a,
+                                  (const float*)raw, g.splits, rows_pad);
+    if (launch_err == cudaSuccess) launch_err = cudaGetLastError();
+    trace_record(MLA_TRACE_APPEND_FINALIZE, true, st);
+    return launch_err;
+  } else if (big) {
     AppendGemm g;
     memset(&g, 0, sizeof(g));
     g.a = a;

@@ -63,8 +63,10 @@ extern "C" int mla_append_latent_noalloc(const mla_dims* dims, const void* h, in
   if (!aligned16(h) || !aligned16(W_dkv) || !aligned16(W_kr) || !aligned16(cache_pool)) return MLA_ERR_ALIGNMENT;
   float* scratch = scratch_on_current_device();
   if (!scratch) return MLA_ERR_CUDA;
+  // scratch capacity 0 for the split-K partials: this entry point keeps the
+  // kernels whose scratch is at most n_tokens * d_c floats
   cudaError_t e = launch_append(*dims, h, n_tokens, seq_idx, pos, W_dkv, W_kr, page_table, batch, max_pages,
-                                cache_pool, num_pages, cache_page_bytes(*dims), scratch, device_status_word(),
+                                cache_pool, num_pages, cache_page_bytes(*dims), scratch, 0, device_status_word(),
                                 (cudaStream_t)stream);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_LAUNCH;
 }

@@ -106,6 +106,13 @@ size_t mla_append_workspace_bytes(const mla_dims* dims, int n_tokens) {
   return align_up(sizeof(float) * append_scratch_floats(*dims, n_tokens), 256);
 }
 
+size_t mla_append_workspace_bytes_fast(const mla_dims* dims, int n_tokens) {
+  if (check_dims(dims) != MLA_OK || n_tokens < 0) return 0;
+  const size_t need = mla_append_workspace_bytes(dims, n_tokens);
+  const size_t fast = align_up(sizeof(float) * append_splitk_floats(*dims, n_tokens), 256);
+  return fast > need ? fast : need;
+}
+
 int mla_append_latent(const mla_dims* dims, const void* h, int n_tokens, const int32_t* seq_idx,
                       const int32_t* pos, const void* W_dkv, const void* W_kr, const int32_t* page_table,
                       int batch, int max_pages, void* cache_pool, int num_pages, void* workspace,
@@ -122,7 +129,8 @@ int mla_append_latent(const mla_dims* dims, const void* h, int n_tokens, const i
     return MLA_ERR_ALIGNMENT;
   return launch_status(launch_append(*dims, h, n_tokens, seq_idx, pos, W_dkv, W_kr, page_table, batch,
                                      max_pages, cache_pool, num_pages, cache_page_bytes(*dims),
-                                     static_cast<float*>(workspace), status_ptr(), (cudaStream_t)stream));
+                                     static_cast<float*>(workspace), workspace ? ws_bytes / sizeof(float) : 0,
+                                     status_ptr(), (cudaStream_t)stream));
 }
 
 int mla_auto_splits(const mla_dims* dims, int batch, int n_q) {

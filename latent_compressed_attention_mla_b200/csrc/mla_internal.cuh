@@ -249,8 +249,11 @@ __device__ __forceinline__ void tl_end_nosync(unsigned long long* tl, int k) {
 cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const int32_t* seq_idx,
                           const int32_t* pos, const void* W_dkv, const void* W_kr,
                           const int32_t* page_table, int batch, int max_pages, void* pool,
-                          int num_pages, size_t page_bytes, float* raw, int* status,
+                          int num_pages, size_t page_bytes, float* raw, size_t raw_floats, int* status,
                           cudaStream_t st);
+// fp32 scratch (floats) with which launch_append takes its split-K path for
+// these dims and token count, or 0 when that path does not apply
+size_t append_splitk_floats(const mla_dims& d, int n_tokens);
 
 // absorb + split plan (+ empty-split initialisation of the lse slots)
 cudaError_t launch_absorb_and_plan(const mla_dims& d, const void* q_nope, const void* q_rope, const void* W_uk,

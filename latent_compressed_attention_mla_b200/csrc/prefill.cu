@@ -150,6 +150,10 @@ struct UpProjGemm {
   CUtensorMap map_wk;  // W_uk [H * 128][512], box 64 x 64
   CUtensorMap map_wv;  // W_uv [H * 128][512], box 64 x 64
 
+  __device__ int chunks(int, int* first) const {
+    *first = 0;
+    return k_chunks;
+  }
   __device__ bool skip(int t) const {
     const int S = a.seq_lens[b];
     const bool ok = S >= a.n_q && S <= a.max_seq_len && (long long)S <= (long long)a.max_pages * kPPage;

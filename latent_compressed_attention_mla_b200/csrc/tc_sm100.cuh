@@ -12,7 +12,9 @@
 // supplies the tile count, the TMA coordinates of a tile's operands and the
 // epilogue:
 //   static constexpr int N, Stages;            N % 64 == 0, N <= 256
-//   int tiles, k_chunks;                        K = 64 * k_chunks
+//   int tiles;
+//   __device__ int chunks(int tile, int* first) const;               the tile's 64-column K chunks:
+//                                                                    [first, first + return value)
 //   int* status; unsigned long long* timeline; int trace;
 //   __device__ bool skip(int tile) const;                                tile left out (by every role)
 //   __device__ const CUtensorMap* a_box(int tile, int* x_row) const;   A rows [x_row, x_row + 128)
@@ -197,20 +199,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) tc_gemm_kernel(const __grid_c
       bool ok = true;
       for (int t = blockIdx.x; t < P.tiles && ok; t += gridDim.x) {
         if (P.skip(t)) continue;
-        int arow = 0;
+        int arow = 0, kc0 = 0;
         const CUtensorMap* amap = P.a_box(t, &arow);
-        for (int kc = 0; kc < P.k_chunks; ++kc, ++g) {
+        const int nk = P.chunks(t, &kc0);
+        for (int kc = 0; kc < nk; ++kc, ++g) {
           const int s = (int)(g % S);
           ok = tc_wait(bar(EMPTY + s), ((g / S) & 1) ^ 1, abort_flag, P.status);
           if (!ok) break;
           const uint32_t dst = sbase + s * L::kStage;
           mbar_expect_local(bar(FULL + s), L::kStage);
-          tma_load_2d(dst, amap, 64 * kc, arow, bar(FULL + s));
+          tma_load_2d(dst, amap, 64 * (kc0 + kc), arow, bar(FULL + s));
 #pragma unroll
           for (int j = 0; j < N / 64; ++j) {
             int brow = 0;
             const CUtensorMap* bmap = P.b_box(t, j, &brow);
-            tma_load_2d(dst + kGemmAChunk + j * 8192, bmap, 64 * kc, brow, bar(FULL + s));
+            tma_load_2d(dst + kGemmAChunk + j * 8192, bmap, 64 * (kc0 + kc), brow, bar(FULL + s));
           }
         }
       }
@@ -227,7 +230,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) tc_gemm_kernel(const __grid_c
         ok = tc_wait(bar(ACC_EMPTY + buf), ((it >> 1) & 1) ^ 1, abort_flag, P.status);
         if (!ok) break;
         tc_fence_after();
-        for (int kc = 0; kc < P.k_chunks; ++kc, ++g) {
+        int kc0 = 0;
+        const int nk = P.chunks(t, &kc0);
+        for (int kc = 0; kc < nk; ++kc, ++g) {
           const int s = (int)(g % S);
           ok = tc_wait(bar(FULL + s), (g / S) & 1, abort_flag, P.status);
           if (!ok) break;

@@ -23,7 +23,9 @@ class MlaDecodeSession:
         self.dims, self.batch, self.n_q, self.num_splits = dims, batch, n_q, num_splits
         self.device = torch.device(device)
         n_tok = batch * n_q
-        self.append_ws = torch.empty(max(B.append_workspace_bytes(dims, n_tok), 256), dtype=torch.uint8,
+        # the workspace of the fastest append path (split-K partial tiles for
+        # steps of 16 to 511 tokens)
+        self.append_ws = torch.empty(max(B.append_workspace_bytes_fast(dims, n_tok), 256), dtype=torch.uint8,
                                      device=self.device)
         self.decode_ws = torch.empty(B.decode_workspace_bytes(dims, batch, n_q, num_splits), dtype=torch.uint8,
                                      device=self.device)

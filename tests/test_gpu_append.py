@@ -43,6 +43,12 @@ CASES = [
     ("bf16-512-tokens", dict(B=8, T=64, L=(0, 1, 63, 64, 65, 127, 500, 3000), cache_dtype="bf16")),
     ("bf16-700-tokens", dict(B=2, T=350, L=(0, 1000), cache_dtype="bf16")),
     ("fp8-1100-tokens", dict(B=4, T=275, L=(5, 64, 300, 2000), cache_dtype="fp8")),
+    # 16 to 511 tokens take the split-K tensor-core projection when the
+    # workspace holds its partials (the session allocates that size); with the
+    # minimum workspace ("-cluster") the cluster kernel runs instead
+    ("bf16-16-tokens", dict(B=8, T=2, L=(0, 1, 62, 63, 64, 127, 500, 3000), cache_dtype="bf16")),
+    ("fp8-129-tokens-cluster", dict(B=129, T=1, L=tuple(int(x) for x in np.arange(129) * 47 % 270), cache_dtype="fp8")),
+    ("bf16-256-tokens-cluster", dict(B=128, T=2, L=tuple(int(x) for x in np.arange(128) * 59 % 480), cache_dtype="bf16")),
 ]
 
 
@@ -68,6 +74,11 @@ def test_append_rows_match_oracle(name, kw):
         pytest.skip("needs a GPU")
     cfg = V3.with_(name=name, seed=70 + len(name), **kw)
     g = GpuProblem(cfg)
+    if name.endswith("-cluster"):
+        n_tok = cfg.B * cfg.T
+        assert B.append_workspace_bytes_fast(g.dims, n_tok) > B.append_workspace_bytes(g.dims, n_tok)
+        g.session.append_ws = torch.empty(max(B.append_workspace_bytes(g.dims, n_tok), 256), dtype=torch.uint8,
+                                          device="cuda")
     before = g.cache.pool.clone()
     g.session.append(g.inputs["h"], g.seq_idx, g.pos, g.weights["W_dkv"], g.weights["W_kr"], g.page_table,
                      g.cache.pool)

@@ -121,3 +121,21 @@ def test_prefill_workspace_query():
     assert n >= 4096 * (1152 + 2 * 128 * 128 * 2)
     assert B.prefill_workspace_bytes(d, 0) == 0
     assert B.prefill_workspace_bytes(B.dims_for(W.TINY_F32), 256) == 0  # fp32 / other dims: no prefill kernel
+
+
+def test_fast_append_workspace_holds_the_split_k_partials():
+    """Steps of 16 to 511 tokens (V3 dims, bf16 activations) have a faster
+    path whose fp32 partial tiles need more scratch: splits x 128-token tiles
+    x 576 outputs, with 3 x tiles x splits CTA tiles at most 144 and at most
+    16 splits.  Outside that range the fast size is the minimum."""
+    for cfg in (W.V3_B1_L4096, W.V3_FP8_B128_T2):
+        d = B.dims_for(cfg)
+        for n in (1, 4, 15, 512, 4096):
+            assert B.append_workspace_bytes_fast(d, n) == B.append_workspace_bytes(d, n)
+        for n in (16, 64, 128, 129, 256, 511):
+            m_tiles = -(-n // 128)
+            splits = min(144 // (3 * m_tiles), 16, d.d_model // 64)
+            fast = B.append_workspace_bytes_fast(d, n)
+            assert fast >= splits * m_tiles * 128 * 576 * 4
+            assert fast >= B.append_workspace_bytes(d, n)
+            assert 3 * m_tiles * splits <= 144
