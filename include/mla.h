@@ -83,6 +83,14 @@ enum {
  *   - mla_combine: the kernel does not fetch its weights, so its bounded wait
  *     for them expires; MLA_ERR_TIMEOUT is recorded and out and lse_out are
  *     left unwritten.
+ *   - mla_prefill: the up-projection GEMM's and the attention kernel's load
+ *     producers issue no loads; both kernels' waits expire (~2 s each), each
+ *     CTA waits (bounded) for the MMAs it issued and frees its tensor memory;
+ *     MLA_ERR_TIMEOUT is recorded and out / lse_out are not valid.
+ *   - mla_append_latent on its tensor-core GEMM paths (16 or more tokens with
+ *     the fast workspace, or 512 or more): the GEMM's producer issues no
+ *     loads and its wait expires the same way; MLA_ERR_TIMEOUT is recorded
+ *     and the step's cache rows are not valid (a later append rewrites them).
  * No copy is in flight when a wait gives up, and the context stays usable.
  * Ignored by the other kernels. */
 #define MLA_FLAG_SELFTEST_STALL 2u

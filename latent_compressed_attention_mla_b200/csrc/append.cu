@@ -92,6 +92,7 @@ struct AppendGemm {
   int* status;
   unsigned long long* timeline;
   int trace;
+  int stall;
   AppendArgs a;
   int fp8;
   CUtensorMap map_h;   // h [n_tokens][d_model], box 64 x 128 (rows past n_tokens read as zero)
@@ -215,6 +216,7 @@ struct AppendSplitGemm {
   int* status;
   unsigned long long* timeline;
   int trace;
+  int stall;
   float* part;  // [splits][m_tiles * 128][576] fp32
   CUtensorMap map_h;   // h [n_tokens][d_model], box 64 x 128 (rows past n_tokens read as zero)
   CUtensorMap map_wd;  // W_dkv [512][d_model], box 64 x 64
@@ -843,6 +845,7 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
     g.status = status;
     g.timeline = a.timeline;
     g.trace = MLA_TRACE_APPEND_PROJECT;
+    g.stall = (d.flags & MLA_FLAG_SELFTEST_STALL) != 0;
     g.part = raw;
     const uint64_t row_bytes = (uint64_t)d.d_model * 2;
     if (!make_tile_map_bf16(&g.map_h, h, d.d_model, n_tokens, row_bytes, 64, 128) ||
@@ -880,6 +883,7 @@ cudaError_t launch_append(const mla_dims& d, const void* h, int n_tokens, const 
     g.status = status;
     g.timeline = a.timeline;
     g.trace = MLA_TRACE_APPEND_PROJECT;
+    g.stall = (d.flags & MLA_FLAG_SELFTEST_STALL) != 0;
     const uint64_t row_bytes = (uint64_t)d.d_model * 2;
     if (!make_tile_map_bf16(&g.map_h, h, d.d_model, n_tokens, row_bytes, 64, 128) ||
         !make_tile_map_bf16(&g.map_wd, W_dkv, d.d_model, 512, row_bytes, 64, 64) ||

@@ -64,6 +64,7 @@ struct PrefillArgs {
   float* lse_out;     // [B, T, H] or null
   int* status;
   unsigned long long* timeline;  // device timeline or null
+  int stall;                     // self-test: the tensor-core kernels' producers issue no loads
 };
 
 // Keys of sequence b, or -1 (recorded) when its length is out of range.
@@ -144,6 +145,7 @@ struct UpProjGemm {
   int* status;
   unsigned long long* timeline;
   int trace;
+  int stall;
   PrefillArgs a;
   int b;
   CUtensorMap map_c;   // C [max_rows][512], box 64 x 128
@@ -291,7 +293,7 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
 
   if (warp == kTKWarp) {
     // ------------------------------------------------------------ TMA: Q, K
-    if (lane == 0) {
+    if (lane == 0 && !a.stall) {
       bool ok = true;
       mbar_expect_local(bar(TQ_FULL), 3 * kTChunk);
       for (int c = 0; c < 3; ++c) tma_load_2d(sbase + kTOffQ + c * kTChunk, &P.map_q, 64 * c, h * T + t0, bar(TQ_FULL));
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
     }
   } else if (warp == kTVWarp) {
     // --------------------------------------------------------------- TMA: V
-    if (lane == 0) {
+    if (lane == 0 && !a.stall) {
       bool ok = true;
       for (int g = 0; g < n_tiles && ok; ++g) {
         ok = tc_wait(bar(TV_EMPTY), (g & 1) ^ 1, abort_flag, a.status);
@@ -648,6 +650,7 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   a.status = device_status_word();
   a.max_rows = L.max_rows;
   a.timeline = timeline_ptr();
+  a.stall = (dims->flags & MLA_FLAG_SELFTEST_STALL) != 0;
   __nv_bfloat16* Qr = reinterpret_cast<__nv_bfloat16*>(ws + L.off_q);
   cudaStream_t st = (cudaStream_t)stream;
   constexpr size_t gsmem = tc_gemm_smem<UpProjGemm>();
@@ -669,6 +672,7 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   up.status = a.status;
   up.timeline = a.timeline;
   up.trace = MLA_TRACE_PREFILL_UPPROJ;
+  up.stall = a.stall;
   if (!make_tile_map_bf16(&up.map_c, a.C, kPDc, R, kPDc * 2, 64, 128) ||
       !make_tile_map_bf16(&up.map_wk, a.W_uk, kPDc, H * kPDn, kPDc * 2, 64, 64) ||
       !make_tile_map_bf16(&up.map_wv, a.W_uv, kPDc, H * kPDv, kPDc * 2, 64, 64))

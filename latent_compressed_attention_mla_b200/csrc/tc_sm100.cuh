@@ -16,6 +16,8 @@
 //   __device__ int chunks(int tile, int* first) const;               the tile's 64-column K chunks:
 //                                                                    [first, first + return value)
 //   int* status; unsigned long long* timeline; int trace;
+//   int stall;                                  self-test: the producer issues no loads, so the
+//                                               MMA issuer's bounded wait expires (MLA_ERR_TIMEOUT)
 //   __device__ bool skip(int tile) const;                                tile left out (by every role)
 //   __device__ const CUtensorMap* a_box(int tile, int* x_row) const;   A rows [x_row, x_row + 128)
 //   __device__ const CUtensorMap* b_box(int tile, int j, int* row) const;  B rows of box j (64 rows)
@@ -194,7 +196,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) tc_gemm_kernel(const __grid_c
 
   if (warp == 4) {
     // ------------------------------------------------------------ TMA loads
-    if (lane == 0) {
+    if (lane == 0 && !P.stall) {
       uint32_t g = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < P.tiles && ok; t += gridDim.x) {
