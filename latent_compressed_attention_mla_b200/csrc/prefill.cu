@@ -213,15 +213,19 @@ constexpr int kTMmaWarp = 8, kTKWarp = 9, kTVWarp = 10, kTPvWarp = 11;  // kTMma
 constexpr uint32_t kTChunk = 128 * 128;            // one 64-column block of 128 rows (16 KB)
 constexpr uint32_t kTOffQ = 0;                     // [3][128 queries][128 B]
 constexpr uint32_t kTOffK = kTOffQ + 3 * kTChunk;  // [2 stages][3][128 keys][128 B]
-constexpr uint32_t kTOffV = kTOffK + 6 * kTChunk;  // [2 column halves][128 keys][128 B]
-constexpr uint32_t kTOffP = kTOffV + 2 * kTChunk;  // [2 key blocks][128 queries][128 B]
+constexpr int kTVSlots = 3;                        // V ring: 64-key half tiles
+constexpr uint32_t kTVSlot = kTChunk;              // [2 column halves][64 keys][128 B]
+constexpr uint32_t kTOffV = kTOffK + 6 * kTChunk;  // [kTVSlots][kTVSlot]
+constexpr uint32_t kTOffP = kTOffV + kTVSlots * kTVSlot;  // [2 key blocks][128 queries][128 B]
 constexpr uint32_t kTOffBar = kTOffP + 2 * kTChunk;
 // TP_FULL / TO_DONE: one per key half (the half's P written / its PV MMAs done)
-enum { TQ_FULL = 0, TK_FULL = 1, TK_EMPTY = 3, TV_FULL = 5, TV_EMPTY = 6, TS_FULL = 7, TS_FREE = 9, TP_FULL = 11,
-       TO_DONE = 13, TDRAIN = 15, TNumBars = 16 };
+enum { TQ_FULL = 0, TK_FULL = 1, TK_EMPTY = 3, TV_FULL = 5, TV_EMPTY = 8, TS_FULL = 11, TS_FREE = 13,
+       TP_FULL = 15, TO_DONE = 17, TDRAIN = 19, TNumBars = 20 };
 constexpr uint32_t kTOffMisc = kTOffBar + 8 * TNumBars;
-constexpr uint32_t kTOffRed = kTOffMisc + 16;      // float [2 halves][128 rows] maxima, then sums
-constexpr size_t kTSmem = kTOffRed + 4 * 128 * 4 + 1024;  // + alignment slack
+constexpr size_t kTSmem = kTOffMisc + 16 + 1024;   // + alignment slack
+// the epilogue's exchange of the halves' maxima and sums, [2][128] floats
+// each, uses the P buffer once the last PV MMAs have read it
+static_assert(kTSmem <= 232448, "shared memory");
 constexpr uint32_t kTColS = 0, kTColO = 256, kTTmemCols = 512;  // S: 0 and 128; O of key half h: 256 + 128 h
 constexpr float kTRescale = 8.0f;                  // log2 units
 
@@ -231,7 +235,7 @@ struct TcAttnParams {
   CUtensorMap map_q;     // Qr [H * T rows][192], box 64 x 128
   CUtensorMap map_kc;    // Kc [H * max_rows][128], box 64 x 128
   CUtensorMap map_kr;    // KR [max_rows][64], box 64 x 128
-  CUtensorMap map_v;     // V  [H * max_rows][128], box 64 x 128
+  CUtensorMap map_v;     // V  [H * max_rows][128], box 64 x 64
 };
 
 // Barrier of the softmax warps (named barrier 1) that also ANDs a flag over them.
@@ -270,8 +274,10 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
       mbar_init_local(bar(TS_FULL + i), 1);
       mbar_init_local(bar(TS_FREE + i), kTSoftThreads / 32);
     }
-    mbar_init_local(bar(TV_FULL), 1);
-    mbar_init_local(bar(TV_EMPTY), 1);
+    for (int i = 0; i < kTVSlots; ++i) {
+      mbar_init_local(bar(TV_FULL + i), 1);
+      mbar_init_local(bar(TV_EMPTY + i), 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init_local(bar(TP_FULL + i), kTSoftThreads / 64);
       mbar_init_local(bar(TO_DONE + i), 1);
@@ -311,13 +317,17 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
   } else if (warp == kTVWarp) {
     // --------------------------------------------------------------- TMA: V
     if (lane == 0 && !a.stall) {
+      // half tile u = 2 g + key half, in slot u % kTVSlots: V(g+1)'s first half
+      // loads while PV(g) runs
       bool ok = true;
-      for (int g = 0; g < n_tiles && ok; ++g) {
-        ok = tc_wait(bar(TV_EMPTY), (g & 1) ^ 1, abort_flag, a.status);
+      for (int u = 0; u < 2 * n_tiles && ok; ++u) {
+        const int vs = u % kTVSlots;
+        ok = tc_wait(bar(TV_EMPTY + vs), ((u / kTVSlots) & 1) ^ 1, abort_flag, a.status);
         if (!ok) break;
-        mbar_expect_local(bar(TV_FULL), 2 * kTChunk);
+        mbar_expect_local(bar(TV_FULL + vs), kTVSlot);
         for (int c = 0; c < 2; ++c)
-          tma_load_2d(sbase + kTOffV + c * kTChunk, &P.map_v, 64 * c, krow0 + kTk * g, bar(TV_FULL));
+          tma_load_2d(sbase + kTOffV + vs * kTVSlot + c * (kTVSlot / 2), &P.map_v, 64 * c, krow0 + 64 * u,
+                      bar(TV_FULL + vs));
       }
     }
   } else if (warp == kTMmaWarp) {
@@ -352,22 +362,22 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
     if (lane == 0) {
       constexpr uint32_t kIdPV = tc_idesc_bf16(128, 128, true);
       const uint64_t pdesc = tc_sdesc(sbase + kTOffP, 16, 1024);      // key block: + 1024; K step: + 2
-      const uint64_t vdesc = tc_sdesc(sbase + kTOffV, kTChunk, 1024);  // 16 keys: + 128
+      const uint64_t vdesc = tc_sdesc(sbase + kTOffV, kTVSlot / 2, 1024);  // slot: + kTVSlot/16; 16 keys: + 128
       bool ok = true;
       for (int g = 0; g < n_tiles && ok; ++g) {
-        ok = tc_wait(bar(TV_FULL), g & 1, abort_flag, a.status);
         for (int hh = 0; hh < 2 && ok; ++hh) {
-          ok = tc_wait(bar(TP_FULL + hh), g & 1, abort_flag, a.status);
+          const int u = 2 * g + hh, vs = u % kTVSlots;
+          ok = tc_wait(bar(TV_FULL + vs), (u / kTVSlots) & 1, abort_flag, a.status) &&
+               tc_wait(bar(TP_FULL + hh), g & 1, abort_flag, a.status);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma1(tmem + kTColO + 128 * hh, pdesc + 1024 * hh + 2 * k, vdesc + 128 * (4 * hh + k), kIdPV,
+            tc_mma1(tmem + kTColO + 128 * hh, pdesc + 1024 * hh + 2 * k, vdesc + (kTVSlot >> 4) * vs + 128 * k, kIdPV,
                     (g | k) ? 1u : 0u);
           tc_commit1(bar(TO_DONE + hh));
+          tc_commit1(bar(TV_EMPTY + vs));
         }
-        if (!ok) break;
-        tc_commit1(bar(TV_EMPTY));
       }
       tc_commit1(bar(TDRAIN));
     }
@@ -385,8 +395,8 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
     const int p = p0 + min(t, T - 1);  // rows past the last query repeat its position (not stored)
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t o_own = tmem + lane_base + kTColO + 128 * half;
-    float* red_m = reinterpret_cast<float*>(smem + kTOffRed);  // [2][128]
-    float* red_l = red_m + 256;                                // [2][128]
+    float* red_m = reinterpret_cast<float*>(smem + kTOffP);  // [2][128], epilogue only (P is read by then)
+    float* red_l = red_m + 256;                              // [2][128]
     float m_ref = -INFINITY, l = 0.f;  // m_ref = -inf: no visible key of this half yet (O_half is 0)
     bool ok = true;
     for (int g = 0; g < n_tiles && ok; ++g) {
@@ -681,7 +691,7 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   if (!make_tile_map_bf16(&tp.map_q, Qr, kPDk, H * n_q, kPDk * 2, 64, kTq) ||
       !make_tile_map_bf16(&tp.map_kc, a.Kc, kPDn, H * R, kPDn * 2, 64, kTk) ||
       !make_tile_map_bf16(&tp.map_kr, a.KR, kPDr, R, kPDr * 2, 64, kTk) ||
-      !make_tile_map_bf16(&tp.map_v, a.V, kPDv, H * R, kPDv * 2, 64, kTk))
+      !make_tile_map_bf16(&tp.map_v, a.V, kPDv, H * R, kPDv * 2, 64, 64))
     return MLA_ERR_LAUNCH;
   // one sequence at a time: the workspace holds one sequence's keys and values
   for (int b = 0; b < batch; ++b) {
