@@ -88,6 +88,7 @@ constexpr int kAgMinTokens = 512;
 
 struct AppendGemm {
   static constexpr int N = kAgN, Stages = 5;
+  static constexpr uint32_t kOutStage = 0;
   int tiles, k_chunks;
   int* status;
   unsigned long long* timeline;
@@ -113,7 +114,7 @@ struct AppendGemm {
     *row = r < 512 ? r : r - 512;
     return r < 512 ? &map_wd : &map_wk;
   }
-  __device__ void epilogue(int t, int r, uint32_t taddr) const {
+  __device__ void epilogue(int t, int r, uint32_t taddr, uint8_t*, uint32_t) const {
     const int n = 128 * (t / 3) + r, nt = t % 3;
     const bool live = n < a.n_tokens;
     int prow = 0, position = 0;
@@ -212,6 +213,7 @@ int append_splitk_splits(const mla_dims& d, int n_tokens) {
 
 struct AppendSplitGemm {
   static constexpr int N = kAgN, Stages = 5;
+  static constexpr uint32_t kOutStage = 0;
   int tiles, m_tiles, splits, k_chunks;
   int* status;
   unsigned long long* timeline;
@@ -239,7 +241,7 @@ struct AppendSplitGemm {
     *row = r < 512 ? r : r - 512;
     return r < 512 ? &map_wd : &map_wk;
   }
-  __device__ void epilogue(int t, int r, uint32_t taddr) const {
+  __device__ void epilogue(int t, int r, uint32_t taddr, uint8_t*, uint32_t) const {
     const int m = t % m_tiles, n = (t / m_tiles) % 3, s = t / (3 * m_tiles);
     float4* dst = reinterpret_cast<float4*>(part + ((size_t)s * m_tiles * 128 + 128 * m + r) * 576 + kAgN * n);
 #pragma unroll 1

@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(256) prefill_gather_kernel(const PrefillArgs a
 // ----------------------------------------------------------------------------
 struct UpProjGemm {
   static constexpr int N = 256, Stages = 4;
+  static constexpr uint32_t kOutStage = 2 * 16384;  // two [128 rows][64 columns] bf16 boxes, 128-byte swizzle
   int tiles, k_chunks;
   int* status;
   unsigned long long* timeline;
@@ -151,6 +152,8 @@ struct UpProjGemm {
   CUtensorMap map_c;   // C [max_rows][512], box 64 x 128
   CUtensorMap map_wk;  // W_uk [H * 128][512], box 64 x 64
   CUtensorMap map_wv;  // W_uv [H * 128][512], box 64 x 64
+  CUtensorMap map_kc_out;  // K^C [H * max_rows][128], box 64 x 128 (stores)
+  CUtensorMap map_v_out;   // V [H * max_rows][128], box 64 x 128 (stores)
 
   __device__ int chunks(int, int* first) const {
     *first = 0;
@@ -169,22 +172,38 @@ struct UpProjGemm {
     *row = 128 * (t % a.n_heads) + 64 * (j & 1);
     return j < 2 ? &map_wk : &map_wv;
   }
-  __device__ void epilogue(int t, int r, uint32_t taddr) const {
-    const int h = t % a.n_heads, s = 128 * (t / a.n_heads) + r;
+  // the tile's four 64-column boxes (K^C 0-63, 64-127, V 0-63, 64-127) leave
+  // through two alternating staging buffers by TMA store: whole 128-byte lines
+  // (a thread writing its own 512-byte row costs ~115 us more on 8192 keys)
+  __device__ void epilogue(int t, int r, uint32_t taddr, uint8_t* ost, uint32_t ost_addr) const {
+    const int h = t % a.n_heads, m0 = 128 * (t / a.n_heads);
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {  // 32-column chunks: 0-3 K^C, 4-7 V
-      uint32_t v[32];
-      tc_ld32(taddr + 32 * c, v);
-      uint32_t w[16];
+    for (int j = 0; j < 4; ++j) {
+      const int buf = j & 1;
+      if (r == 0) gemm_bulk_wait_read<1>();  // the store of two boxes back has read this buffer
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      uint32_t v[64];
+      tc_ld32_nw(taddr + 64 * j, v);
+      tc_ld32_nw(taddr + 64 * j + 32, v + 32);
+      tc_wait_ld();
+      uint8_t* row = ost + buf * 16384 + r * 128;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-        w[j] = *reinterpret_cast<const uint32_t*>(&b2);
+      for (int u = 0; u < 8; ++u) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 b2 =
+              __floats2bfloat162_rn(__uint_as_float(v[8 * u + 2 * e]), __uint_as_float(v[8 * u + 2 * e + 1]));
+          w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        *reinterpret_cast<uint4*>(row + ((u ^ (r & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      __nv_bfloat16* out = (c < 4 ? a.Kc : a.V) + ((size_t)h * a.max_rows + s) * kPDn + 32 * (c & 3);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        reinterpret_cast<uint4*>(out)[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the TMA store reads it
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (r == 0) {
+        gemm_tma_store_2d(j < 2 ? &map_kc_out : &map_v_out, 64 * (j & 1), h * a.max_rows + m0, ost_addr + buf * 16384);
+        gemm_bulk_commit();
+      }
     }
   }
 };
@@ -685,7 +704,9 @@ extern "C" int mla_prefill(const mla_dims* dims, const void* q_nope, const void*
   up.stall = a.stall;
   if (!make_tile_map_bf16(&up.map_c, a.C, kPDc, R, kPDc * 2, 64, 128) ||
       !make_tile_map_bf16(&up.map_wk, a.W_uk, kPDc, H * kPDn, kPDc * 2, 64, 64) ||
-      !make_tile_map_bf16(&up.map_wv, a.W_uv, kPDc, H * kPDv, kPDc * 2, 64, 64))
+      !make_tile_map_bf16(&up.map_wv, a.W_uv, kPDc, H * kPDv, kPDc * 2, 64, 64) ||
+      !make_tile_map_bf16(&up.map_kc_out, a.Kc, kPDn, H * R, kPDn * 2, 64, 128) ||
+      !make_tile_map_bf16(&up.map_v_out, a.V, kPDv, H * R, kPDv * 2, 64, 128))
     return MLA_ERR_LAUNCH;
   const int up_grid = up.tiles < device_sm_count() ? up.tiles : device_sm_count();
   if (!make_tile_map_bf16(&tp.map_q, Qr, kPDk, H * n_q, kPDk * 2, 64, kTq) ||

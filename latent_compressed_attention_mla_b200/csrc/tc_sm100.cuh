@@ -21,8 +21,13 @@
 //   __device__ bool skip(int tile) const;                                tile left out (by every role)
 //   __device__ const CUtensorMap* a_box(int tile, int* x_row) const;   A rows [x_row, x_row + 128)
 //   __device__ const CUtensorMap* b_box(int tile, int j, int* row) const;  B rows of box j (64 rows)
-//   __device__ void epilogue(int tile, int row, uint32_t taddr) const;  taddr: TMEM lane/column of row's
-//                                                                        accumulator column 0
+//   static constexpr uint32_t kOutStage;        bytes of shared memory for the epilogue's output
+//                                               staging (0: none)
+//   __device__ void epilogue(int tile, int row, uint32_t taddr, uint8_t* ost, uint32_t ost_addr) const;
+//                                               taddr: TMEM lane/column of row's accumulator column 0;
+//                                               ost: the staging region (generic, shared address).
+//                                               The four epilogue warps run it together and may
+//                                               synchronise on named barrier 1 (128 threads).
 // Every wait is bounded; a CTA that gives up records MLA_ERR_TIMEOUT, waits
 // (bounded) for the MMAs it issued and frees its tensor memory.
 #pragma once
@@ -136,17 +141,42 @@ constexpr uint32_t tc_idesc_bf16(int M, int N, bool b_mn) {
 }
 
 
+// TMA bulk stores from shared memory (a bulk async-group per issuing thread)
+__device__ __forceinline__ void gemm_tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void gemm_bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int K>
+__device__ __forceinline__ void gemm_bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(K) : "memory");
+}
+__device__ __forceinline__ void gemm_bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Barrier of the GEMM's four epilogue warps (named barrier 1) that also ANDs a flag over them.
+__device__ __forceinline__ bool gemm_epi_sync_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
 // ---------------------------------------------------------------------------
 // persistent GEMM
 // ---------------------------------------------------------------------------
 constexpr int kGemmThreads = 192;  // warps 0-3 epilogue, 4 TMA, 5 TMEM allocation + MMA issue
 constexpr uint32_t kGemmAChunk = 128 * 128;  // 128 rows x 64 bf16 columns
 
-template <int N, int Stages>
+template <int N, int Stages, uint32_t OutStage = 0>
 struct GemmSmem {
   static constexpr uint32_t kB = (uint32_t)N * 128;
   static constexpr uint32_t kStage = kGemmAChunk + kB;
-  static constexpr uint32_t kOffBar = Stages * kStage;
+  static constexpr uint32_t kOffOut = Stages * kStage;  // the epilogue's output staging
+  static constexpr uint32_t kOffBar = kOffOut + OutStage;
   // FULL[Stages], EMPTY[Stages], ACC_FULL[2], ACC_EMPTY[2], DRAIN
   static constexpr int kBars = 2 * Stages + 5;
   static constexpr uint32_t kOffMisc = kOffBar + 8 * kBars;
@@ -157,7 +187,7 @@ struct GemmSmem {
 template <class Prob>
 __global__ void __launch_bounds__(kGemmThreads, 1) tc_gemm_kernel(const __grid_constant__ Prob P) {
   constexpr int N = Prob::N, S = Prob::Stages;
-  using L = GemmSmem<N, S>;
+  using L = GemmSmem<N, S, Prob::kOutStage>;
   static_assert(N % 64 == 0 && N <= 256, "tile N");
   static_assert(L::kBytes <= 232448, "shared memory");
   extern __shared__ uint8_t gemm_smem_raw[];
@@ -259,14 +289,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) tc_gemm_kernel(const __grid_c
     for (int t = blockIdx.x; t < P.tiles; t += gridDim.x) {
       if (P.skip(t)) continue;
       const uint32_t buf = it & 1;
-      if (!__all_sync(0xffffffffu, tc_wait(bar(ACC_FULL + buf), (it >> 1) & 1, abort_flag, P.status))) break;
+      const bool okw = __all_sync(0xffffffffu, tc_wait(bar(ACC_FULL + buf), (it >> 1) & 1, abort_flag, P.status));
+      if (!gemm_epi_sync_and(okw)) break;  // the four warps agree, so none is left at a barrier of the epilogue
       tc_fence_after();
-      P.epilogue(t, row, tmem + lane_base + buf * N);
+      P.epilogue(t, row, tmem + lane_base + buf * N, smem + L::kOffOut, sbase + L::kOffOut);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) tc_arrive(bar(ACC_EMPTY + buf));
       ++it;
     }
+    if (Prob::kOutStage > 0 && threadIdx.x == 0) gemm_bulk_wait_all();  // the epilogue's stores are complete
   }
 
   // teardown: every tensor-memory access finished before deallocation; after
@@ -301,7 +333,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) tc_gemm_kernel(const __grid_c
 // Shared memory a tc_gemm_kernel<Prob> launch needs.
 template <class Prob>
 constexpr size_t tc_gemm_smem() {
-  return GemmSmem<Prob::N, Prob::Stages>::kBytes;
+  return GemmSmem<Prob::N, Prob::Stages, Prob::kOutStage>::kBytes;
 }
 
 }  // namespace mla
