@@ -212,18 +212,19 @@ struct UpProjGemm {
 // 3. attention on the 5th-generation tensor cores: one CTA per (head, block of
 //    128 queries).  The 128 queries are the M dimension of tcgen05 MMAs with
 //    accumulators in tensor memory (query i in TMEM lane i):
-//      S[128 x 128 keys] = Q[128 x 192] . K^T     (12 MMAs of K = 16)
-//      O[128 x 128]     += P[128 x 128 keys] . V  (8 MMAs of K = 16)
-//    S is double-buffered (columns 0 and 128), O sits in columns 256-383.
-//    Warps 0-7 run the softmax (two threads per query row, each with half
-//    of the tile's keys and half of O's columns; a lazily updated reference
-//    max as in the decode: O is rescaled only when a row's tile maximum
-//    exceeds its reference by more than 2^8), write P as bf16 into shared
-//    memory and finish; warp 8 allocates tensor memory and one of its
-//    threads issues the QK MMAs, one thread of warp 11 the PV MMAs; warps 9
-//    and 10 bring K and V tiles by TMA (128-byte swizzle).  Every wait is bounded; a CTA that gives up records
-//    MLA_ERR_TIMEOUT, waits (bounded) for the MMAs it issued and frees its
-//    tensor memory.
+//      S[128 x 128 keys] = Q[128 x 192] . K^T        (12 MMAs of K = 16)
+//      O_h[128 x 128]   += P_h[128 x 64 keys] . V_h  (4 MMAs of K = 16 per key half h)
+//    S is double-buffered (columns 0 and 128); O_0 and O_1 sit in columns
+//    256 and 384.  Warps 0-7 run the softmax: two threads per query row, one
+//    per key half, each with its own running max and sum (lazily updated as
+//    in the decode: O_h is rescaled only when a tile maximum exceeds the
+//    reference by more than 2^8); they write P as bf16 into shared memory
+//    and, at the end, merge the halves.  Warp 8 allocates tensor memory and
+//    one of its threads issues the QK MMAs, one thread of warp 11 the PV
+//    MMAs; warps 9 and 10 bring K tiles (two stages) and 64-key V half tiles
+//    (a ring of three) by TMA with the 128-byte swizzle.  Every wait is
+//    bounded; a CTA that gives up records MLA_ERR_TIMEOUT, waits (bounded)
+//    for the MMAs it issued and frees its tensor memory.
 // ----------------------------------------------------------------------------
 constexpr int kTq = 128, kTk = 128;
 constexpr int kTSoftThreads = 256;                 // warps 0-7
