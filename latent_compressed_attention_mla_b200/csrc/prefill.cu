@@ -268,6 +268,23 @@ __device__ __forceinline__ bool softmax_sync_and(bool v) {
       : "memory");
   return r != 0;
 }
+// d = a * b + c and d += a on two fp32 lanes in one instruction (sm_100
+// packed fp32; measured: the softmax's scale-and-shift and row sums in this
+// form took the attention from 1,888 to 1,856 us on a 4,096-token chunk)
+__device__ __forceinline__ void fma_x2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                       float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add_x2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
+      "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+
 __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __grid_constant__ TcAttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -456,9 +473,11 @@ __global__ void __launch_bounds__(kTThreads, 1) prefill_attn_tc_kernel(const __g
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float e0 = tc_exp2(fmaf(__uint_as_float(r[2 * j]), a.scale_log2, -m_use));
-        const float e1 = tc_exp2(fmaf(__uint_as_float(r[2 * j + 1]), a.scale_log2, -m_use));
-        s4[j & 3] += e0 + e1;
+        float x0, x1;
+        fma_x2(x0, x1, __uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]), a.scale_log2, a.scale_log2, -m_use,
+               -m_use);
+        const float e0 = tc_exp2(x0), e1 = tc_exp2(x1);
+        add_x2(s4[2 * (j & 1)], s4[2 * (j & 1) + 1], e0, e1);
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
         pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
       }
