@@ -141,3 +141,46 @@ def test_append_f32_cache_matches_oracle():
     rows = torch.tensor([s[4] for s in slots], device="cuda")
     assert np.abs(v["c"][pages, rows].double().cpu().numpy() - c).max() <= 1e-5 * np.abs(c).max()
     assert np.abs(v["kr"][pages, rows].double().cpu().numpy() - kr).max() <= 1e-5 * np.abs(kr).max()
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("gemv-3", dict(B=3, T=1, L=(10, 70, 200), cache_dtype="bf16")),
+    ("cluster-8", dict(B=8, T=1, L=tuple(range(5, 800, 100)), cache_dtype="bf16")),
+    ("splitk-64", dict(B=32, T=2, L=tuple(int(x) for x in np.arange(32) * 29 % 300), cache_dtype="fp8")),
+    ("gemm-600", dict(B=3, T=200, L=(0, 100, 1000), cache_dtype="bf16")),
+], ids=lambda v: v if isinstance(v, str) else "")
+def test_out_of_range_tokens_are_skipped_and_reported(name, kw):
+    """A token whose sequence index or position is out of range is skipped and
+    MLA_ERR_BOUNDS recorded, on every append path (register GEMV, cluster
+    kernel, split-K and long-chunk tcgen05 GEMMs): no byte outside the valid
+    tokens' rows changes, and the valid rows hold the oracle's values."""
+    cfg = V3.with_(name=name, seed=81 + len(name), **kw)
+    g = GpuProblem(cfg)
+    n = cfg.B * cfg.T
+    seq_idx = g.seq_idx.clone()
+    pos = g.pos.clone()
+    seq_idx[1] = cfg.B            # no such sequence
+    pos[n - 1] = 1 << 24          # past the page table
+    before = g.cache.pool.clone()
+    g.session.append(g.inputs["h"], seq_idx, pos, g.weights["W_dkv"], g.weights["W_kr"], g.page_table, g.cache.pool)
+    torch.cuda.synchronize()
+    assert g.status() == B.MLA_ERR_BOUNDS
+    o = OracleProblem(cfg)
+    valid = [k for k in range(n) if k not in (1, n - 1)]
+    slots = [s for s in appended_slots(cfg, g.pt_host, o.seq_idx, o.pos) if s[0] in valid]
+    allowed = torch.zeros_like(before, dtype=torch.bool)
+    for _, _, _, page, row in slots:
+        for off, nb in row_byte_ranges(cfg, g.cache.page_bytes, page, row):
+            allowed[off:off + nb] = True
+    assert not bool(((before != g.cache.pool) & ~allowed).any()), "bytes outside the valid tokens' rows changed"
+    c, kr = O.append_latent(o.inp["h"][valid], o.w["W_dkv"], o.w["W_kr"], o.pos[valid], cfg.rope_base)
+    v = g.cache.views()
+    pages = torch.tensor([s[3] for s in slots], device="cuda")
+    rows = torch.tensor([s[4] for s in slots], device="cuda")
+    kr_gpu = v["kr"][pages, rows].double().cpu().numpy()
+    assert np.allclose(kr_gpu, kr, rtol=2.0 ** -7, atol=2.0 ** -12 * np.abs(kr).max())
+    if cfg.cache_dtype == "fp8":
+        got = O.fp8_dequantise_latent(v["codes"][pages, rows].cpu().numpy(), v["scales"][pages, rows].double().cpu().numpy())
+        assert np.abs(got - c).max() <= 2.0 ** -3 * np.abs(c).max()
+    else:
+        assert np.allclose(v["c"][pages, rows].double().cpu().numpy(), c, rtol=2.0 ** -7, atol=2.0 ** -12 * np.abs(c).max())
