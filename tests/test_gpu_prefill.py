@@ -8,6 +8,7 @@ import torch
 
 from latent_compressed_attention_mla_b200 import binding as B
 from latent_compressed_attention_mla_b200 import workloads as W
+from oracle import mla_oracle as O
 from tests.gpu_harness import GpuProblem, OracleProblem, rel_err
 
 pytestmark = pytest.mark.gpu
@@ -83,3 +84,27 @@ def test_prefill_length_beyond_bound_is_reported():
     o = OracleProblem(cfg)
     heads = list(range(0, 128, 16))
     assert rel_err(g.session.out[0][:, heads].float().cpu().numpy(), o.expected(0, heads)[0]) <= 1e-2
+
+
+def test_prefill_full_size_sampled_queries():
+    """The bench's prefill workload at full size (4,096 new tokens over 4,096
+    cached, in the launch configuration the bench times), on sampled queries
+    (the first and last of the chunk and of 128-query blocks) of three heads
+    against the oracle's explicit form; a query at position p is the last
+    query of the sequence's first p + 1 keys."""
+    cfg = W.V3_PREFILL_CHUNK
+    g = GpuProblem(cfg)
+    out, lse = run_prefill(g)
+    assert g.status() == 0
+    got_all = out[0].float().cpu().numpy()
+    assert np.isfinite(got_all).all()
+    o = OracleProblem(cfg)
+    C, KR = o.cache_values(0)
+    S, T = int(cfg.seq_lens[0]), cfg.T
+    heads = [0, 57, 127]
+    for t in (0, 1, 127, 128, 1023, 2048, 3071, 4094, 4095):
+        p = S - T + t
+        ref, ref_lse = O.decode_explicit(o.inp["q_nope"][0][t:t + 1], o.inp["q_rope"][0][t:t + 1], C, KR,
+                                         o.w["W_uk"], o.w["W_uv"], p + 1, cfg.softmax_scale, cfg.rope_base, heads)
+        assert rel_err(got_all[t][heads], ref[0]) <= 1e-2, t
+        assert np.allclose(lse[0, t, heads].cpu().numpy(), ref_lse[0], rtol=1e-2, atol=1e-2), t
