@@ -26,9 +26,16 @@ CASES = [
     # passes of at most 4 tokens take the register-resident projection
     ("bf16-1-token", dict(B=1, T=1, L=(4000,), cache_dtype="bf16")),
     ("fp8-4-tokens", dict(B=2, T=2, L=(1, 1000), cache_dtype="fp8")),
-    # the smallest pass of the tensor-core projection, and one past a 16-row tile
+    # 5 to 15 tokens take the cluster kernel (mma.sync, 16-row tiles): one
+    # partial tile, and tiles of 8, 9 and 14 tokens
     ("bf16-5-tokens", dict(B=5, T=1, L=(0, 63, 64, 65, 511), cache_dtype="bf16")),
+    ("fp8-8-tokens", dict(B=8, T=1, L=(0, 1, 63, 64, 65, 127, 500, 3000), cache_dtype="fp8")),
+    ("fp8-14-tokens", dict(B=7, T=2, L=(1, 2, 63, 64, 200, 1000, 4000), cache_dtype="fp8")),
+    ("bf16-9-tokens", dict(B=9, T=1, L=tuple(int(x) for x in np.arange(9) * 61 % 300), cache_dtype="bf16")),
+    # one past a 16-row tile: the split-K projection, and with the minimum
+    # workspace the cluster kernel
     ("bf16-17-tokens", dict(B=17, T=1, L=tuple(int(x) for x in np.arange(17) * 29 % 250), cache_dtype="bf16")),
+    ("bf16-17-tokens-cluster", dict(B=17, T=1, L=tuple(int(x) for x in np.arange(17) * 23 % 250), cache_dtype="bf16")),
     # more tokens than one 64-token pass of the tensor-core projection
     ("bf16-70-tokens", dict(B=70, T=1, L=tuple(int(x) for x in np.arange(70) * 37 % 300), cache_dtype="bf16")),
     ("fp8-70-tokens", dict(B=35, T=2, L=tuple(int(x) for x in np.arange(35) * 53 % 400), cache_dtype="fp8")),
@@ -145,7 +152,8 @@ def test_append_f32_cache_matches_oracle():
 
 @pytest.mark.parametrize("name,kw", [
     ("gemv-3", dict(B=3, T=1, L=(10, 70, 200), cache_dtype="bf16")),
-    ("cluster-8", dict(B=8, T=1, L=tuple(range(5, 800, 100)), cache_dtype="bf16")),
+    ("cluster-12", dict(B=6, T=2, L=(3, 64, 65, 300, 700, 1000), cache_dtype="fp8")),
+    ("cluster-17", dict(B=17, T=1, L=tuple(range(5, 1700, 100)), cache_dtype="bf16")),
     ("splitk-64", dict(B=32, T=2, L=tuple(int(x) for x in np.arange(32) * 29 % 300), cache_dtype="fp8")),
     ("gemm-600", dict(B=3, T=200, L=(0, 100, 1000), cache_dtype="bf16")),
 ], ids=lambda v: v if isinstance(v, str) else "")
@@ -157,6 +165,9 @@ def test_out_of_range_tokens_are_skipped_and_reported(name, kw):
     cfg = V3.with_(name=name, seed=81 + len(name), **kw)
     g = GpuProblem(cfg)
     n = cfg.B * cfg.T
+    if name.startswith("cluster"):  # the minimum workspace: the cluster kernel, not split-K
+        g.session.append_ws = torch.empty(max(B.append_workspace_bytes(g.dims, n), 256), dtype=torch.uint8,
+                                          device="cuda")
     seq_idx = g.seq_idx.clone()
     pos = g.pos.clone()
     seq_idx[1] = cfg.B            # no such sequence
